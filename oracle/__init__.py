@@ -1,0 +1,179 @@
+"""fp64 CPU oracle for block top-k sparse decode attention (TEST INFRASTRUCTURE).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline /
+reference leg may import this package.  The product library never calls it.
+It wraps ``kin_oracle.c`` (plain C, fp64, OpenMP over (batch, kv head) pairs),
+which shares no code with the CUDA library.
+
+Every function takes bf16 inputs as ``np.uint16`` bit patterns, exactly as the
+GPU path receives them, and widens them exactly to double.
+
+Parity pins: see tests/test_oracle_pins.py.  Every function here is pinned by
+at least one check that does not restate its own formula (dense attention
+from a library routine, brute-force subset search, one-hot V weights against
+scipy's softmax, per-token logits averaged per block, chunked LSE merges,
+incremental vs from-scratch means).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB = os.path.join(_HERE, "libkin_oracle.so")
+SRC = os.path.join(_HERE, "kin_oracle.c")
+
+
+def build(verbose: bool = False) -> None:
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-fvisibility=hidden",
+           SRC, "-o", LIB, "-lm"]
+    if verbose:
+        print(" ".join(cmd))
+    subprocess.run(cmd, check=True)
+
+
+_lib = None
+
+
+def _L():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
+            build()
+        lib = ctypes.CDLL(LIB)
+        vp, i32, dbl = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
+        lib.kin_oracle_block_means.argtypes = [vp, i32, i32, i32, vp]
+        lib.kin_oracle_block_scores.argtypes = [vp, i32, vp, i32, i32, vp]
+        lib.kin_oracle_select.argtypes = [vp, i32, i32, vp]
+        lib.kin_oracle_select.restype = i32
+        lib.kin_oracle_attend_partial.argtypes = [vp, i32, vp, vp, i32, i32, i32, vp, i32, dbl,
+                                                  vp, vp, vp]
+        lib.kin_oracle_merge.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp]
+        lib.kin_oracle_attend.argtypes = [vp, i32, vp, vp, i32, i32, i32, vp, i32, dbl, vp, vp]
+        lib.kin_oracle_means_update.argtypes = [vp, vp, i32, i32, vp, vp, i32, i32, vp]
+        lib.kin_oracle_decode_pairs.argtypes = [i32, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp,
+                                                vp, i32, dbl, vp, i32, vp, vp, vp, vp, vp, i32]
+        lib.kin_oracle_decode_pairs.restype = i32
+        _lib = lib
+    return _lib
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _p(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def block_means(K: np.ndarray, L: int, bs: int) -> np.ndarray:
+    """K [>=L, D] bf16 bits -> means [ceil(L/bs), D] fp64 over valid rows."""
+    K = _c(K, np.uint16)
+    D = K.shape[-1]
+    nb = -(-L // bs)
+    out = np.zeros((nb, D), dtype=np.float64)
+    _L().kin_oracle_block_means(_p(K), L, D, bs, _p(out))
+    return out
+
+
+def block_scores(q_group: np.ndarray, means: np.ndarray) -> np.ndarray:
+    """q_group [g, D] bf16 bits, means [nb, D] fp64 -> scores [nb] (scale 1/sqrt(D))."""
+    q = _c(q_group, np.uint16)
+    m = _c(means, np.float64)
+    g, D = q.shape
+    out = np.zeros(m.shape[0], dtype=np.float64)
+    _L().kin_oracle_block_scores(_p(q), g, _p(m), m.shape[0], D, _p(out))
+    return out
+
+
+def select(scores: np.ndarray, k: int):
+    """-> (sel [k] int32 ascending, -1 padded; count).  count -1: k < 2 < nb."""
+    s = _c(scores, np.float64)
+    sel = np.full(max(k, 1), -1, dtype=np.int32)
+    c = _L().kin_oracle_select(_p(s), s.shape[0], k, _p(sel))
+    return sel[:k], c
+
+
+def attend_partial(q_group, K, V, L, bs, blocks, scale):
+    q = _c(q_group, np.uint16)
+    K = _c(K, np.uint16)
+    V = _c(V, np.uint16)
+    blk = _c(blocks, np.int32)
+    g, D = q.shape
+    o = np.zeros((g, D), dtype=np.float64)
+    m = np.zeros(g, dtype=np.float64)
+    l = np.zeros(g, dtype=np.float64)
+    _L().kin_oracle_attend_partial(_p(q), g, _p(K), _p(V), L, D, bs, _p(blk), blk.shape[0],
+                                   float(scale), _p(o), _p(m), _p(l))
+    return o, m, l
+
+
+def merge(o_parts, m_parts, l_parts):
+    o = _c(o_parts, np.float64)
+    m = _c(m_parts, np.float64)
+    l = _c(l_parts, np.float64)
+    n, g, D = o.shape
+    out = np.zeros((g, D), dtype=np.float64)
+    lse = np.zeros(g, dtype=np.float64)
+    _L().kin_oracle_merge(n, g, D, _p(o), _p(m), _p(l), _p(out), _p(lse))
+    return out, lse
+
+
+def attend(q_group, K, V, L, bs, blocks, scale):
+    q = _c(q_group, np.uint16)
+    K = _c(K, np.uint16)
+    V = _c(V, np.uint16)
+    blk = _c(blocks, np.int32)
+    g, D = q.shape
+    out = np.zeros((g, D), dtype=np.float64)
+    lse = np.zeros(g, dtype=np.float64)
+    _L().kin_oracle_attend(_p(q), g, _p(K), _p(V), L, D, bs, _p(blk), blk.shape[0],
+                           float(scale), _p(out), _p(lse))
+    return out, lse
+
+
+def means_update(Kc, Vc, L0, knew, vnew, bs, means):
+    """In place on Kc, Vc [Lcap, D] (uint16) and means [nbcap, D] (fp64)."""
+    assert Kc.flags["C_CONTIGUOUS"] and Vc.flags["C_CONTIGUOUS"] and means.flags["C_CONTIGUOUS"]
+    kn = _c(knew, np.uint16)
+    vn = _c(vnew, np.uint16)
+    n, D = kn.shape
+    _L().kin_oracle_means_update(_p(Kc), _p(Vc), L0, n, _p(kn), _p(vn), D, bs, _p(means))
+
+
+def decode_pairs(*, Hkv, Hq, bs, seq_lens, q, Kc, Vc, means, k, scale, pairs, threads=0,
+                 want_scores=False):
+    """One decode step (scores, select, attend) for the listed (b*Hkv+h) pairs.
+
+    q [B,Hq,D]; Kc, Vc [B,Hkv,Lcap,D] (or any array whose pair p rows are at
+    [p]); means [B,Hkv,nbcap,D] fp64.  Returns dict(sel, cnt, out, lse[, scores]).
+    """
+    q = _c(q, np.uint16)
+    Kc = _c(Kc, np.uint16)
+    Vc = _c(Vc, np.uint16)
+    means = _c(means, np.float64)
+    lens = _c(seq_lens, np.int32)
+    pairs = _c(pairs, np.int32)
+    B, _, D = q.shape
+    Lcap = Kc.shape[-2]
+    nbcap = means.shape[-2]
+    g = Hq // Hkv
+    n = pairs.shape[0]
+    sel = np.full((n, k), -1, dtype=np.int32)
+    cnt = np.zeros(n, dtype=np.int32)
+    out = np.zeros((n, g, D), dtype=np.float64)
+    lse = np.zeros((n, g), dtype=np.float64)
+    sc = np.zeros((n, nbcap), dtype=np.float64) if want_scores else None
+    rc = _L().kin_oracle_decode_pairs(B, Hkv, Hq, D, bs, Lcap, nbcap, _p(lens), _p(q), _p(Kc),
+                                      _p(Vc), _p(means), k, float(scale), _p(pairs), n, _p(sel),
+                                      _p(cnt), _p(out), _p(lse), _p(sc) if sc is not None else None,
+                                      threads)
+    if rc != 0:
+        raise ValueError("oracle: budget k < 2 with more blocks than k")
+    res = dict(sel=sel, cnt=cnt, out=out, lse=lse)
+    if sc is not None:
+        res["scores"] = sc
+    return res

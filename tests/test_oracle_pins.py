@@ -1,0 +1,265 @@
+"""Pins for the fp64 oracle, each against something other than the oracle's
+own formula: a library routine (torch SDPA, scipy softmax, logsumexp), brute
+force over all block subsets, a different but equivalent computation (mean of
+per-token logits vs logit of the mean key), invariants (convex hull, constant
+V, split-K merge invariance, incremental == from-scratch means) and a
+constructed case (a planted block).
+
+The method (block top-k sparse decode attention) is described on the pages
+"Kinetics: Memory-Aware Test-Time Scaling" (Architecture Overview;
+Implementation, BlockTopKAttention) and "Kinetics: Rethinking Test-Time
+Scaling Law" (author response Q4, KV block size and grouping strategy).
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import kin_inputs as ki
+import oracle
+
+D = 128
+
+
+def rand_bf16(rng, shape, scale=1.0):
+    return ki.bf16_from_f32((rng.standard_normal(shape) * scale).astype(np.float32))
+
+
+def f64(bits):
+    return ki.bf16_to_f32(bits).astype(np.float64)
+
+
+# --------------------------------------------------------------- dense == SDPA
+@pytest.mark.parametrize("g,bs,lens", [(4, 16, (83, 130)), (1, 32, (64, 31)), (5, 64, (200, 1)),
+                                       (8, 16, (16, 17))])
+def test_full_budget_is_dense_attention(g, bs, lens):
+    """With k >= nb the method is plain softmax(q K^T / sqrt(d)) V over all
+    tokens (budget = block size x blocks covers the whole cache)."""
+    rng = np.random.default_rng(1 + g + bs)
+    B, Hkv = len(lens), 2
+    Hq = Hkv * g
+    lens = np.array(lens, np.int32)
+    Lcap = int(lens.max()) + 7
+    q = rand_bf16(rng, (B, Hq, D))
+    Kc = rand_bf16(rng, (B, Hkv, Lcap, D))
+    Vc = rand_bf16(rng, (B, Hkv, Lcap, D))
+    for b in range(B):  # rows beyond the length are poison and must be ignored
+        Kc[b, :, lens[b]:] = ki.BF16_NAN
+        Vc[b, :, lens[b]:] = ki.BF16_NAN
+    nbcap = -(-Lcap // bs)
+    means = np.zeros((B, Hkv, nbcap, D))
+    for b in range(B):
+        for h in range(Hkv):
+            m = oracle.block_means(Kc[b, h], int(lens[b]), bs)
+            means[b, h, :m.shape[0]] = m
+    k = nbcap + 3
+    res = oracle.decode_pairs(Hkv=Hkv, Hq=Hq, bs=bs, seq_lens=lens, q=q, Kc=Kc, Vc=Vc, means=means,
+                              k=k, scale=1 / math.sqrt(D), pairs=np.arange(B * Hkv))
+    for b in range(B):
+        L = int(lens[b])
+        qt = torch.from_numpy(f64(q[b])).view(1, Hq, 1, D)
+        Kt = torch.from_numpy(f64(Kc[b, :, :L])).repeat_interleave(g, dim=0).view(1, Hq, L, D)
+        Vt = torch.from_numpy(f64(Vc[b, :, :L])).repeat_interleave(g, dim=0).view(1, Hq, L, D)
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt).view(Hq, D).numpy()
+        lse_ref = torch.logsumexp((qt @ Kt.transpose(-1, -2)) / math.sqrt(D), dim=-1).view(Hq).numpy()
+        for h in range(Hkv):
+            p = b * Hkv + h
+            nb = -(-L // bs)
+            assert res["cnt"][p] == nb
+            assert list(res["sel"][p, :nb]) == list(range(nb))
+            assert np.all(res["sel"][p, nb:] == -1)
+            np.testing.assert_allclose(res["out"][p], ref[h * g:(h + 1) * g], rtol=0, atol=1e-12)
+            np.testing.assert_allclose(res["lse"][p], lse_ref[h * g:(h + 1) * g], rtol=1e-13, atol=1e-12)
+
+
+# ------------------------------------------------------- selection brute force
+def brute_force_select(scores, k):
+    nb = len(scores)
+    if k >= nb:
+        return list(range(nb))
+    forced = [0, nb - 1]
+    best = None
+    for combo in itertools.combinations(range(1, nb - 1), k - 2):
+        s = sorted(forced + list(combo))
+        tot = sum(scores[i] for i in s)
+        key = (-tot, tuple(s))
+        if best is None or key < best[0]:
+            best = (key, s)
+    return best[1]
+
+
+@pytest.mark.parametrize("trial", range(300))
+def test_select_maximises_summed_score(trial):
+    rng = np.random.default_rng(1000 + trial)
+    nb = int(rng.integers(1, 15))
+    k = int(rng.integers(2, 7))
+    if trial % 3 == 0:
+        scores = rng.integers(-3, 4, nb) / 8.0           # many exact ties
+    elif trial % 3 == 1:
+        scores = rng.standard_normal(nb)
+    else:
+        scores = np.full(nb, 0.25)                        # all equal
+        scores[rng.integers(0, nb)] = -1.0
+    sel, cnt = oracle.select(scores, k)
+    expect = brute_force_select(list(scores), k)
+    assert cnt == len(expect)
+    assert list(sel[:cnt]) == expect
+    assert np.all(sel[cnt:] == -1)
+
+
+def test_select_rejects_budget_below_forced_pair():
+    _, c = oracle.select(np.zeros(5), 1)
+    assert c == -1
+    sel, c = oracle.select(np.zeros(1), 1)   # one block fits a budget of one
+    assert c == 1 and sel[0] == 0
+
+
+def test_select_all_equal_prefers_low_indices():
+    sel, c = oracle.select(np.zeros(300), 10)
+    assert c == 10
+    assert list(sel) == list(range(9)) + [299]
+
+
+def test_select_large_topk_property():
+    rng = np.random.default_rng(5)
+    nb, k = 2048, 256
+    scores = np.round(rng.standard_normal(nb) * 16) / 16   # ties at the boundary
+    sel, c = oracle.select(scores, k)
+    assert c == k and sel[0] == 0 and sel[-1] == nb - 1
+    assert np.all(np.diff(sel) > 0)
+    chosen = set(int(i) for i in sel) - {0, nb - 1}
+    tau = min(scores[i] for i in chosen)
+    for i in range(1, nb - 1):
+        if scores[i] > tau:
+            assert i in chosen
+    eq = [i for i in range(1, nb - 1) if scores[i] == tau]
+    taken = [i for i in eq if i in chosen]
+    assert taken == eq[:len(taken)]
+
+
+# ------------------------------------------------------------------ linearity
+@pytest.mark.parametrize("L,bs,g", [(150, 16, 5), (64, 32, 1), (257, 64, 8)])
+def test_scores_equal_group_sum_of_mean_token_logits(L, bs, g):
+    """score(block) from the mean key == sum over the group of the mean of the
+    per-token logits q_j . K_t / sqrt(D) over the block's valid tokens."""
+    rng = np.random.default_rng(L)
+    q = rand_bf16(rng, (g, D))
+    K = rand_bf16(rng, (L + 5, D))
+    K[L:] = ki.BF16_NAN
+    s = oracle.block_scores(q, oracle.block_means(K, L, bs))
+    z = f64(q) @ f64(K[:L]).T / math.sqrt(D)           # [g, L]
+    nb = -(-L // bs)
+    ref = np.array([z[:, i * bs:min((i + 1) * bs, L)].mean(axis=1).sum() for i in range(nb)])
+    np.testing.assert_allclose(s, ref, rtol=1e-12, atol=1e-13)
+
+
+# ------------------------------------------------------- softmax weights pins
+def test_onehot_values_expose_softmax_weights():
+    """V_t = e_t makes o_j[t] the weight of token t: compare with scipy's
+    softmax of the logits, dense and sparse."""
+    rng = np.random.default_rng(3)
+    L, bs, g = 100, 16, 3
+    q = rand_bf16(rng, (g, D))
+    K = rand_bf16(rng, (L, D), 0.7)
+    V = np.zeros((L, D), np.uint16)
+    V[np.arange(L), np.arange(L)] = 0x3F80        # bf16 1.0
+    z = f64(q) @ f64(K).T / math.sqrt(D)
+    nb = -(-L // bs)
+    out, lse = oracle.attend(q, K, V, L, bs, np.arange(nb), 1 / math.sqrt(D))
+    w = out[:, :L]
+    np.testing.assert_allclose(w, scipy.special.softmax(z, axis=1), rtol=1e-13, atol=1e-15)
+    assert np.all(w >= 0)
+    np.testing.assert_allclose(w.sum(axis=1), 1.0, atol=1e-14)
+    np.testing.assert_allclose(lse, scipy.special.logsumexp(z, axis=1), rtol=1e-14)
+    blocks = np.array([0, 2, 6])
+    out, _ = oracle.attend(q, K, V, L, bs, blocks, 1 / math.sqrt(D))
+    toks = np.concatenate([np.arange(b * bs, min((b + 1) * bs, L)) for b in blocks])
+    ref = np.zeros((g, L))
+    ref[:, toks] = scipy.special.softmax(z[:, toks], axis=1)
+    np.testing.assert_allclose(out[:, :L], ref, rtol=1e-13, atol=1e-15)
+
+
+def test_output_in_convex_hull_and_constant_values():
+    rng = np.random.default_rng(4)
+    L, bs, g = 333, 32, 4
+    q = rand_bf16(rng, (g, D), 2.0)
+    K = rand_bf16(rng, (L, D))
+    V = rand_bf16(rng, (L, D))
+    blocks = np.array([0, 3, 4, 9, 10])
+    out, _ = oracle.attend(q, K, V, L, bs, blocks, 1 / math.sqrt(D))
+    toks = np.concatenate([np.arange(b * bs, min((b + 1) * bs, L)) for b in blocks])
+    vs = f64(V[toks])
+    assert np.all(out >= vs.min(axis=0) - 1e-12)
+    assert np.all(out <= vs.max(axis=0) + 1e-12)
+    Vc = np.full((L, D), ki.bf16_from_f32(np.array([1.375], np.float32))[0], np.uint16)
+    out, _ = oracle.attend(q, K, Vc, L, bs, blocks, 1 / math.sqrt(D))
+    np.testing.assert_allclose(out, 1.375, rtol=0, atol=1e-14)
+
+
+# ------------------------------------------------------------ split-K merge
+@pytest.mark.parametrize("nchunks", [1, 2, 7, 13])
+def test_chunked_merge_equals_single_pass(nchunks):
+    rng = np.random.default_rng(nchunks)
+    L, bs, g = 16 * 40 - 5, 16, 5
+    q = rand_bf16(rng, (g, D), 1.5)
+    K = rand_bf16(rng, (L, D))
+    V = rand_bf16(rng, (L, D))
+    blocks = np.array(sorted(rng.choice(np.arange(1, 39), 11, replace=False).tolist()) + [0, 39])
+    blocks.sort()
+    full, lse_full = oracle.attend(q, K, V, L, bs, blocks, 1 / math.sqrt(D))
+    parts = np.array_split(blocks, nchunks)
+    os_, ms, ls = zip(*[oracle.attend_partial(q, K, V, L, bs, p, 1 / math.sqrt(D)) for p in parts])
+    out, lse = oracle.merge(np.stack(os_), np.stack(ms), np.stack(ls))
+    np.testing.assert_allclose(out, full, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(lse, lse_full, rtol=1e-14)
+
+
+# --------------------------------------------------------------- means update
+@pytest.mark.parametrize("bs", [16, 32])
+def test_incremental_update_equals_build_from_scratch(bs):
+    rng = np.random.default_rng(bs)
+    Lcap = 130
+    Kall = rand_bf16(rng, (Lcap, D))
+    Vall = rand_bf16(rng, (Lcap, D))
+    for steps in ([1] * Lcap, [7, 1, 30, 2, 16, 1, 73]):
+        Kc = np.zeros((Lcap, D), np.uint16)
+        Vc = np.zeros((Lcap, D), np.uint16)
+        means = np.zeros((-(-Lcap // bs), D))
+        L = 0
+        for n in steps:
+            oracle.means_update(Kc, Vc, L, Kall[L:L + n], Vall[L:L + n], bs, means)
+            L += n
+            ref = oracle.block_means(Kall, L, bs)
+            assert np.array_equal(means[:ref.shape[0]], ref)
+        assert np.array_equal(Kc, Kall) and np.array_equal(Vc, Vall)
+
+
+def test_means_are_plain_averages():
+    """The mean of a block is the arithmetic mean of its valid rows (numpy)."""
+    rng = np.random.default_rng(11)
+    L, bs = 75, 16
+    K = rand_bf16(rng, (L, D))
+    m = oracle.block_means(K, L, bs)
+    for i in range(m.shape[0]):
+        np.testing.assert_allclose(m[i], f64(K[i * bs:min((i + 1) * bs, L)]).mean(axis=0), rtol=1e-15, atol=1e-16)
+
+
+# ------------------------------------------------------------- planted block
+def test_planted_block_is_selected_and_dominates():
+    rng = np.random.default_rng(12)
+    L, bs, g, k = 16 * 64, 16, 4, 8
+    q = rand_bf16(rng, (g, D))
+    K = rand_bf16(rng, (L, D))
+    V = rand_bf16(rng, (L, D))
+    planted = 37
+    q0 = f64(q[0])
+    K[planted * bs:(planted + 1) * bs] = ki.bf16_from_f32((8.0 * q0).astype(np.float32))
+    means = oracle.block_means(K, L, bs)
+    scores = oracle.block_scores(q, means)
+    sel, c = oracle.select(scores, k)
+    assert c == k and planted in sel
+    out, _ = oracle.attend(q[:1], K, V, L, bs, sel, 1 / math.sqrt(D))
+    np.testing.assert_allclose(out[0], f64(V[planted * bs:(planted + 1) * bs]).mean(axis=0), atol=1e-12)
