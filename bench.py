@@ -1,0 +1,496 @@
+"""Benchmark: block top-k sparse decode attention on B200.
+
+One step = the whole decode hot path for one batch: group-summed block scores
++ exact block top-k (kin_block_topk_select), then the split-K sparse decode
+attention with its log-sum-exp merge (kin_sparse_decode_attn); workloads with
+an append first run kin_block_means_update.  The block means and KV cache are
+resident decode state built before timing.
+
+Metric: query-heads/s = B * Hq / t_step (whole job: summed over ranks, time =
+max over ranks).  Timing: CUDA events on the launching stream, one event pair
+per kernel per step, L2 flushed (a 256 MiB write, outside the events) before
+every step; W warm-up steps; barrier + synchronize around the K timed steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--k K]
+  python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
+Multi-GPU: torchrun, one rank per GPU, each rank an independent batch shard
+(weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import kin_inputs as ki  # noqa: E402
+
+DEFAULT_WORKLOAD = "qwen3_8b_32k"
+METRIC = "block-top-k decode attn query-heads/s"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ---------------------------------------------------------------- bytes model
+def algorithmic_bytes(w: ki.Workload, k: int, lens: np.ndarray):
+    """Algorithmic HBM bytes per launch: (select, attention).
+
+    select: fp32 means of every block (skipped when k >= nb), q, indices.
+    attention: K+V rows of the kept tokens, q, bf16 out, indices.
+    """
+    nb = -(-lens.astype(np.int64) // w.bs)
+    scan = nb > k
+    means = int((w.Hkv * nb[scan] * w.D * 4).sum())
+    q_bytes = w.B * w.Hq * w.D * 2
+    idx_bytes = w.B * w.Hkv * k * 4
+    sel_bytes = means + q_bytes + idx_bytes
+    # kept tokens per pair: k full blocks incl. the (maybe partial) last one
+    toks = np.where(scan, (k - 1) * w.bs + (lens - (nb - 1) * w.bs), lens).astype(np.int64)
+    kv = int((w.Hkv * toks * w.D * 2 * 2).sum())
+    attn_bytes = kv + q_bytes + w.B * w.Hq * w.D * 2 + idx_bytes
+    return sel_bytes, attn_bytes
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_digest(name: str) -> str:
+    path = os.path.join(ROOT, "block_top_sparse_kin_b200", "csrc", name)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(kernel_file: str, workload: str, k: int):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the
+    current kernel source (profiles/traffic.txt: file workload k sha bytes)."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    digest = kernel_source_digest(kernel_file)
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) == 5 and not line.startswith("#"):
+                if parts[0] == kernel_file and parts[1] == workload and int(parts[2]) == k and parts[3] == digest:
+                    return int(float(parts[4]))
+    return None
+
+
+# -------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                mx = float(p[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, p[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_smi_id(local: int) -> str:
+    import torch
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        return str(local)
+
+
+# --------------------------------------------------------------- GPU arm
+def setup_dist(args):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def shard_workload(w: ki.Workload, rank: int) -> ki.Workload:
+    """Weak scaling: every rank decodes its own batch of the same shape
+    (independent sequences; seed offset by rank)."""
+    return w.with_(seed=w.seed + 1000 * rank) if rank else w
+
+
+def build_device_state(w: ki.Workload, k: int):
+    import torch
+    import block_top_sparse_kin_b200 as kin
+    lens_final, lens_pre, hh = ki.case_meta(w)
+    dims = kin.make_dims(w.B, w.Hkv, w.Hq, w.D, w.bs, w.cap)
+    q_host = ki.fill_q(w.seed, w.B, w.Hq, w.D)
+    st = dict(w=w, k=k, dims=dims, lens_final=lens_final, lens_pre=lens_pre, q_host=q_host)
+    st["q"] = torch.from_numpy(q_host.view(np.int16)).cuda().view(torch.bfloat16)
+    st["seq_pre"] = torch.from_numpy(lens_pre.copy()).cuda()
+    st["seq"] = st["seq_pre"].clone()
+    hh_dev = torch.from_numpy(hh).cuda()
+    kc = torch.empty((w.B, w.Hkv, w.cap, w.D), dtype=torch.bfloat16, device="cuda")
+    vc = torch.empty_like(kc)
+    ki.kv_cache_device(w.seed, True, w.B, w.Hkv, w.cap, w.D, w.bs, st["seq"], hh_dev, False, kc)
+    ki.kv_cache_device(w.seed, False, w.B, w.Hkv, w.cap, w.D, w.bs, st["seq"], hh_dev, False, vc)
+    st["k_cache"], st["v_cache"] = kc, vc
+    st["means"] = torch.zeros((w.B, w.Hkv, w.nbcap, w.D), dtype=torch.float32, device="cuda")
+    kin.kin_block_means_build(dims, kc, st["seq"], st["means"])
+    if w.n_append:
+        kn = np.empty((w.B, w.Hkv, w.n_append, w.D), np.uint16)
+        vn = np.empty_like(kn)
+        for b in range(w.B):
+            for h in range(w.Hkv):
+                t0 = int(lens_pre[b])
+                kn[b, h] = ki.kv_rows(w.seed, True, b * w.Hkv + h, t0, t0 + w.n_append, w.D, w.bs, hh[b, h])
+                vn[b, h] = ki.kv_rows(w.seed, False, b * w.Hkv + h, t0, t0 + w.n_append, w.D, w.bs, None)
+        st["k_new"] = torch.from_numpy(kn.view(np.int16)).cuda().view(torch.bfloat16)
+        st["v_new"] = torch.from_numpy(vn.view(np.int16)).cuda().view(torch.bfloat16)
+    st["sel"] = torch.empty((w.B, w.Hkv, k), dtype=torch.int32, device="cuda")
+    st["cnt"] = torch.empty((w.B, w.Hkv), dtype=torch.int32, device="cuda")
+    st["out"] = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
+    st["lse"] = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
+    st["status"] = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st["ws"] = kin.alloc_workspace(dims, k)
+    torch.cuda.synchronize()
+    return st
+
+
+def run_step(st, ev=None):
+    """One decode step.  ev: optional list of 3 or 4 events to record between kernels."""
+    import block_top_sparse_kin_b200 as kin
+    w, dims, k = st["w"], st["dims"], st["k"]
+    i = 0
+    if ev is not None:
+        ev[i].record(); i += 1
+    if w.n_append:
+        kin.kin_block_means_update(dims, st["k_cache"], st["v_cache"], st["means"], st["seq"],
+                                   st["k_new"], st["v_new"], w.n_append, st["status"])
+        if ev is not None:
+            ev[i].record(); i += 1
+    kin.kin_block_topk_select(dims, st["q"], st["means"], st["seq"], k, st["sel"], st["cnt"], st["ws"],
+                              st["status"])
+    if ev is not None:
+        ev[i].record(); i += 1
+    kin.kin_sparse_decode_attn(dims, st["q"], st["k_cache"], st["v_cache"], st["seq"], st["sel"], st["cnt"],
+                               k, 0.0, st["out"], st["lse"], st["ws"], st["status"])
+    if ev is not None:
+        ev[i].record()
+
+
+def reset_state(st):
+    if st["w"].n_append:
+        st["seq"].copy_(st["seq_pre"])
+
+
+def gpu_arm(args):
+    import torch
+    import torch.distributed as dist
+    rank, world, local = setup_dist(args)
+    w0 = ki.WORKLOADS[args.workload]
+    k = args.k or w0.k
+    w = shard_workload(w0, rank)
+    st = build_device_state(w, k)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    n_ev = 4 if w.n_append else 3
+    launches_per_step = 3 if w.n_append else 2
+
+    for _ in range(args.warmup):
+        reset_state(st)
+        run_step(st)
+    torch.cuda.synchronize()
+    if int(st["status"].item()) != 0:
+        raise RuntimeError(f"device status {int(st['status'].item())} after warm-up")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_smi_id(local)) as clk:
+        wall0 = time.perf_counter()
+        for s in range(args.steps):
+            reset_state(st)
+            flush.fill_(s & 0xFF)          # L2 flush (outside the events)
+            run_step(st, events[s])
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - wall0
+    if world > 1:
+        dist.barrier()
+    per_step = [ev[0].elapsed_time(ev[-1]) for ev in events]
+    sel_ms = [ev[-3].elapsed_time(ev[-2]) for ev in events]
+    attn_ms = [ev[-2].elapsed_time(ev[-1]) for ev in events]
+    upd_ms = [ev[0].elapsed_time(ev[1]) for ev in events] if w.n_append else []
+    total_ms = sum(per_step)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    qh_per_step = w.B * w.Hq
+    value = world * qh_per_step * args.steps / (total_ms / 1e3)
+
+    # ---- e2e: the same step through the public API with host buffers:
+    # pinned q -> device, step, device out -> pinned host, all on one stream.
+    q_pin = torch.from_numpy(st["q_host"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    out_pin = torch.empty(st["out"].shape, dtype=torch.bfloat16).pin_memory()
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for _ in range(args.warmup):
+        reset_state(st)
+        st["q"].copy_(q_pin, non_blocking=True)
+        run_step(st)
+        out_pin.copy_(st["out"], non_blocking=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    for s in range(args.steps):
+        reset_state(st)
+        flush.fill_(s & 0xFF)
+        e2e_ev[s][0].record()
+        st["q"].copy_(q_pin, non_blocking=True)
+        run_step(st)
+        out_pin.copy_(st["out"], non_blocking=True)
+        e2e_ev[s][1].record()
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * qh_per_step * args.steps / (e2e_ms / 1e3)
+    status = int(st["status"].item())
+
+    if rank == 0:
+        sel_b, attn_b = algorithmic_bytes(w, k, st["lens_final"])
+        peak, peak_kind = measured_peak()
+        sel_avg = statistics.mean(sel_ms)
+        attn_avg = statistics.mean(attn_ms)
+        attn_gbs = attn_b / (attn_avg * 1e-3) / 1e9
+        sel_gbs = sel_b / (sel_avg * 1e-3) / 1e9
+        step_gbs = (sel_b + attn_b) / (ms_per_step * 1e-3) / 1e9
+        dominant = "attn" if attn_avg >= sel_avg else "select"
+        dom_file = "kin_attn.cu" if dominant == "attn" else "kin_select.cu"
+        dom_bytes, dom_ms, dom_gbs = (attn_b, attn_avg, attn_gbs) if dominant == "attn" else (sel_b, sel_avg, sel_gbs)
+        line = {
+            "metric": METRIC,
+            "value": value,
+            "unit": "query-heads/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_per_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded Philox N(0,1) q/K/V, 5% heavy-hitter key-bias blocks)",
+            "config": {
+                "workload": w0.name, "batch": w0.B, "kv_heads": w0.Hkv, "q_heads": w0.Hq,
+                "head_dim": w0.D, "context": [w0.Lmin, w0.Lmax], "block_size": w0.bs,
+                "top_k_blocks": k, "append_tokens": w0.n_append,
+                "global_batch": w0.B * world, "parallelism": f"dp{world}",
+                "l2": "flushed before every step (256 MiB write outside the timed events)",
+            },
+            "impl": "kin",
+            "gpu_launches": launches_per_step * args.steps,
+            "kernel_ms": {"select": sel_avg, "attn": attn_avg, **({"update": statistics.mean(upd_ms)} if upd_ms else {})},
+            "hbm_gbs": {"select": sel_gbs, "attn": attn_gbs, "step": step_gbs},
+            "hbm_frac": {"select": sel_gbs / peak, "attn": attn_gbs / peak, "step": step_gbs / peak,
+                         "peak_gbs": peak, "peak_kind": peak_kind},
+            "roofline": {
+                "kernel": dominant, "bound": "hbm", "achieved": dom_gbs, "peak": peak, "unit": "GB/s",
+                "frac": dom_gbs / peak, "peak_kind": peak_kind,
+                "algorithmic_bytes_per_launch": dom_bytes,
+                "traffic": profiled_traffic(dom_file, w0.name, k),
+            },
+            "e2e": {"value": e2e_value, "unit": "query-heads/s",
+                    "h2d_bytes_per_step": int(q_pin.numel() * 2), "d2h_bytes_per_step": int(out_pin.numel() * 2)},
+            "clocks": clk.summary(),
+            "wall_s_timed_region": wall,
+            "device_status": status,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w0, k, budget_s=args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------- oracle (CPU) arm
+class OracleSample:
+    """A bounded sample of (batch, kv-head) pairs of a workload, prepared on
+    the host for the fp64 oracle: K/V rows regenerated from the seeded
+    generator and block means precomputed (resident state, as on the GPU)."""
+
+    def __init__(self, w: ki.Workload, k: int, max_pairs: int):
+        import oracle
+        self.oracle = oracle
+        self.w, self.k = w, k
+        lens_final, _, hh = ki.case_meta(w)
+        P = w.B * w.Hkv
+        n = min(max_pairs, P)
+        pairs = sorted(set(int(round(i * (P - 1) / max(n - 1, 1))) for i in range(n)))
+        self.n, self.P = len(pairs), P
+        Lmax = int(max(lens_final[p // w.Hkv] for p in pairs))
+        nbcap = -(-Lmax // w.bs)
+        q_all = ki.fill_q(w.seed, w.B, w.Hq, w.D)
+        self.Kc = np.zeros((self.n, 1, Lmax, w.D), np.uint16)
+        self.Vc = np.zeros_like(self.Kc)
+        self.means = np.zeros((self.n, 1, nbcap, w.D))
+        self.qs = np.zeros((self.n, w.g, w.D), np.uint16)
+        self.lens = np.zeros(self.n, np.int32)
+        for i, p in enumerate(pairs):
+            b, h = divmod(p, w.Hkv)
+            L = int(lens_final[b])
+            self.Kc[i, 0, :L], self.Vc[i, 0, :L] = ki.pair_rows(w, hh, b, h, L)
+            self.means[i, 0, :-(-L // w.bs)] = oracle.block_means(self.Kc[i, 0], L, w.bs)
+            self.qs[i] = q_all[b, h * w.g:(h + 1) * w.g]
+            self.lens[i] = L
+        self.threads = os.cpu_count() or 1
+
+    def run_pass(self):
+        w = self.w
+        self.oracle.decode_pairs(Hkv=1, Hq=w.g, bs=w.bs, seq_lens=self.lens, q=self.qs, Kc=self.Kc,
+                                 Vc=self.Vc, means=self.means, k=self.k, scale=1 / math.sqrt(w.D),
+                                 pairs=np.arange(self.n), threads=self.threads)
+        return self.n * w.g  # query heads processed
+
+    def describe(self, passes, seconds):
+        return (f"{self.n} of {self.P} (batch, kv-head) pairs of {self.w.name} (k={self.k}), {passes} "
+                f"passes in {seconds:.1f} s; scores + top-k + attention in fp64, block means precomputed")
+
+
+def cpu_baseline(w: ki.Workload, k: int, budget_s: float = 12.0, max_pairs: int = 32):
+    """The oracle (as it stands) on the host cores: whole passes over the
+    sample until `budget_s` has elapsed; query-heads/s."""
+    smp = OracleSample(w, k, max_pairs)
+    t0 = time.perf_counter()
+    passes, qh = 0, 0
+    while True:
+        qh += smp.run_pass()
+        passes += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return {"value": qh / el, "unit": "query-heads/s", "cores": smp.threads, "kind": "oracle",
+            "sample": smp.describe(passes, el)}
+
+
+def reference_arm(args):
+    """The oracle as the reference arm: each step is one pass over a bounded
+    sample of the workload's pairs, timed on the host clock."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = ki.WORKLOADS[args.workload]
+    k = args.k or w.k
+    t0 = time.perf_counter()
+    smp = OracleSample(w, k, max_pairs=args.ref_pairs)
+    for _ in range(args.warmup):
+        smp.run_pass()
+    el, qh = 0.0, 0
+    for _ in range(args.steps):
+        a = time.perf_counter()
+        qh += smp.run_pass()
+        el += time.perf_counter() - a
+    value = qh / el
+    line = {
+        "metric": METRIC, "value": value, "unit": "query-heads/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": w.B * w.Hq / value * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.B, "kv_heads": w.Hkv, "q_heads": w.Hq, "head_dim": w.D,
+                   "context": [w.Lmin, w.Lmax], "block_size": w.bs, "top_k_blocks": k},
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "query-heads/s", "cores": smp.threads, "kind": "oracle",
+                         "sample": smp.describe(args.steps, el)},
+        "e2e": {"value": value, "unit": "query-heads/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": time.perf_counter() - t0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="kin", choices=["kin", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(ki.WORKLOADS))
+    ap.add_argument("--k", type=int, default=0, help="override the workload's block budget")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-pairs", type=int, default=8, help="pairs per reference-arm step")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "kin":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        reference_arm(args)
+    else:
+        gpu_arm(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,171 @@
+"""Python binding of libkin.so: block top-k sparse decode attention on B200.
+
+Argument marshalling only.  Every function has the name of the C entry point
+it wraps (see include/kin.h for the exact semantics, layouts and errors),
+takes CUDA tensors, passes their device pointers and the current CUDA stream,
+and raises KinError when the library returns a non-OK status.  All
+arithmetic runs in the library's CUDA kernels; there is no fallback: if
+libkin.so is missing or cannot be loaded, the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkin.so")
+
+KIN_OK = 0
+STATUS_NAMES = {
+    0: "KIN_OK", 1: "KIN_ERR_INVALID_ARG", 2: "KIN_ERR_WORKSPACE", 3: "KIN_ERR_CAPACITY",
+    4: "KIN_ERR_CUDA", 5: "KIN_ERR_DEVICE_DATA", 6: "KIN_ERR_TIMEOUT",
+}
+EXPORTED = (
+    "kin_status_string", "kin_workspace_bytes", "kin_block_means_build",
+    "kin_block_means_update", "kin_block_topk_select", "kin_sparse_decode_attn",
+)
+
+
+class KinError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+class kin_dims(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32),
+        ("num_q_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("block_size", ctypes.c_int32),
+        ("max_seq_len", ctypes.c_int32),
+    ]
+
+    def __repr__(self):
+        return "kin_dims(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+def make_dims(batch, num_kv_heads, num_q_heads, head_dim, block_size, max_seq_len) -> kin_dims:
+    return kin_dims(batch, num_kv_heads, num_q_heads, head_dim, block_size, max_seq_len)
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libkin.so (once) and declare the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"libkin.so not found at {path}: build it with "
+            "`python -m block_top_sparse_kin_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(path)
+    vp, i32, sz, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_float
+    dp = ctypes.POINTER(kin_dims)
+    lib.kin_status_string.argtypes = [ctypes.c_int]
+    lib.kin_status_string.restype = ctypes.c_char_p
+    lib.kin_workspace_bytes.argtypes = [dp, i32]
+    lib.kin_workspace_bytes.restype = sz
+    lib.kin_block_means_build.argtypes = [dp, vp, vp, vp, vp, vp]
+    lib.kin_block_means_build.restype = ctypes.c_int
+    lib.kin_block_means_update.argtypes = [dp, vp, vp, vp, vp, vp, vp, i32, vp, vp]
+    lib.kin_block_means_update.restype = ctypes.c_int
+    lib.kin_block_topk_select.argtypes = [dp, vp, vp, vp, i32, vp, vp, vp, sz, vp, vp]
+    lib.kin_block_topk_select.restype = ctypes.c_int
+    lib.kin_sparse_decode_attn.argtypes = [dp, vp, vp, vp, vp, vp, vp, i32, f32, vp, vp, vp, sz,
+                                           vp, vp]
+    lib.kin_sparse_decode_attn.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _dev(t: Optional[torch.Tensor], name: str, dtype=None, nullable=False):
+    if t is None:
+        if nullable:
+            return None
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(rc: int, where: str):
+    if rc != KIN_OK:
+        raise KinError(rc, where)
+
+
+_BF16 = (torch.bfloat16, torch.uint16, torch.int16)
+
+
+def kin_status_string(status: int) -> str:
+    return load_library().kin_status_string(status).decode()
+
+
+def kin_workspace_bytes(dims: kin_dims, k_blocks: int) -> int:
+    return int(load_library().kin_workspace_bytes(ctypes.byref(dims), k_blocks))
+
+
+def alloc_workspace(dims: kin_dims, k_blocks: int, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace tensor of kin_workspace_bytes (torch allocations are 256-B aligned)."""
+    n = kin_workspace_bytes(dims, k_blocks)
+    if n == 0:
+        raise KinError(1, "kin_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def kin_block_means_build(dims, k_cache, seq_lens, block_means, dev_status=None, stream=None):
+    rc = load_library().kin_block_means_build(
+        ctypes.byref(dims), _dev(k_cache, "k_cache", _BF16), _dev(seq_lens, "seq_lens", torch.int32),
+        _dev(block_means, "block_means", torch.float32),
+        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+    _check(rc, "kin_block_means_build")
+
+
+def kin_block_means_update(dims, k_cache, v_cache, block_means, seq_lens, k_new, v_new, n_new,
+                           dev_status=None, stream=None):
+    rc = load_library().kin_block_means_update(
+        ctypes.byref(dims), _dev(k_cache, "k_cache", _BF16), _dev(v_cache, "v_cache", _BF16),
+        _dev(block_means, "block_means", torch.float32), _dev(seq_lens, "seq_lens", torch.int32),
+        _dev(k_new, "k_new", _BF16), _dev(v_new, "v_new", _BF16), int(n_new),
+        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+    _check(rc, "kin_block_means_update")
+
+
+def kin_block_topk_select(dims, q, block_means, seq_lens, k_blocks, sel_idx, sel_cnt, workspace,
+                          dev_status=None, stream=None):
+    rc = load_library().kin_block_topk_select(
+        ctypes.byref(dims), _dev(q, "q", _BF16), _dev(block_means, "block_means", torch.float32),
+        _dev(seq_lens, "seq_lens", torch.int32), int(k_blocks), _dev(sel_idx, "sel_idx", torch.int32),
+        _dev(sel_cnt, "sel_cnt", torch.int32), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(),
+        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+    _check(rc, "kin_block_topk_select")
+
+
+def kin_sparse_decode_attn(dims, q, k_cache, v_cache, seq_lens, sel_idx, sel_cnt, k_blocks,
+                           softmax_scale, out, lse, workspace, dev_status=None, stream=None):
+    rc = load_library().kin_sparse_decode_attn(
+        ctypes.byref(dims), _dev(q, "q", _BF16), _dev(k_cache, "k_cache", _BF16),
+        _dev(v_cache, "v_cache", _BF16), _dev(seq_lens, "seq_lens", torch.int32),
+        _dev(sel_idx, "sel_idx", torch.int32), _dev(sel_cnt, "sel_cnt", torch.int32),
+        int(k_blocks), float(softmax_scale), _dev(out, "out", _BF16),
+        _dev(lse, "lse", torch.float32, nullable=True), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(),
+        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+    _check(rc, "kin_sparse_decode_attn")

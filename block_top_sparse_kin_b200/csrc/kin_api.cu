@@ -1,0 +1,273 @@
+// kin_api.cu -- the extern "C" boundary of libkin.so: argument checks,
+// workspace layout, launch-shape heuristics, TMA descriptors and launches.
+// Semantics of every call are documented in include/kin.h.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+
+#include "kin_internal.cuh"
+
+#define KIN_EXPORT extern "C" __attribute__((visibility("default")))
+
+namespace {
+
+using namespace kin;
+
+constexpr int kTargetSMs = 148;  // B200 SM count, used only to shape grids
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+kin_status check_dims(const kin_dims* d) {
+  if (!d) return KIN_ERR_INVALID_ARG;
+  if (d->batch < 1 || d->num_kv_heads < 1 || d->num_q_heads < 1 || d->max_seq_len < 1)
+    return KIN_ERR_INVALID_ARG;
+  if (d->num_q_heads % d->num_kv_heads != 0) return KIN_ERR_INVALID_ARG;
+  if (d->head_dim != kHeadDim) return KIN_ERR_INVALID_ARG;
+  const int bs = d->block_size;
+  if (bs != 16 && bs != 32 && bs != 64 && bs != 128) return KIN_ERR_INVALID_ARG;
+  if (d->num_q_heads / d->num_kv_heads > kMaxGroup) return KIN_ERR_CAPACITY;
+  if ((d->max_seq_len + bs - 1) / bs > kMaxBlocksPerSeq) return KIN_ERR_CAPACITY;
+  if ((int64_t)d->batch * d->num_kv_heads * d->max_seq_len >= (int64_t)1 << 31) return KIN_ERR_CAPACITY;
+  return KIN_OK;
+}
+
+int nbcap_of(const kin_dims& d) { return (d.max_seq_len + d.block_size - 1) / d.block_size; }
+int pairs_of(const kin_dims& d) { return d.batch * d.num_kv_heads; }
+
+// Blocks of means per select CTA: 128 (64 KB of fp32 means), halved down to
+// 32 while the grid would hold fewer than 4 CTAs per SM.
+int select_chunk_blocks(const kin_dims& d) {
+  const int nbcap = nbcap_of(d);
+  int ch = 128;
+  while (ch > 32 && (int64_t)pairs_of(d) * ((nbcap + ch - 1) / ch) < 4 * kTargetSMs) ch >>= 1;
+  return ch;
+}
+
+// Kept blocks per attention CTA: 512 tokens (256 KB of K+V), fewer when the
+// grid would hold fewer than 2 CTAs per SM.
+int attn_chunk_blocks(const kin_dims& d, int k) {
+  const int k_eff = k < nbcap_of(d) ? k : nbcap_of(d);
+  const int by_tokens = 512 / d.block_size > 0 ? 512 / d.block_size : 1;
+  const int64_t by_grid = (int64_t)k_eff * pairs_of(d) / (2 * kTargetSMs);
+  int ch = by_tokens;
+  if (by_grid < ch) ch = by_grid > 0 ? (int)by_grid : 1;
+  return ch;
+}
+
+int attn_max_chunks(const kin_dims& d, int k) {
+  const int k_eff = k < nbcap_of(d) ? k : nbcap_of(d);
+  const int ch = attn_chunk_blocks(d, k);
+  return (k_eff + ch - 1) / ch;
+}
+
+struct WsLayout {
+  size_t sel_counters, attn_counters, scores, partials, total;
+};
+
+WsLayout ws_layout(const kin_dims& d, int k) {
+  WsLayout w;
+  const size_t pairs = (size_t)pairs_of(d);
+  const size_t g = (size_t)(d.num_q_heads / d.num_kv_heads);
+  size_t off = 0;
+  w.sel_counters = off;
+  off = align_up(off + pairs * sizeof(uint32_t));
+  w.attn_counters = off;
+  off = align_up(off + pairs * sizeof(uint32_t));
+  w.scores = off;
+  off = align_up(off + pairs * (size_t)nbcap_of(d) * sizeof(float));
+  w.partials = off;
+  off = align_up(off + pairs * (size_t)attn_max_chunks(d, k) * g * (kHeadDim + 2) * sizeof(float));
+  w.total = off;
+  return w;
+}
+
+kin_status check_ws(const kin_dims& d, int k, void* ws, size_t ws_bytes, WsLayout* out) {
+  *out = ws_layout(d, k);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return KIN_ERR_WORKSPACE;
+  if (ws_bytes < out->total) return KIN_ERR_WORKSPACE;
+  return KIN_OK;
+}
+
+kin_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KIN_OK : KIN_ERR_CUDA; }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point, so the
+// library needs no link-time dependency on libcuda.
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+// 2-D view [rows, 128] of a bf16 cache; box 16 rows x 64 columns (128 bytes,
+// the 128-byte swizzle span).
+bool encode_cache_map(CUtensorMap* m, const void* base, uint64_t rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)kTileTokens};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+KIN_EXPORT const char* kin_status_string(kin_status s) {
+  switch (s) {
+    case KIN_OK: return "KIN_OK";
+    case KIN_ERR_INVALID_ARG: return "KIN_ERR_INVALID_ARG";
+    case KIN_ERR_WORKSPACE: return "KIN_ERR_WORKSPACE";
+    case KIN_ERR_CAPACITY: return "KIN_ERR_CAPACITY";
+    case KIN_ERR_CUDA: return "KIN_ERR_CUDA";
+    case KIN_ERR_DEVICE_DATA: return "KIN_ERR_DEVICE_DATA";
+    case KIN_ERR_TIMEOUT: return "KIN_ERR_TIMEOUT";
+  }
+  return "KIN_ERR_UNKNOWN";
+}
+
+KIN_EXPORT size_t kin_workspace_bytes(const kin_dims* dims, int32_t k_blocks) {
+  if (check_dims(dims) != KIN_OK || k_blocks < 2) return 0;
+  return ws_layout(*dims, k_blocks).total;
+}
+
+KIN_EXPORT kin_status kin_block_means_build(const kin_dims* dims, const void* k_cache,
+                                            const int32_t* seq_lens, float* block_means,
+                                            int32_t* dev_status, void* stream) {
+  kin_status st = check_dims(dims);
+  if (st != KIN_OK) return st;
+  if (!k_cache || !seq_lens || !block_means) return KIN_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(block_means)) return KIN_ERR_INVALID_ARG;
+  MeansBuildParams p;
+  p.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
+  p.seq_lens = seq_lens;
+  p.means = block_means;
+  p.dev_status = dev_status;
+  p.B = dims->batch;
+  p.Hkv = dims->num_kv_heads;
+  p.Lcap = dims->max_seq_len;
+  p.bs = dims->block_size;
+  p.nbcap = nbcap_of(*dims);
+  return from_cuda(launch_means_build(p, static_cast<cudaStream_t>(stream)));
+}
+
+KIN_EXPORT kin_status kin_block_means_update(const kin_dims* dims, void* k_cache, void* v_cache,
+                                             float* block_means, int32_t* seq_lens,
+                                             const void* k_new, const void* v_new, int32_t n_new,
+                                             int32_t* dev_status, void* stream) {
+  kin_status st = check_dims(dims);
+  if (st != KIN_OK) return st;
+  if (n_new < 0) return KIN_ERR_INVALID_ARG;
+  if (n_new > dims->max_seq_len) return KIN_ERR_CAPACITY;
+  if (n_new == 0) return KIN_OK;
+  if (!k_cache || !v_cache || !block_means || !seq_lens || !k_new || !v_new) return KIN_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(block_means) || !aligned16(k_new) ||
+      !aligned16(v_new))
+    return KIN_ERR_INVALID_ARG;
+  MeansUpdateParams p;
+  p.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+  p.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  p.means = block_means;
+  p.seq_lens = seq_lens;
+  p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  p.dev_status = dev_status;
+  p.B = dims->batch;
+  p.Hkv = dims->num_kv_heads;
+  p.Lcap = dims->max_seq_len;
+  p.bs = dims->block_size;
+  p.nbcap = nbcap_of(*dims);
+  p.n_new = n_new;
+  return from_cuda(launch_means_update(p, static_cast<cudaStream_t>(stream)));
+}
+
+KIN_EXPORT kin_status kin_block_topk_select(const kin_dims* dims, const void* q, const float* block_means,
+                                            const int32_t* seq_lens, int32_t k_blocks, int32_t* sel_idx,
+                                            int32_t* sel_cnt, void* workspace, size_t ws_bytes,
+                                            int32_t* dev_status, void* stream) {
+  kin_status st = check_dims(dims);
+  if (st != KIN_OK) return st;
+  if (k_blocks < 2) return KIN_ERR_INVALID_ARG;
+  if (!q || !block_means || !seq_lens || !sel_idx || !sel_cnt) return KIN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(block_means)) return KIN_ERR_INVALID_ARG;
+  WsLayout w;
+  st = check_ws(*dims, k_blocks, workspace, ws_bytes, &w);
+  if (st != KIN_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  SelectParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.means = block_means;
+  p.seq_lens = seq_lens;
+  p.sel_idx = sel_idx;
+  p.sel_cnt = sel_cnt;
+  p.scores = reinterpret_cast<float*>(ws + w.scores);
+  p.counters = reinterpret_cast<uint32_t*>(ws + w.sel_counters);
+  p.dev_status = dev_status;
+  p.B = dims->batch;
+  p.Hkv = dims->num_kv_heads;
+  p.Hq = dims->num_q_heads;
+  p.g = dims->num_q_heads / dims->num_kv_heads;
+  p.bs = dims->block_size;
+  p.Lcap = dims->max_seq_len;
+  p.nbcap = nbcap_of(*dims);
+  p.k = k_blocks;
+  p.chunk_blocks = select_chunk_blocks(*dims);
+  p.score_scale = 1.0f / std::sqrt((float)kHeadDim);
+  const int grid_x = (p.nbcap + p.chunk_blocks - 1) / p.chunk_blocks;
+  return from_cuda(launch_select(p, grid_x, static_cast<cudaStream_t>(stream)));
+}
+
+KIN_EXPORT kin_status kin_sparse_decode_attn(const kin_dims* dims, const void* q, const void* k_cache,
+                                             const void* v_cache, const int32_t* seq_lens,
+                                             const int32_t* sel_idx, const int32_t* sel_cnt,
+                                             int32_t k_blocks, float softmax_scale, void* out, float* lse,
+                                             void* workspace, size_t ws_bytes, int32_t* dev_status,
+                                             void* stream) {
+  kin_status st = check_dims(dims);
+  if (st != KIN_OK) return st;
+  if (k_blocks < 2) return KIN_ERR_INVALID_ARG;
+  if (!q || !k_cache || !v_cache || !seq_lens || !sel_idx || !sel_cnt || !out) return KIN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+    return KIN_ERR_INVALID_ARG;
+  if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale)) return KIN_ERR_INVALID_ARG;
+  WsLayout w;
+  st = check_ws(*dims, k_blocks, workspace, ws_bytes, &w);
+  if (st != KIN_OK) return st;
+  const uint64_t rows = (uint64_t)dims->batch * dims->num_kv_heads * dims->max_seq_len;
+  CUtensorMap tmk, tmv;
+  if (!encode_cache_map(&tmk, k_cache, rows) || !encode_cache_map(&tmv, v_cache, rows)) return KIN_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  AttnParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.seq_lens = seq_lens;
+  p.sel_idx = sel_idx;
+  p.sel_cnt = sel_cnt;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.partials = reinterpret_cast<float*>(ws + w.partials);
+  p.counters = reinterpret_cast<uint32_t*>(ws + w.attn_counters);
+  p.dev_status = dev_status;
+  p.B = dims->batch;
+  p.Hkv = dims->num_kv_heads;
+  p.Hq = dims->num_q_heads;
+  p.g = dims->num_q_heads / dims->num_kv_heads;
+  p.bs = dims->block_size;
+  p.Lcap = dims->max_seq_len;
+  p.k = k_blocks;
+  p.chunk_blocks = attn_chunk_blocks(*dims, k_blocks);
+  p.max_chunks = attn_max_chunks(*dims, k_blocks);
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)kHeadDim);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  return from_cuda(launch_attn(p, tmk, tmv, p.max_chunks, static_cast<cudaStream_t>(stream)));
+}

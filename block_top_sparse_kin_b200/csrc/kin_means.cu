@@ -1,0 +1,117 @@
+// kin_means.cu -- block mean keys: build for a prefilled cache, and the
+// append-and-refresh update of a decode step.
+//
+// The block summary is the mean key over the block's valid tokens (the block
+// mean of "Kinetics: Memory-Aware Test-Time Scaling", Implementation,
+// BlockTopKAttention, read along the key axis).  Means are summed in fp32 in
+// token order and divided by the valid-row count, so a refreshed block is
+// bit-identical to one built from scratch.
+//
+// Layout: one warp per block; lane l owns dims 4l..4l+3, so every cache row is
+// one coalesced 256-byte warp load and every mean one 512-byte warp store.
+#include "kin_internal.cuh"
+
+namespace kin {
+
+__device__ __forceinline__ void add_row4(float (&acc)[4], uint2 raw) {
+  __nv_bfloat162 lo = *reinterpret_cast<__nv_bfloat162*>(&raw.x);
+  __nv_bfloat162 hi = *reinterpret_cast<__nv_bfloat162*>(&raw.y);
+  float2 a = __bfloat1622float2(lo), b = __bfloat1622float2(hi);
+  acc[0] += a.x;
+  acc[1] += a.y;
+  acc[2] += b.x;
+  acc[3] += b.y;
+}
+
+// grid (ceil(nbcap / 8), Hkv, B), 256 threads: warp w of CTA x owns block 8x + w.
+__global__ void __launch_bounds__(256) means_build_kernel(MeansBuildParams p) {
+  const int b = blockIdx.z, h = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int L = p.seq_lens[b];
+  if (L < 0 || L > p.Lcap) {
+    if (blockIdx.x == 0 && h == 0 && threadIdx.x == 0) set_status(p.dev_status, KIN_ERR_DEVICE_DATA);
+    return;
+  }
+  const int i = blockIdx.x * 8 + warp;
+  const int nb = (L + p.bs - 1) / p.bs;
+  if (i >= nb) return;
+  const int64_t pair = (int64_t)b * p.Hkv + h;
+  const int t0 = i * p.bs;
+  const int t1 = min(t0 + p.bs, L);
+  const uint2* src = reinterpret_cast<const uint2*>(p.k_cache + (pair * p.Lcap + t0) * kHeadDim) + lane;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  int t = t0;
+  for (; t + 8 <= t1; t += 8) {  // 8 rows in flight per lane
+    uint2 r[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) r[u] = __ldg(src + (int64_t)(t - t0 + u) * (kHeadDim / 4));
+#pragma unroll
+    for (int u = 0; u < 8; ++u) add_row4(acc, r[u]);
+  }
+  for (; t < t1; ++t) add_row4(acc, __ldg(src + (int64_t)(t - t0) * (kHeadDim / 4)));
+  const float n = (float)(t1 - t0);
+  float4 m = make_float4(__fdiv_rn(acc[0], n), __fdiv_rn(acc[1], n), __fdiv_rn(acc[2], n),
+                         __fdiv_rn(acc[3], n));
+  reinterpret_cast<float4*>(p.means + (pair * p.nbcap + i) * kHeadDim)[lane] = m;
+}
+
+// grid (B), 256 threads.  One CTA owns a whole sequence so that the length
+// it reads and the length it writes back cannot race with another CTA.
+__global__ void __launch_bounds__(256) means_update_kernel(MeansUpdateParams p) {
+  const int b = blockIdx.x;
+  const int L0 = p.seq_lens[b];
+  const int n = p.n_new;
+  if (L0 < 0 || (int64_t)L0 + n > p.Lcap) {
+    if (threadIdx.x == 0) set_status(p.dev_status, KIN_ERR_DEVICE_DATA);
+    return;
+  }
+  const int L1 = L0 + n;
+  // 1. copy the new rows into the caches (16-byte chunks, 16 per row)
+  const int64_t chunks = (int64_t)p.Hkv * n * (kHeadDim / 8);
+  for (int64_t c = threadIdx.x; c < chunks; c += blockDim.x) {
+    const int h = (int)(c / ((int64_t)n * 16));
+    const int64_t rem = c - (int64_t)h * n * 16;
+    const int r = (int)(rem / 16), q16 = (int)(rem % 16);
+    const int64_t pair = (int64_t)b * p.Hkv + h;
+    const int64_t src = (((int64_t)b * p.Hkv + h) * n + r) * 16 + q16;
+    const int64_t dst = (pair * p.Lcap + L0 + r) * 16 + q16;
+    reinterpret_cast<uint4*>(p.k_cache)[dst] = reinterpret_cast<const uint4*>(p.k_new)[src];
+    reinterpret_cast<uint4*>(p.v_cache)[dst] = reinterpret_cast<const uint4*>(p.v_new)[src];
+  }
+  // 2. recompute the mean of every touched block from its valid rows; rows
+  //    below L0 come from the cache, newer rows straight from k_new.
+  const int first = L0 / p.bs, last = (L1 - 1) / p.bs;
+  const int nblk = last - first + 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  for (int task = warp; task < p.Hkv * nblk; task += nwarps) {
+    const int h = task / nblk, i = first + task % nblk;
+    const int64_t pair = (int64_t)b * p.Hkv + h;
+    const int t0 = i * p.bs, t1 = min(t0 + p.bs, L1);
+    const uint2* cache = reinterpret_cast<const uint2*>(p.k_cache + pair * p.Lcap * kHeadDim) + lane;
+    const uint2* fresh = reinterpret_cast<const uint2*>(p.k_new + pair * n * kHeadDim) + lane;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int t = t0; t < t1; ++t) {
+      uint2 raw = t < L0 ? cache[(int64_t)t * (kHeadDim / 4)] : fresh[(int64_t)(t - L0) * (kHeadDim / 4)];
+      add_row4(acc, raw);
+    }
+    const float cnt = (float)(t1 - t0);
+    float4 m = make_float4(__fdiv_rn(acc[0], cnt), __fdiv_rn(acc[1], cnt), __fdiv_rn(acc[2], cnt),
+                           __fdiv_rn(acc[3], cnt));
+    reinterpret_cast<float4*>(p.means + (pair * p.nbcap + i) * kHeadDim)[lane] = m;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) p.seq_lens[b] = L1;
+}
+
+cudaError_t launch_means_build(const MeansBuildParams& p, cudaStream_t s) {
+  dim3 grid((p.nbcap + 7) / 8, p.Hkv, p.B);
+  means_build_kernel<<<grid, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_means_update(const MeansUpdateParams& p, cudaStream_t s) {
+  means_update_kernel<<<p.B, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace kin

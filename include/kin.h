@@ -1,0 +1,153 @@
+/*
+ * kin.h -- C ABI of the B200 (sm_100a) block top-k sparse decode attention
+ * library libkin.so.
+ *
+ * The method: for every sequence b and KV head h of a decode batch, keep one
+ * mean key per fixed-size KV block, score each block against the GQA query
+ * group, keep the top-k blocks (the first block and the block holding the
+ * newest token always among them), and run softmax(q K^T / sqrt(d)) V over
+ * the tokens of the kept blocks only.
+ *   - "Kinetics: Memory-Aware Test-Time Scaling", Architecture Overview
+ *     (block-level top-k sparsity) and Implementation, BlockTopKAttention
+ *     (1/sqrt(head_dim) scaling, mean over a block, top-k over blocks,
+ *     softmax then the weighted sum of V).
+ *   - "Kinetics: Rethinking Test-Time Scaling Law", author response Q4
+ *     "KV block size and grouping strategy" (KV budget = block size x number
+ *     of top-k blocks, e.g. (16, 64), (32, 32), (64, 16)) and response Q3
+ *     (decode batches with ragged KV lengths).
+ * Readings where the pages are silent: the block summary is the mean key of
+ * the block's valid tokens; a group's block score is the sum over its query
+ * heads; the budget k counts the two forced blocks; ties go to the lower
+ * block index; query head j reads KV head j / (Hq / Hkv).
+ *
+ * Conventions shared by every call
+ *  - All tensor pointers are caller-owned DEVICE memory (e.g. PyTorch
+ *    tensors), C-contiguous, 16-byte aligned.  The library never allocates,
+ *    frees or synchronises; every call is asynchronous on `stream` (a
+ *    cudaStream_t; NULL means the legacy default stream).
+ *  - Layouts (bf16 = 2-byte bfloat16):
+ *      q            [B][Hq][D]            bf16
+ *      k_cache/v_cache [B][Hkv][Lcap][D]  bf16  (Lcap = dims.max_seq_len)
+ *      block_means  [B][Hkv][NBcap][D]    fp32  (NBcap = ceil(Lcap / bs))
+ *      seq_lens     [B]                   int32 (valid tokens per sequence)
+ *      sel_idx      [B][Hkv][k]           int32 ascending, -1 padded
+ *      sel_cnt      [B][Hkv]              int32
+ *      out          [B][Hq][D]            bf16
+ *      lse          [B][Hq]               fp32  natural-log log-sum-exp
+ *  - The host checks every argument it can before launching and returns a
+ *    status; after launching it returns KIN_ERR_CUDA if the launch failed.
+ *  - Data that only the device can see (a sequence length outside
+ *    [1, Lcap], a block index outside [0, nb)) makes the kernel skip that
+ *    item and write the status code into *dev_status (first error wins) when
+ *    dev_status is not NULL.  Kernels never trap; every wait is bounded.
+ *  - No C++ exception crosses this boundary; the library keeps no state
+ *    between calls other than what the caller's buffers hold.
+ *  - Limits: head_dim == 128; Hq % Hkv == 0 with 1 <= Hq/Hkv <= 8;
+ *    block_size in {16, 32, 64, 128}; ceil(Lcap / bs) <= 32768;
+ *    B * Hkv * Lcap < 2^31.
+ */
+#ifndef KIN_H
+#define KIN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KIN_OK = 0,
+  KIN_ERR_INVALID_ARG = 1,  /* null pointer, bad dimension, k < 2, misaligned */
+  KIN_ERR_WORKSPACE = 2,    /* workspace NULL, too small or misaligned */
+  KIN_ERR_CAPACITY = 3,     /* a size beyond a documented limit */
+  KIN_ERR_CUDA = 4,         /* a CUDA runtime/driver call or launch failed */
+  KIN_ERR_DEVICE_DATA = 5,  /* (device) bad seq_len / block index: item skipped */
+  KIN_ERR_TIMEOUT = 6       /* (device) a bounded wait expired: item skipped */
+} kin_status;
+
+typedef struct {
+  int32_t batch;         /* B */
+  int32_t num_kv_heads;  /* Hkv */
+  int32_t num_q_heads;   /* Hq, a multiple of Hkv */
+  int32_t head_dim;      /* D, must be 128 */
+  int32_t block_size;    /* bs, tokens per KV block: 16, 32, 64 or 128 */
+  int32_t max_seq_len;   /* Lcap, cache capacity in tokens per sequence */
+} kin_dims;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* kin_status_string(kin_status s);
+
+/* Bytes of scratch the select and attention calls need for budget k_blocks
+ * (one buffer serves both calls: each uses its own disjoint region).  Returns
+ * 0 if the dims are invalid.  The buffer must be 256-byte aligned and filled
+ * with zeros before its first use; every call leaves its completion counters
+ * at zero again, so the same buffer can be reused by later calls on the same
+ * stream without re-zeroing.  Calls that share one workspace must not run
+ * concurrently. */
+size_t kin_workspace_bytes(const kin_dims* dims, int32_t k_blocks);
+
+/* Block means of a prefilled cache: for every (b, h) and block
+ * i < ceil(seq_lens[b] / bs), block_means[b][h][i][:] = mean of K rows
+ * i*bs .. min((i+1)*bs, seq_lens[b]) - 1, summed in fp32 in token order and
+ * divided by the number of valid rows.  Blocks at or beyond the length are
+ * left untouched.  Reads k_cache; writes block_means.  This is the prefill
+ * counterpart of kin_block_means_update (the same definition applied to
+ * every block at once). */
+kin_status kin_block_means_build(const kin_dims* dims, const void* k_cache,
+                                 const int32_t* seq_lens, float* block_means,
+                                 int32_t* dev_status, void* stream);
+
+/* Append n_new tokens to every sequence and refresh the block means they
+ * touch.  For each b with L0 = seq_lens[b] (read on the device):
+ * k_new[b][h][r] / v_new[b][h][r] ([B][Hkv][n_new][D] bf16) are written to
+ * cache rows L0 + r; the mean of every block that holds one of those rows is
+ * recomputed from all its valid rows (fp32, token order, divided by the
+ * count); then seq_lens[b] = L0 + n_new.  A sequence with L0 < 0 or
+ * L0 + n_new > Lcap is skipped and flagged KIN_ERR_DEVICE_DATA.
+ * seq_lens is device memory, read and written.  n_new == 0 is a no-op. */
+kin_status kin_block_means_update(const kin_dims* dims, void* k_cache, void* v_cache,
+                                  float* block_means, int32_t* seq_lens,
+                                  const void* k_new, const void* v_new, int32_t n_new,
+                                  int32_t* dev_status, void* stream);
+
+/* Group-summed block scores then exact block top-k.  For pair (b, h) with
+ * nb = ceil(seq_lens[b] / bs):
+ *   s_i = (1/sqrt(D)) * sum_{j < g} q[b][h*g + j] . block_means[b][h][i],
+ * computed in fp32 from the fp32 means.
+ * If k_blocks >= nb, all nb blocks are kept.  Otherwise blocks 0 and nb-1
+ * are kept and the other k_blocks - 2 are the best of 1..nb-2 by
+ * (s descending, index ascending).  sel_idx[b][h][:] receives the kept
+ * indices ascending followed by -1 padding to k_blocks; sel_cnt[b][h] the
+ * count.  k_blocks < 2 is KIN_ERR_INVALID_ARG.  A sequence whose length is
+ * outside [1, Lcap] gets sel_cnt 0 and is flagged KIN_ERR_DEVICE_DATA.
+ * workspace: see kin_workspace_bytes. */
+kin_status kin_block_topk_select(const kin_dims* dims, const void* q, const float* block_means,
+                                 const int32_t* seq_lens, int32_t k_blocks, int32_t* sel_idx,
+                                 int32_t* sel_cnt, void* workspace, size_t ws_bytes,
+                                 int32_t* dev_status, void* stream);
+
+/* Split-K flash-decode over the selected blocks, then a log-sum-exp merge.
+ * For query head j of pair (b, h = j / g), over the tokens t < seq_lens[b]
+ * of the blocks sel_idx[b][h][0 .. sel_cnt[b][h]-1]:
+ *   z_t = softmax_scale * q[b][j] . K_t,
+ *   out[b][j] = sum_t e^{z_t - max z} V_t / sum_t e^{z_t - max z}   (bf16, RNE),
+ *   lse[b][j] = max z + ln sum_t e^{z_t - max z}                  (fp32).
+ * softmax_scale <= 0 selects 1/sqrt(D).  lse may be NULL.  Work is split
+ * into chunks of selected blocks whose partial (o, max, sum) are merged by
+ * the last chunk to finish (no extra launch).  A pair with sel_cnt 0 gets
+ * out = 0 and lse = -inf.  A block index outside [0, nb) is skipped and
+ * flagged KIN_ERR_DEVICE_DATA.  k_blocks is the sel_idx row stride.
+ * workspace: see kin_workspace_bytes. */
+kin_status kin_sparse_decode_attn(const kin_dims* dims, const void* q, const void* k_cache,
+                                  const void* v_cache, const int32_t* seq_lens,
+                                  const int32_t* sel_idx, const int32_t* sel_cnt,
+                                  int32_t k_blocks, float softmax_scale, void* out, float* lse,
+                                  void* workspace, size_t ws_bytes, int32_t* dev_status,
+                                  void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KIN_H */

@@ -222,6 +222,7 @@ class Workload:
     Lcap: int = 0
     hh_num: int = 5
     hh_den: int = 100
+    lens: tuple = ()   # explicit final lengths (overrides the draw when given)
 
     @property
     def g(self) -> int:
@@ -268,7 +269,11 @@ class HostCase:
 
 
 def case_meta(w: Workload):
-    lens_final = seq_lens(w.seed, w.B, w.Lmin, w.Lmax)
+    if w.lens:
+        lens_final = np.array(w.lens, dtype=np.int32)
+        assert lens_final.shape == (w.B,)
+    else:
+        lens_final = seq_lens(w.seed, w.B, w.Lmin, w.Lmax)
     lens_pre = (lens_final - w.n_append).astype(np.int32)
     hh = heavy_flags(w.seed, w.B, w.Hkv, w.nbcap, w.bs, lens_final, w.hh_num, w.hh_den)
     return lens_final, lens_pre, hh

@@ -1,0 +1,189 @@
+"""Helpers shared by the GPU parity tests: build a seeded case on the device,
+run the CUDA path through the C ABI binding, and compare with the fp64 oracle
+on the same bf16 bits (regenerated on the host for any (batch, kv head)).
+
+Tolerances (from the arithmetic: bf16 inputs, fp32 accumulation, bf16 out):
+  * outputs: max |gpu - oracle| <= 2e-2 and mean |gpu - oracle| <= 2e-3;
+  * lse: |gpu - oracle| <= 1e-3 + 1e-4 |oracle|;
+  * block means: |gpu - oracle| <= 1e-5 (fp32 sums of <= 128 bf16 rows);
+  * selected indices: bit-exact, except that a block may be swapped only when
+    its oracle score lies within delta of the k-th / (k+1)-th best score,
+    delta = 1e-4 * max(|tau_k|, |tau_k+1|, eps) with eps the mean over blocks
+    of (1/sqrt(D)) sum_j sum_d |q_jd| |m_d| (the scores' natural magnitude).
+    When sets differ, the output is compared with the oracle recomputed on
+    the GPU's set.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+import block_top_sparse_kin_b200 as kin
+import kin_inputs as ki
+import oracle
+
+D = 128
+OUT_MAX_ABS = 2e-2
+OUT_MEAN_ABS = 2e-3
+MEANS_ABS = 1e-5
+TIE_REL = 1e-4
+
+
+@dataclass
+class DeviceCase:
+    w: ki.Workload
+    dims: kin.kin_dims
+    q: torch.Tensor
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    means: torch.Tensor
+    seq_lens: torch.Tensor       # device, pre-append lengths (updated in place by append)
+    lens_pre: np.ndarray
+    lens_final: np.ndarray
+    hh: np.ndarray
+    q_host: np.ndarray
+    k_new: torch.Tensor | None
+    v_new: torch.Tensor | None
+
+
+def to_dev_bf16(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def make_device_case(w: ki.Workload, poison: bool = True) -> DeviceCase:
+    lens_final, lens_pre, hh = ki.case_meta(w)
+    q_host = ki.fill_q(w.seed, w.B, w.Hq, w.D)
+    dims = kin.make_dims(w.B, w.Hkv, w.Hq, w.D, w.bs, w.cap)
+    seq = torch.from_numpy(lens_pre.copy()).cuda()
+    hh_dev = torch.from_numpy(hh).cuda()
+    kc = torch.empty((w.B, w.Hkv, w.cap, w.D), dtype=torch.bfloat16, device="cuda")
+    vc = torch.empty_like(kc)
+    ki.kv_cache_device(w.seed, True, w.B, w.Hkv, w.cap, w.D, w.bs, seq, hh_dev, poison, kc)
+    ki.kv_cache_device(w.seed, False, w.B, w.Hkv, w.cap, w.D, w.bs, seq, hh_dev, poison, vc)
+    means = torch.full((w.B, w.Hkv, w.nbcap, w.D), float("nan"), dtype=torch.float32, device="cuda")
+    kn = vn = None
+    if w.n_append:
+        kn_h = np.empty((w.B, w.Hkv, w.n_append, w.D), np.uint16)
+        vn_h = np.empty_like(kn_h)
+        for b in range(w.B):
+            for h in range(w.Hkv):
+                t0 = int(lens_pre[b])
+                kn_h[b, h] = ki.kv_rows(w.seed, True, b * w.Hkv + h, t0, t0 + w.n_append, w.D, w.bs, hh[b, h])
+                vn_h[b, h] = ki.kv_rows(w.seed, False, b * w.Hkv + h, t0, t0 + w.n_append, w.D, w.bs, None)
+        kn, vn = to_dev_bf16(kn_h), to_dev_bf16(vn_h)
+    return DeviceCase(w, dims, to_dev_bf16(q_host), kc, vc, means, seq, lens_pre, lens_final, hh, q_host, kn, vn)
+
+
+@dataclass
+class GpuResult:
+    sel: np.ndarray
+    cnt: np.ndarray
+    out: np.ndarray     # float32 [B,Hq,D]
+    lse: np.ndarray
+    status: int
+
+
+def gpu_step(dc: DeviceCase, k: int, ws: torch.Tensor | None = None, build_means: bool = True) -> GpuResult:
+    """Means (build, then append if the workload has one), select, attend."""
+    w = dc.w
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    if build_means:
+        kin.kin_block_means_build(dc.dims, dc.k_cache, dc.seq_lens, dc.means, st)
+        if w.n_append:
+            kin.kin_block_means_update(dc.dims, dc.k_cache, dc.v_cache, dc.means, dc.seq_lens,
+                                       dc.k_new, dc.v_new, w.n_append, st)
+    if ws is None:
+        ws = kin.alloc_workspace(dc.dims, k)
+    sel = torch.empty((w.B, w.Hkv, k), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((w.B, w.Hkv), dtype=torch.int32, device="cuda")
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
+    kin.kin_block_topk_select(dc.dims, dc.q, dc.means, dc.seq_lens, k, sel, cnt, ws, st)
+    kin.kin_sparse_decode_attn(dc.dims, dc.q, dc.k_cache, dc.v_cache, dc.seq_lens, sel, cnt, k, 0.0,
+                               out, lse, ws, st)
+    torch.cuda.synchronize()
+    return GpuResult(sel.cpu().numpy(), cnt.cpu().numpy(), out.float().cpu().numpy(),
+                     lse.cpu().numpy(), int(st.item()))
+
+
+@dataclass
+class PairRef:
+    means: np.ndarray
+    scores: np.ndarray
+    sel: np.ndarray
+    cnt: int
+    K: np.ndarray
+    V: np.ndarray
+    L: int
+
+
+def oracle_pair(dc: DeviceCase, b: int, h: int, k: int) -> PairRef:
+    w = dc.w
+    L = int(dc.lens_final[b])
+    K, V = ki.pair_rows(w, dc.hh, b, h, L)
+    means = oracle.block_means(K, L, w.bs)
+    qg = dc.q_host[b, h * w.g:(h + 1) * w.g]
+    scores = oracle.block_scores(qg, means)
+    sel, cnt = oracle.select(scores, k)
+    return PairRef(means, scores, sel, cnt, K, V, L)
+
+
+def tie_delta(dc: DeviceCase, b: int, h: int, ref: PairRef):
+    w = dc.w
+    qg = ki.bf16_to_f32(dc.q_host[b, h * w.g:(h + 1) * w.g]).astype(np.float64)
+    eps = (np.abs(qg).sum(axis=0) @ np.abs(ref.means).T).mean() / math.sqrt(D)
+    nb = ref.means.shape[0]
+    cand = np.sort(ref.scores[1:nb - 1])[::-1]
+    kk = ref.cnt - 2
+    tau_k = cand[kk - 1] if kk >= 1 else 0.0
+    tau_k1 = cand[kk] if kk < len(cand) else tau_k
+    return TIE_REL * max(abs(tau_k), abs(tau_k1), eps), tau_k, tau_k1
+
+
+def check_selection(dc: DeviceCase, b: int, h: int, k: int, ref: PairRef, gsel: np.ndarray, gcnt: int):
+    """Returns True if identical, False if an allowed near-tie swap; raises otherwise."""
+    nb = ref.means.shape[0]
+    assert gcnt == ref.cnt, (b, h, gcnt, ref.cnt)
+    assert np.all(gsel[gcnt:] == -1), (b, h)
+    g = gsel[:gcnt]
+    assert np.all(np.diff(g) > 0), (b, h, "not ascending")
+    if np.array_equal(g, ref.sel[:ref.cnt]):
+        return True
+    assert g[0] == 0 and g[-1] == nb - 1, (b, h, "forced blocks missing")
+    delta, tau_k, tau_k1 = tie_delta(dc, b, h, ref)
+    diff = set(g.tolist()) ^ set(ref.sel[:ref.cnt].tolist())
+    for i in diff:
+        s = ref.scores[i]
+        assert min(abs(s - tau_k), abs(s - tau_k1)) <= delta, \
+            (b, h, i, s, tau_k, tau_k1, delta, "selection differs beyond the tie tolerance")
+    return False
+
+
+def check_pair(dc: DeviceCase, gr: GpuResult, b: int, h: int, k: int, gpu_means: np.ndarray | None = None):
+    """Full parity of one (b, h): means, selection, outputs, lse."""
+    w = dc.w
+    ref = oracle_pair(dc, b, h, k)
+    nb = ref.means.shape[0]
+    if gpu_means is not None:
+        err = np.abs(gpu_means[b, h, :nb].astype(np.float64) - ref.means).max()
+        assert err <= MEANS_ABS, (b, h, err)
+    same = check_selection(dc, b, h, k, ref, gr.sel[b, h], int(gr.cnt[b, h]))
+    blocks = gr.sel[b, h, :gr.cnt[b, h]] if not same else ref.sel[:ref.cnt]
+    qg = dc.q_host[b, h * w.g:(h + 1) * w.g]
+    o_ref, lse_ref = oracle.attend(qg, ref.K, ref.V, ref.L, w.bs, blocks, 1 / math.sqrt(D))
+    o_gpu = gr.out[b, h * w.g:(h + 1) * w.g].astype(np.float64)
+    err = np.abs(o_gpu - o_ref)
+    assert err.max() <= OUT_MAX_ABS and err.mean() <= OUT_MEAN_ABS, (b, h, err.max(), err.mean())
+    lse_gpu = gr.lse[b, h * w.g:(h + 1) * w.g].astype(np.float64)
+    assert np.all(np.abs(lse_gpu - lse_ref) <= 1e-3 + 1e-4 * np.abs(lse_ref)), (b, h, lse_gpu, lse_ref)
+    return same, err.max(), err.mean()
+
+
+def sample_pairs(w: ki.Workload, n: int):
+    """Deterministic spread of (b, h) pairs: first, last and evenly spaced."""
+    P = w.B * w.Hkv
+    idx = sorted(set([0, P - 1] + [int(round(i * (P - 1) / max(n - 1, 1))) for i in range(n)]))
+    return [(p // w.Hkv, p % w.Hkv) for p in idx]

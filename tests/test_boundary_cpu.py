@@ -1,0 +1,131 @@
+"""The C ABI library without a GPU: it loads, exports every entry point that
+include/kin.h declares, and its host-side checks reject bad arguments before
+any CUDA call is made."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import block_top_sparse_kin_b200 as kin
+from block_top_sparse_kin_b200 import build as kbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kin.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    srcs = [os.path.join(kbuild.CSRC, s) for s in kbuild.SOURCES] + [HEADER]
+    if not os.path.exists(kbuild.LIB) or os.path.getmtime(kbuild.LIB) < max(map(os.path.getmtime, srcs)):
+        kbuild.build()
+    return kin.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kin_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    assert declared_functions() == sorted(kin.EXPORTED)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", kbuild.LIB], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(l.split()[-1] for l in out.splitlines() if " T " in l)
+    for name in declared_functions():
+        assert name in exported, name
+        assert getattr(lib, name) is not None
+    # nothing else of ours leaks out of the library
+    assert not [s for s in exported if s.startswith("_ZN3kin")]
+
+
+def test_status_strings(lib):
+    for code, name in kin.STATUS_NAMES.items():
+        assert kin.kin_status_string(code) == name
+    assert kin.kin_status_string(99) == "KIN_ERR_UNKNOWN"
+
+
+def dims(B=2, Hkv=2, Hq=8, D=128, bs=16, L=256):
+    return kin.make_dims(B, Hkv, Hq, D, bs, L)
+
+
+def test_workspace_bytes(lib):
+    assert kin.kin_workspace_bytes(dims(), 1) == 0
+    assert kin.kin_workspace_bytes(dims(D=64), 8) == 0
+    assert kin.kin_workspace_bytes(dims(bs=24), 8) == 0
+    assert kin.kin_workspace_bytes(dims(Hq=7), 8) == 0
+    assert kin.kin_workspace_bytes(dims(Hq=32, Hkv=2), 8) == 0       # g = 16
+    n8 = kin.kin_workspace_bytes(dims(), 8)
+    pairs, nbcap = 4, 16
+    assert n8 >= pairs * nbcap * 4 + 2 * pairs * 4
+    assert n8 % 256 == 0
+    assert kin.kin_workspace_bytes(dims(), 16) >= n8
+    big = kin.make_dims(32, 8, 32, 128, 16, 32768)
+    assert kin.kin_workspace_bytes(big, 256) >= 32 * 8 * 2048 * 4
+
+
+FAKE = ctypes.c_void_p(1 << 20)   # aligned, never dereferenced: every call below fails its host checks
+
+
+def test_select_rejects_before_launch(lib):
+    d = dims()
+    args = lambda k=8, q=FAKE, ws=FAKE, n=1 << 30: (ctypes.byref(d), q, FAKE, FAKE, k, FAKE, FAKE, ws, n,
+                                                   None, None)
+    assert lib.kin_block_topk_select(*args(k=1)) == 1
+    assert lib.kin_block_topk_select(*args(q=None)) == 1
+    assert lib.kin_block_topk_select(*args(q=ctypes.c_void_p((1 << 20) + 2))) == 1
+    assert lib.kin_block_topk_select(*args(ws=None)) == 2
+    assert lib.kin_block_topk_select(*args(ws=ctypes.c_void_p((1 << 20) + 16))) == 2
+    assert lib.kin_block_topk_select(*args(n=64)) == 2
+    bad = kin.make_dims(2, 2, 8, 128, 16, 0)
+    assert lib.kin_block_topk_select(ctypes.byref(bad), FAKE, FAKE, FAKE, 8, FAKE, FAKE, FAKE, 1 << 30,
+                                     None, None) == 1
+    huge = kin.make_dims(1, 1, 1, 128, 16, 16 * 32768 + 1)
+    assert lib.kin_block_topk_select(ctypes.byref(huge), FAKE, FAKE, FAKE, 8, FAKE, FAKE, FAKE, 1 << 40,
+                                     None, None) == 3
+    assert lib.kin_block_topk_select(None, FAKE, FAKE, FAKE, 8, FAKE, FAKE, FAKE, 1 << 30, None, None) == 1
+
+
+def test_attn_rejects_before_launch(lib):
+    d = dims()
+    def call(scale=0.0, ws=FAKE, n=1 << 30, out=FAKE, k=8):
+        return lib.kin_sparse_decode_attn(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, k, scale,
+                                          out, None, ws, n, None, None)
+    assert call(k=0) == 1
+    assert call(out=None) == 1
+    assert call(scale=float("nan")) == 1
+    assert call(scale=float("inf")) == 1
+    assert call(ws=None) == 2
+    assert call(n=100) == 2
+
+
+def test_means_calls_reject_before_launch(lib):
+    d = dims()
+    assert lib.kin_block_means_update(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, -1, None, None) == 1
+    assert lib.kin_block_means_update(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, None, None) == 0
+    assert lib.kin_block_means_update(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 257, None, None) == 3
+    assert lib.kin_block_means_update(ctypes.byref(d), None, FAKE, FAKE, FAKE, FAKE, FAKE, 1, None, None) == 1
+    assert lib.kin_block_means_build(ctypes.byref(d), None, FAKE, FAKE, None, None) == 1
+    assert lib.kin_block_means_build(ctypes.byref(dims(bs=8)), FAKE, FAKE, FAKE, None, None) == 1
+
+
+def test_binding_refuses_host_tensors(lib):
+    import torch
+    with pytest.raises(ValueError):
+        kin.kin_block_means_build(dims(), torch.zeros(4, dtype=torch.bfloat16),
+                                  torch.zeros(2, dtype=torch.int32), torch.zeros(4))
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    saved = kin._lib
+    try:
+        kin._lib = None
+        with pytest.raises(RuntimeError):
+            kin.load_library(str(tmp_path / "nope.so"))
+    finally:
+        kin._lib = saved
