@@ -11,7 +11,7 @@ LIB = os.path.join(HERE, "libkin.so")
 SOURCES = ["kin_api.cu", "kin_means.cu", "kin_select.cu", "kin_attn.cu"]
 
 
-def nvcc_command(out: str = LIB, ptxas_verbose: bool = False) -> list:
+def nvcc_command(out: str = LIB, ptxas_verbose: bool = False, defines=()) -> list:
     cmd = [
         "nvcc", "-O3", "-std=c++17", "-shared", "-Xcompiler", "-fPIC,-fvisibility=hidden",
         "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
@@ -19,6 +19,7 @@ def nvcc_command(out: str = LIB, ptxas_verbose: bool = False) -> list:
     ]
     if ptxas_verbose:
         cmd += ["-Xptxas", "-v"]
+    cmd += [f"-D{d}" for d in defines]
     cmd += [os.path.join(CSRC, s) for s in SOURCES] + ["-o", out]
     return cmd
 

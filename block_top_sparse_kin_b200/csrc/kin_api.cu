@@ -1,8 +1,6 @@
 // kin_api.cu -- the extern "C" boundary of libkin.so: argument checks,
 // workspace layout, launch-shape heuristics, TMA descriptors and launches.
 // Semantics of every call are documented in include/kin.h.
-#include <cudaTypedefs.h>
-
 #include <cmath>
 
 #include "kin_internal.cuh"
@@ -36,24 +34,32 @@ kin_status check_dims(const kin_dims* d) {
 int nbcap_of(const kin_dims& d) { return (d.max_seq_len + d.block_size - 1) / d.block_size; }
 int pairs_of(const kin_dims& d) { return d.batch * d.num_kv_heads; }
 
-// Blocks of means per select CTA: 128 (64 KB of fp32 means), halved down to
-// 32 while the grid would hold fewer than 4 CTAs per SM.
+#ifndef KIN_SEL_CHUNK
+#define KIN_SEL_CHUNK 128
+#endif
+#ifndef KIN_ATTN_CHUNK_TOKENS
+#define KIN_ATTN_CHUNK_TOKENS 512
+#endif
+
+// Blocks of means per select CTA: KIN_SEL_CHUNK (128 -> 64 KB of fp32 means),
+// halved down to 32 while the grid would hold fewer than 4 CTAs per SM.
 int select_chunk_blocks(const kin_dims& d) {
   const int nbcap = nbcap_of(d);
-  int ch = 128;
+  int ch = KIN_SEL_CHUNK;
   while (ch > 32 && (int64_t)pairs_of(d) * ((nbcap + ch - 1) / ch) < 4 * kTargetSMs) ch >>= 1;
   return ch;
 }
 
-// Kept blocks per attention CTA: 512 tokens (256 KB of K+V), fewer when the
-// grid would hold fewer than 2 CTAs per SM.
+// Kept blocks per attention CTA: KIN_ATTN_CHUNK_TOKENS tokens (512 -> 256 KB
+// of K+V), fewer when the grid would hold fewer than 2 CTAs per SM.
 int attn_chunk_blocks(const kin_dims& d, int k) {
   const int k_eff = k < nbcap_of(d) ? k : nbcap_of(d);
-  const int by_tokens = 512 / d.block_size > 0 ? 512 / d.block_size : 1;
+  const int by_tokens = KIN_ATTN_CHUNK_TOKENS / d.block_size > 0 ? KIN_ATTN_CHUNK_TOKENS / d.block_size : 1;
   const int64_t by_grid = (int64_t)k_eff * pairs_of(d) / (2 * kTargetSMs);
   int ch = by_tokens;
   if (by_grid < ch) ch = by_grid > 0 ? (int)by_grid : 1;
-  return ch;
+  const int cap = kMaxItemTiles / (d.block_size / kTileTokens);  // tiles per item <= 64
+  return ch < cap ? ch : cap;
 }
 
 int attn_max_chunks(const kin_dims& d, int k) {
@@ -91,36 +97,6 @@ kin_status check_ws(const kin_dims& d, int k, void* ws, size_t ws_bytes, WsLayou
 }
 
 kin_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KIN_OK : KIN_ERR_CUDA; }
-
-// cuTensorMapEncodeTiled through the runtime's driver entry point, so the
-// library needs no link-time dependency on libcuda.
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return nullptr;
-    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  }();
-  return fn;
-}
-
-// 2-D view [rows, 128] of a bf16 cache; box 16 rows x 64 columns (128 bytes,
-// the 128-byte swizzle span).
-bool encode_cache_map(CUtensorMap* m, const void* base, uint64_t rows) {
-  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)kTileTokens};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
 
 }  // namespace
 
@@ -244,12 +220,11 @@ KIN_EXPORT kin_status kin_sparse_decode_attn(const kin_dims* dims, const void* q
   WsLayout w;
   st = check_ws(*dims, k_blocks, workspace, ws_bytes, &w);
   if (st != KIN_OK) return st;
-  const uint64_t rows = (uint64_t)dims->batch * dims->num_kv_heads * dims->max_seq_len;
-  CUtensorMap tmk, tmv;
-  if (!encode_cache_map(&tmk, k_cache, rows) || !encode_cache_map(&tmv, v_cache, rows)) return KIN_ERR_CUDA;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   AttnParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
+  p.v_cache = static_cast<const __nv_bfloat16*>(v_cache);
   p.seq_lens = seq_lens;
   p.sel_idx = sel_idx;
   p.sel_cnt = sel_cnt;
@@ -269,5 +244,6 @@ KIN_EXPORT kin_status kin_sparse_decode_attn(const kin_dims* dims, const void* q
   p.max_chunks = attn_max_chunks(*dims, k_blocks);
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)kHeadDim);
   p.scale_log2 = scale * 1.4426950408889634f;
-  return from_cuda(launch_attn(p, tmk, tmv, p.max_chunks, static_cast<cudaStream_t>(stream)));
+  const int num_items = pairs_of(*dims) * p.max_chunks;
+  return from_cuda(launch_attn(p, num_items, static_cast<cudaStream_t>(stream)));
 }

@@ -8,52 +8,78 @@
 // merged: o = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c, M = max_c m_c
 // (base-2 logits: the scale is folded with log2(e)).
 //
-// Work split (HBM-bound gather, ~8 KB of K+V per 16 tokens):
-//   grid (chunk, kv head, batch); 4 warps per CTA.  A chunk is
-//   `chunk_blocks` consecutive entries of the pair's ascending kept-block
-//   list; its 16-token tiles are dealt round-robin to the 4 warps.
-//   Each warp runs its own STAGES-deep pipeline: lane 0 issues four 2-D TMA
-//   loads per tile (K and V, two 64-column halves each, 128-byte swizzle) that
-//   complete on the slot's mbarrier; all lanes wait on it (bounded).
-//   Per tile and warp: S^T[16 tok x 8 heads] = K Q^T with 8 mma.sync m16n8k16
-//   (tokens are M, the GQA group is N, so g <= 8 wastes no rows), online
-//   softmax across the 16 tokens with quad shuffles, P^T moved into the B
-//   operand with movmatrix, then O^T[128 x 8] += V^T P^T with 8 more MMAs.
-//   The 4 warps merge in shared memory; a chunk's partial (o, m, l) goes to
-//   workspace and the pair's last chunk to finish (atomic counter, no spin)
-//   merges all chunks and writes bf16 out and fp32 lse.
+// Design (an HBM-bound gather of scattered 4 KB K and V tiles, ~1 flop/byte
+// per query head):
+//  * One CTA per work item = (kv pair, chunk of `chunk_blocks` consecutive
+//    entries of the pair's ascending kept-block list); several CTAs share an
+//    SM so one CTA's merge overlaps the others' streaming.
+//  * Each warp streams its own 16-token tiles (tiles w, w + W, ...) through a
+//    KIN_ATTN_STAGES-deep ring in shared memory with 16-byte cp.async copies
+//    issued by all 32 lanes (16 per lane per tile), written straight into a
+//    128-byte XOR-swizzled layout so ldmatrix reads are bank-conflict free.
+//    Rows past the sequence end are zero-filled, never read.  (Measured on
+//    B200: one thread issuing TMA/bulk copies of such small tiles tops out
+//    near 2 copies/us, so spreading the issue over all lanes is what lets the
+//    gather approach HBM speed.)
+//  * Per tile: S^T[16 tok x 8 heads] = K Q^T with 8 mma.sync m16n8k16 (tokens
+//    are M, the GQA group is N), online softmax over the 16 tokens with quad
+//    shuffles, P^T moved into the B operand with movmatrix, O^T[128 x 8] +=
+//    V^T P^T with 8 more MMAs.
+//  * The warps merge in shared memory.  A single-chunk pair writes bf16 out
+//    and fp32 lse directly; otherwise the chunk's partial (o, m, l) goes to
+//    workspace and the pair's last chunk to finish (atomic counter, no
+//    spinning) merges all of them with batched, independent loads.
 #include "kin_internal.cuh"
 
 namespace kin {
 
-constexpr int kAttnWarps = 4;
+#ifndef KIN_ATTN_WARPS
+#define KIN_ATTN_WARPS 4
+#endif
+#ifndef KIN_ATTN_STAGES
+#define KIN_ATTN_STAGES 2
+#endif
+#ifndef KIN_ATTN_CTAS_PER_SM
+#define KIN_ATTN_CTAS_PER_SM 3
+#endif
+
+constexpr int kAttnWarps = KIN_ATTN_WARPS;
 constexpr int kAttnThreads = kAttnWarps * 32;
-constexpr int kHalfBox = 16 * 64 * 2;        // bytes of one 16-row x 64-col bf16 box
-constexpr int kStageBytes = 4 * kHalfBox;    // K0 K1 V0 V1
+constexpr int kStages = KIN_ATTN_STAGES;
+constexpr int kHalfBox = 16 * 64 * 2;       // bytes of a 16-row x 64-column bf16 half tile
+constexpr int kStageBytes = 4 * kHalfBox;   // K0 K1 V0 V1
+constexpr int kRowPad = kHeadDim + 4;       // combine rows padded against bank conflicts
+constexpr int kMergeBatch = 32;             // chunks whose (m, l) are staged per merge round
+constexpr size_t kPipeBytes = (size_t)kAttnWarps * kStages * kStageBytes;
+constexpr size_t kCombBytes = (size_t)kAttnWarps * kMaxGroup * kRowPad * sizeof(float);
+static_assert(kAttnThreads >= kHeadDim, "one thread per output dim in the merge");
+static_assert(kMaxItemTiles / kAttnWarps <= 32, "a warp's tiles of one item fit one per lane");
 #define kNegInf (-__int_as_float(0x7f800000))
 
-template <int STAGES>
-constexpr size_t attn_smem_bytes() {
-  return (size_t)kAttnWarps * STAGES * kStageBytes + 1024;  // + alignment slack
-}
+size_t attn_smem_bytes() { return (kPipeBytes > kCombBytes ? kPipeBytes : kCombBytes) + 1024; }
 
-struct TileInfo {
-  int64_t grow;  // row in the [B*Hkv*Lcap, D] view
-  int nvalid;    // valid tokens in the tile, 0 => skip
-  bool bad;      // block index out of range
+struct ItemInfo {
+  int64_t pair;
+  int b, h, c, L, nb, cnt, nchunks, j0, ntiles;
 };
 
-__device__ __forceinline__ TileInfo tile_info(const AttnParams& p, int64_t pair, int warp, int n,
-                                              int j0, int tpb, int nb, int L) {
-  TileInfo t;
-  const int T = warp + kAttnWarps * n;
-  const int jj = j0 + T / tpb, sub = T % tpb;
-  const int blk = __ldg(p.sel_idx + pair * p.k + jj);
-  t.bad = blk < 0 || blk >= nb;
-  const int row0 = blk * p.bs + sub * kTileTokens;
-  t.nvalid = (t.bad || row0 >= L) ? 0 : min(kTileTokens, L - row0);
-  t.grow = pair * p.Lcap + (t.nvalid ? row0 : 0);
-  return t;
+__device__ __forceinline__ ItemInfo item_info(const AttnParams& p, int u) {
+  ItemInfo it;
+  it.pair = u / p.max_chunks;
+  it.c = u - (int)it.pair * p.max_chunks;
+  it.b = (int)(it.pair / p.Hkv);
+  it.h = (int)(it.pair - (int64_t)it.b * p.Hkv);
+  it.L = __ldg(p.seq_lens + it.b);
+  int cnt = __ldg(p.sel_cnt + it.pair);
+  if (it.L < 1 || it.L > p.Lcap) cnt = 0;
+  if (cnt > p.k) cnt = p.k;
+  it.cnt = cnt;
+  it.nchunks = cnt > 0 ? (cnt + p.chunk_blocks - 1) / p.chunk_blocks : 0;
+  it.nb = (it.L + p.bs - 1) / p.bs;
+  it.j0 = it.c * p.chunk_blocks;
+  const int j1 = min(it.j0 + p.chunk_blocks, cnt);
+  it.ntiles = it.c < it.nchunks ? (j1 - it.j0) * (p.bs / kTileTokens) : 0;
+  return it;
 }
 
 // Zero the bf16 halves of a V^T fragment register whose token is invalid.
@@ -61,47 +87,56 @@ __device__ __forceinline__ uint32_t tok_mask(int t, int nvalid) {
   return (t < nvalid ? 0x0000FFFFu : 0u) | (t + 1 < nvalid ? 0xFFFF0000u : 0u);
 }
 
-template <int STAGES>
-__global__ void __launch_bounds__(kAttnThreads)
-    attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-                AttnParams p) {
+// 16-byte async copy global -> shared; src_bytes 0 writes zeros and reads nothing.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kernel(AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bars[kAttnWarps][STAGES];
   __shared__ float s_m[kAttnWarps][kMaxGroup], s_l[kAttnWarps][kMaxGroup];
   __shared__ int s_last;
+  __shared__ float s_pm[kMergeBatch * kMaxGroup], s_pl[kMergeBatch * kMaxGroup];  // merge staging
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int b = blockIdx.z, h = blockIdx.y, c = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t pair = (int64_t)b * p.Hkv + h;
   const int g = p.g;
-  const int L = p.seq_lens[b];
-  int cnt = p.sel_cnt[pair];
-  if (L < 1 || L > p.Lcap) cnt = 0;
-  if (cnt > p.k) cnt = p.k;
-  if (cnt <= 0) {  // nothing selected (flagged upstream): out = 0, lse = -inf
-    if (c == 0) {
-      for (int j = 0; j < g; ++j)
-        p.out[((int64_t)b * p.Hq + (int64_t)h * g + j) * kHeadDim + tid] = __float2bfloat16_rn(0.f);
-      if (p.lse && tid < g) p.lse[(int64_t)b * p.Hq + (int64_t)h * g + tid] = kNegInf;
+  const ItemInfo it = item_info(p, blockIdx.x);
+  const int64_t qh0 = (int64_t)it.b * p.Hq + (int64_t)it.h * g;
+  if (it.cnt <= 0) {  // nothing selected (flagged upstream): out = 0, lse = -inf
+    if (it.c == 0 && tid < kHeadDim) {
+      for (int j = 0; j < g; ++j) p.out[(qh0 + j) * kHeadDim + tid] = __float2bfloat16_rn(0.f);
+      if (p.lse && tid < g) p.lse[qh0 + tid] = kNegInf;
     }
     return;
   }
-  const int nchunks = (cnt + p.chunk_blocks - 1) / p.chunk_blocks;
-  if (c >= nchunks) return;
-  const int nb = (L + p.bs - 1) / p.bs;
-  const int tpb = p.bs / kTileTokens;
-  const int j0 = c * p.chunk_blocks;
-  const int j1 = min(j0 + p.chunk_blocks, cnt);
-  const int total_tiles = (j1 - j0) * tpb;
-  const int n_w = warp < total_tiles ? (total_tiles - 1 - warp) / kAttnWarps + 1 : 0;
+  if (it.ntiles == 0) return;  // a chunk index past this pair's chunks
 
-  // Q fragments (B operand, "col" layout): head = lane/4, dims 16kk + 2(lane%4) (+8).
+  // ---- this warp's tiles t = warp + W n; lane n holds tile n's source row and valid count
+  const int tpb = p.bs / kTileTokens;
+  const int n_w = warp < it.ntiles ? (it.ntiles - 1 - warp) / kAttnWarps + 1 : 0;
+  int my_row = 0, my_nvalid = 0;
+  if (lane < n_w) {
+    const int t = warp + kAttnWarps * lane;
+    const int blk = __ldg(p.sel_idx + it.pair * p.k + it.j0 + t / tpb);
+    const bool bad = blk < 0 || blk >= it.nb;
+    if (bad) set_status(p.dev_status, KIN_ERR_DEVICE_DATA);
+    const int row0 = blk * p.bs + (t - (t / tpb) * tpb) * kTileTokens;
+    my_nvalid = (bad || row0 >= it.L) ? 0 : min(kTileTokens, it.L - row0);
+    my_row = my_nvalid ? row0 : 0;
+  }
+
+  // Q fragments (B operand, "col" layout): head = lane/4, dims 16kk + 2(lane%4) (+8)
   uint32_t qf[8][2];
   {
     const int n = lane >> 2;
-    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-        p.q + ((int64_t)b * p.Hq + (int64_t)h * g + (n < g ? n : 0)) * kHeadDim);
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(p.q + (qh0 + (n < g ? n : 0)) * kHeadDim);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
       qf[kk][0] = n < g ? __ldg(qrow + kk * 8 + (lane & 3)) : 0u;
@@ -109,34 +144,33 @@ __global__ void __launch_bounds__(kAttnThreads)
     }
   }
 
-  const uint32_t stage0 = smem_u32(smem) + (uint32_t)(warp * STAGES * kStageBytes);
-  const uint32_t bar0 = smem_u32(&bars[warp][0]);
-  if (lane == 0) {
-#pragma unroll
-    for (int s = 0; s < STAGES; ++s) mbar_init(bar0 + 8 * s, 1);
-    fence_mbar_init();
-  }
-  __syncwarp();
+  const uint32_t ring = smem_u32(smem) + (uint32_t)(warp * kStages * kStageBytes);
+  const __nv_bfloat16* kbase = p.k_cache + it.pair * (int64_t)p.Lcap * kHeadDim;
+  const __nv_bfloat16* vbase = p.v_cache + it.pair * (int64_t)p.Lcap * kHeadDim;
 
-  auto issue = [&](int n) {  // lane 0 only
-    const int slot = n % STAGES;
-    const uint32_t bar = bar0 + 8 * slot;
-    const TileInfo t = tile_info(p, pair, warp, n, j0, tpb, nb, L);
-    if (t.nvalid == 0) {
-      mbar_arrive(bar);
-      return;
+  // Issue tile n into its ring slot: lane l copies pieces l + 32 i (i < 8) of
+  // the K tile and of the V tile; piece = (row r, 16-byte column cc).
+  auto issue = [&](int n) {
+    const int row0 = __shfl_sync(0xffffffffu, my_row, n & 31);
+    const int nv = __shfl_sync(0xffffffffu, my_nvalid, n & 31);
+    if (n < n_w && nv > 0) {
+      const uint32_t base = ring + (uint32_t)((n % kStages) * kStageBytes);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int piece = lane + 32 * i;
+        const int r = piece >> 4, cc = piece & 15;
+        const uint32_t off = (uint32_t)((cc >> 3) * kHalfBox + r * 128 + (((cc & 7) ^ (r & 7)) << 4));
+        const int64_t src = (int64_t)(row0 + (r < nv ? r : 0)) * kHeadDim + cc * 8;
+        const uint32_t bytes = r < nv ? 16u : 0u;
+        cp_async16(base + off, kbase + src, bytes);
+        cp_async16(base + 2 * kHalfBox + off, vbase + src, bytes);
+      }
     }
-    const uint32_t dst = stage0 + (uint32_t)(slot * kStageBytes);
-    mbar_arrive_expect_tx(bar, kStageBytes);
-    const int32_t y = (int32_t)t.grow;
-    tma_load_2d(dst, &tmk, 0, y, bar);
-    tma_load_2d(dst + kHalfBox, &tmk, 64, y, bar);
-    tma_load_2d(dst + 2 * kHalfBox, &tmv, 0, y, bar);
-    tma_load_2d(dst + 3 * kHalfBox, &tmv, 64, y, bar);
+    cp_async_commit();  // one group per tile, empty or not, keeps the accounting uniform
   };
 
-  if (lane == 0)
-    for (int n = 0; n < n_w && n < STAGES; ++n) issue(n);
+#pragma unroll
+  for (int n = 0; n < kStages; ++n) issue(n);
 
   float o[8][4];
 #pragma unroll
@@ -144,25 +178,18 @@ __global__ void __launch_bounds__(kAttnThreads)
   float m0 = kNegInf, m1 = kNegInf, l0 = 0.f, l1 = 0.f;
   const float sl2 = p.scale_log2;
   const int tq = lane >> 2;                        // token row of C fragments
-  const int ta = 2 * (lane & 3);                   // token col of A(V^T) fragments
-  const int kr = lane & 15, khi = lane >> 4;       // ldmatrix row/col-chunk for K
+  const int ta = 2 * (lane & 3);                   // token col of A(V^T) / head col of C
+  const int kr = lane & 15, khi = lane >> 4;       // ldmatrix row / column chunk for K
   const int vt = (lane & 7) + ((lane >> 4) << 3);  // ldmatrix row for V^T
   const int vsel = (lane >> 3) & 1;
 
-  int n_done = 0;
-  bool timed_out = false;
   for (int n = 0; n < n_w; ++n) {
-    const int slot = n % STAGES;
-    const TileInfo t = tile_info(p, pair, warp, n, j0, tpb, nb, L);
-    if (t.bad && lane == 0) set_status(p.dev_status, KIN_ERR_DEVICE_DATA);
-    if (!mbar_wait_bounded(bar0 + 8 * slot, (uint32_t)((n / STAGES) & 1), p.dev_status)) {
-      timed_out = true;
-      break;
-    }
-    n_done = n + 1;
-    if (t.nvalid > 0) {
-      const uint32_t base = stage0 + (uint32_t)(slot * kStageBytes);
-      // ---- S^T = K Q^T (two accumulator chains to halve the MMA dependency chain)
+    cp_async_wait<kStages - 1>();  // this lane's copies of tile n have landed
+    __syncwarp();                  // ... and every other lane's
+    const int nvalid = __shfl_sync(0xffffffffu, my_nvalid, n & 31);
+    if (nvalid > 0) {
+      const uint32_t base = ring + (uint32_t)((n % kStages) * kStageBytes);
+      // ---- S^T = K Q^T (two accumulator chains halve the MMA dependency chain)
       float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
@@ -175,7 +202,7 @@ __global__ void __launch_bounds__(kAttnThreads)
         else
           mma_bf16_16816(sa, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
       }
-      const bool v0 = tq < t.nvalid, v1 = tq + 8 < t.nvalid;
+      const bool v0 = tq < nvalid, v1 = tq + 8 < nvalid;
       const float s0 = v0 ? (sa[0] + sb[0]) * sl2 : kNegInf;
       const float s1 = v0 ? (sa[1] + sb[1]) * sl2 : kNegInf;
       const float s2 = v1 ? (sa[2] + sb[2]) * sl2 : kNegInf;
@@ -205,7 +232,7 @@ __global__ void __launch_bounds__(kAttnThreads)
       // ---- P^T into the B operand (k = token, n = head) by 8x8 transposes
       const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));
       const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2, p3));
-      const uint32_t mlo = tok_mask(ta, t.nvalid), mhi = tok_mask(ta + 8, t.nvalid);
+      const uint32_t mlo = tok_mask(ta, nvalid), mhi = tok_mask(ta + 8, nvalid);
       // ---- O^T += V^T P^T
 #pragma unroll
       for (int dm = 0; dm < 8; ++dm) {
@@ -214,7 +241,7 @@ __global__ void __launch_bounds__(kAttnThreads)
         const int ch = (d0 & 63) >> 3;
         uint32_t a0, a1, a2, a3;
         ldmatrix_x4_trans(box + vt * 128 + ((ch ^ (vt & 7)) << 4), a0, a1, a2, a3);
-        if (t.nvalid < kTileTokens) {  // invalid rows may hold anything: zero them
+        if (nvalid < kTileTokens) {  // zero-filled rows: keep them out exactly
           a0 &= mlo;
           a1 &= mlo;
           a2 &= mhi;
@@ -223,35 +250,27 @@ __global__ void __launch_bounds__(kAttnThreads)
         mma_bf16_16816(o[dm], a0, a1, a2, a3, pb0, pb1);
       }
     }
-    fence_proxy_async_smem();  // our generic reads of the slot precede the next async write
-    __syncwarp();
-    if (lane == 0 && n + STAGES < n_w) issue(n + STAGES);
+    __syncwarp();  // every lane is done reading slot n % S before it is refilled
+    issue(n + kStages);
   }
-  if (timed_out) {
-    if (lane == 0) set_status(p.dev_status, KIN_ERR_TIMEOUT);
-    // drain the copies this warp still has in flight before its smem is reused
-    for (int n = n_done; n < n_w && n < n_done + STAGES; ++n)
-      mbar_wait_bounded(bar0 + 8 * (n % STAGES), (uint32_t)((n / STAGES) & 1), nullptr);
-    m0 = m1 = kNegInf;
-    l0 = l1 = 0.f;
-  }
+  cp_async_wait<0>();
 
-  // ---- per-warp totals of l over the 8 token rows
+  // ---- per-warp totals of l over the 8 token rows, then the cross-warp merge
 #pragma unroll
   for (int off = 4; off < 32; off <<= 1) {
     l0 += __shfl_xor_sync(0xffffffffu, l0, off);
     l1 += __shfl_xor_sync(0xffffffffu, l1, off);
   }
-  __syncthreads();  // every warp is done with its pipeline smem
-  float* so = reinterpret_cast<float*>(smem);  // [warp][head 8][128]
+  __syncthreads();  // every warp is done with its ring; the combine area reuses it
+  float* comb = reinterpret_cast<float*>(smem);  // [warp][head][kRowPad]
 #pragma unroll
   for (int dm = 0; dm < 8; ++dm) {
     const int d = dm * 16 + tq;
-    float* w0 = so + ((warp * kMaxGroup) + ta) * kHeadDim;
+    float* w0 = comb + ((warp * kMaxGroup) + ta) * kRowPad;
     w0[d] = o[dm][0];
-    w0[kHeadDim + d] = o[dm][1];
+    w0[kRowPad + d] = o[dm][1];
     w0[d + 8] = o[dm][2];
-    w0[kHeadDim + d + 8] = o[dm][3];
+    w0[kRowPad + d + 8] = o[dm][3];
   }
   if (lane < 4) {
     s_m[warp][2 * lane] = m0;
@@ -261,10 +280,10 @@ __global__ void __launch_bounds__(kAttnThreads)
   }
   __syncthreads();
 
-  const int d = tid;  // one output dim per thread
-  const int64_t qh0 = (int64_t)b * p.Hq + (int64_t)h * g;
-  if (nchunks == 1) {
-    for (int j = 0; j < g; ++j) {
+  const int d = tid;  // one output dim per thread (threads >= kHeadDim idle)
+  const int gd = d < kHeadDim ? g : 0;
+  if (it.nchunks == 1) {
+    for (int j = 0; j < gd; ++j) {
       float M = kNegInf;
 #pragma unroll
       for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, s_m[w][j]);
@@ -273,7 +292,7 @@ __global__ void __launch_bounds__(kAttnThreads)
 #pragma unroll
         for (int w = 0; w < kAttnWarps; ++w) {
           const float e = exp2f(s_m[w][j] - M);
-          num += e * so[(w * kMaxGroup + j) * kHeadDim + d];
+          num += e * comb[(w * kMaxGroup + j) * kRowPad + d];
           den += e * s_l[w][j];
         }
       }
@@ -283,9 +302,9 @@ __global__ void __launch_bounds__(kAttnThreads)
     return;
   }
 
-  // ---- write this chunk's partial, then the last chunk merges all of them
-  float* part = p.partials + (pair * p.max_chunks + c) * (int64_t)g * (kHeadDim + 2);
-  for (int j = 0; j < g; ++j) {
+  // ---- write this chunk's partial; the pair's last chunk merges all of them
+  float* part = p.partials + (it.pair * p.max_chunks + it.c) * (int64_t)g * (kHeadDim + 2);
+  for (int j = 0; j < gd; ++j) {
     float M = kNegInf;
 #pragma unroll
     for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, s_m[w][j]);
@@ -294,7 +313,7 @@ __global__ void __launch_bounds__(kAttnThreads)
 #pragma unroll
       for (int w = 0; w < kAttnWarps; ++w) {
         const float e = exp2f(s_m[w][j] - M);
-        num += e * so[(w * kMaxGroup + j) * kHeadDim + d];
+        num += e * comb[(w * kMaxGroup + j) * kRowPad + d];
         den += e * s_l[w][j];
       }
     }
@@ -306,42 +325,75 @@ __global__ void __launch_bounds__(kAttnThreads)
   }
   __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(&p.counters[pair], 1u) == (unsigned)(nchunks - 1));
+  if (tid == 0) s_last = (atomicAdd(&p.counters[it.pair], 1u) == (unsigned)(it.nchunks - 1));
   __syncthreads();
   if (!s_last) return;
+
+  // Merge all chunks of the pair: the (m, l) of up to kMergeBatch chunks are
+  // staged in shared memory with one round of independent loads, then every
+  // thread folds its output dim over the batch with independent, unrolled
+  // loads, so a merge costs a few L2 round trips rather than one per chunk.
   __threadfence();
-  if (tid == 0) p.counters[pair] = 0u;
-  const float* pp = p.partials + pair * p.max_chunks * (int64_t)g * (kHeadDim + 2);
-  for (int j = 0; j < g; ++j) {
-    float M = kNegInf;
-    for (int cc = 0; cc < nchunks; ++cc)
-      M = fmaxf(M, __ldcg(pp + ((int64_t)cc * g + j) * (kHeadDim + 2) + kHeadDim));
-    float num = 0.f, den = 0.f;
-    if (M != kNegInf) {
-      for (int cc = 0; cc < nchunks; ++cc) {
-        const float* q = pp + ((int64_t)cc * g + j) * (kHeadDim + 2);
-        const float mc = __ldcg(q + kHeadDim);
-        if (mc == kNegInf) continue;
-        const float e = exp2f(mc - M);
-        num += e * __ldcg(q + d);
-        den += e * __ldcg(q + kHeadDim + 1);
+  if (tid == 0) p.counters[it.pair] = 0u;  // ready for the next call
+  const float* pp = p.partials + it.pair * p.max_chunks * (int64_t)g * (kHeadDim + 2);
+  float Mr[kMaxGroup], num[kMaxGroup], den[kMaxGroup];
+#pragma unroll
+  for (int j = 0; j < kMaxGroup; ++j) {
+    Mr[j] = kNegInf;
+    num[j] = 0.f;
+    den[j] = 0.f;
+  }
+  for (int cb = 0; cb < it.nchunks; cb += kMergeBatch) {
+    const int nbat = min(kMergeBatch, it.nchunks - cb);
+    for (int i = tid; i < nbat * g; i += kAttnThreads) {
+      const float* q = pp + ((int64_t)cb * g + i) * (kHeadDim + 2);
+      s_pm[i] = __ldcg(q + kHeadDim);
+      s_pl[i] = __ldcg(q + kHeadDim + 1);
+    }
+    __syncthreads();
+    if (d < kHeadDim) {
+#pragma unroll
+      for (int j = 0; j < kMaxGroup; ++j) {
+        if (j < g) {
+          float Mb = kNegInf;
+          for (int c = 0; c < nbat; ++c) Mb = fmaxf(Mb, s_pm[c * g + j]);
+          const float Mn = fmaxf(Mr[j], Mb);
+          if (Mn != kNegInf) {
+            const float a = exp2f(Mr[j] - Mn);
+            float nn = num[j] * a, dd = den[j] * a;
+#pragma unroll 8
+            for (int c = 0; c < nbat; ++c) {
+              const float mc = s_pm[c * g + j];
+              const float e = mc == kNegInf ? 0.f : exp2f(mc - Mn);
+              nn += e * __ldcg(pp + ((int64_t)(cb + c) * g + j) * (kHeadDim + 2) + d);
+              dd += e * s_pl[c * g + j];
+            }
+            num[j] = nn;
+            den[j] = dd;
+            Mr[j] = Mn;
+          }
+        }
       }
     }
-    p.out[(qh0 + j) * kHeadDim + d] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
-    if (p.lse && d == 0) p.lse[qh0 + j] = den > 0.f ? (M + log2f(den)) * 0.6931471805599453f : kNegInf;
+    __syncthreads();
+  }
+  if (d < kHeadDim) {
+#pragma unroll
+    for (int j = 0; j < kMaxGroup; ++j) {
+      if (j < g) {
+        p.out[(qh0 + j) * kHeadDim + d] = __float2bfloat16_rn(den[j] > 0.f ? num[j] / den[j] : 0.f);
+        if (p.lse && d == 0)
+          p.lse[qh0 + j] = den[j] > 0.f ? (Mr[j] + log2f(den[j])) * 0.6931471805599453f : kNegInf;
+      }
+    }
   }
 }
 
-constexpr int kAttnStages = 4;
-
-cudaError_t launch_attn(const AttnParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
-                        int grid_x, cudaStream_t s) {
-  const size_t smem = attn_smem_bytes<kAttnStages>();
-  cudaError_t e = cudaFuncSetAttribute(attn_kernel<kAttnStages>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+cudaError_t launch_attn(const AttnParams& p, int num_items, cudaStream_t s) {
+  const size_t smem = attn_smem_bytes();
+  cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(grid_x, p.Hkv, p.B);
-  attn_kernel<kAttnStages><<<grid, kAttnThreads, smem, s>>>(tmk, tmv, p);
+  attn_kernel<<<num_items, kAttnThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 

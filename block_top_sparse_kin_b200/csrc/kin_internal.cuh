@@ -2,7 +2,6 @@
 // libkin.so (sm_100a).  Not part of the public ABI (see include/kin.h).
 #pragma once
 
-#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -15,9 +14,7 @@ constexpr int kHeadDim = 128;
 constexpr int kMaxGroup = 8;
 constexpr int kMaxBlocksPerSeq = 32768;
 constexpr int kTileTokens = 16;  // tokens per attention tile (one m16 MMA row block)
-
-// Bounded waits give up after this many SM clock cycles (about 0.5 s at 2 GHz).
-constexpr long long kWaitLimitCycles = 1000000000LL;
+constexpr int kMaxItemTiles = 64;  // attention tiles per work item (chunk of kept blocks)
 
 // ----------------------------------------------------------------- status
 __device__ __forceinline__ void set_status(int32_t* st, int32_t code) {
@@ -31,69 +28,8 @@ __device__ __forceinline__ uint32_t float_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// ------------------------------------------------------- PTX: mbarriers, TMA
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void fence_mbar_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Waits for phase `parity` of the barrier.  Gives up (returns false) after
-// kWaitLimitCycles, or early once another warp has recorded KIN_ERR_TIMEOUT
-// in *abort_flag (nullable), so one stuck copy cannot stall a whole grid.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
-                                                  const int32_t* abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0) {
-      if (clock64() - t0 > kWaitLimitCycles) return false;
-      if (abort_flag && *reinterpret_cast<const volatile int32_t*>(abort_flag) == KIN_ERR_TIMEOUT)
-        return false;
-    }
-  }
-}
-
-// 2-D tiled TMA load global -> shared, completion counted on an mbarrier.
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int32_t x,
-                                            int32_t y, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
 }
 
 // -------------------------------------------------- PTX: warp-level MMA path
@@ -168,6 +104,8 @@ struct SelectParams {
 
 struct AttnParams {
   const __nv_bfloat16* q;
+  const __nv_bfloat16* k_cache;
+  const __nv_bfloat16* v_cache;
   const int32_t* seq_lens;
   const int32_t* sel_idx;
   const int32_t* sel_cnt;
@@ -184,7 +122,6 @@ struct AttnParams {
 cudaError_t launch_means_build(const MeansBuildParams& p, cudaStream_t s);
 cudaError_t launch_means_update(const MeansUpdateParams& p, cudaStream_t s);
 cudaError_t launch_select(const SelectParams& p, int grid_x, cudaStream_t s);
-cudaError_t launch_attn(const AttnParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
-                        int grid_x, cudaStream_t s);
+cudaError_t launch_attn(const AttnParams& p, int num_items, cudaStream_t s);
 
 }  // namespace kin

@@ -97,7 +97,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectParams p) {
   const int i1 = min(i0 + p.chunk_blocks, nb);
   const float4* mrow = reinterpret_cast<const float4*>(p.means + pair * p.nbcap * kHeadDim) + lane;
   float* sc = p.scores + pair * p.nbcap;
-  constexpr int U = 4;
+#ifndef KIN_SEL_UNROLL
+#define KIN_SEL_UNROLL 4
+#endif
+  constexpr int U = KIN_SEL_UNROLL;  // mean rows in flight per warp
   for (int i = i0 + warp; i < i1; i += kSelWarps * U) {
     float4 m[U];
 #pragma unroll
