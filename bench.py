@@ -8,8 +8,9 @@ resident decode state built before timing.
 
 Metric: query-heads/s = B * Hq / t_step (whole job: summed over ranks, time =
 max over ranks).  Timing: CUDA events on the launching stream, one event pair
-per kernel per step, L2 flushed (a 256 MiB write, outside the events) before
-every step; W warm-up steps; barrier + synchronize around the K timed steps.
+per kernel per step, L2 flushed (a 256 MiB write then a 256 MiB read, outside
+the events) before every step; W warm-up steps; barrier + synchronize around
+the K timed steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--k K]
   python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
@@ -39,7 +40,7 @@ import kin_inputs as ki  # noqa: E402
 DEFAULT_WORKLOAD = "qwen3_8b_32k"
 METRIC = "block-top-k decode attn query-heads/s"
 FALLBACK_HBM_GBS = 6650.0
-L2_FLUSH_BYTES = 256 << 20
+L2_FLUSH_BYTES = 256 << 20  # > 2x the 126 MB L2
 
 
 # ---------------------------------------------------------------- bytes model
@@ -252,9 +253,19 @@ def gpu_arm(args):
     k = args.k or w0.k
     w = shard_workload(w0, rank)
     st = build_device_state(w, k)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+
+    def flush_l2(i):
+        """Write a buffer larger than L2, then read another one, so a timed
+        step starts with a cold L2 holding no dirty lines to write back."""
+        flush_w.fill_(i & 0xFF)
+        flush_sink.copy_(flush_r.sum())
+
+    flush_sink = torch.zeros((), dtype=torch.float32, device="cuda")
     n_ev = 4 if w.n_append else 3
-    launches_per_step = 3 if w.n_append else 2
+    # select = scan + top-k kernels, then attention (+ the append update)
+    launches_per_step = 4 if w.n_append else 3
 
     for _ in range(args.warmup):
         reset_state(st)
@@ -271,7 +282,7 @@ def gpu_arm(args):
         wall0 = time.perf_counter()
         for s in range(args.steps):
             reset_state(st)
-            flush.fill_(s & 0xFF)          # L2 flush (outside the events)
+            flush_l2(s)                    # outside the events
             run_step(st, events[s])
         torch.cuda.synchronize()
         wall = time.perf_counter() - wall0
@@ -305,7 +316,7 @@ def gpu_arm(args):
         dist.barrier()
     for s in range(args.steps):
         reset_state(st)
-        flush.fill_(s & 0xFF)
+        flush_l2(s)
         e2e_ev[s][0].record()
         st["q"].copy_(q_pin, non_blocking=True)
         run_step(st)
@@ -349,7 +360,7 @@ def gpu_arm(args):
                 "head_dim": w0.D, "context": [w0.Lmin, w0.Lmax], "block_size": w0.bs,
                 "top_k_blocks": k, "append_tokens": w0.n_append,
                 "global_batch": w0.B * world, "parallelism": f"dp{world}",
-                "l2": "flushed before every step (256 MiB write outside the timed events)",
+                "l2": "flushed before every step (256 MiB write + 256 MiB read, outside the timed events)",
             },
             "impl": "kin",
             "gpu_launches": launches_per_step * args.steps,

@@ -200,8 +200,8 @@ KIN_EXPORT kin_status kin_block_topk_select(const kin_dims* dims, const void* q,
   p.k = k_blocks;
   p.chunk_blocks = select_chunk_blocks(*dims);
   p.score_scale = 1.0f / std::sqrt((float)kHeadDim);
-  const int grid_x = (p.nbcap + p.chunk_blocks - 1) / p.chunk_blocks;
-  return from_cuda(launch_select(p, grid_x, static_cast<cudaStream_t>(stream)));
+  const int chunks_per_pair = (p.nbcap + p.chunk_blocks - 1) / p.chunk_blocks;
+  return from_cuda(launch_select(p, chunks_per_pair, static_cast<cudaStream_t>(stream)));
 }
 
 KIN_EXPORT kin_status kin_sparse_decode_attn(const kin_dims* dims, const void* q, const void* k_cache,

@@ -121,7 +121,7 @@ struct AttnParams {
 // Launchers (one per kernel family); return the launch error.
 cudaError_t launch_means_build(const MeansBuildParams& p, cudaStream_t s);
 cudaError_t launch_means_update(const MeansUpdateParams& p, cudaStream_t s);
-cudaError_t launch_select(const SelectParams& p, int grid_x, cudaStream_t s);
+cudaError_t launch_select(const SelectParams& p, int chunks_per_pair, cudaStream_t s);
 cudaError_t launch_attn(const AttnParams& p, int num_items, cudaStream_t s);
 
 }  // namespace kin

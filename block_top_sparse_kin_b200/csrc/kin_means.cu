@@ -89,11 +89,19 @@ __global__ void __launch_bounds__(256) means_update_kernel(MeansUpdateParams p) 
     const int t0 = i * p.bs, t1 = min(t0 + p.bs, L1);
     const uint2* cache = reinterpret_cast<const uint2*>(p.k_cache + pair * p.Lcap * kHeadDim) + lane;
     const uint2* fresh = reinterpret_cast<const uint2*>(p.k_new + pair * n * kHeadDim) + lane;
+    auto row = [&](int t) {
+      return t < L0 ? cache[(int64_t)t * (kHeadDim / 4)] : fresh[(int64_t)(t - L0) * (kHeadDim / 4)];
+    };
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int t = t0; t < t1; ++t) {
-      uint2 raw = t < L0 ? cache[(int64_t)t * (kHeadDim / 4)] : fresh[(int64_t)(t - L0) * (kHeadDim / 4)];
-      add_row4(acc, raw);
+    int t = t0;
+    for (; t + 8 <= t1; t += 8) {  // 8 rows in flight per lane, summed in token order
+      uint2 r[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) r[u] = row(t + u);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) add_row4(acc, r[u]);
     }
+    for (; t < t1; ++t) add_row4(acc, row(t));
     const float cnt = (float)(t1 - t0);
     float4 m = make_float4(__fdiv_rn(acc[0], cnt), __fdiv_rn(acc[1], cnt), __fdiv_rn(acc[2], cnt),
                            __fdiv_rn(acc[3], cnt));
