@@ -274,16 +274,33 @@ def gpu_arm(args):
     if int(st["status"].item()) != 0:
         raise RuntimeError(f"device status {int(st['status'].item())} after warm-up")
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    # Each timed step is one CUDA graph (captured once, as a decode loop
+    # would): the kernels of the step with timing events between them.  The
+    # L2 flush runs eagerly before each replay, outside the events.
+    events = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ev)]
+              for _ in range(args.steps)]
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    graphs = []
+    with torch.cuda.stream(cap):
+        for s in range(args.steps):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                reset_state(st)
+                run_step(st, events[s])
+            graphs.append(g)
+    torch.cuda.current_stream().wait_stream(cap)
+    for g in graphs[: min(len(graphs), args.warmup)]:  # warm the graphs themselves
+        g.replay()
+    torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         wall0 = time.perf_counter()
         for s in range(args.steps):
-            reset_state(st)
             flush_l2(s)                    # outside the events
-            run_step(st, events[s])
+            graphs[s].replay()
         torch.cuda.synchronize()
         wall = time.perf_counter() - wall0
     if world > 1:

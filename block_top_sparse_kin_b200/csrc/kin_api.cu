@@ -100,6 +100,40 @@ kin_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KIN_OK : KIN_ERR
 
 }  // namespace
 
+namespace kin {
+
+constexpr int kMaxDevices = 64;
+
+int device_sm_count() {
+  static int cache[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return kTargetSMs;
+  if (dev >= kMaxDevices) {
+    int n = 0;
+    return cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? n : kTargetSMs;
+  }
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return kTargetSMs;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+cudaError_t ensure_smem_limit(const void* kernel, int slot, size_t bytes) {
+  // slot: a small per-kernel index; the cache remembers the largest limit set
+  static size_t done[8][kMaxDevices] = {{0}};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < kMaxDevices && slot >= 0 && slot < 8 && done[slot][dev] >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess && dev < kMaxDevices && slot >= 0 && slot < 8) done[slot][dev] = bytes;
+  return e;
+}
+
+}  // namespace kin
+
 KIN_EXPORT const char* kin_status_string(kin_status s) {
   switch (s) {
     case KIN_OK: return "KIN_OK";

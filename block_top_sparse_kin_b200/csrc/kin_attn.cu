@@ -107,6 +107,7 @@ __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kerne
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = p.g;
+  pdl_wait();  // the selection comes from the select kernels
   const ItemInfo it = item_info(p, blockIdx.x);
   const int64_t qh0 = (int64_t)it.b * p.Hq + (int64_t)it.h * g;
   if (it.cnt <= 0) {  // nothing selected (flagged upstream): out = 0, lse = -inf
@@ -391,10 +392,9 @@ __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kerne
 
 cudaError_t launch_attn(const AttnParams& p, int num_items, cudaStream_t s) {
   const size_t smem = attn_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(attn_kernel), 1, smem);
   if (e != cudaSuccess) return e;
-  attn_kernel<<<num_items, kAttnThreads, smem, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(attn_kernel, dim3(num_items), dim3(kAttnThreads), smem, s, p);
 }
 
 }  // namespace kin

@@ -32,6 +32,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ------------------------------------------- programmatic dependent launch
+// Kernels of a step are launched with programmatic stream serialization: a
+// kernel may be scheduled while its predecessor drains, and waits here (a
+// hardware dependency wait, not a spin) before touching the predecessor's
+// results; each kernel signals once its own results are written.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // -------------------------------------------------- PTX: warp-level MMA path
 __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1,
                                             uint32_t& r2, uint32_t& r3) {
@@ -117,6 +125,29 @@ struct AttnParams {
   int B, Hkv, Hq, g, bs, Lcap, k, chunk_blocks, max_chunks;
   float scale_log2;     // softmax_scale * log2(e)
 };
+
+// Launch with programmatic stream serialization (see pdl_wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// Per-device facts the launchers need, cached after the first query (a
+// device's SM count never changes; racing first calls store the same value).
+int device_sm_count();
+// Raises a kernel's dynamic shared memory limit once per device.
+cudaError_t ensure_smem_limit(const void* kernel, int slot, size_t bytes);
 
 // Launchers (one per kernel family); return the launch error.
 cudaError_t launch_means_build(const MeansBuildParams& p, cudaStream_t s);

@@ -25,6 +25,7 @@ __device__ __forceinline__ void add_row4(float (&acc)[4], uint2 raw) {
 
 // grid (ceil(nbcap / 8), Hkv, B), 256 threads: warp w of CTA x owns block 8x + w.
 __global__ void __launch_bounds__(256) means_build_kernel(MeansBuildParams p) {
+  pdl_wait();
   const int b = blockIdx.z, h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int L = p.seq_lens[b];
@@ -58,6 +59,7 @@ __global__ void __launch_bounds__(256) means_build_kernel(MeansBuildParams p) {
 // grid (B), 256 threads.  One CTA owns a whole sequence so that the length
 // it reads and the length it writes back cannot race with another CTA.
 __global__ void __launch_bounds__(256) means_update_kernel(MeansUpdateParams p) {
+  pdl_wait();
   const int b = blockIdx.x;
   const int L0 = p.seq_lens[b];
   const int n = p.n_new;
@@ -109,17 +111,15 @@ __global__ void __launch_bounds__(256) means_update_kernel(MeansUpdateParams p) 
   }
   __syncthreads();
   if (threadIdx.x == 0) p.seq_lens[b] = L1;
+  pdl_trigger();
 }
 
 cudaError_t launch_means_build(const MeansBuildParams& p, cudaStream_t s) {
-  dim3 grid((p.nbcap + 7) / 8, p.Hkv, p.B);
-  means_build_kernel<<<grid, 256, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(means_build_kernel, dim3((p.nbcap + 7) / 8, p.Hkv, p.B), dim3(256), 0, s, p);
 }
 
 cudaError_t launch_means_update(const MeansUpdateParams& p, cudaStream_t s) {
-  means_update_kernel<<<p.B, 256, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(means_update_kernel, dim3(p.B), dim3(256), 0, s, p);
 }
 
 }  // namespace kin

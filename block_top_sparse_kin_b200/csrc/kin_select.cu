@@ -8,19 +8,18 @@
 // response Q4).  The group score uses linearity: sum_j q_j . m_i =
 // (sum_j q_j) . m_i, so each block costs one 128-wide dot product.
 //
-// Work split: a work item is a chunk of `chunk_blocks` blocks of one pair;
-// a grid of KIN_SEL_CTAS_PER_SM resident CTAs per SM walks the items.  Warp
-// w scans rows w, w + 8, ... of the chunk, one 512-byte mean row per warp
-// load (lane l reads dims 4l..4l+3 as one float4), double-buffered so the
-// next U rows are in flight while the current U are reduced; a butterfly
-// that halves the rows per lane at each level sums U rows in U + 4 - log2 U
-// shuffles.  Scores go to workspace (they stay in L2).  The pair's last
-// chunk to finish (atomic completion counter, no waiting) runs the top-k: a
-// 4-pass 8-bit radix select over order-preserving uint32 keys in shared
-// memory finds the threshold key T and how many keys equal to T to take; the
-// lowest-index equal keys are taken, which is the (score desc, index asc)
-// rule.  Output positions come from two block-wide prefix sums, so indices
-// leave ascending.
+// Two kernels, the second launched with programmatic dependent launch:
+//  1. select_scan_kernel streams every block mean once: the (pair, block)
+//     rows are cut into one contiguous, pair-aligned range per warp; a warp
+//     reads one 512-byte mean row per load (lane l owns dims 4l..4l+3) and
+//     keeps the next 8 rows in flight while reducing the current 8, with a
+//     butterfly that halves the rows per lane at each level (8 rows in 9
+//     shuffles).  Scores go to workspace, where they stay in L2.
+//  2. select_topk_kernel, one CTA per pair, loads the pair's scores as
+//     order-preserving uint32 keys into shared memory and runs an exact
+//     radix select (see topk_emit): the first block and the block holding
+//     the newest token are always kept, ties go to the lower index, and the
+//     kept indices leave ascending.
 #include "kin_internal.cuh"
 
 namespace kin {
@@ -35,24 +34,6 @@ namespace kin {
 constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelU = KIN_SEL_UNROLL;  // mean rows per warp per step
-
-// Exclusive prefix sum over the CTA (256 threads); returns this thread's base.
-__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int inc = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int t = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += t;
-  }
-  if (lane == 31) warp_tot[warp] = inc;
-  __syncthreads();
-  int base = 0;
-#pragma unroll
-  for (int w = 0; w < kSelWarps; ++w) base += (w < warp) ? warp_tot[w] : 0;
-  __syncthreads();
-  return base + inc - v;
-}
 
 // Sums U per-lane partials (one per mean row) over the warp with
 // U + 4 - log2(U) shuffles instead of 5 U: each butterfly level halves the
@@ -79,34 +60,45 @@ __device__ __forceinline__ float warp_sum_rows(float (&v)[U], int lane) {
 }
 
 struct SelectSmem {
-  int hist[256];
-  int warp_tot[kSelWarps];
-  int digit, above, last;
+  int hist[2][256];          // double-buffered radix histogram
+  int warp_cnt[3][kSelWarps];  // per-warp counts: forced, > T, == T
+  int digit, above;
 };
 
 // Exact top-(k-2) over keys[1..nb-2] plus the forced blocks 0 and nb-1,
 // written ascending to sel[0..k).  keys live in shared memory.
+//  * Radix select, 4 passes of 8 bits from the top: each pass histograms the
+//    keys that still match the chosen prefix (shared atomics into one of two
+//    alternating histograms, so zeroing the next needs no extra barrier),
+//    then warp 0 finds the digit holding the kr-th largest.  This yields the threshold key T and kr, the
+//    number of keys equal to T to take.
+//  * Emit with ballots: warp w owns a contiguous index range; one pass counts
+//    its forced / greater / equal keys, one barrier publishes the counts, and
+//    a second pass writes the taken indices in order (keys == T are taken in
+//    index order while their rank is below kr, i.e. ties go to lower indices).
 __device__ __forceinline__ void topk_emit(const uint32_t* keys, int nb, int k, int32_t* sel,
                                           SelectSmem& sm, int32_t* dev_status) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // ---- radix select: threshold key T and the number kr of keys == T to take
   uint32_t prefix = 0u, mask = 0u;
   int kr = k - 2;
+  sm.hist[0][tid] = 0;
+  sm.hist[1][tid] = 0;
+  __syncthreads();
 #pragma unroll 1
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
-    sm.hist[tid] = 0;
-    __syncthreads();
+    int* hist = sm.hist[pass & 1];
     for (int i = 1 + tid; i < nb - 1; i += kSelThreads) {
       const uint32_t key = keys[i];
-      if ((key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 0xFFu], 1);
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFFu], 1);
     }
+    sm.hist[(pass + 1) & 1][tid] = 0;  // the other buffer is free: ready it for the next pass
     __syncthreads();
     if (warp == 0) {
       int cnt[8], tot = 0;
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        cnt[u] = sm.hist[255 - (lane * 8 + u)];  // descending digits
+        cnt[u] = hist[255 - (lane * 8 + u)];  // descending digits
         tot += cnt[u];
       }
       int inc = tot;
@@ -133,45 +125,55 @@ __device__ __forceinline__ void topk_emit(const uint32_t* keys, int nb, int k, i
     prefix |= (uint32_t)sm.digit << shift;
     mask |= 0xFFu << shift;
     kr -= sm.above;
-    __syncthreads();
   }
   const uint32_t T = prefix;
 
-  // ---- emit: forced {0, nb-1}, keys > T, and the kr lowest-index keys == T
-  const int per = (nb + kSelThreads - 1) / kSelThreads;
-  const int j0 = min(tid * per, nb), j1 = min(j0 + per, nb);
-  int eq = 0;
-  for (int i = j0; i < j1; ++i)
-    if (i >= 1 && i <= nb - 2 && keys[i] == T) ++eq;
-  const int eq_base = block_exclusive_scan(eq, sm.warp_tot);
-  int r = eq_base, mine = 0;
-  for (int i = j0; i < j1; ++i) {
-    const bool cand = i >= 1 && i <= nb - 2;
-    const uint32_t key = keys[i];
-    bool take = !cand || key > T;
-    if (cand && key == T) {
-      take = r < kr;
-      ++r;
-    }
-    mine += take;
+  // ---- emit
+  const int span = ((nb + kSelWarps - 1) / kSelWarps + 31) & ~31;  // per-warp range, whole batches
+  const int w0 = min(warp * span, nb), w1 = min(w0 + span, nb);
+  const unsigned lt = (1u << lane) - 1u;
+  int n_forced = 0, n_gt = 0, n_eq = 0;
+  for (int base = w0; base < w1; base += 32) {
+    const int i = base + lane;
+    const bool in = i < w1;
+    const uint32_t key = in ? keys[i] : 0u;
+    const bool cand = in && i >= 1 && i <= nb - 2;
+    n_forced += __popc(__ballot_sync(0xffffffffu, in && !cand));
+    n_gt += __popc(__ballot_sync(0xffffffffu, cand && key > T));
+    n_eq += __popc(__ballot_sync(0xffffffffu, cand && key == T));
   }
-  int pos = block_exclusive_scan(mine, sm.warp_tot);
-  r = eq_base;
-  for (int i = j0; i < j1; ++i) {
-    const bool cand = i >= 1 && i <= nb - 2;
-    const uint32_t key = keys[i];
-    bool take = !cand || key > T;
-    if (cand && key == T) {
-      take = r < kr;
-      ++r;
-    }
+  if (lane == 0) {
+    sm.warp_cnt[0][warp] = n_forced;
+    sm.warp_cnt[1][warp] = n_gt;
+    sm.warp_cnt[2][warp] = n_eq;
+  }
+  __syncthreads();
+  int eq_base = 0, out_base = 0;
+  for (int w = 0; w < warp; ++w) {
+    const int e = sm.warp_cnt[2][w];
+    const int eq_take = min(max(kr - eq_base, 0), e);  // equal keys warp w takes
+    out_base += sm.warp_cnt[0][w] + sm.warp_cnt[1][w] + eq_take;
+    eq_base += e;
+  }
+  int pos = out_base, eq_rank = eq_base;
+  for (int base = w0; base < w1; base += 32) {
+    const int i = base + lane;
+    const bool in = i < w1;
+    const uint32_t key = in ? keys[i] : 0u;
+    const bool cand = in && i >= 1 && i <= nb - 2;
+    const bool eq = cand && key == T;
+    const unsigned eq_mask = __ballot_sync(0xffffffffu, eq);
+    const bool take = (in && !cand) || (cand && key > T) || (eq && eq_rank + __popc(eq_mask & lt) < kr);
+    const unsigned take_mask = __ballot_sync(0xffffffffu, take);
     if (take) {
-      if (pos < k) sel[pos] = i;  // never write past the pair's row
-      ++pos;
+      const int o = pos + __popc(take_mask & lt);
+      if (o < k) sel[o] = i;  // never write past the pair's row
     }
+    pos += __popc(take_mask);
+    eq_rank += __popc(eq_mask);
   }
-  // self-check: exactly k blocks were emitted (the last thread ends at k)
-  if (tid == kSelThreads - 1 && pos != k) set_status(dev_status, KIN_ERR_DEVICE_DATA);
+  // self-check: exactly k blocks were emitted (the last warp ends at k)
+  if (warp == kSelWarps - 1 && lane == 0 && pos != k) set_status(dev_status, KIN_ERR_DEVICE_DATA);
 }
 
 // ---- kernel 1: the scan.  Rows are numbered per pair in steps of U
@@ -203,6 +205,7 @@ __device__ __forceinline__ void pair_qsum(const SelectParams& p, int pair, int l
 }
 
 __global__ void __launch_bounds__(kSelThreads, KIN_SEL_CTAS_PER_SM) select_scan_kernel(SelectParams p) {
+  pdl_wait();  // means, lengths and q come from earlier work on the stream
   const int lane = threadIdx.x & 31;
   const int nwarps = gridDim.x * kSelWarps;
   const int gw = blockIdx.x * kSelWarps + (threadIdx.x >> 5);
@@ -210,7 +213,10 @@ __global__ void __launch_bounds__(kSelThreads, KIN_SEL_CTAS_PER_SM) select_scan_
   const int steps = p.B * p.Hkv * (nbp / kSelU);
   const int per = (steps + nwarps - 1) / nwarps;
   const int s0 = gw * per, s1 = min(s0 + per, steps);
-  if (s0 >= s1) return;
+  if (s0 >= s1) {
+    pdl_trigger();
+    return;
+  }
 
   // step s covers slots s*U .. s*U+U-1 of pair (s*U) / nbp
   int pair = (s0 * kSelU) / nbp;
@@ -259,6 +265,7 @@ __global__ void __launch_bounds__(kSelThreads, KIN_SEL_CTAS_PER_SM) select_scan_
 #pragma unroll
     for (int u = 0; u < kSelU; ++u) cur[u] = nxt[u];
   }
+  pdl_trigger();
 }
 
 // ---- kernel 2: one CTA per pair: dense shortcut, bad-length flag, or the
@@ -267,6 +274,7 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(SelectParams p
   extern __shared__ uint32_t skey[];  // [nbcap]
   __shared__ SelectSmem sm;
   const int tid = threadIdx.x;
+  pdl_wait();  // scores come from the scan kernel
   const int64_t pair = blockIdx.x;
   const int b = (int)(pair / p.Hkv);
   const int k = p.k;
@@ -296,22 +304,16 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(SelectParams p
 cudaError_t launch_select(const SelectParams& p, int /*chunks_per_pair*/, cudaStream_t s) {
   const size_t smem = (size_t)p.nbcap * sizeof(uint32_t);
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(select_topk_kernel), 0, smem);
     if (e != cudaSuccess) return e;
   }
-  int dev = 0, sms = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
   const int64_t rows = (int64_t)p.B * p.Hkv * p.nbcap;
   const int64_t want = (rows + kSelWarps * kSelU * 4 - 1) / (kSelWarps * kSelU * 4);  // >= 4 steps per warp
-  const int64_t resident = (int64_t)sms * KIN_SEL_CTAS_PER_SM;
+  const int64_t resident = (int64_t)device_sm_count() * KIN_SEL_CTAS_PER_SM;
   const int grid = (int)(want < resident ? (want > 0 ? want : 1) : resident);
-  select_scan_kernel<<<grid, kSelThreads, 0, s>>>(p);
-  e = cudaGetLastError();
+  cudaError_t e = launch_pdl(select_scan_kernel, dim3(grid), dim3(kSelThreads), 0, s, p);
   if (e != cudaSuccess) return e;
-  select_topk_kernel<<<p.B * p.Hkv, kSelThreads, smem, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(select_topk_kernel, dim3(p.B * p.Hkv), dim3(kSelThreads), smem, s, p);
 }
 
 }  // namespace kin
