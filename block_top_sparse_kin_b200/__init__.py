@@ -26,7 +26,9 @@ STATUS_NAMES = {
 EXPORTED = (
     "kin_status_string", "kin_workspace_bytes", "kin_block_means_build",
     "kin_block_means_update", "kin_block_topk_select", "kin_sparse_decode_attn",
+    "kin_block_topk_select_noalloc",
 )
+NOALLOC_SCRATCH_FLOATS = 1 << 21  # KIN_NOALLOC_SCRATCH_FLOATS in include/kin.h
 
 
 class KinError(RuntimeError):
@@ -81,6 +83,8 @@ def load_library(path: str = LIB_PATH):
     lib.kin_sparse_decode_attn.argtypes = [dp, vp, vp, vp, vp, vp, vp, i32, f32, vp, vp, vp, sz,
                                            vp, vp]
     lib.kin_sparse_decode_attn.restype = ctypes.c_int
+    lib.kin_block_topk_select_noalloc.argtypes = [dp, vp, vp, vp, i32, vp, vp, vp, vp]
+    lib.kin_block_topk_select_noalloc.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -169,3 +173,16 @@ def kin_sparse_decode_attn(dims, q, k_cache, v_cache, seq_lens, sel_idx, sel_cnt
         workspace.numel() * workspace.element_size(),
         _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
     _check(rc, "kin_sparse_decode_attn")
+
+
+def kin_block_topk_select_noalloc(dims, q, block_means, seq_lens, k_blocks, sel_idx, sel_cnt,
+                                  dev_status=None, stream=None):
+    """kin_block_topk_select without a workspace, for callers that may not
+    allocate device memory: the scratch lives in a fixed array inside
+    libkin.so (see include/kin.h for its limit and its sharing rules)."""
+    rc = load_library().kin_block_topk_select_noalloc(
+        ctypes.byref(dims), _dev(q, "q", _BF16), _dev(block_means, "block_means", torch.float32),
+        _dev(seq_lens, "seq_lens", torch.int32), int(k_blocks), _dev(sel_idx, "sel_idx", torch.int32),
+        _dev(sel_cnt, "sel_cnt", torch.int32),
+        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+    _check(rc, "kin_block_topk_select_noalloc")

@@ -41,7 +41,8 @@
  *    item and write the status code into *dev_status (first error wins) when
  *    dev_status is not NULL.  Kernels never trap; every wait is bounded.
  *  - No C++ exception crosses this boundary; the library keeps no state
- *    between calls other than what the caller's buffers hold.
+ *    between calls other than what the caller's buffers hold (except the
+ *    scratch array of kin_block_topk_select_noalloc, described there).
  *  - Limits: head_dim == 128; Hq % Hkv == 0 with 1 <= Hq/Hkv <= 8;
  *    block_size in {16, 32, 64, 128}; ceil(Lcap / bs) <= 32768;
  *    B * Hkv * Lcap < 2^31.
@@ -145,6 +146,33 @@ kin_status kin_sparse_decode_attn(const kin_dims* dims, const void* q, const voi
                                   int32_t k_blocks, float softmax_scale, void* out, float* lse,
                                   void* workspace, size_t ws_bytes, int32_t* dev_status,
                                   void* stream);
+
+/* ------------------------------------------------------------------------
+ * Allocation-free variant of kin_block_topk_select (the pages describe no
+ * counterpart; it exists for callers, not for the method).
+ *
+ * For callers that cannot allocate device memory: code running under a host
+ * that plans and owns all device memory up front (a runtime with a fixed
+ * memory plan, a plugin that may not call cudaMalloc, a decode loop that
+ * must never reach the allocator), or that has no workspace to pass.  It
+ * computes exactly what kin_block_topk_select computes, with the same
+ * kernels, but keeps its scratch (one fp32 score per block) in a fixed array
+ * inside libkin.so: KIN_NOALLOC_SCRATCH_FLOATS floats (8 MiB) that every
+ * GPU which loads the library holds until the process exits.
+ *  - Requires batch * num_kv_heads * ceil(max_seq_len / block_size) <=
+ *    KIN_NOALLOC_SCRATCH_FLOATS, else KIN_ERR_CAPACITY (nothing launched).
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *  - The first call on each device is a one-time set-up (it looks up the
+ *    array's device address) and should come before any stream capture.
+ *  - Every call shares the one array, which keeps the last call's contents;
+ *    nothing in it needs to start at zero.  Calls whose kernels overlap on
+ *    the GPU (other streams, other threads) race on it: serialize them.
+ * Arguments, layouts and errors are those of kin_block_topk_select, without
+ * the workspace. */
+#define KIN_NOALLOC_SCRATCH_FLOATS (1 << 21)
+kin_status kin_block_topk_select_noalloc(const kin_dims* dims, const void* q, const float* block_means,
+                                         const int32_t* seq_lens, int32_t k_blocks, int32_t* sel_idx,
+                                         int32_t* sel_cnt, int32_t* dev_status, void* stream);
 
 #ifdef __cplusplus
 }

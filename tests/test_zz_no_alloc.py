@@ -1,0 +1,64 @@
+"""kin_block_topk_select_noalloc: the select for callers that may not
+allocate device memory (a runtime that owns a fixed memory plan, a plugin
+without allocation rights, a decode loop that must never reach the
+allocator).  It must return exactly what the workspace-based
+kin_block_topk_select returns, call after call, even though every call
+reuses the same scratch array inside the library.  This file sorts last so a
+run that stops at the first failure has run every other test first."""
+import numpy as np
+import pytest
+import torch
+
+import block_top_sparse_kin_b200 as kin
+import kin_inputs as ki
+from kin_testlib import D, make_device_case
+
+pytestmark = pytest.mark.gpu
+
+
+def _reference(dc, k):
+    ws = kin.alloc_workspace(dc.dims, k)
+    sel = torch.full((dc.w.B, dc.w.Hkv, k), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.full((dc.w.B, dc.w.Hkv), -7, dtype=torch.int32, device="cuda")
+    kin.kin_block_topk_select(dc.dims, dc.q, dc.means, dc.seq_lens, k, sel, cnt, ws)
+    torch.cuda.synchronize()
+    return sel.cpu().numpy(), cnt.cpu().numpy()
+
+
+def _noalloc(dc, k):
+    sel = torch.full((dc.w.B, dc.w.Hkv, k), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.full((dc.w.B, dc.w.Hkv), -7, dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kin.kin_block_topk_select_noalloc(dc.dims, dc.q, dc.means, dc.seq_lens, k, sel, cnt, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    return sel.cpu().numpy(), cnt.cpu().numpy()
+
+
+def test_noalloc_select_matches_workspace_select_on_consecutive_calls():
+    cases = [
+        ki.Workload("noalloc_a", 4, 4, 16, D, 16, 1500, 3000, 24, 31, Lcap=3072),
+        ki.Workload("noalloc_b", 3, 2, 10, D, 32, 300, 900, 6, 32, Lcap=960),
+    ]
+    devs = [make_device_case(w) for w in cases]
+    for dc in devs:
+        kin.kin_block_means_build(dc.dims, dc.k_cache, dc.seq_lens, dc.means)
+    torch.cuda.synchronize()
+    refs = [_reference(dc, dc.w.k) for dc in devs]
+    # two calls in a row on the same inputs, then a call on other inputs whose
+    # scratch rows overlap the previous call's: indices are integer results,
+    # so they must match bit for bit
+    for dc, ref in ((devs[0], refs[0]), (devs[0], refs[0]), (devs[1], refs[1])):
+        sel, cnt = _noalloc(dc, dc.w.k)
+        assert np.array_equal(cnt, ref[1])
+        assert np.array_equal(sel, ref[0])
+
+
+def test_noalloc_select_rejects_problems_beyond_its_scratch():
+    # B * Hkv * ceil(Lcap / bs) = 64 * 8 * 8192 > 2^21 scores
+    dims = kin.make_dims(64, 8, 32, D, 16, 8192 * 16)
+    t = torch.zeros(16, dtype=torch.int32, device="cuda")
+    q = torch.zeros((1, D), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(kin.KinError) as e:
+        kin.kin_block_topk_select_noalloc(dims, q, torch.zeros(4, device="cuda"), t, 8, t, t)
+    assert e.value.status == 3
