@@ -59,74 +59,119 @@ __device__ __forceinline__ float warp_sum_rows(float (&v)[U], int lane) {
   return r;
 }
 
+constexpr int kListCap = 4096;  // candidates kept in a compact list after the first pass
+
 struct SelectSmem {
-  int hist[2][256];          // double-buffered radix histogram
+  int hist[2][256];            // double-buffered radix histogram
+  int list[kListCap];          // indices whose key matches the first chosen digit
+  int list_n;
   int warp_cnt[3][kSelWarps];  // per-warp counts: forced, > T, == T
-  int digit, above;
+  int digit, above, bin;
 };
 
+// Warp 0: the digit (descending) whose bin holds the kr-th largest key of the
+// histogram, the count of keys in higher digits, and the bin's own count.
+__device__ __forceinline__ void find_digit(const int* hist, int kr, SelectSmem& sm) {
+  const int lane = threadIdx.x & 31;
+  int cnt[8], tot = 0;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    cnt[u] = hist[255 - (lane * 8 + u)];
+    tot += cnt[u];
+  }
+  int inc = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int t = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += t;
+  }
+  const int excl = inc - tot;
+  if (excl < kr && kr <= inc) {
+    int run = excl;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (run + cnt[u] >= kr) {
+        sm.digit = 255 - (lane * 8 + u);
+        sm.above = run;
+        sm.bin = cnt[u];
+        break;
+      }
+      run += cnt[u];
+    }
+  }
+}
+
 // Exact top-(k-2) over keys[1..nb-2] plus the forced blocks 0 and nb-1,
-// written ascending to sel[0..k).  keys live in shared memory.
-//  * Radix select, 4 passes of 8 bits from the top: each pass histograms the
-//    keys that still match the chosen prefix (shared atomics into one of two
-//    alternating histograms, so zeroing the next needs no extra barrier),
-//    then warp 0 finds the digit holding the kr-th largest.  This yields the threshold key T and kr, the
-//    number of keys equal to T to take.
+// written ascending to sel[0..k).  keys live in shared memory; hist[0] must
+// already hold the histogram of the candidates' top byte and hist[1] zeros.
+//  * Radix select, up to 4 passes of 8 bits from the top: each pass finds the
+//    digit whose bin holds the kr-th largest remaining key.  After the first
+//    pass the indices matching the chosen prefix go to a compact list, so the
+//    later passes visit only those.  A pass whose bin holds exactly the keys
+//    still needed ends the search: they are all taken.  The result is a
+//    prefix T over the top `mask` bits and kr, the number of keys equal to T
+//    (under the mask) to take.
 //  * Emit with ballots: warp w owns a contiguous index range; one pass counts
 //    its forced / greater / equal keys, one barrier publishes the counts, and
-//    a second pass writes the taken indices in order (keys == T are taken in
-//    index order while their rank is below kr, i.e. ties go to lower indices).
+//    a second pass writes the taken indices in order (keys equal to T under
+//    the mask are taken in index order while their rank is below kr: ties go
+//    to lower indices, and indices leave ascending).
 __device__ __forceinline__ void topk_emit(const uint32_t* keys, int nb, int k, int32_t* sel,
                                           SelectSmem& sm, int32_t* dev_status) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t prefix = 0u, mask = 0u;
   int kr = k - 2;
-  sm.hist[0][tid] = 0;
-  sm.hist[1][tid] = 0;
-  __syncthreads();
+  bool use_list = false;
+  if (kr == 0) {  // budget of two: only the forced blocks; no candidate key can pass
+    prefix = 0xFFFFFFFFu;
+    mask = 0xFFFFFFFFu;
+  }
 #pragma unroll 1
-  for (int pass = 0; pass < 4; ++pass) {
+  for (int pass = 0; pass < 4 && kr > 0; ++pass) {
     const int shift = 24 - 8 * pass;
     int* hist = sm.hist[pass & 1];
-    for (int i = 1 + tid; i < nb - 1; i += kSelThreads) {
-      const uint32_t key = keys[i];
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFFu], 1);
-    }
-    sm.hist[(pass + 1) & 1][tid] = 0;  // the other buffer is free: ready it for the next pass
-    __syncthreads();
-    if (warp == 0) {
-      int cnt[8], tot = 0;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        cnt[u] = hist[255 - (lane * 8 + u)];  // descending digits
-        tot += cnt[u];
-      }
-      int inc = tot;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        int t = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += t;
-      }
-      const int excl = inc - tot;
-      if (excl < kr && kr <= inc) {
-        int run = excl;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          if (run + cnt[u] >= kr) {
-            sm.digit = 255 - (lane * 8 + u);
-            sm.above = run;
-            break;
+    if (pass > 0) {
+      if (pass == 1) {  // visit every key once more, keep the matching indices
+        if (tid == 0) sm.list_n = 0;
+        __syncthreads();
+        for (int base = 0; base < nb; base += kSelThreads) {  // uniform trip count per warp
+          const int i = base + tid;
+          const uint32_t key = i < nb ? keys[i] : 0u;
+          const bool match = i >= 1 && i <= nb - 2 && (key & mask) == prefix;
+          if (match) atomicAdd(&hist[(key >> shift) & 0xFFu], 1);
+          if (use_list) {  // one list reservation per warp, lanes take slots in order
+            const unsigned m = __ballot_sync(0xffffffffu, match);
+            int slot = 0;
+            if (lane == 0 && m) slot = atomicAdd(&sm.list_n, __popc(m));
+            slot = __shfl_sync(0xffffffffu, slot, 0);
+            if (match) sm.list[slot + __popc(m & ((1u << lane) - 1u))] = i;
           }
-          run += cnt[u];
+        }
+      } else if (use_list) {
+        for (int j = tid; j < sm.list_n; j += kSelThreads) {
+          const uint32_t key = keys[sm.list[j]];
+          if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFFu], 1);
+        }
+      } else {
+        for (int i = 1 + tid; i < nb - 1; i += kSelThreads) {
+          const uint32_t key = keys[i];
+          if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFFu], 1);
         }
       }
+      sm.hist[(pass + 1) & 1][tid] = 0;  // the other buffer is free: ready it for the next pass
+      __syncthreads();
     }
+    if (warp == 0) find_digit(hist, kr, sm);
+    if (pass == 0) sm.hist[1][tid] = 0;
     __syncthreads();
     prefix |= (uint32_t)sm.digit << shift;
     mask |= 0xFFu << shift;
     kr -= sm.above;
+    if (pass == 0) use_list = sm.bin <= kListCap;
+    const bool done = sm.bin == kr;  // every key in the bin is taken
+    __syncthreads();                 // all threads have read digit/above/bin
+    if (done) break;
   }
-  const uint32_t T = prefix;
 
   // ---- emit
   const int span = ((nb + kSelWarps - 1) / kSelWarps + 31) & ~31;  // per-warp range, whole batches
@@ -136,11 +181,11 @@ __device__ __forceinline__ void topk_emit(const uint32_t* keys, int nb, int k, i
   for (int base = w0; base < w1; base += 32) {
     const int i = base + lane;
     const bool in = i < w1;
-    const uint32_t key = in ? keys[i] : 0u;
+    const uint32_t key = in ? (keys[i] & mask) : 0u;
     const bool cand = in && i >= 1 && i <= nb - 2;
     n_forced += __popc(__ballot_sync(0xffffffffu, in && !cand));
-    n_gt += __popc(__ballot_sync(0xffffffffu, cand && key > T));
-    n_eq += __popc(__ballot_sync(0xffffffffu, cand && key == T));
+    n_gt += __popc(__ballot_sync(0xffffffffu, cand && key > prefix));
+    n_eq += __popc(__ballot_sync(0xffffffffu, cand && key == prefix));
   }
   if (lane == 0) {
     sm.warp_cnt[0][warp] = n_forced;
@@ -159,11 +204,11 @@ __device__ __forceinline__ void topk_emit(const uint32_t* keys, int nb, int k, i
   for (int base = w0; base < w1; base += 32) {
     const int i = base + lane;
     const bool in = i < w1;
-    const uint32_t key = in ? keys[i] : 0u;
+    const uint32_t key = in ? (keys[i] & mask) : 0u;
     const bool cand = in && i >= 1 && i <= nb - 2;
-    const bool eq = cand && key == T;
+    const bool eq = cand && key == prefix;
     const unsigned eq_mask = __ballot_sync(0xffffffffu, eq);
-    const bool take = (in && !cand) || (cand && key > T) || (eq && eq_rank + __popc(eq_mask & lt) < kr);
+    const bool take = (in && !cand) || (cand && key > prefix) || (eq && eq_rank + __popc(eq_mask & lt) < kr);
     const unsigned take_mask = __ballot_sync(0xffffffffu, take);
     if (take) {
       const int o = pos + __popc(take_mask & lt);
@@ -294,8 +339,27 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(SelectParams p
     if (tid == 0) p.sel_cnt[pair] = nb;
     return;
   }
+  // load the scores as keys, building the first pass's histogram on the way
   const float* sc = p.scores + pair * p.nbcap;
-  for (int i = tid; i < nb; i += kSelThreads) skey[i] = float_key(__ldcg(sc + i));
+  sm.hist[0][tid] = 0;
+  __syncthreads();
+  for (int base = 0; base < nb; base += 4 * kSelThreads) {
+    float v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = base + u * kSelThreads + tid;
+      v[u] = i < nb ? __ldcg(sc + i) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = base + u * kSelThreads + tid;
+      if (i < nb) {
+        const uint32_t key = float_key(v[u]);
+        skey[i] = key;
+        if (i >= 1 && i <= nb - 2) atomicAdd(&sm.hist[0][key >> 24], 1);
+      }
+    }
+  }
   __syncthreads();
   topk_emit(skey, nb, k, sel, sm, p.dev_status);
   if (tid == 0) p.sel_cnt[pair] = k;

@@ -1,0 +1,139 @@
+"""More GPU parity cases: minimal budgets, odd group sizes, multi-block
+appends, very long block lists (the top-k path without a candidate list),
+a multi-step decode loop (append -> select -> attend, checked every step),
+and a whole step captured in a CUDA graph (as the benchmark replays it)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import block_top_sparse_kin_b200 as kin
+import kin_inputs as ki
+import oracle
+from kin_testlib import D, check_pair, gpu_step, make_device_case, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+W = ki.Workload
+
+
+@pytest.mark.parametrize("w", [
+    W("k2_ragged", 3, 2, 6, D, 16, 40, 700, 2, 40, Lcap=704),
+    W("g3", 2, 3, 9, D, 16, 500, 900, 7, 41, Lcap=912),
+    W("g6_bs32", 2, 2, 12, D, 32, 300, 1000, 5, 42, Lcap=1024),
+    W("g7_bs64", 2, 1, 7, D, 64, 129, 1200, 4, 43, Lcap=1280),
+    W("append_100_bs64", 2, 2, 4, D, 64, 0, 0, 5, 44, Lcap=640, n_append=100, lens=(300, 500)),
+    W("append_130_bs128", 1, 2, 8, D, 128, 0, 0, 3, 45, Lcap=1024, n_append=130, lens=(900,)),
+], ids=lambda w: w.name)
+def test_edge_shapes_every_pair(w):
+    dc = make_device_case(w)
+    gr = gpu_step(dc, w.k)
+    assert gr.status == 0
+    means = dc.means.cpu().numpy()
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            check_pair(dc, gr, b, h, w.k, gpu_means=means)
+
+
+def test_long_block_list_with_all_equal_scores():
+    """16384 blocks whose scores all tie: the top-k cannot keep a compact
+    candidate list and must still pick blocks 0..k-2 and the last one."""
+    L = 16384 * 16
+    w = W("long_ties", 1, 2, 4, D, 16, 0, 0, 100, 46, Lcap=L, lens=(L,))
+    dc = make_device_case(w)
+    dc.q.zero_()
+    dc.q_host[:] = 0
+    gr = gpu_step(dc, w.k)
+    assert gr.status == 0
+    for h in range(w.Hkv):
+        assert list(gr.sel[0, h]) == list(range(99)) + [16383]
+        check_pair(dc, gr, 0, h, w.k)
+
+
+def test_long_block_list_random():
+    L = 16384 * 16 - 5
+    w = W("long_rand", 1, 2, 8, D, 16, 0, 0, 300, 47, Lcap=16384 * 16, lens=(L,))
+    dc = make_device_case(w)
+    gr = gpu_step(dc, w.k)
+    assert gr.status == 0
+    for h in range(w.Hkv):
+        check_pair(dc, gr, 0, h, w.k)
+
+
+def test_decode_loop_append_select_attend():
+    """Three decode steps in a row on one stream (each kernel launched with
+    programmatic dependent launch): every step's selection and output match
+    the oracle on the grown cache."""
+    w = W("loop", 2, 2, 8, D, 16, 0, 0, 6, 48, Lcap=400, lens=(200, 95))
+    lens0 = np.array(w.lens, np.int32)
+    steps = 3
+    wf = w.with_(lens=tuple(int(x) + steps for x in lens0), n_append=steps)
+    dc = make_device_case(wf)               # cache holds lens0 rows; the field runs to lens0 + 3
+    kin.kin_block_means_build(dc.dims, dc.k_cache, dc.seq_lens, dc.means)
+    ws = kin.alloc_workspace(dc.dims, w.k)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for s in range(steps):
+        kn = dc.k_new[:, :, s:s + 1].contiguous()
+        vn = dc.v_new[:, :, s:s + 1].contiguous()
+        kin.kin_block_means_update(dc.dims, dc.k_cache, dc.v_cache, dc.means, dc.seq_lens, kn, vn, 1, st)
+        sel = torch.empty((w.B, w.Hkv, w.k), dtype=torch.int32, device="cuda")
+        cnt = torch.empty((w.B, w.Hkv), dtype=torch.int32, device="cuda")
+        out = torch.empty((w.B, w.Hq, D), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
+        kin.kin_block_topk_select(dc.dims, dc.q, dc.means, dc.seq_lens, w.k, sel, cnt, ws, st)
+        kin.kin_sparse_decode_attn(dc.dims, dc.q, dc.k_cache, dc.v_cache, dc.seq_lens, sel, cnt, w.k, 0.0,
+                                   out, lse, ws, st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        lens = lens0 + s + 1
+        assert np.array_equal(dc.seq_lens.cpu().numpy(), lens)
+        sel_h, out_h = sel.cpu().numpy(), out.float().cpu().numpy()
+        for b in range(w.B):
+            L = int(lens[b])
+            for h in range(w.Hkv):
+                K, V = ki.pair_rows(wf, dc.hh, b, h, L)
+                qg = dc.q_host[b, h * w.g:(h + 1) * w.g]
+                ref_sel, c = oracle.select(oracle.block_scores(qg, oracle.block_means(K, L, w.bs)), w.k)
+                assert np.array_equal(sel_h[b, h], ref_sel)
+                o_ref, _ = oracle.attend(qg, K, V, L, w.bs, ref_sel[:c], 1 / math.sqrt(D))
+                err = np.abs(out_h[b, h * w.g:(h + 1) * w.g] - o_ref)
+                assert err.max() <= 2e-2 and err.mean() <= 2e-3
+
+
+def test_step_captured_in_a_cuda_graph_matches_eager():
+    w = W("graph", 4, 2, 8, D, 16, 2000, 4000, 40, 49, Lcap=4096)
+    dc = make_device_case(w)
+    kin.kin_block_means_build(dc.dims, dc.k_cache, dc.seq_lens, dc.means)
+    ws = kin.alloc_workspace(dc.dims, w.k)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def bufs():
+        return (torch.empty((w.B, w.Hkv, w.k), dtype=torch.int32, device="cuda"),
+                torch.empty((w.B, w.Hkv), dtype=torch.int32, device="cuda"),
+                torch.empty((w.B, w.Hq, D), dtype=torch.bfloat16, device="cuda"),
+                torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda"))
+
+    def step(sel, cnt, out, lse):
+        kin.kin_block_topk_select(dc.dims, dc.q, dc.means, dc.seq_lens, w.k, sel, cnt, ws, st)
+        kin.kin_sparse_decode_attn(dc.dims, dc.q, dc.k_cache, dc.v_cache, dc.seq_lens, sel, cnt, w.k, 0.0,
+                                   out, lse, ws, st)
+
+    eager = bufs()
+    step(*eager)
+    torch.cuda.synchronize()
+    graphed = bufs()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            step(*graphed)
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(3):
+        for t in graphed:
+            t.fill_(0)
+        g.replay()
+        torch.cuda.synchronize()
+        for a, b in zip(eager, graphed):
+            assert torch.equal(a, b)
+    assert int(st.item()) == 0
