@@ -27,9 +27,9 @@ LIB = os.path.join(_HERE, "libkin_oracle.so")
 SRC = os.path.join(_HERE, "kin_oracle.c")
 
 
-def build(verbose: bool = False) -> None:
+def build(verbose: bool = False, src: str = SRC, out: str = LIB) -> None:
     cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-fvisibility=hidden",
-           SRC, "-o", LIB, "-lm"]
+           src, "-o", out, "-lm"]
     if verbose:
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)
@@ -43,22 +43,26 @@ def _L():
     if _lib is None:
         if not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
             build()
-        lib = ctypes.CDLL(LIB)
-        vp, i32, dbl = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
-        lib.kin_oracle_block_means.argtypes = [vp, i32, i32, i32, vp]
-        lib.kin_oracle_block_scores.argtypes = [vp, i32, vp, i32, i32, vp]
-        lib.kin_oracle_select.argtypes = [vp, i32, i32, vp]
-        lib.kin_oracle_select.restype = i32
-        lib.kin_oracle_attend_partial.argtypes = [vp, i32, vp, vp, i32, i32, i32, vp, i32, dbl,
-                                                  vp, vp, vp]
-        lib.kin_oracle_merge.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp]
-        lib.kin_oracle_attend.argtypes = [vp, i32, vp, vp, i32, i32, i32, vp, i32, dbl, vp, vp]
-        lib.kin_oracle_means_update.argtypes = [vp, vp, i32, i32, vp, vp, i32, i32, vp]
-        lib.kin_oracle_decode_pairs.argtypes = [i32, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp,
-                                                vp, i32, dbl, vp, i32, vp, vp, vp, vp, vp, i32]
-        lib.kin_oracle_decode_pairs.restype = i32
-        _lib = lib
+        _lib = load(LIB)
     return _lib
+
+
+def load(path: str):
+    """Load an oracle library build (the default one, or a test's variant) and declare its C signatures."""
+    lib = ctypes.CDLL(path)
+    vp, i32, dbl = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
+    lib.kin_oracle_block_means.argtypes = [vp, i32, i32, i32, vp]
+    lib.kin_oracle_block_scores.argtypes = [vp, i32, vp, i32, i32, vp]
+    lib.kin_oracle_select.argtypes = [vp, i32, i32, vp]
+    lib.kin_oracle_select.restype = i32
+    lib.kin_oracle_attend_partial.argtypes = [vp, i32, vp, vp, i32, i32, i32, vp, i32, dbl, vp, vp, vp]
+    lib.kin_oracle_merge.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp]
+    lib.kin_oracle_attend.argtypes = [vp, i32, vp, vp, i32, i32, i32, vp, i32, dbl, vp, vp]
+    lib.kin_oracle_means_update.argtypes = [vp, vp, i32, i32, vp, vp, i32, i32, vp]
+    lib.kin_oracle_decode_pairs.argtypes = [i32, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp,
+                                            vp, i32, dbl, vp, i32, vp, vp, vp, vp, vp, i32]
+    lib.kin_oracle_decode_pairs.restype = i32
+    return lib
 
 
 def _c(a, dtype):
