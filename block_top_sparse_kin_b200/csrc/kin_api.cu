@@ -34,21 +34,9 @@ kin_status check_dims(const kin_dims* d) {
 int nbcap_of(const kin_dims& d) { return (d.max_seq_len + d.block_size - 1) / d.block_size; }
 int pairs_of(const kin_dims& d) { return d.batch * d.num_kv_heads; }
 
-#ifndef KIN_SEL_CHUNK
-#define KIN_SEL_CHUNK 128
-#endif
 #ifndef KIN_ATTN_CHUNK_TOKENS
 #define KIN_ATTN_CHUNK_TOKENS 512
 #endif
-
-// Blocks of means per select CTA: KIN_SEL_CHUNK (128 -> 64 KB of fp32 means),
-// halved down to 32 while the grid would hold fewer than 4 CTAs per SM.
-int select_chunk_blocks(const kin_dims& d) {
-  const int nbcap = nbcap_of(d);
-  int ch = KIN_SEL_CHUNK;
-  while (ch > 32 && (int64_t)pairs_of(d) * ((nbcap + ch - 1) / ch) < 4 * kTargetSMs) ch >>= 1;
-  return ch;
-}
 
 // Kept blocks per attention CTA: KIN_ATTN_CHUNK_TOKENS tokens (512 -> 256 KB
 // of K+V), fewer when the grid would hold fewer than 2 CTAs per SM.
@@ -69,7 +57,7 @@ int attn_max_chunks(const kin_dims& d, int k) {
 }
 
 struct WsLayout {
-  size_t sel_counters, attn_counters, scores, partials, total;
+  size_t attn_counters, scores, partials, total;
 };
 
 WsLayout ws_layout(const kin_dims& d, int k) {
@@ -77,8 +65,6 @@ WsLayout ws_layout(const kin_dims& d, int k) {
   const size_t pairs = (size_t)pairs_of(d);
   const size_t g = (size_t)(d.num_q_heads / d.num_kv_heads);
   size_t off = 0;
-  w.sel_counters = off;
-  off = align_up(off + pairs * sizeof(uint32_t));
   w.attn_counters = off;
   off = align_up(off + pairs * sizeof(uint32_t));
   w.scores = off;
@@ -222,7 +208,6 @@ KIN_EXPORT kin_status kin_block_topk_select(const kin_dims* dims, const void* q,
   p.sel_idx = sel_idx;
   p.sel_cnt = sel_cnt;
   p.scores = reinterpret_cast<float*>(ws + w.scores);
-  p.counters = reinterpret_cast<uint32_t*>(ws + w.sel_counters);
   p.dev_status = dev_status;
   p.B = dims->batch;
   p.Hkv = dims->num_kv_heads;
@@ -232,10 +217,8 @@ KIN_EXPORT kin_status kin_block_topk_select(const kin_dims* dims, const void* q,
   p.Lcap = dims->max_seq_len;
   p.nbcap = nbcap_of(*dims);
   p.k = k_blocks;
-  p.chunk_blocks = select_chunk_blocks(*dims);
   p.score_scale = 1.0f / std::sqrt((float)kHeadDim);
-  const int chunks_per_pair = (p.nbcap + p.chunk_blocks - 1) / p.chunk_blocks;
-  return from_cuda(launch_select(p, chunks_per_pair, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_select(p, static_cast<cudaStream_t>(stream)));
 }
 
 KIN_EXPORT kin_status kin_sparse_decode_attn(const kin_dims* dims, const void* q, const void* k_cache,

@@ -108,6 +108,7 @@ __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kerne
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = p.g;
   pdl_wait();  // the selection comes from the select kernels
+  pdl_trigger_early();
   const ItemInfo it = item_info(p, blockIdx.x);
   const int64_t qh0 = (int64_t)it.b * p.Hq + (int64_t)it.h * g;
   if (it.cnt <= 0) {  // nothing selected (flagged upstream): out = 0, lse = -inf

@@ -39,6 +39,21 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 // results; each kernel signals once its own results are written.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// Where a kernel lets the next one launch.  griddepcontrol.wait returns
+// only once every prerequisite grid has completed and its memory is visible,
+// so the signal's place never changes results, only overlap: with
+// KIN_PDL_EARLY 1 a kernel signals right after its own wait, and the next
+// kernel's CTAs are scheduled onto free SM slots while this grid runs (they
+// sit in their wait); with 0 it signals as its CTAs finish.
+#ifndef KIN_PDL_EARLY
+#define KIN_PDL_EARLY 1
+#endif
+__device__ __forceinline__ void pdl_trigger_early() {
+  if (KIN_PDL_EARLY) pdl_trigger();
+}
+__device__ __forceinline__ void pdl_trigger_late() {
+  if (!KIN_PDL_EARLY) pdl_trigger();
+}
 
 // -------------------------------------------------- PTX: warp-level MMA path
 __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1,
@@ -104,9 +119,8 @@ struct SelectParams {
   int32_t* sel_idx;
   int32_t* sel_cnt;
   float* scores;        // workspace [B*Hkv][nbcap]
-  uint32_t* counters;   // workspace [B*Hkv], zero between calls
   int32_t* dev_status;
-  int B, Hkv, Hq, g, bs, Lcap, nbcap, k, chunk_blocks;
+  int B, Hkv, Hq, g, bs, Lcap, nbcap, k;
   float score_scale;
 };
 
@@ -152,7 +166,7 @@ cudaError_t ensure_smem_limit(const void* kernel, int slot, size_t bytes);
 // Launchers (one per kernel family); return the launch error.
 cudaError_t launch_means_build(const MeansBuildParams& p, cudaStream_t s);
 cudaError_t launch_means_update(const MeansUpdateParams& p, cudaStream_t s);
-cudaError_t launch_select(const SelectParams& p, int chunks_per_pair, cudaStream_t s);
+cudaError_t launch_select(const SelectParams& p, cudaStream_t s);
 cudaError_t launch_attn(const AttnParams& p, int num_items, cudaStream_t s);
 
 }  // namespace kin

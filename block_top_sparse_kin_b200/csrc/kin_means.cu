@@ -26,6 +26,7 @@ __device__ __forceinline__ void add_row4(float (&acc)[4], uint2 raw) {
 // grid (ceil(nbcap / 8), Hkv, B), 256 threads: warp w of CTA x owns block 8x + w.
 __global__ void __launch_bounds__(256) means_build_kernel(MeansBuildParams p) {
   pdl_wait();
+  pdl_trigger_early();
   const int b = blockIdx.z, h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int L = p.seq_lens[b];
@@ -60,6 +61,7 @@ __global__ void __launch_bounds__(256) means_build_kernel(MeansBuildParams p) {
 // it reads and the length it writes back cannot race with another CTA.
 __global__ void __launch_bounds__(256) means_update_kernel(MeansUpdateParams p) {
   pdl_wait();
+  pdl_trigger_early();
   const int b = blockIdx.x;
   const int L0 = p.seq_lens[b];
   const int n = p.n_new;
@@ -111,7 +113,7 @@ __global__ void __launch_bounds__(256) means_update_kernel(MeansUpdateParams p) 
   }
   __syncthreads();
   if (threadIdx.x == 0) p.seq_lens[b] = L1;
-  pdl_trigger();
+  pdl_trigger_late();
 }
 
 cudaError_t launch_means_build(const MeansBuildParams& p, cudaStream_t s) {

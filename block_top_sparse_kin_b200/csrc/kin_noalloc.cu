@@ -88,7 +88,6 @@ KIN_EXPORT kin_status kin_block_topk_select_noalloc(const kin_dims* dims, const 
   p.sel_idx = sel_idx;
   p.sel_cnt = sel_cnt;
   p.scores = scratch;
-  p.counters = nullptr;  // the select kernels keep no completion counters
   p.dev_status = dev_status;
   p.B = dims->batch;
   p.Hkv = dims->num_kv_heads;
@@ -98,7 +97,6 @@ KIN_EXPORT kin_status kin_block_topk_select_noalloc(const kin_dims* dims, const 
   p.Lcap = dims->max_seq_len;
   p.nbcap = nbcap;
   p.k = k_blocks;
-  p.chunk_blocks = 0;  // unused by the select kernels
   p.score_scale = 1.0f / sqrtf((float)kHeadDim);
-  return launch_select(p, 1, static_cast<cudaStream_t>(stream)) == cudaSuccess ? KIN_OK : KIN_ERR_CUDA;
+  return launch_select(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? KIN_OK : KIN_ERR_CUDA;
 }

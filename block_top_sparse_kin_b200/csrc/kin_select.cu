@@ -1,5 +1,5 @@
 // kin_select.cu -- group-summed block scores (HBM scan of the fp32 block
-// means) fused with an exact per-(batch, kv-head) block top-k.
+// means) followed by an exact per-(batch, kv-head) block top-k.
 //
 // Method: block-level top-k sparsity ("Kinetics: Memory-Aware Test-Time
 // Scaling", Architecture Overview; Implementation, BlockTopKAttention: scores
@@ -15,11 +15,15 @@
 //     keeps the next 8 rows in flight while reducing the current 8, with a
 //     butterfly that halves the rows per lane at each level (8 rows in 9
 //     shuffles).  Scores go to workspace, where they stay in L2.
-//  2. select_topk_kernel, one CTA per pair, loads the pair's scores as
-//     order-preserving uint32 keys into shared memory and runs an exact
-//     radix select (see topk_emit): the first block and the block holding
-//     the newest token are always kept, ties go to the lower index, and the
-//     kept indices leave ascending.
+//  2. select_topk_kernel, one CTA per pair (256, 512 or 1024 threads, so
+//     that each thread holds 4 of a 4096-block pair's keys), turns the
+//     pair's scores into order-preserving uint32 keys, finds the exact
+//     threshold (equal-width score bins, then a pairwise rank of the
+//     boundary bin; a radix search over the key bits when the range is
+//     crowded or degenerate) and writes the kept indices.
+// The top-k: the first block and the block holding the newest token are
+// always kept, ties go to the lower index, and the kept indices leave
+// ascending.
 #include "kin_internal.cuh"
 
 namespace kin {
@@ -59,73 +63,96 @@ __device__ __forceinline__ float warp_sum_rows(float (&v)[U], int lane) {
   return r;
 }
 
-constexpr int kListCap = 4096;  // candidates kept in a compact list after the first pass
 
-struct SelectSmem {
-  int hist[2][256];            // double-buffered radix histogram
-  int list[kListCap];          // indices whose key matches the first chosen digit
+// ------------------------------------------------------------------ top-k
+// One CTA of NT threads (256, 512 or 1024, chosen from the block capacity)
+// per pair.  Scores become order-preserving uint32 keys (float_key); the
+// threshold is found by a search over 256 equal-width score bins, with a
+// radix search over the key bits for crowded or degenerate ranges.
+constexpr int kListCap = 4096;  // radix: candidates kept after the first pass
+constexpr int kRankCap = 512;   // equal-width bins: boundary-bin keys ranked pairwise
+constexpr int kMaxKPT = 8;      // keys per thread on the register path
+
+template <int NT>
+struct TopkSmem {
+  static constexpr int NW = NT / 32;
+  int hist[2][256];          // histograms (equal-width bins, or radix digits double-buffered)
+  uint32_t list[kListCap];   // radix: candidate indices; equal-width bins: boundary-bin keys
   int list_n;
-  int warp_cnt[3][kSelWarps];  // per-warp counts: forced, > T, == T
+  int warp_cnt[3][NW];       // per-warp counts: forced, > T, == T
+  uint32_t wmin[NW], wmax[NW];
   int digit, above, bin;
+  uint32_t thresh;
+  int thresh_take;
+  int slot_cnt[kMaxKPT * NW];  // register path: packed (> T, == T) counts per 32-block slot
 };
 
-// Warp 0: the digit (descending) whose bin holds the kr-th largest key of the
-// histogram, the count of keys in higher digits, and the bin's own count.
-__device__ __forceinline__ void find_digit(const int* hist, int kr, SelectSmem& sm) {
+// Inverse of float_key.
+__device__ __forceinline__ float key_float(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// Order-preserving key of the fp32 value whose bits are u.
+__device__ __forceinline__ uint32_t key_of_bits(uint32_t u) {
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+template <int NT>
+__device__ __forceinline__ void zero_hist(TopkSmem<NT>& sm, int which) {
+  if (threadIdx.x < 256) sm.hist[which][threadIdx.x] = 0;
+}
+
+// Every lane of the calling warp gets the bin (counted from the top of a
+// 256-bin histogram) holding the kr-th largest key, the count of keys in
+// higher bins, and the bin's own count.  Needs 1 <= kr <= total count.
+__device__ __forceinline__ void warp_find_bin(const int* hist, int kr, int& bin, int& above, int& cnt) {
   const int lane = threadIdx.x & 31;
-  int cnt[8], tot = 0;
+  int c[8], tot = 0;
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
-    cnt[u] = hist[255 - (lane * 8 + u)];
-    tot += cnt[u];
+    c[u] = hist[255 - (lane * 8 + u)];
+    tot += c[u];
   }
   int inc = tot;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    int t = __shfl_up_sync(0xffffffffu, inc, o);
+    const int t = __shfl_up_sync(0xffffffffu, inc, o);
     if (lane >= o) inc += t;
   }
   const int excl = inc - tot;
-  if (excl < kr && kr <= inc) {
-    int run = excl;
+  const bool mine = excl < kr && kr <= inc;
+  int b = 0, ab = 0, cn = 0, run = excl;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (run + cnt[u] >= kr) {
-        sm.digit = 255 - (lane * 8 + u);
-        sm.above = run;
-        sm.bin = cnt[u];
-        break;
-      }
-      run += cnt[u];
+  for (int u = 0; u < 8; ++u) {
+    if (mine && cn == 0 && run + c[u] >= kr) {
+      b = 255 - (lane * 8 + u);
+      ab = run;
+      cn = c[u];
     }
+    run += c[u];
   }
+  const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+  bin = __shfl_sync(0xffffffffu, b, src);
+  above = __shfl_sync(0xffffffffu, ab, src);
+  cnt = __shfl_sync(0xffffffffu, cn, src);
 }
 
-// Exact top-(k-2) over keys[1..nb-2] plus the forced blocks 0 and nb-1,
-// written ascending to sel[0..k).  keys live in shared memory; hist[0] must
-// already hold the histogram of the candidates' top byte and hist[1] zeros.
-//  * Radix select, up to 4 passes of 8 bits from the top: each pass finds the
-//    digit whose bin holds the kr-th largest remaining key.  After the first
-//    pass the indices matching the chosen prefix go to a compact list, so the
-//    later passes visit only those.  A pass whose bin holds exactly the keys
-//    still needed ends the search: they are all taken.  The result is a
-//    prefix T over the top `mask` bits and kr, the number of keys equal to T
-//    (under the mask) to take.
-//  * Emit with ballots: warp w owns a contiguous index range; one pass counts
-//    its forced / greater / equal keys, one barrier publishes the counts, and
-//    a second pass writes the taken indices in order (keys equal to T under
-//    the mask are taken in index order while their rank is below kr: ties go
-//    to lower indices, and indices leave ascending).
-__device__ __forceinline__ void topk_emit(const uint32_t* keys, int nb, int k, int32_t* sel,
-                                          SelectSmem& sm, int32_t* dev_status) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  uint32_t prefix = 0u, mask = 0u;
-  int kr = k - 2;
+// Radix select over the candidate keys keys[1..nb-2]: on entry kr (> 0) is
+// how many of them to keep, sm.hist[0] holds the histogram of their top
+// bytes and sm.hist[1] is zero.  Up to 4 passes of 8 bits from the top: each
+// pass finds the digit whose bin holds the kr-th largest remaining key.
+// After the first pass the indices matching the chosen prefix go to a
+// compact list, so the later passes visit only those.  A pass whose bin
+// holds exactly the keys still needed ends the search: they are all taken.
+// On return every key above `prefix` under `mask` is kept, and the first kr
+// keys equal to it under the mask (by index).
+template <int NT>
+__device__ __forceinline__ void radix_threshold(const uint32_t* keys, int nb, TopkSmem<NT>& sm,
+                                                uint32_t& prefix, uint32_t& mask, int& kr) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  prefix = 0u;
+  mask = 0u;
   bool use_list = false;
-  if (kr == 0) {  // budget of two: only the forced blocks; no candidate key can pass
-    prefix = 0xFFFFFFFFu;
-    mask = 0xFFFFFFFFu;
-  }
 #pragma unroll 1
   for (int pass = 0; pass < 4 && kr > 0; ++pass) {
     const int shift = 24 - 8 * pass;
@@ -134,7 +161,7 @@ __device__ __forceinline__ void topk_emit(const uint32_t* keys, int nb, int k, i
       if (pass == 1) {  // visit every key once more, keep the matching indices
         if (tid == 0) sm.list_n = 0;
         __syncthreads();
-        for (int base = 0; base < nb; base += kSelThreads) {  // uniform trip count per warp
+        for (int base = 0; base < nb; base += NT) {  // uniform trip count per warp
           const int i = base + tid;
           const uint32_t key = i < nb ? keys[i] : 0u;
           const bool match = i >= 1 && i <= nb - 2 && (key & mask) == prefix;
@@ -148,21 +175,29 @@ __device__ __forceinline__ void topk_emit(const uint32_t* keys, int nb, int k, i
           }
         }
       } else if (use_list) {
-        for (int j = tid; j < sm.list_n; j += kSelThreads) {
+        for (int j = tid; j < sm.list_n; j += NT) {
           const uint32_t key = keys[sm.list[j]];
           if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFFu], 1);
         }
       } else {
-        for (int i = 1 + tid; i < nb - 1; i += kSelThreads) {
+        for (int i = 1 + tid; i < nb - 1; i += NT) {
           const uint32_t key = keys[i];
           if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFFu], 1);
         }
       }
-      sm.hist[(pass + 1) & 1][tid] = 0;  // the other buffer is free: ready it for the next pass
+      zero_hist(sm, (pass + 1) & 1);  // the other buffer is free: ready it for the next pass
       __syncthreads();
     }
-    if (warp == 0) find_digit(hist, kr, sm);
-    if (pass == 0) sm.hist[1][tid] = 0;
+    if (tid < 32) {
+      int d, a, c;
+      warp_find_bin(hist, kr, d, a, c);
+      if (tid == 0) {
+        sm.digit = d;
+        sm.above = a;
+        sm.bin = c;
+      }
+    }
+    if (pass == 0) zero_hist(sm, 1);
     __syncthreads();
     prefix |= (uint32_t)sm.digit << shift;
     mask |= 0xFFu << shift;
@@ -172,9 +207,21 @@ __device__ __forceinline__ void topk_emit(const uint32_t* keys, int nb, int k, i
     __syncthreads();                 // all threads have read digit/above/bin
     if (done) break;
   }
+}
 
-  // ---- emit
-  const int span = ((nb + kSelWarps - 1) / kSelWarps + 31) & ~31;  // per-warp range, whole batches
+// Writes the kept blocks ascending to sel[0..k): the forced blocks 0 and
+// nb-1, every candidate whose key under `mask` is above `prefix`, and the
+// first kr candidates (by index) whose key under the mask equals it.  Warp w
+// owns a contiguous index range; one pass of ballots counts its forced /
+// greater / equal keys, one barrier publishes the counts, and a second pass
+// writes the taken indices in order (so ties go to lower indices).
+template <int NT>
+__device__ __forceinline__ void emit_selection(const uint32_t* keys, int nb, int k, uint32_t prefix,
+                                               uint32_t mask, int kr, int32_t* sel, TopkSmem<NT>& sm,
+                                               int32_t* dev_status) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int span = ((nb + NW - 1) / NW + 31) & ~31;  // per-warp range, whole batches
   const int w0 = min(warp * span, nb), w1 = min(w0 + span, nb);
   const unsigned lt = (1u << lane) - 1u;
   int n_forced = 0, n_gt = 0, n_eq = 0;
@@ -218,7 +265,308 @@ __device__ __forceinline__ void topk_emit(const uint32_t* keys, int nb, int k, i
     eq_rank += __popc(eq_mask);
   }
   // self-check: exactly k blocks were emitted (the last warp ends at k)
-  if (warp == kSelWarps - 1 && lane == 0 && pos != k) set_status(dev_status, KIN_ERR_DEVICE_DATA);
+  if (warp == NW - 1 && lane == 0 && pos != k) set_status(dev_status, KIN_ERR_DEVICE_DATA);
+}
+
+// Ranks the boundary bin's c keys (sm.list[0..c)) pairwise: the need-th
+// largest, with multiplicity, is the threshold T, and need - #{keys > T} of
+// the keys equal to T are kept.  Every thread that finds it writes the same
+// values.  Ends with a barrier.
+template <int NT>
+__device__ __forceinline__ void rank_boundary_bin(int c, int need, TopkSmem<NT>& sm) {
+  for (int j = threadIdx.x; j < c; j += NT) {
+    const uint32_t kj = sm.list[j];
+    int gt = 0, ge = 0;
+    for (int i = 0; i < c; ++i) {
+      const uint32_t ki = sm.list[i];
+      gt += ki > kj;
+      ge += ki >= kj;
+    }
+    if (gt < need && need <= ge) {
+      sm.thresh = kj;
+      sm.thresh_take = need - gt;
+    }
+  }
+  __syncthreads();
+}
+
+// One-pass threshold search for score distributions without extreme
+// outliers, over keys in memory.  The candidates' scores are cut into 256
+// equal-width bins between the smallest (kmin) and largest (kmax) candidate
+// key; the bin of a score, trunc((s - s_min) * (256 / (s_max - s_min))), is a
+// non-decreasing function of s (a correctly rounded subtract and multiply,
+// then truncation), so every key in a higher bin is larger than every key in
+// a lower one.  One histogram finds the bin holding the kr-th largest key;
+// its keys (at most kRankCap) are ranked pairwise to find the exact
+// threshold key and how many keys equal to it to keep.  Returns false
+// (CTA-uniform) when the range is empty or not finite, or the boundary bin
+// is too crowded: the caller then runs the radix search.  Expects
+// sm.hist[0] zero.
+template <int NT>
+__device__ __forceinline__ bool linear_threshold(const uint32_t* keys, int nb, int kr, uint32_t kmin,
+                                                 uint32_t kmax, TopkSmem<NT>& sm, uint32_t& thresh,
+                                                 int& take) {
+  const float lo = key_float(kmin), hi = key_float(kmax);
+  const float range = hi - lo;
+  const float inv = 256.f / range;
+  if (!(isfinite(lo) && isfinite(hi) && range > 0.f && isfinite(range) && isfinite(inv))) return false;
+  const int tid = threadIdx.x, lane = tid & 31;
+  auto bin_of = [&](uint32_t key) { return min((int)((key_float(key) - lo) * inv), 255); };
+  for (int i = 1 + tid; i <= nb - 2; i += NT) atomicAdd(&sm.hist[0][bin_of(keys[i])], 1);
+  if (tid == 0) sm.list_n = 0;
+  __syncthreads();
+  int bstar, above, c;
+  warp_find_bin(sm.hist[0], kr, bstar, above, c);  // every warp, same result
+  if (c > kRankCap) return false;
+  for (int base = 1; base <= nb - 2; base += NT) {  // uniform trip count per warp
+    const int i = base + tid;
+    const bool in = i <= nb - 2;
+    const uint32_t key = in ? keys[i] : 0u;
+    const bool match = in && bin_of(key) == bstar;
+    const unsigned m = __ballot_sync(0xffffffffu, match);
+    int slot = 0;
+    if (lane == 0 && m) slot = atomicAdd(&sm.list_n, __popc(m));
+    slot = __shfl_sync(0xffffffffu, slot, 0);
+    if (match) sm.list[slot + __popc(m & ((1u << lane) - 1u))] = key;
+  }
+  __syncthreads();
+  rank_boundary_bin(c, kr - above, sm);
+  thresh = sm.thresh;
+  take = sm.thresh_take;
+  return true;
+}
+
+// Exact top-(k-2) over keys[1..nb-2] plus the forced blocks 0 and nb-1,
+// written ascending to sel[0..k).  kmin / kmax: the smallest and largest
+// candidate key.  Expects sm.hist[0] and sm.hist[1] zero.
+template <int NT>
+__device__ __forceinline__ void select_from_keys(const uint32_t* keys, int nb, int k, uint32_t kmin,
+                                                 uint32_t kmax, int32_t* sel, TopkSmem<NT>& sm,
+                                                 int32_t* dev_status) {
+  uint32_t prefix = 0xFFFFFFFFu, mask = 0xFFFFFFFFu;  // budget of two: no candidate passes
+  int kr = k - 2;
+  if (kr > 0 && !linear_threshold(keys, nb, kr, kmin, kmax, sm, prefix, kr)) {
+    __syncthreads();  // every warp is done with the bin histogram
+    zero_hist(sm, 0);
+    __syncthreads();
+    for (int i = 1 + threadIdx.x; i <= nb - 2; i += NT) atomicAdd(&sm.hist[0][keys[i] >> 24], 1);
+    __syncthreads();
+    kr = k - 2;
+    radix_threshold(keys, nb, sm, prefix, mask, kr);
+  }
+  emit_selection(keys, nb, k, prefix, mask, kr, sel, sm, dev_status);
+}
+
+// Loads a pair's nb scores (written by the scan kernel: read from L2) as
+// keys into keys[] (shared memory, or the score row itself), returns the
+// smallest and largest candidate key, and zeroes both histograms.
+template <int NT>
+__device__ __forceinline__ void load_keys(const uint32_t* sc, uint32_t* keys, int nb, TopkSmem<NT>& sm,
+                                          uint32_t& kmin, uint32_t& kmax) {
+  constexpr int NW = NT / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int kBatch = 8;
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  for (int base = 0; base < nb; base += kBatch * NT) {
+    uint32_t v[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = base + u * NT + tid;
+      v[u] = i < nb ? __ldcg(sc + i) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = base + u * NT + tid;
+      if (i < nb) {
+        const uint32_t key = key_of_bits(v[u]);
+        keys[i] = key;
+        if (i >= 1 && i <= nb - 2) {
+          lo = min(lo, key);
+          hi = max(hi, key);
+        }
+      }
+    }
+  }
+  lo = __reduce_min_sync(0xffffffffu, lo);
+  hi = __reduce_max_sync(0xffffffffu, hi);
+  if (lane == 0) {
+    sm.wmin[warp] = lo;
+    sm.wmax[warp] = hi;
+  }
+  zero_hist(sm, 0);
+  zero_hist(sm, 1);
+  __syncthreads();
+  kmin = sm.wmin[0];
+  kmax = sm.wmax[0];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) {
+    kmin = min(kmin, sm.wmin[w]);
+    kmax = max(kmax, sm.wmax[w]);
+  }
+}
+
+// The top-k of one pair with any nb, keys in memory: shared memory when
+// nb <= key_cap, else the pair's own score row (which nothing else reads
+// afterwards).
+template <int NT>
+__device__ __forceinline__ void topk_memory(const uint32_t* row, int nb, int k, int32_t* sel, uint32_t* skey,
+                                            int key_cap, TopkSmem<NT>& sm, int32_t* dev_status) {
+  uint32_t* keys = nb <= key_cap ? skey : const_cast<uint32_t*>(row);
+  uint32_t kmin, kmax;
+  load_keys(row, keys, nb, sm, kmin, kmax);
+  select_from_keys(keys, nb, k, kmin, kmax, sel, sm, dev_status);
+}
+
+// The top-k of one pair with nb <= KPT * NT blocks, keys held in registers:
+// thread t owns blocks u * NT + t (u < KPT), so every load and ballot walks
+// the blocks in index order.  Same threshold search as the memory path
+// (equal-width bins; the radix search on a crowded or degenerate range runs
+// from shared memory), and an emit without a second trip through memory:
+// per 32-block slot (u, warp) one ballot pair counts the keys above the
+// threshold (or forced) and the keys equal to it, one barrier publishes the
+// packed counts, every warp scans them, and every thread writes its taken
+// indices at their final positions.
+template <int NT, int KPT>
+__device__ __forceinline__ void topk_regs(const uint32_t* row, int nb, int k, int32_t* sel, uint32_t* skey,
+                                          TopkSmem<NT>& sm, int32_t* dev_status) {
+  constexpr int NW = NT / 32;
+  constexpr int kPerLane = KPT * NW / 32;  // slots per lane in the emit's scan
+  static_assert(KPT <= kMaxKPT && kPerLane >= 1 && NW % kPerLane == 0, "slot layout");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t key[KPT];
+#pragma unroll
+  for (int u = 0; u < KPT; ++u) {
+    const int i = u * NT + tid;
+    key[u] = i < nb ? __ldcg(row + i) : 0u;
+  }
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+#pragma unroll
+  for (int u = 0; u < KPT; ++u) {
+    const int i = u * NT + tid;
+    key[u] = key_of_bits(key[u]);
+    if (i >= 1 && i <= nb - 2) {
+      lo = min(lo, key[u]);
+      hi = max(hi, key[u]);
+    }
+  }
+  lo = __reduce_min_sync(0xffffffffu, lo);
+  hi = __reduce_max_sync(0xffffffffu, hi);
+  if (lane == 0) {
+    sm.wmin[warp] = lo;
+    sm.wmax[warp] = hi;
+  }
+  zero_hist(sm, 0);
+  if (tid == 0) sm.list_n = 0;
+  __syncthreads();
+  uint32_t kmin = sm.wmin[0], kmax = sm.wmax[0];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) {
+    kmin = min(kmin, sm.wmin[w]);
+    kmax = max(kmax, sm.wmax[w]);
+  }
+
+  const int kr = k - 2;
+  uint32_t T = 0xFFFFFFFFu;  // budget of two: no candidate is above T, none equal is taken
+  int take = 0;
+  if (kr > 0) {
+    const float flo = key_float(kmin), fhi = key_float(kmax);
+    const float range = fhi - flo;
+    const float inv = 256.f / range;
+    bool ok = isfinite(flo) && isfinite(fhi) && range > 0.f && isfinite(range) && isfinite(inv);
+    auto bin_of = [&](uint32_t kk) { return min((int)((key_float(kk) - flo) * inv), 255); };
+    int bstar = 0, above = 0, c = 0;
+    if (ok) {
+#pragma unroll
+      for (int u = 0; u < KPT; ++u) {
+        const int i = u * NT + tid;
+        if (i >= 1 && i <= nb - 2) atomicAdd(&sm.hist[0][bin_of(key[u])], 1);
+      }
+      __syncthreads();
+      warp_find_bin(sm.hist[0], kr, bstar, above, c);  // every warp, same result
+      ok = c <= kRankCap;
+    }
+    if (!ok) {  // crowded or degenerate range: radix search from shared memory
+      __syncthreads();  // every warp is done with the bin histogram
+#pragma unroll
+      for (int u = 0; u < KPT; ++u) {
+        const int i = u * NT + tid;
+        if (i < nb) skey[i] = key[u];
+      }
+      zero_hist(sm, 0);
+      zero_hist(sm, 1);
+      __syncthreads();
+      for (int i = 1 + tid; i <= nb - 2; i += NT) atomicAdd(&sm.hist[0][skey[i] >> 24], 1);
+      __syncthreads();
+      uint32_t prefix, mask;
+      int kr2 = kr;
+      radix_threshold(skey, nb, sm, prefix, mask, kr2);
+      emit_selection(skey, nb, k, prefix, mask, kr2, sel, sm, dev_status);
+      return;
+    }
+#pragma unroll
+    for (int u = 0; u < KPT; ++u) {
+      const int i = u * NT + tid;
+      const bool match = i >= 1 && i <= nb - 2 && bin_of(key[u]) == bstar;
+      const unsigned m = __ballot_sync(0xffffffffu, match);
+      int slot = 0;
+      if (lane == 0 && m) slot = atomicAdd(&sm.list_n, __popc(m));
+      slot = __shfl_sync(0xffffffffu, slot, 0);
+      if (match) sm.list[slot + __popc(m & ((1u << lane) - 1u))] = key[u];
+    }
+    __syncthreads();
+    rank_boundary_bin(c, kr - above, sm);
+    T = sm.thresh;
+    take = sm.thresh_take;
+  }
+
+  // ---- emit: slot s = u * NW + warp covers blocks 32 s .. 32 s + 31, in index order
+  const unsigned lt = (1u << lane) - 1u;
+  auto flags = [&](int u, bool& g, bool& e) {
+    const int i = u * NT + tid;
+    const bool cand = i >= 1 && i <= nb - 2;
+    g = (i < nb && !cand) || (cand && key[u] > T);
+    e = cand && key[u] == T;
+  };
+#pragma unroll
+  for (int u = 0; u < KPT; ++u) {
+    bool g, e;
+    flags(u, g, e);
+    const unsigned gb = __ballot_sync(0xffffffffu, g), eb = __ballot_sync(0xffffffffu, e);
+    if (lane == 0) sm.slot_cnt[u * NW + warp] = __popc(gb) | (__popc(eb) << 16);
+  }
+  __syncthreads();
+  // this warp's slots all sit at offset warp % kPerLane within their owner lane
+  const int jw = warp % kPerLane;
+  int tot = 0, mine = 0;
+#pragma unroll
+  for (int j = 0; j < kPerLane; ++j) {
+    const int v = sm.slot_cnt[lane * kPerLane + j];
+    if (j < jw) mine += v;
+    tot += v;
+  }
+  int inc = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += t;
+  }
+  mine += inc - tot;
+  const int all = __shfl_sync(0xffffffffu, inc, 31);
+#pragma unroll
+  for (int u = 0; u < KPT; ++u) {
+    const int base = __shfl_sync(0xffffffffu, mine, (u * NW + warp) / kPerLane);
+    bool g, e;
+    flags(u, g, e);
+    const unsigned gb = __ballot_sync(0xffffffffu, g), eb = __ballot_sync(0xffffffffu, e);
+    const int gt_before = (base & 0xFFFF) + __popc(gb & lt);
+    const int eq_before = (base >> 16) + __popc(eb & lt);
+    if (g || (e && eq_before < take)) {
+      const int pos = gt_before + min(eq_before, take);
+      if (pos < k) sel[pos] = u * NT + tid;  // never write past the pair's row
+    }
+  }
+  // self-check: exactly k blocks were emitted
+  if (tid == 0 && (all & 0xFFFF) + min(all >> 16, take) != k) set_status(dev_status, KIN_ERR_DEVICE_DATA);
 }
 
 // ---- kernel 1: the scan.  Rows are numbered per pair in steps of U
@@ -251,6 +599,7 @@ __device__ __forceinline__ void pair_qsum(const SelectParams& p, int pair, int l
 
 __global__ void __launch_bounds__(kSelThreads, KIN_SEL_CTAS_PER_SM) select_scan_kernel(SelectParams p) {
   pdl_wait();  // means, lengths and q come from earlier work on the stream
+  pdl_trigger_early();
   const int lane = threadIdx.x & 31;
   const int nwarps = gridDim.x * kSelWarps;
   const int gw = blockIdx.x * kSelWarps + (threadIdx.x >> 5);
@@ -259,7 +608,7 @@ __global__ void __launch_bounds__(kSelThreads, KIN_SEL_CTAS_PER_SM) select_scan_
   const int per = (steps + nwarps - 1) / nwarps;
   const int s0 = gw * per, s1 = min(s0 + per, steps);
   if (s0 >= s1) {
-    pdl_trigger();
+    pdl_trigger_late();
     return;
   }
 
@@ -310,23 +659,27 @@ __global__ void __launch_bounds__(kSelThreads, KIN_SEL_CTAS_PER_SM) select_scan_
 #pragma unroll
     for (int u = 0; u < kSelU; ++u) cur[u] = nxt[u];
   }
-  pdl_trigger();
+  pdl_trigger_late();
 }
 
-// ---- kernel 2: one CTA per pair: dense shortcut, bad-length flag, or the
-// exact top-k over the scores the scan left in workspace (L2-resident).
-__global__ void __launch_bounds__(kSelThreads) select_topk_kernel(SelectParams p) {
+
+// ---- kernel 2: one CTA of NT threads per pair: dense shortcut, bad-length
+// flag, or the exact top-k over the scores the scan left in workspace
+// (L2-resident), in registers when nb <= 8 NT.
+template <int NT>
+__global__ void __launch_bounds__(NT, 1024 / NT) select_topk_kernel(SelectParams p) {
   extern __shared__ uint32_t skey[];  // [nbcap]
-  __shared__ SelectSmem sm;
+  __shared__ TopkSmem<NT> sm;
   const int tid = threadIdx.x;
   pdl_wait();  // scores come from the scan kernel
+  pdl_trigger_early();
   const int64_t pair = blockIdx.x;
   const int b = (int)(pair / p.Hkv);
   const int k = p.k;
   int32_t* sel = p.sel_idx + pair * k;
   const int L = __ldg(p.seq_lens + b);
   if (L < 1 || L > p.Lcap) {
-    for (int i = tid; i < k; i += kSelThreads) sel[i] = -1;
+    for (int i = tid; i < k; i += NT) sel[i] = -1;
     if (tid == 0) {
       p.sel_cnt[pair] = 0;
       set_status(p.dev_status, KIN_ERR_DEVICE_DATA);
@@ -335,49 +688,43 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(SelectParams p
   }
   const int nb = (L + p.bs - 1) / p.bs;
   if (nb <= k) {  // the budget covers every block: dense
-    for (int i = tid; i < k; i += kSelThreads) sel[i] = i < nb ? i : -1;
+    for (int i = tid; i < k; i += NT) sel[i] = i < nb ? i : -1;
     if (tid == 0) p.sel_cnt[pair] = nb;
     return;
   }
-  // load the scores as keys, building the first pass's histogram on the way
-  const float* sc = p.scores + pair * p.nbcap;
-  sm.hist[0][tid] = 0;
-  __syncthreads();
-  for (int base = 0; base < nb; base += 4 * kSelThreads) {
-    float v[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = base + u * kSelThreads + tid;
-      v[u] = i < nb ? __ldcg(sc + i) : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = base + u * kSelThreads + tid;
-      if (i < nb) {
-        const uint32_t key = float_key(v[u]);
-        skey[i] = key;
-        if (i >= 1 && i <= nb - 2) atomicAdd(&sm.hist[0][key >> 24], 1);
-      }
-    }
-  }
-  __syncthreads();
-  topk_emit(skey, nb, k, sel, sm, p.dev_status);
+  const uint32_t* row = reinterpret_cast<const uint32_t*>(p.scores + pair * p.nbcap);
+  if (nb <= 4 * NT) topk_regs<NT, 4>(row, nb, k, sel, skey, sm, p.dev_status);
+  else if (nb <= 8 * NT) topk_regs<NT, 8>(row, nb, k, sel, skey, sm, p.dev_status);
+  else topk_memory<NT>(row, nb, k, sel, skey, p.nbcap, sm, p.dev_status);
   if (tid == 0) p.sel_cnt[pair] = k;
 }
 
-cudaError_t launch_select(const SelectParams& p, int /*chunks_per_pair*/, cudaStream_t s) {
+// Threads per top-k CTA: 4 keys per thread up to 4096 blocks.
+int topk_threads(int nbcap) { return nbcap <= 1024 ? 256 : nbcap <= 2048 ? 512 : 1024; }
+
+template <int NT>
+cudaError_t launch_topk(const SelectParams& p, cudaStream_t s) {
   const size_t smem = (size_t)p.nbcap * sizeof(uint32_t);
-  if (smem > 48 * 1024) {
-    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(select_topk_kernel), 0, smem);
+  if (smem > 16 * 1024) {
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(select_topk_kernel<NT>),
+                                      NT == 256 ? 0 : NT == 512 ? 2 : 3, smem);
     if (e != cudaSuccess) return e;
   }
+  return launch_pdl(select_topk_kernel<NT>, dim3(p.B * p.Hkv), dim3(NT), smem, s, p);
+}
+
+cudaError_t launch_select(const SelectParams& p, cudaStream_t s) {
   const int64_t rows = (int64_t)p.B * p.Hkv * p.nbcap;
   const int64_t want = (rows + kSelWarps * kSelU * 4 - 1) / (kSelWarps * kSelU * 4);  // >= 4 steps per warp
   const int64_t resident = (int64_t)device_sm_count() * KIN_SEL_CTAS_PER_SM;
   const int grid = (int)(want < resident ? (want > 0 ? want : 1) : resident);
   cudaError_t e = launch_pdl(select_scan_kernel, dim3(grid), dim3(kSelThreads), 0, s, p);
   if (e != cudaSuccess) return e;
-  return launch_pdl(select_topk_kernel, dim3(p.B * p.Hkv), dim3(kSelThreads), smem, s, p);
+  switch (topk_threads(p.nbcap)) {
+    case 256: return launch_topk<256>(p, s);
+    case 512: return launch_topk<512>(p, s);
+    default: return launch_topk<1024>(p, s);
+  }
 }
 
 }  // namespace kin
