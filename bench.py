@@ -290,58 +290,61 @@ def gpu_arm(args):
     if int(st["status"].item()) != 0:
         raise RuntimeError(f"device status {int(st['status'].item())} after warm-up")
 
-    # Each timed step is one CUDA graph (captured once, as a decode loop
-    # would run it) bracketed by two timing events, so the step's kernels
-    # chain back to back.  A second set of graphs, replayed after the timed
-    # loop, carries an event between every kernel for the per-kernel times
-    # the roofline uses.  The L2 flush runs eagerly before every replay,
-    # outside the events.
+    # A step is one CUDA graph, captured once and replayed every step as a
+    # decode loop would, with two timing events inside it around the step's
+    # kernels, so the kernels chain back to back.  A second graph carries an
+    # event between every kernel for the per-kernel times the roofline uses.
+    # Both graphs are replayed during warm-up, so no timed step pays a
+    # graph's first launch.  The L2 flush runs eagerly before every replay,
+    # outside the events, and each replay's events are read back (a host
+    # synchronize, also outside the events) before the next replay.
     def ext_events(n):
         return [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n)]
 
-    step_ev = [ext_events(2) for _ in range(args.steps)]
-    kern_ev = [ext_events(n_ev) for _ in range(args.steps)]
+    step_ev = ext_events(2)
+    kern_ev = ext_events(n_ev)
     cap = torch.cuda.Stream()
     cap.wait_stream(torch.cuda.current_stream())
-    graphs, diag_graphs = [], []
     with torch.cuda.stream(cap):
-        for s in range(args.steps):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=cap):
-                reset_state(st)
-                step_ev[s][0].record()
-                run_step(st)
-                step_ev[s][1].record()
-            graphs.append(g)
-            g2 = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g2, stream=cap):
-                reset_state(st)
-                run_step(st, kern_ev[s])
-            diag_graphs.append(g2)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cap):
+            reset_state(st)
+            step_ev[0].record()
+            run_step(st)
+            step_ev[1].record()
+        diag_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(diag_graph, stream=cap):
+            reset_state(st)
+            run_step(st, kern_ev)
     torch.cuda.current_stream().wait_stream(cap)
-    for g in graphs[: min(len(graphs), args.warmup)] + diag_graphs[: min(len(graphs), args.warmup)]:
-        g.replay()  # warm the graphs themselves
+    for _ in range(args.warmup):
+        flush_l2(0)
+        graph.replay()
+        diag_graph.replay()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    per_step = []
     with ClockSampler(local) as clk:
         wall0 = time.perf_counter()
         for s in range(args.steps):
             flush_l2(s)                    # outside the events
-            graphs[s].replay()
-        torch.cuda.synchronize()
+            graph.replay()
+            torch.cuda.synchronize()
+            per_step.append(step_ev[0].elapsed_time(step_ev[1]))
         wall = time.perf_counter() - wall0
     if world > 1:
         dist.barrier()
+    sel_ms, attn_ms, upd_ms = [], [], []
     for s in range(args.steps):            # per-kernel timing pass (not in `value`)
         flush_l2(s)
-        diag_graphs[s].replay()
-    torch.cuda.synchronize()
-    per_step = [ev[0].elapsed_time(ev[1]) for ev in step_ev]
-    sel_ms = [ev[-3].elapsed_time(ev[-2]) for ev in kern_ev]
-    attn_ms = [ev[-2].elapsed_time(ev[-1]) for ev in kern_ev]
-    upd_ms = [ev[0].elapsed_time(ev[1]) for ev in kern_ev] if w.n_append else []
+        diag_graph.replay()
+        torch.cuda.synchronize()
+        sel_ms.append(kern_ev[-3].elapsed_time(kern_ev[-2]))
+        attn_ms.append(kern_ev[-2].elapsed_time(kern_ev[-1]))
+        if w.n_append:
+            upd_ms.append(kern_ev[0].elapsed_time(kern_ev[1]))
     total_ms = reduce_max(sum(per_step), "cuda")
     ms_per_step = total_ms / args.steps
     qh_per_step = w.B * w.Hq

@@ -70,7 +70,7 @@ WsLayout ws_layout(const kin_dims& d, int k) {
   w.scores = off;
   off = align_up(off + pairs * (size_t)nbcap_of(d) * sizeof(float));
   w.partials = off;
-  off = align_up(off + pairs * (size_t)attn_max_chunks(d, k) * g * (kHeadDim + 2) * sizeof(float));
+  off = align_up(off + pairs * (size_t)attn_max_chunks(d, k) * g * kPartStride * sizeof(float));
   w.total = off;
   return w;
 }

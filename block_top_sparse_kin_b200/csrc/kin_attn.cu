@@ -28,7 +28,8 @@
 //  * The warps merge in shared memory.  A single-chunk pair writes bf16 out
 //    and fp32 lse directly; otherwise the chunk's partial (o, m, l) goes to
 //    workspace and the pair's last chunk to finish (atomic counter, no
-//    spinning) merges all of them with batched, independent loads.
+//    spinning) merges all of them, staged in shared memory with one round
+//    of independent 16-byte loads.
 #include "kin_internal.cuh"
 
 namespace kin {
@@ -49,7 +50,6 @@ constexpr int kStages = KIN_ATTN_STAGES;
 constexpr int kHalfBox = 16 * 64 * 2;       // bytes of a 16-row x 64-column bf16 half tile
 constexpr int kStageBytes = 4 * kHalfBox;   // K0 K1 V0 V1
 constexpr int kRowPad = kHeadDim + 4;       // combine rows padded against bank conflicts
-constexpr int kMergeBatch = 32;             // chunks whose (m, l) are staged per merge round
 constexpr size_t kPipeBytes = (size_t)kAttnWarps * kStages * kStageBytes;
 constexpr size_t kCombBytes = (size_t)kAttnWarps * kMaxGroup * kRowPad * sizeof(float);
 static_assert(kAttnThreads >= kHeadDim, "one thread per output dim in the merge");
@@ -102,7 +102,6 @@ __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kerne
   extern __shared__ uint8_t smem_raw[];
   __shared__ float s_m[kAttnWarps][kMaxGroup], s_l[kAttnWarps][kMaxGroup];
   __shared__ int s_last;
-  __shared__ float s_pm[kMergeBatch * kMaxGroup], s_pl[kMergeBatch * kMaxGroup];  // merge staging
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -305,7 +304,7 @@ __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kerne
   }
 
   // ---- write this chunk's partial; the pair's last chunk merges all of them
-  float* part = p.partials + (it.pair * p.max_chunks + it.c) * (int64_t)g * (kHeadDim + 2);
+  float* part = p.partials + (it.pair * p.max_chunks + it.c) * (int64_t)g * kPartStride;
   for (int j = 0; j < gd; ++j) {
     float M = kNegInf;
 #pragma unroll
@@ -319,10 +318,10 @@ __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kerne
         den += e * s_l[w][j];
       }
     }
-    part[j * (kHeadDim + 2) + d] = num;
+    part[j * kPartStride + d] = num;
     if (d == 0) {
-      part[j * (kHeadDim + 2) + kHeadDim] = M;
-      part[j * (kHeadDim + 2) + kHeadDim + 1] = den;
+      part[j * kPartStride + kHeadDim] = M;
+      part[j * kPartStride + kHeadDim + 1] = den;
     }
   }
   __threadfence();
@@ -331,13 +330,18 @@ __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kerne
   __syncthreads();
   if (!s_last) return;
 
-  // Merge all chunks of the pair: the (m, l) of up to kMergeBatch chunks are
-  // staged in shared memory with one round of independent loads, then every
-  // thread folds its output dim over the batch with independent, unrolled
-  // loads, so a merge costs a few L2 round trips rather than one per chunk.
+  // Merge all chunks of the pair: their partial records are staged in shared
+  // memory (the idle ring and combine area: every thread passed the two
+  // barriers above after its last read of the combine rows) with one round of independent 16-byte loads per
+  // batch of chunks that fits, then every thread folds its output dim over
+  // the batch from shared memory, so a merge costs about one L2 round trip.
   __threadfence();
   if (tid == 0) p.counters[it.pair] = 0u;  // ready for the next call
-  const float* pp = p.partials + it.pair * p.max_chunks * (int64_t)g * (kHeadDim + 2);
+  const int rec = g * kPartStride;                        // floats per chunk
+  const int per_batch = (int)(kPipeBytes / (sizeof(float) * rec));  // chunks staged at once
+  const float4* src4 = reinterpret_cast<const float4*>(p.partials + it.pair * p.max_chunks * (int64_t)rec);
+  float* stage = reinterpret_cast<float*>(smem);
+  float4* stage4 = reinterpret_cast<float4*>(smem);
   float Mr[kMaxGroup], num[kMaxGroup], den[kMaxGroup];
 #pragma unroll
   for (int j = 0; j < kMaxGroup; ++j) {
@@ -345,12 +349,23 @@ __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kerne
     num[j] = 0.f;
     den[j] = 0.f;
   }
-  for (int cb = 0; cb < it.nchunks; cb += kMergeBatch) {
-    const int nbat = min(kMergeBatch, it.nchunks - cb);
-    for (int i = tid; i < nbat * g; i += kAttnThreads) {
-      const float* q = pp + ((int64_t)cb * g + i) * (kHeadDim + 2);
-      s_pm[i] = __ldcg(q + kHeadDim);
-      s_pl[i] = __ldcg(q + kHeadDim + 1);
+  for (int cb = 0; cb < it.nchunks; cb += per_batch) {
+    const int nbat = min(per_batch, it.nchunks - cb);
+    const int n4 = nbat * rec / 4;
+    const float4* s4 = src4 + (int64_t)cb * (rec / 4);
+    constexpr int kLoads = 16;  // float4 loads in flight per thread
+    for (int base = 0; base < n4; base += kLoads * kAttnThreads) {
+      float4 v[kLoads];
+#pragma unroll
+      for (int u = 0; u < kLoads; ++u) {
+        const int i = base + u * kAttnThreads + tid;
+        if (i < n4) v[u] = __ldcg(s4 + i);
+      }
+#pragma unroll
+      for (int u = 0; u < kLoads; ++u) {
+        const int i = base + u * kAttnThreads + tid;
+        if (i < n4) stage4[i] = v[u];
+      }
     }
     __syncthreads();
     if (d < kHeadDim) {
@@ -358,17 +373,17 @@ __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kerne
       for (int j = 0; j < kMaxGroup; ++j) {
         if (j < g) {
           float Mb = kNegInf;
-          for (int c = 0; c < nbat; ++c) Mb = fmaxf(Mb, s_pm[c * g + j]);
+          for (int c = 0; c < nbat; ++c) Mb = fmaxf(Mb, stage[(c * g + j) * kPartStride + kHeadDim]);
           const float Mn = fmaxf(Mr[j], Mb);
           if (Mn != kNegInf) {
             const float a = exp2f(Mr[j] - Mn);
             float nn = num[j] * a, dd = den[j] * a;
-#pragma unroll 8
             for (int c = 0; c < nbat; ++c) {
-              const float mc = s_pm[c * g + j];
+              const float* r = stage + (c * g + j) * kPartStride;
+              const float mc = r[kHeadDim];
               const float e = mc == kNegInf ? 0.f : exp2f(mc - Mn);
-              nn += e * __ldcg(pp + ((int64_t)(cb + c) * g + j) * (kHeadDim + 2) + d);
-              dd += e * s_pl[c * g + j];
+              nn += e * r[d];
+              dd += e * r[kHeadDim + 1];
             }
             num[j] = nn;
             den[j] = dd;
@@ -377,7 +392,7 @@ __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kerne
         }
       }
     }
-    __syncthreads();
+    __syncthreads();  // the next batch overwrites the staging area
   }
   if (d < kHeadDim) {
 #pragma unroll

@@ -15,6 +15,9 @@ constexpr int kMaxGroup = 8;
 constexpr int kMaxBlocksPerSeq = 32768;
 constexpr int kTileTokens = 16;  // tokens per attention tile (one m16 MMA row block)
 constexpr int kMaxItemTiles = 64;  // attention tiles per work item (chunk of kept blocks)
+// floats per (chunk, query head) attention partial: o[D], max, sum, 2 pad
+// (a multiple of 4, so every record starts on a 16-byte boundary)
+constexpr int kPartStride = kHeadDim + 4;
 
 // ----------------------------------------------------------------- status
 __device__ __forceinline__ void set_status(int32_t* st, int32_t code) {
@@ -133,7 +136,7 @@ struct AttnParams {
   const int32_t* sel_cnt;
   __nv_bfloat16* out;
   float* lse;
-  float* partials;      // workspace [B*Hkv][max_chunks][g][D + 2]
+  float* partials;      // workspace [B*Hkv][max_chunks][g][kPartStride]
   uint32_t* counters;   // workspace [B*Hkv], zero between calls
   int32_t* dev_status;
   int B, Hkv, Hq, g, bs, Lcap, k, chunk_blocks, max_chunks;
