@@ -53,6 +53,8 @@ constexpr int kRowPad = kHeadDim + 4;       // combine rows padded against bank 
 constexpr size_t kPipeBytes = (size_t)kAttnWarps * kStages * kStageBytes;
 constexpr size_t kCombBytes = (size_t)kAttnWarps * kMaxGroup * kRowPad * sizeof(float);
 static_assert(kAttnThreads >= kHeadDim, "one thread per output dim in the merge");
+// (chunk, head) records staged per merge batch: kPipeBytes / (4 kPartStride)
+constexpr int kMaxMergeWeights = (int)(kPipeBytes / (sizeof(float) * kPartStride));
 static_assert(kMaxItemTiles / kAttnWarps <= 32, "a warp's tiles of one item fit one per lane");
 #define kNegInf (-__int_as_float(0x7f800000))
 
@@ -102,6 +104,10 @@ __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kerne
   extern __shared__ uint8_t smem_raw[];
   __shared__ float s_m[kAttnWarps][kMaxGroup], s_l[kAttnWarps][kMaxGroup];
   __shared__ int s_last;
+  // merge: per head running max, sum and rescale; per (chunk, head) weight
+  __shared__ float s_mr[kMaxGroup], s_den[kMaxGroup], s_a[kMaxGroup], s_w[kMaxMergeWeights];
+  // warp combine: per (warp, head) weight, per head maximum and sum
+  __shared__ float s_ww[kAttnWarps][kMaxGroup], s_cm[kMaxGroup], s_cden[kMaxGroup];
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -281,24 +287,37 @@ __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kerne
   }
   __syncthreads();
 
+  // per head j (thread j < g): the maximum over the warps, each warp's
+  // weight and the weighted sum; then every thread combines its output dim
+  if (tid < g) {
+    const int j = tid;
+    float M = kNegInf;
+#pragma unroll
+    for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, s_m[w][j]);
+    float den = 0.f;
+#pragma unroll
+    for (int w = 0; w < kAttnWarps; ++w) {
+      const float e = M == kNegInf ? 0.f : exp2f(s_m[w][j] - M);
+      s_ww[w][j] = e;
+      den += e * s_l[w][j];
+    }
+    s_cm[j] = M;
+    s_cden[j] = den;
+  }
+  __syncthreads();
   const int d = tid;  // one output dim per thread (threads >= kHeadDim idle)
   const int gd = d < kHeadDim ? g : 0;
+  auto combined = [&](int j) {
+    float num = 0.f;
+#pragma unroll
+    for (int w = 0; w < kAttnWarps; ++w) num += s_ww[w][j] * comb[(w * kMaxGroup + j) * kRowPad + d];
+    return num;
+  };
   if (it.nchunks == 1) {
     for (int j = 0; j < gd; ++j) {
-      float M = kNegInf;
-#pragma unroll
-      for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, s_m[w][j]);
-      float num = 0.f, den = 0.f;
-      if (M != kNegInf) {
-#pragma unroll
-        for (int w = 0; w < kAttnWarps; ++w) {
-          const float e = exp2f(s_m[w][j] - M);
-          num += e * comb[(w * kMaxGroup + j) * kRowPad + d];
-          den += e * s_l[w][j];
-        }
-      }
+      const float num = combined(j), den = s_cden[j];
       p.out[(qh0 + j) * kHeadDim + d] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
-      if (p.lse && d == 0) p.lse[qh0 + j] = den > 0.f ? (M + log2f(den)) * 0.6931471805599453f : kNegInf;
+      if (p.lse && d == 0) p.lse[qh0 + j] = den > 0.f ? (s_cm[j] + log2f(den)) * 0.6931471805599453f : kNegInf;
     }
     return;
   }
@@ -306,22 +325,10 @@ __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kerne
   // ---- write this chunk's partial; the pair's last chunk merges all of them
   float* part = p.partials + (it.pair * p.max_chunks + it.c) * (int64_t)g * kPartStride;
   for (int j = 0; j < gd; ++j) {
-    float M = kNegInf;
-#pragma unroll
-    for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, s_m[w][j]);
-    float num = 0.f, den = 0.f;
-    if (M != kNegInf) {
-#pragma unroll
-      for (int w = 0; w < kAttnWarps; ++w) {
-        const float e = exp2f(s_m[w][j] - M);
-        num += e * comb[(w * kMaxGroup + j) * kRowPad + d];
-        den += e * s_l[w][j];
-      }
-    }
-    part[j * kPartStride + d] = num;
+    part[j * kPartStride + d] = combined(j);
     if (d == 0) {
-      part[j * kPartStride + kHeadDim] = M;
-      part[j * kPartStride + kHeadDim + 1] = den;
+      part[j * kPartStride + kHeadDim] = s_cm[j];
+      part[j * kPartStride + kHeadDim + 1] = s_cden[j];
     }
   }
   __threadfence();
@@ -332,75 +339,73 @@ __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kerne
 
   // Merge all chunks of the pair: their partial records are staged in shared
   // memory (the idle ring and combine area: every thread passed the two
-  // barriers above after its last read of the combine rows) with one round of independent 16-byte loads per
-  // batch of chunks that fits, then every thread folds its output dim over
-  // the batch from shared memory, so a merge costs about one L2 round trip.
+  // barriers above after its last read of the combine rows) with one round
+  // of 16-byte cp.async copies per batch of chunks that fits.  Threads j < g
+  // then fold head j's maxima and sums and leave one weight per (chunk,
+  // head) in shared memory, and every thread folds its output dim with
+  // independent, unrolled reads, so a merge costs about one L2 round trip.
   __threadfence();
   if (tid == 0) p.counters[it.pair] = 0u;  // ready for the next call
-  const int rec = g * kPartStride;                        // floats per chunk
+  const int rec = g * kPartStride;                                  // floats per chunk
   const int per_batch = (int)(kPipeBytes / (sizeof(float) * rec));  // chunks staged at once
   const float4* src4 = reinterpret_cast<const float4*>(p.partials + it.pair * p.max_chunks * (int64_t)rec);
-  float* stage = reinterpret_cast<float*>(smem);
-  float4* stage4 = reinterpret_cast<float4*>(smem);
-  float Mr[kMaxGroup], num[kMaxGroup], den[kMaxGroup];
+  const float* stage = reinterpret_cast<const float*>(smem);
+  const uint32_t stage_s = smem_u32(smem);
+  float num[kMaxGroup];
 #pragma unroll
-  for (int j = 0; j < kMaxGroup; ++j) {
-    Mr[j] = kNegInf;
-    num[j] = 0.f;
-    den[j] = 0.f;
+  for (int j = 0; j < kMaxGroup; ++j) num[j] = 0.f;
+  if (tid < g) {
+    s_mr[tid] = kNegInf;
+    s_den[tid] = 0.f;
   }
   for (int cb = 0; cb < it.nchunks; cb += per_batch) {
     const int nbat = min(per_batch, it.nchunks - cb);
     const int n4 = nbat * rec / 4;
     const float4* s4 = src4 + (int64_t)cb * (rec / 4);
-    constexpr int kLoads = 16;  // float4 loads in flight per thread
-    for (int base = 0; base < n4; base += kLoads * kAttnThreads) {
-      float4 v[kLoads];
-#pragma unroll
-      for (int u = 0; u < kLoads; ++u) {
-        const int i = base + u * kAttnThreads + tid;
-        if (i < n4) v[u] = __ldcg(s4 + i);
+    for (int i = tid; i < n4; i += kAttnThreads) cp_async16(stage_s + 16u * (uint32_t)i, s4 + i, 16u);
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    if (tid < g) {  // head j: batch maximum, rescale of the running sums, chunk weights
+      const int j = tid;
+      float Mb = kNegInf;
+      for (int c = 0; c < nbat; ++c) Mb = fmaxf(Mb, stage[(c * g + j) * kPartStride + kHeadDim]);
+      const float Mr = s_mr[j];
+      const float Mn = fmaxf(Mr, Mb);
+      const float a = Mn == kNegInf ? 0.f : exp2f(Mr - Mn);
+      float dd = s_den[j] * a;
+      for (int c = 0; c < nbat; ++c) {
+        const float* r = stage + (c * g + j) * kPartStride;
+        const float e = (Mn == kNegInf || r[kHeadDim] == kNegInf) ? 0.f : exp2f(r[kHeadDim] - Mn);
+        s_w[c * g + j] = e;
+        dd += e * r[kHeadDim + 1];
       }
-#pragma unroll
-      for (int u = 0; u < kLoads; ++u) {
-        const int i = base + u * kAttnThreads + tid;
-        if (i < n4) stage4[i] = v[u];
-      }
+      s_a[j] = a;
+      s_mr[j] = Mn;
+      s_den[j] = dd;
     }
     __syncthreads();
     if (d < kHeadDim) {
 #pragma unroll
       for (int j = 0; j < kMaxGroup; ++j) {
         if (j < g) {
-          float Mb = kNegInf;
-          for (int c = 0; c < nbat; ++c) Mb = fmaxf(Mb, stage[(c * g + j) * kPartStride + kHeadDim]);
-          const float Mn = fmaxf(Mr[j], Mb);
-          if (Mn != kNegInf) {
-            const float a = exp2f(Mr[j] - Mn);
-            float nn = num[j] * a, dd = den[j] * a;
-            for (int c = 0; c < nbat; ++c) {
-              const float* r = stage + (c * g + j) * kPartStride;
-              const float mc = r[kHeadDim];
-              const float e = mc == kNegInf ? 0.f : exp2f(mc - Mn);
-              nn += e * r[d];
-              dd += e * r[kHeadDim + 1];
-            }
-            num[j] = nn;
-            den[j] = dd;
-            Mr[j] = Mn;
-          }
+          float nn = num[j] * s_a[j];
+#pragma unroll 8
+          for (int c = 0; c < nbat; ++c) nn += s_w[c * g + j] * stage[(c * g + j) * kPartStride + d];
+          num[j] = nn;
         }
       }
     }
-    __syncthreads();  // the next batch overwrites the staging area
+    __syncthreads();  // the next batch overwrites the staging area and the weights
   }
   if (d < kHeadDim) {
 #pragma unroll
     for (int j = 0; j < kMaxGroup; ++j) {
       if (j < g) {
-        p.out[(qh0 + j) * kHeadDim + d] = __float2bfloat16_rn(den[j] > 0.f ? num[j] / den[j] : 0.f);
+        const float den = s_den[j];
+        p.out[(qh0 + j) * kHeadDim + d] = __float2bfloat16_rn(den > 0.f ? num[j] / den : 0.f);
         if (p.lse && d == 0)
-          p.lse[qh0 + j] = den[j] > 0.f ? (Mr[j] + log2f(den[j])) * 0.6931471805599453f : kNegInf;
+          p.lse[qh0 + j] = den > 0.f ? (s_mr[j] + log2f(den)) * 0.6931471805599453f : kNegInf;
       }
     }
   }
