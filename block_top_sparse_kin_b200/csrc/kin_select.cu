@@ -72,11 +72,15 @@ __device__ __forceinline__ float warp_sum_rows(float (&v)[U], int lane) {
 constexpr int kListCap = 4096;  // radix: candidates kept after the first pass
 constexpr int kRankCap = 512;   // equal-width bins: boundary-bin keys ranked pairwise
 constexpr int kMaxKPT = 8;      // keys per thread on the register path
+// 256-bin histograms padded by one word per 8 bins, so a lane reading 8
+// consecutive bins (stride 9 words between lanes) hits 32 distinct banks
+constexpr int kHistWords = 256 + 32;
+__device__ __forceinline__ int hidx(int bin) { return bin + (bin >> 3); }
 
 template <int NT>
 struct TopkSmem {
   static constexpr int NW = NT / 32;
-  int hist[2][256];          // histograms (equal-width bins, or radix digits double-buffered)
+  int hist[2][kHistWords];   // histograms (equal-width bins, or radix digits double-buffered), hidx-padded
   uint32_t list[kListCap];   // radix: candidate indices; equal-width bins: boundary-bin keys
   int list_n;
   int warp_cnt[3][NW];       // per-warp counts: forced, > T, == T
@@ -99,7 +103,7 @@ __device__ __forceinline__ uint32_t key_of_bits(uint32_t u) {
 
 template <int NT>
 __device__ __forceinline__ void zero_hist(TopkSmem<NT>& sm, int which) {
-  if (threadIdx.x < 256) sm.hist[which][threadIdx.x] = 0;
+  for (int i = threadIdx.x; i < kHistWords; i += NT) sm.hist[which][i] = 0;
 }
 
 // Every lane of the calling warp gets the bin (counted from the top of a
@@ -110,7 +114,7 @@ __device__ __forceinline__ void warp_find_bin(const int* hist, int kr, int& bin,
   int c[8], tot = 0;
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
-    c[u] = hist[255 - (lane * 8 + u)];
+    c[u] = hist[hidx(255 - (lane * 8 + u))];
     tot += c[u];
   }
   int inc = tot;
@@ -165,7 +169,7 @@ __device__ __forceinline__ void radix_threshold(const uint32_t* keys, int nb, To
           const int i = base + tid;
           const uint32_t key = i < nb ? keys[i] : 0u;
           const bool match = i >= 1 && i <= nb - 2 && (key & mask) == prefix;
-          if (match) atomicAdd(&hist[(key >> shift) & 0xFFu], 1);
+          if (match) atomicAdd(&hist[hidx((key >> shift) & 0xFFu)], 1);
           if (use_list) {  // one list reservation per warp, lanes take slots in order
             const unsigned m = __ballot_sync(0xffffffffu, match);
             int slot = 0;
@@ -177,12 +181,12 @@ __device__ __forceinline__ void radix_threshold(const uint32_t* keys, int nb, To
       } else if (use_list) {
         for (int j = tid; j < sm.list_n; j += NT) {
           const uint32_t key = keys[sm.list[j]];
-          if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFFu], 1);
+          if ((key & mask) == prefix) atomicAdd(&hist[hidx((key >> shift) & 0xFFu)], 1);
         }
       } else {
         for (int i = 1 + tid; i < nb - 1; i += NT) {
           const uint32_t key = keys[i];
-          if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFFu], 1);
+          if ((key & mask) == prefix) atomicAdd(&hist[hidx((key >> shift) & 0xFFu)], 1);
         }
       }
       zero_hist(sm, (pass + 1) & 1);  // the other buffer is free: ready it for the next pass
@@ -312,7 +316,7 @@ __device__ __forceinline__ bool linear_threshold(const uint32_t* keys, int nb, i
   if (!(isfinite(lo) && isfinite(hi) && range > 0.f && isfinite(range) && isfinite(inv))) return false;
   const int tid = threadIdx.x, lane = tid & 31;
   auto bin_of = [&](uint32_t key) { return min((int)((key_float(key) - lo) * inv), 255); };
-  for (int i = 1 + tid; i <= nb - 2; i += NT) atomicAdd(&sm.hist[0][bin_of(keys[i])], 1);
+  for (int i = 1 + tid; i <= nb - 2; i += NT) atomicAdd(&sm.hist[0][hidx(bin_of(keys[i]))], 1);
   if (tid == 0) sm.list_n = 0;
   __syncthreads();
   int bstar, above, c;
@@ -349,7 +353,7 @@ __device__ __forceinline__ void select_from_keys(const uint32_t* keys, int nb, i
     __syncthreads();  // every warp is done with the bin histogram
     zero_hist(sm, 0);
     __syncthreads();
-    for (int i = 1 + threadIdx.x; i <= nb - 2; i += NT) atomicAdd(&sm.hist[0][keys[i] >> 24], 1);
+    for (int i = 1 + threadIdx.x; i <= nb - 2; i += NT) atomicAdd(&sm.hist[0][hidx(keys[i] >> 24)], 1);
     __syncthreads();
     kr = k - 2;
     radix_threshold(keys, nb, sm, prefix, mask, kr);
@@ -479,7 +483,7 @@ __device__ __forceinline__ void topk_regs(const uint32_t* row, int nb, int k, in
 #pragma unroll
       for (int u = 0; u < KPT; ++u) {
         const int i = u * NT + tid;
-        if (i >= 1 && i <= nb - 2) atomicAdd(&sm.hist[0][bin_of(key[u])], 1);
+        if (i >= 1 && i <= nb - 2) atomicAdd(&sm.hist[0][hidx(bin_of(key[u]))], 1);
       }
       __syncthreads();
       warp_find_bin(sm.hist[0], kr, bstar, above, c);  // every warp, same result
@@ -495,7 +499,7 @@ __device__ __forceinline__ void topk_regs(const uint32_t* row, int nb, int k, in
       zero_hist(sm, 0);
       zero_hist(sm, 1);
       __syncthreads();
-      for (int i = 1 + tid; i <= nb - 2; i += NT) atomicAdd(&sm.hist[0][skey[i] >> 24], 1);
+      for (int i = 1 + tid; i <= nb - 2; i += NT) atomicAdd(&sm.hist[0][hidx(skey[i] >> 24)], 1);
       __syncthreads();
       uint32_t prefix, mask;
       int kr2 = kr;
@@ -699,8 +703,14 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_topk_kernel(SelectParams
   if (tid == 0) p.sel_cnt[pair] = k;
 }
 
-// Threads per top-k CTA: 4 keys per thread up to 4096 blocks.
-int topk_threads(int nbcap) { return nbcap <= 1024 ? 256 : nbcap <= 2048 ? 512 : 1024; }
+// Threads per top-k CTA: enough for 4 keys per thread (up to 4096 blocks),
+// halved (8 keys per thread) while the pairs would need more than one wave
+// of CTAs (the launch bounds allow 1024 / NT CTAs per SM).
+int topk_threads(int nbcap, int64_t pairs) {
+  int nt = nbcap <= 1024 ? 256 : nbcap <= 2048 ? 512 : 1024;
+  while (nt > 256 && nbcap <= 8 * (nt / 2) && pairs > (int64_t)device_sm_count() * (1024 / nt)) nt /= 2;
+  return nt;
+}
 
 template <int NT>
 cudaError_t launch_topk(const SelectParams& p, cudaStream_t s) {
@@ -720,7 +730,7 @@ cudaError_t launch_select(const SelectParams& p, cudaStream_t s) {
   const int grid = (int)(want < resident ? (want > 0 ? want : 1) : resident);
   cudaError_t e = launch_pdl(select_scan_kernel, dim3(grid), dim3(kSelThreads), 0, s, p);
   if (e != cudaSuccess) return e;
-  switch (topk_threads(p.nbcap)) {
+  switch (topk_threads(p.nbcap, (int64_t)p.B * p.Hkv)) {
     case 256: return launch_topk<256>(p, s);
     case 512: return launch_topk<512>(p, s);
     default: return launch_topk<1024>(p, s);
