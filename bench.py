@@ -41,6 +41,7 @@ DEFAULT_WORKLOAD = "qwen3_8b_32k"
 METRIC = "block-top-k decode attn query-heads/s"
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20  # > 2x the 126 MB L2
+KERNEL_REPEATS = 4  # back-to-back calls per per-kernel timing graph
 
 
 # ---------------------------------------------------------------- bytes model
@@ -279,7 +280,6 @@ def gpu_arm(args):
         flush_sink.copy_(flush_r.sum())
 
     flush_sink = torch.zeros((), dtype=torch.float32, device="cuda")
-    n_ev = 4 if w.n_append else 3
     # select = scan + top-k kernels, then attention (+ the append update)
     launches_per_step = 4 if w.n_append else 3
 
@@ -292,17 +292,33 @@ def gpu_arm(args):
 
     # A step is one CUDA graph, captured once and replayed every step as a
     # decode loop would, with two timing events inside it around the step's
-    # kernels, so the kernels chain back to back.  A second graph carries an
-    # event between every kernel for the per-kernel times the roofline uses.
-    # Both graphs are replayed during warm-up, so no timed step pays a
-    # graph's first launch.  The L2 flush runs eagerly before every replay,
-    # outside the events, and each replay's events are read back (a host
-    # synchronize, also outside the events) before the next replay.
+    # kernels, so the kernels chain back to back.  Both this graph and the
+    # per-kernel graphs below are replayed during warm-up, so no timed replay
+    # pays a graph's first launch.  The L2 flush runs eagerly before every
+    # replay, outside the events, and each replay's events are read back (a
+    # host synchronize, also outside the events) before the next replay.
     def ext_events(n):
         return [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n)]
 
+    import block_top_sparse_kin_b200 as kin
+
+    def call_select():
+        kin.kin_block_topk_select(st["dims"], st["q"], st["means"], st["seq"], k, st["sel"], st["cnt"],
+                                  st["ws"], st["status"])
+
+    def call_attn():
+        kin.kin_sparse_decode_attn(st["dims"], st["q"], st["k_cache"], st["v_cache"], st["seq"], st["sel"],
+                                   st["cnt"], k, 0.0, st["out"], st["lse"], st["ws"], st["status"])
+
+    # Per-kernel times for the roofline: a graph per kernel family holding
+    # KERNEL_REPEATS back-to-back calls between two events.  The means and the
+    # kept K/V are larger than L2 and are streamed (means with evict-first
+    # loads), so every call reads HBM; the events' few-us launch edges are
+    # spread over the calls, as in a decode pipeline.  The append update is
+    # timed once per replay (its calls would move the lengths).
     step_ev = ext_events(2)
-    kern_ev = ext_events(n_ev)
+    sel_ev, attn_ev = ext_events(2), ext_events(2)
+    upd_ev = ext_events(2)
     cap = torch.cuda.Stream()
     cap.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(cap):
@@ -312,15 +328,34 @@ def gpu_arm(args):
             step_ev[0].record()
             run_step(st)
             step_ev[1].record()
-        diag_graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(diag_graph, stream=cap):
-            reset_state(st)
-            run_step(st, kern_ev)
+        sel_graph, attn_graph = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(sel_graph, stream=cap):
+            sel_ev[0].record()
+            for _ in range(KERNEL_REPEATS):
+                call_select()
+            sel_ev[1].record()
+        with torch.cuda.graph(attn_graph, stream=cap):
+            attn_ev[0].record()
+            for _ in range(KERNEL_REPEATS):
+                call_attn()
+            attn_ev[1].record()
+        upd_graph = None
+        if w.n_append:
+            upd_graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(upd_graph, stream=cap):
+                reset_state(st)
+                upd_ev[0].record()
+                kin.kin_block_means_update(st["dims"], st["k_cache"], st["v_cache"], st["means"], st["seq"],
+                                           st["k_new"], st["v_new"], w.n_append, st["status"])
+                upd_ev[1].record()
     torch.cuda.current_stream().wait_stream(cap)
+    diag = [g for g in (sel_graph, attn_graph, upd_graph) if g is not None]
     for _ in range(args.warmup):
         flush_l2(0)
         graph.replay()
-        diag_graph.replay()
+        for g in diag:
+            flush_l2(0)
+            g.replay()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -338,13 +373,18 @@ def gpu_arm(args):
         dist.barrier()
     sel_ms, attn_ms, upd_ms = [], [], []
     for s in range(args.steps):            # per-kernel timing pass (not in `value`)
-        flush_l2(s)
-        diag_graph.replay()
-        torch.cuda.synchronize()
-        sel_ms.append(kern_ev[-3].elapsed_time(kern_ev[-2]))
-        attn_ms.append(kern_ev[-2].elapsed_time(kern_ev[-1]))
-        if w.n_append:
-            upd_ms.append(kern_ev[0].elapsed_time(kern_ev[1]))
+        for g, ev, out, reps in ((sel_graph, sel_ev, sel_ms, KERNEL_REPEATS),
+                                 (attn_graph, attn_ev, attn_ms, KERNEL_REPEATS),
+                                 (upd_graph, upd_ev, upd_ms, 1)):
+            if g is None:
+                continue
+            flush_l2(s)
+            g.replay()
+            torch.cuda.synchronize()
+            out.append(ev[0].elapsed_time(ev[1]) / reps)
+    reset_state(st)
+    run_step(st)                           # leave the state as one step leaves it
+    torch.cuda.synchronize()
     total_ms = reduce_max(sum(per_step), "cuda")
     ms_per_step = total_ms / args.steps
     qh_per_step = w.B * w.Hq

@@ -89,16 +89,6 @@ __device__ __forceinline__ uint32_t tok_mask(int t, int nvalid) {
   return (t < nvalid ? 0x0000FFFFu : 0u) | (t + 1 < nvalid ? 0xFFFF0000u : 0u);
 }
 
-// 16-byte async copy global -> shared; src_bytes 0 writes zeros and reads nothing.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kernel(AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -385,15 +375,15 @@ __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kerne
       s_den[j] = dd;
     }
     __syncthreads();
-    if (d < kHeadDim) {
+    if (d < kHeadDim) {  // chunk-outer, head-inner: g independent accumulation chains
 #pragma unroll
-      for (int j = 0; j < kMaxGroup; ++j) {
-        if (j < g) {
-          float nn = num[j] * s_a[j];
-#pragma unroll 8
-          for (int c = 0; c < nbat; ++c) nn += s_w[c * g + j] * stage[(c * g + j) * kPartStride + d];
-          num[j] = nn;
-        }
+      for (int j = 0; j < kMaxGroup; ++j)
+        if (j < g) num[j] *= s_a[j];
+      for (int c = 0; c < nbat; ++c) {
+        const float* rc = stage + c * g * kPartStride + d;
+#pragma unroll
+        for (int j = 0; j < kMaxGroup; ++j)
+          if (j < g) num[j] += s_w[c * g + j] * rc[j * kPartStride];
       }
     }
     __syncthreads();  // the next batch overwrites the staging area and the weights

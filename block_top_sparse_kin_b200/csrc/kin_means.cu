@@ -59,7 +59,13 @@ __global__ void __launch_bounds__(256) means_build_kernel(MeansBuildParams p) {
 
 // grid (B), 256 threads.  One CTA owns a whole sequence so that the length
 // it reads and the length it writes back cannot race with another CTA.
-__global__ void __launch_bounds__(256) means_update_kernel(MeansUpdateParams p) {
+constexpr int kUpdRows = 32;                // rows staged per warp and batch
+constexpr int kRowBytes = kHeadDim * 2;     // one bf16 K row
+constexpr int kUpdThreads = 256;
+constexpr size_t kUpdSmem = (size_t)(kUpdThreads / 32) * kUpdRows * kRowBytes;  // 64 KB
+
+__global__ void __launch_bounds__(kUpdThreads) means_update_kernel(MeansUpdateParams p) {
+  extern __shared__ __align__(16) uint8_t upd_rows[];  // [warp][kUpdRows][kRowBytes]
   pdl_wait();
   pdl_trigger_early();
   const int b = blockIdx.x;
@@ -83,29 +89,34 @@ __global__ void __launch_bounds__(256) means_update_kernel(MeansUpdateParams p) 
     reinterpret_cast<uint4*>(p.v_cache)[dst] = reinterpret_cast<const uint4*>(p.v_new)[src];
   }
   // 2. recompute the mean of every touched block from its valid rows; rows
-  //    below L0 come from the cache, newer rows straight from k_new.
+  //    below L0 come from the cache, newer rows straight from k_new.  A warp
+  //    copies up to 32 rows of its block into shared memory with 16-byte
+  //    cp.async (one memory round trip), then sums them in token order.
   const int first = L0 / p.bs, last = (L1 - 1) / p.bs;
   const int nblk = last - first + 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  const uint32_t rows_s = smem_u32(upd_rows) + (uint32_t)(warp * kUpdRows * kRowBytes);
+  const uint2* rows_r = reinterpret_cast<const uint2*>(upd_rows + warp * kUpdRows * kRowBytes) + lane;
   for (int task = warp; task < p.Hkv * nblk; task += nwarps) {
     const int h = task / nblk, i = first + task % nblk;
     const int64_t pair = (int64_t)b * p.Hkv + h;
     const int t0 = i * p.bs, t1 = min(t0 + p.bs, L1);
-    const uint2* cache = reinterpret_cast<const uint2*>(p.k_cache + pair * p.Lcap * kHeadDim) + lane;
-    const uint2* fresh = reinterpret_cast<const uint2*>(p.k_new + pair * n * kHeadDim) + lane;
-    auto row = [&](int t) {
-      return t < L0 ? cache[(int64_t)t * (kHeadDim / 4)] : fresh[(int64_t)(t - L0) * (kHeadDim / 4)];
-    };
+    const uint8_t* cache = reinterpret_cast<const uint8_t*>(p.k_cache + pair * p.Lcap * kHeadDim);
+    const uint8_t* fresh = reinterpret_cast<const uint8_t*>(p.k_new + pair * n * kHeadDim);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    int t = t0;
-    for (; t + 8 <= t1; t += 8) {  // 8 rows in flight per lane, summed in token order
-      uint2 r[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) r[u] = row(t + u);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) add_row4(acc, r[u]);
+    for (int t = t0; t < t1; t += kUpdRows) {
+      const int nrows = min(kUpdRows, t1 - t);
+      for (int c = lane; c < nrows * 16; c += 32) {  // 16 pieces of 16 bytes per row
+        const int r = t + (c >> 4), piece = c & 15;
+        const uint8_t* src = r < L0 ? cache + (int64_t)r * kRowBytes : fresh + (int64_t)(r - L0) * kRowBytes;
+        cp_async16(rows_s + (uint32_t)(c * 16), src + piece * 16, 16u);
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
+      __syncwarp();
+      for (int r = 0; r < nrows; ++r) add_row4(acc, rows_r[r * (kRowBytes / 8)]);
+      __syncwarp();  // every lane is done reading before the next batch lands
     }
-    for (; t < t1; ++t) add_row4(acc, row(t));
     const float cnt = (float)(t1 - t0);
     float4 m = make_float4(__fdiv_rn(acc[0], cnt), __fdiv_rn(acc[1], cnt), __fdiv_rn(acc[2], cnt),
                            __fdiv_rn(acc[3], cnt));
@@ -121,7 +132,9 @@ cudaError_t launch_means_build(const MeansBuildParams& p, cudaStream_t s) {
 }
 
 cudaError_t launch_means_update(const MeansUpdateParams& p, cudaStream_t s) {
-  return launch_pdl(means_update_kernel, dim3(p.B), dim3(256), 0, s, p);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(means_update_kernel), 4, kUpdSmem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(means_update_kernel, dim3(p.B), dim3(kUpdThreads), kUpdSmem, s, p);
 }
 
 }  // namespace kin
