@@ -195,7 +195,43 @@ def shard_workload(w: ki.Workload, rank: int) -> ki.Workload:
     return w.with_(seed=w.seed + 1000 * rank) if rank else w
 
 
-def build_device_state(w: ki.Workload, k: int):
+def make_page_pool(st, seed: int):
+    """Moves the contiguous K/V caches into a shuffled page pool (page = one
+    KV block, [num_pages, Hkv, bs, D]) with a block table [B, nbcap]: every
+    block a sequence holds after the step's append gets a page, in random
+    order.  Frees the contiguous caches."""
+    import torch
+    w = st["w"]
+    B, Hkv, cap, D = st["k_cache"].shape
+    bs, nbcap = w.bs, w.nbcap
+    nbs = [-(-int(L) // bs) for L in st["lens_final"]]
+    P = sum(nbs)
+    order = np.random.default_rng(seed).permutation(P)
+    table = np.full((B, nbcap), -1, np.int32)
+    j = 0
+    for b in range(B):
+        table[b, :nbs[b]] = order[j:j + nbs[b]]
+        j += nbs[b]
+    ib, ii = np.nonzero(table >= 0)
+    dst = torch.from_numpy(table[ib, ii].astype(np.int64)).cuda()
+    tb, ti = torch.from_numpy(ib).cuda(), torch.from_numpy(ii).cuda()
+    for name in ("k_cache", "v_cache"):
+        cache = st.pop(name)
+        if cap % bs:
+            cache = torch.nn.functional.pad(cache, (0, 0, 0, nbcap * bs - cap))
+        blocks = cache.view(B, Hkv, nbcap, bs, D)
+        pool = torch.empty((P, Hkv, bs, D), dtype=torch.bfloat16, device="cuda")
+        for c0 in range(0, len(ib), 1 << 16):  # bounded temporaries
+            sl = slice(c0, c0 + (1 << 16))
+            pool[dst[sl]] = blocks[tb[sl], :, ti[sl]]
+        st[name.replace("cache", "pages")] = pool
+        del cache, blocks
+    st["table"] = torch.from_numpy(table).cuda()
+    st["num_pages"] = P
+    torch.cuda.empty_cache()
+
+
+def build_device_state(w: ki.Workload, k: int, paged: bool = False):
     import torch
     import block_top_sparse_kin_b200 as kin
     lens_final, lens_pre, hh = ki.case_meta(w)
@@ -229,6 +265,8 @@ def build_device_state(w: ki.Workload, k: int):
     st["lse"] = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
     st["status"] = torch.zeros(1, dtype=torch.int32, device="cuda")
     st["ws"] = kin.alloc_workspace(dims, k)
+    if paged:
+        make_page_pool(st, w.seed)
     torch.cuda.synchronize()
     return st
 
@@ -240,19 +278,35 @@ def run_step(st, ev=None):
     i = 0
     if ev is not None:
         ev[i].record(); i += 1
+    paged = "table" in st
     if w.n_append:
-        kin.kin_block_means_update(dims, st["k_cache"], st["v_cache"], st["means"], st["seq"],
-                                   st["k_new"], st["v_new"], w.n_append, st["status"])
+        if paged:
+            kin.kin_block_means_update_paged(dims, st["k_pages"], st["v_pages"], st["table"], st["means"],
+                                             st["seq"], st["k_new"], st["v_new"], w.n_append, st["status"])
+        else:
+            kin.kin_block_means_update(dims, st["k_cache"], st["v_cache"], st["means"], st["seq"],
+                                       st["k_new"], st["v_new"], w.n_append, st["status"])
         if ev is not None:
             ev[i].record(); i += 1
     kin.kin_block_topk_select(dims, st["q"], st["means"], st["seq"], k, st["sel"], st["cnt"], st["ws"],
                               st["status"])
     if ev is not None:
         ev[i].record(); i += 1
-    kin.kin_sparse_decode_attn(dims, st["q"], st["k_cache"], st["v_cache"], st["seq"], st["sel"], st["cnt"],
-                               k, 0.0, st["out"], st["lse"], st["ws"], st["status"])
+    attend(st)
     if ev is not None:
         ev[i].record()
+
+
+def attend(st):
+    """The step's attention call, over the contiguous cache or the page pool."""
+    import block_top_sparse_kin_b200 as kin
+    if "table" in st:
+        kin.kin_sparse_decode_attn_paged(st["dims"], st["q"], st["k_pages"], st["v_pages"], st["table"], st["seq"],
+                                         st["sel"], st["cnt"], st["k"], 0.0, st["out"], st["lse"], st["ws"],
+                                         st["status"])
+    else:
+        kin.kin_sparse_decode_attn(st["dims"], st["q"], st["k_cache"], st["v_cache"], st["seq"], st["sel"],
+                                   st["cnt"], st["k"], 0.0, st["out"], st["lse"], st["ws"], st["status"])
 
 
 def reset_state(st):
@@ -269,7 +323,7 @@ def gpu_arm(args):
         w0 = w0.with_(B=args.batch, name=f"{w0.name}_b{args.batch}")
     k = args.k or w0.k
     w = shard_workload(w0, rank)
-    st = build_device_state(w, k)
+    st = build_device_state(w, k, paged=args.paged)
     flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
 
@@ -307,8 +361,7 @@ def gpu_arm(args):
                                   st["ws"], st["status"])
 
     def call_attn():
-        kin.kin_sparse_decode_attn(st["dims"], st["q"], st["k_cache"], st["v_cache"], st["seq"], st["sel"],
-                                   st["cnt"], k, 0.0, st["out"], st["lse"], st["ws"], st["status"])
+        attend(st)
 
     # Per-kernel times for the roofline: a graph per kernel family holding
     # KERNEL_REPEATS back-to-back calls between two events.  The means and the
@@ -345,8 +398,13 @@ def gpu_arm(args):
             with torch.cuda.graph(upd_graph, stream=cap):
                 reset_state(st)
                 upd_ev[0].record()
-                kin.kin_block_means_update(st["dims"], st["k_cache"], st["v_cache"], st["means"], st["seq"],
-                                           st["k_new"], st["v_new"], w.n_append, st["status"])
+                if "table" in st:
+                    kin.kin_block_means_update_paged(st["dims"], st["k_pages"], st["v_pages"], st["table"],
+                                                     st["means"], st["seq"], st["k_new"], st["v_new"],
+                                                     w.n_append, st["status"])
+                else:
+                    kin.kin_block_means_update(st["dims"], st["k_cache"], st["v_cache"], st["means"],
+                                               st["seq"], st["k_new"], st["v_new"], w.n_append, st["status"])
                 upd_ev[1].record()
     torch.cuda.current_stream().wait_stream(cap)
     diag = [g for g in (sel_graph, attn_graph, upd_graph) if g is not None]
@@ -446,6 +504,8 @@ def gpu_arm(args):
                 "top_k_blocks": k, "append_tokens": w0.n_append,
                 "global_batch": w0.B * world, "parallelism": f"dp{world}",
                 "l2": "flushed before every step (256 MiB write + 256 MiB read, outside the timed events)",
+                "kv_layout": (f"paged: {st['num_pages']} pages of one {w.bs}-token block, shuffled pool + block table"
+                              if args.paged else "contiguous [B][Hkv][Lcap][D]"),
             },
             "impl": "kin",
             "gpu_launches": launches_per_step * args.steps,  # in the timed region
@@ -579,6 +639,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-pairs", type=int, default=8, help="pairs per reference-arm step")
+    ap.add_argument("--paged", action="store_true", help="KV cache in a shuffled page pool with a block table")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "kin":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

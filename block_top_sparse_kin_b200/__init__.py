@@ -26,7 +26,8 @@ STATUS_NAMES = {
 EXPORTED = (
     "kin_status_string", "kin_workspace_bytes", "kin_block_means_build",
     "kin_block_means_update", "kin_block_topk_select", "kin_sparse_decode_attn",
-    "kin_block_topk_select_noalloc",
+    "kin_block_topk_select_noalloc", "kin_block_means_build_paged", "kin_block_means_update_paged",
+    "kin_sparse_decode_attn_paged",
 )
 NOALLOC_SCRATCH_FLOATS = 1 << 21  # KIN_NOALLOC_SCRATCH_FLOATS in include/kin.h
 
@@ -85,6 +86,13 @@ def load_library(path: str = LIB_PATH):
     lib.kin_sparse_decode_attn.restype = ctypes.c_int
     lib.kin_block_topk_select_noalloc.argtypes = [dp, vp, vp, vp, i32, vp, vp, vp, vp]
     lib.kin_block_topk_select_noalloc.restype = ctypes.c_int
+    lib.kin_block_means_build_paged.argtypes = [dp, vp, i32, vp, vp, vp, vp, vp]
+    lib.kin_block_means_build_paged.restype = ctypes.c_int
+    lib.kin_block_means_update_paged.argtypes = [dp, vp, vp, i32, vp, vp, vp, vp, vp, i32, vp, vp]
+    lib.kin_block_means_update_paged.restype = ctypes.c_int
+    lib.kin_sparse_decode_attn_paged.argtypes = [dp, vp, vp, vp, i32, vp, vp, vp, vp, i32, f32, vp, vp, vp,
+                                                 sz, vp, vp]
+    lib.kin_sparse_decode_attn_paged.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -186,3 +194,41 @@ def kin_block_topk_select_noalloc(dims, q, block_means, seq_lens, k_blocks, sel_
         _dev(sel_cnt, "sel_cnt", torch.int32),
         _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
     _check(rc, "kin_block_topk_select_noalloc")
+
+
+# ---------------------------------------------------------------- paged KV
+# k_pages / v_pages [num_pages, Hkv, bs, D] bf16; block_table [B, ceil(Lcap / bs)]
+# int32 (page of each logical block).  See include/kin.h.
+
+def kin_block_means_build_paged(dims, k_pages, block_table, seq_lens, block_means, dev_status=None,
+                                stream=None):
+    rc = load_library().kin_block_means_build_paged(
+        ctypes.byref(dims), _dev(k_pages, "k_pages", _BF16), int(k_pages.shape[0]),
+        _dev(block_table, "block_table", torch.int32), _dev(seq_lens, "seq_lens", torch.int32),
+        _dev(block_means, "block_means", torch.float32),
+        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+    _check(rc, "kin_block_means_build_paged")
+
+
+def kin_block_means_update_paged(dims, k_pages, v_pages, block_table, block_means, seq_lens, k_new, v_new,
+                                 n_new, dev_status=None, stream=None):
+    rc = load_library().kin_block_means_update_paged(
+        ctypes.byref(dims), _dev(k_pages, "k_pages", _BF16), _dev(v_pages, "v_pages", _BF16),
+        int(k_pages.shape[0]), _dev(block_table, "block_table", torch.int32),
+        _dev(block_means, "block_means", torch.float32), _dev(seq_lens, "seq_lens", torch.int32),
+        _dev(k_new, "k_new", _BF16), _dev(v_new, "v_new", _BF16), int(n_new),
+        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+    _check(rc, "kin_block_means_update_paged")
+
+
+def kin_sparse_decode_attn_paged(dims, q, k_pages, v_pages, block_table, seq_lens, sel_idx, sel_cnt, k_blocks,
+                                 softmax_scale, out, lse, workspace, dev_status=None, stream=None):
+    rc = load_library().kin_sparse_decode_attn_paged(
+        ctypes.byref(dims), _dev(q, "q", _BF16), _dev(k_pages, "k_pages", _BF16),
+        _dev(v_pages, "v_pages", _BF16), int(k_pages.shape[0]), _dev(block_table, "block_table", torch.int32),
+        _dev(seq_lens, "seq_lens", torch.int32), _dev(sel_idx, "sel_idx", torch.int32),
+        _dev(sel_cnt, "sel_cnt", torch.int32), int(k_blocks), float(softmax_scale), _dev(out, "out", _BF16),
+        _dev(lse, "lse", torch.float32, nullable=True), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(),
+        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+    _check(rc, "kin_sparse_decode_attn_paged")

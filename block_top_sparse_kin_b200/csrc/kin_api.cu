@@ -84,6 +84,25 @@ kin_status check_ws(const kin_dims& d, int k, void* ws, size_t ws_bytes, WsLayou
 
 kin_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KIN_OK : KIN_ERR_CUDA; }
 
+PageTable contiguous() {
+  PageTable pt;
+  pt.table = nullptr;
+  pt.max_blocks = 0;
+  pt.num_pages = 0;
+  return pt;
+}
+
+// A page pool [num_pages][Hkv][bs][D] bf16 and its table [B][ceil(Lcap / bs)].
+kin_status check_pages(const kin_dims& d, const void* pool, int32_t num_pages, const int32_t* table,
+                       PageTable* out) {
+  if (!pool || !table || num_pages < 1) return KIN_ERR_INVALID_ARG;
+  if (!aligned16(pool)) return KIN_ERR_INVALID_ARG;
+  out->table = table;
+  out->max_blocks = nbcap_of(d);
+  out->num_pages = num_pages;
+  return KIN_OK;
+}
+
 }  // namespace
 
 namespace kin {
@@ -138,18 +157,16 @@ KIN_EXPORT size_t kin_workspace_bytes(const kin_dims* dims, int32_t k_blocks) {
   return ws_layout(*dims, k_blocks).total;
 }
 
-KIN_EXPORT kin_status kin_block_means_build(const kin_dims* dims, const void* k_cache,
-                                            const int32_t* seq_lens, float* block_means,
-                                            int32_t* dev_status, void* stream) {
-  kin_status st = check_dims(dims);
-  if (st != KIN_OK) return st;
-  if (!k_cache || !seq_lens || !block_means) return KIN_ERR_INVALID_ARG;
-  if (!aligned16(k_cache) || !aligned16(block_means)) return KIN_ERR_INVALID_ARG;
+namespace {
+
+kin_status means_build(const kin_dims* dims, const void* k_rows, const PageTable& pt, const int32_t* seq_lens,
+                       float* block_means, int32_t* dev_status, void* stream) {
   MeansBuildParams p;
-  p.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
+  p.k_cache = static_cast<const __nv_bfloat16*>(k_rows);
   p.seq_lens = seq_lens;
   p.means = block_means;
   p.dev_status = dev_status;
+  p.pages = pt;
   p.B = dims->batch;
   p.Hkv = dims->num_kv_heads;
   p.Lcap = dims->max_seq_len;
@@ -158,27 +175,18 @@ KIN_EXPORT kin_status kin_block_means_build(const kin_dims* dims, const void* k_
   return from_cuda(launch_means_build(p, static_cast<cudaStream_t>(stream)));
 }
 
-KIN_EXPORT kin_status kin_block_means_update(const kin_dims* dims, void* k_cache, void* v_cache,
-                                             float* block_means, int32_t* seq_lens,
-                                             const void* k_new, const void* v_new, int32_t n_new,
-                                             int32_t* dev_status, void* stream) {
-  kin_status st = check_dims(dims);
-  if (st != KIN_OK) return st;
-  if (n_new < 0) return KIN_ERR_INVALID_ARG;
-  if (n_new > dims->max_seq_len) return KIN_ERR_CAPACITY;
-  if (n_new == 0) return KIN_OK;
-  if (!k_cache || !v_cache || !block_means || !seq_lens || !k_new || !v_new) return KIN_ERR_INVALID_ARG;
-  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(block_means) || !aligned16(k_new) ||
-      !aligned16(v_new))
-    return KIN_ERR_INVALID_ARG;
+kin_status means_update(const kin_dims* dims, void* k_rows, void* v_rows, const PageTable& pt,
+                        float* block_means, int32_t* seq_lens, const void* k_new, const void* v_new,
+                        int32_t n_new, int32_t* dev_status, void* stream) {
   MeansUpdateParams p;
-  p.k_cache = static_cast<__nv_bfloat16*>(k_cache);
-  p.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  p.k_cache = static_cast<__nv_bfloat16*>(k_rows);
+  p.v_cache = static_cast<__nv_bfloat16*>(v_rows);
   p.means = block_means;
   p.seq_lens = seq_lens;
   p.k_new = static_cast<const __nv_bfloat16*>(k_new);
   p.v_new = static_cast<const __nv_bfloat16*>(v_new);
   p.dev_status = dev_status;
+  p.pages = pt;
   p.B = dims->batch;
   p.Hkv = dims->num_kv_heads;
   p.Lcap = dims->max_seq_len;
@@ -186,6 +194,77 @@ KIN_EXPORT kin_status kin_block_means_update(const kin_dims* dims, void* k_cache
   p.nbcap = nbcap_of(*dims);
   p.n_new = n_new;
   return from_cuda(launch_means_update(p, static_cast<cudaStream_t>(stream)));
+}
+
+kin_status check_update_count(const kin_dims* dims, int32_t n_new) {
+  if (n_new < 0) return KIN_ERR_INVALID_ARG;
+  if (n_new > dims->max_seq_len) return KIN_ERR_CAPACITY;
+  return KIN_OK;
+}
+
+kin_status check_update_args(const void* k_rows, const void* v_rows, const float* block_means,
+                             const int32_t* seq_lens, const void* k_new, const void* v_new) {
+  if (!k_rows || !v_rows || !block_means || !seq_lens || !k_new || !v_new) return KIN_ERR_INVALID_ARG;
+  if (!aligned16(k_rows) || !aligned16(v_rows) || !aligned16(block_means) || !aligned16(k_new) ||
+      !aligned16(v_new))
+    return KIN_ERR_INVALID_ARG;
+  return KIN_OK;
+}
+
+}  // namespace
+
+KIN_EXPORT kin_status kin_block_means_build(const kin_dims* dims, const void* k_cache,
+                                            const int32_t* seq_lens, float* block_means,
+                                            int32_t* dev_status, void* stream) {
+  kin_status st = check_dims(dims);
+  if (st != KIN_OK) return st;
+  if (!k_cache || !seq_lens || !block_means) return KIN_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(block_means)) return KIN_ERR_INVALID_ARG;
+  return means_build(dims, k_cache, contiguous(), seq_lens, block_means, dev_status, stream);
+}
+
+KIN_EXPORT kin_status kin_block_means_build_paged(const kin_dims* dims, const void* k_pages, int32_t num_pages,
+                                                  const int32_t* block_table, const int32_t* seq_lens,
+                                                  float* block_means, int32_t* dev_status, void* stream) {
+  kin_status st = check_dims(dims);
+  if (st != KIN_OK) return st;
+  PageTable pt;
+  st = check_pages(*dims, k_pages, num_pages, block_table, &pt);
+  if (st != KIN_OK) return st;
+  if (!seq_lens || !block_means || !aligned16(block_means)) return KIN_ERR_INVALID_ARG;
+  return means_build(dims, k_pages, pt, seq_lens, block_means, dev_status, stream);
+}
+
+KIN_EXPORT kin_status kin_block_means_update(const kin_dims* dims, void* k_cache, void* v_cache,
+                                             float* block_means, int32_t* seq_lens,
+                                             const void* k_new, const void* v_new, int32_t n_new,
+                                             int32_t* dev_status, void* stream) {
+  kin_status st = check_dims(dims);
+  if (st != KIN_OK) return st;
+  st = check_update_count(dims, n_new);
+  if (st != KIN_OK || n_new == 0) return st;
+  st = check_update_args(k_cache, v_cache, block_means, seq_lens, k_new, v_new);
+  if (st != KIN_OK) return st;
+  return means_update(dims, k_cache, v_cache, contiguous(), block_means, seq_lens, k_new, v_new, n_new,
+                      dev_status, stream);
+}
+
+KIN_EXPORT kin_status kin_block_means_update_paged(const kin_dims* dims, void* k_pages, void* v_pages,
+                                                   int32_t num_pages, const int32_t* block_table,
+                                                   float* block_means, int32_t* seq_lens, const void* k_new,
+                                                   const void* v_new, int32_t n_new, int32_t* dev_status,
+                                                   void* stream) {
+  kin_status st = check_dims(dims);
+  if (st != KIN_OK) return st;
+  st = check_update_count(dims, n_new);
+  if (st != KIN_OK || n_new == 0) return st;
+  PageTable pt;
+  st = check_pages(*dims, k_pages, num_pages, block_table, &pt);
+  if (st != KIN_OK) return st;
+  st = check_update_args(k_pages, v_pages, block_means, seq_lens, k_new, v_new);
+  if (st != KIN_OK) return st;
+  return means_update(dims, k_pages, v_pages, pt, block_means, seq_lens, k_new, v_new, n_new, dev_status,
+                      stream);
 }
 
 KIN_EXPORT kin_status kin_block_topk_select(const kin_dims* dims, const void* q, const float* block_means,
@@ -221,27 +300,24 @@ KIN_EXPORT kin_status kin_block_topk_select(const kin_dims* dims, const void* q,
   return from_cuda(launch_select(p, static_cast<cudaStream_t>(stream)));
 }
 
-KIN_EXPORT kin_status kin_sparse_decode_attn(const kin_dims* dims, const void* q, const void* k_cache,
-                                             const void* v_cache, const int32_t* seq_lens,
-                                             const int32_t* sel_idx, const int32_t* sel_cnt,
-                                             int32_t k_blocks, float softmax_scale, void* out, float* lse,
-                                             void* workspace, size_t ws_bytes, int32_t* dev_status,
-                                             void* stream) {
-  kin_status st = check_dims(dims);
-  if (st != KIN_OK) return st;
+namespace {
+
+kin_status sparse_decode_attn(const kin_dims* dims, const void* q, const void* k_rows, const void* v_rows,
+                              const PageTable& pt, const int32_t* seq_lens, const int32_t* sel_idx,
+                              const int32_t* sel_cnt, int32_t k_blocks, float softmax_scale, void* out,
+                              float* lse, void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
   if (k_blocks < 2) return KIN_ERR_INVALID_ARG;
-  if (!q || !k_cache || !v_cache || !seq_lens || !sel_idx || !sel_cnt || !out) return KIN_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
-    return KIN_ERR_INVALID_ARG;
+  if (!q || !k_rows || !v_rows || !seq_lens || !sel_idx || !sel_cnt || !out) return KIN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_rows) || !aligned16(v_rows) || !aligned16(out)) return KIN_ERR_INVALID_ARG;
   if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale)) return KIN_ERR_INVALID_ARG;
   WsLayout w;
-  st = check_ws(*dims, k_blocks, workspace, ws_bytes, &w);
+  kin_status st = check_ws(*dims, k_blocks, workspace, ws_bytes, &w);
   if (st != KIN_OK) return st;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   AttnParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
-  p.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
-  p.v_cache = static_cast<const __nv_bfloat16*>(v_cache);
+  p.k_cache = static_cast<const __nv_bfloat16*>(k_rows);
+  p.v_cache = static_cast<const __nv_bfloat16*>(v_rows);
   p.seq_lens = seq_lens;
   p.sel_idx = sel_idx;
   p.sel_cnt = sel_cnt;
@@ -250,6 +326,7 @@ KIN_EXPORT kin_status kin_sparse_decode_attn(const kin_dims* dims, const void* q
   p.partials = reinterpret_cast<float*>(ws + w.partials);
   p.counters = reinterpret_cast<uint32_t*>(ws + w.attn_counters);
   p.dev_status = dev_status;
+  p.pages = pt;
   p.B = dims->batch;
   p.Hkv = dims->num_kv_heads;
   p.Hq = dims->num_q_heads;
@@ -263,4 +340,34 @@ KIN_EXPORT kin_status kin_sparse_decode_attn(const kin_dims* dims, const void* q
   p.scale_log2 = scale * 1.4426950408889634f;
   const int num_items = pairs_of(*dims) * p.max_chunks;
   return from_cuda(launch_attn(p, num_items, static_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+KIN_EXPORT kin_status kin_sparse_decode_attn(const kin_dims* dims, const void* q, const void* k_cache,
+                                             const void* v_cache, const int32_t* seq_lens,
+                                             const int32_t* sel_idx, const int32_t* sel_cnt,
+                                             int32_t k_blocks, float softmax_scale, void* out, float* lse,
+                                             void* workspace, size_t ws_bytes, int32_t* dev_status,
+                                             void* stream) {
+  kin_status st = check_dims(dims);
+  if (st != KIN_OK) return st;
+  return sparse_decode_attn(dims, q, k_cache, v_cache, contiguous(), seq_lens, sel_idx, sel_cnt, k_blocks,
+                            softmax_scale, out, lse, workspace, ws_bytes, dev_status, stream);
+}
+
+KIN_EXPORT kin_status kin_sparse_decode_attn_paged(const kin_dims* dims, const void* q, const void* k_pages,
+                                                   const void* v_pages, int32_t num_pages,
+                                                   const int32_t* block_table, const int32_t* seq_lens,
+                                                   const int32_t* sel_idx, const int32_t* sel_cnt,
+                                                   int32_t k_blocks, float softmax_scale, void* out,
+                                                   float* lse, void* workspace, size_t ws_bytes,
+                                                   int32_t* dev_status, void* stream) {
+  kin_status st = check_dims(dims);
+  if (st != KIN_OK) return st;
+  PageTable pt;
+  st = check_pages(*dims, k_pages, num_pages, block_table, &pt);
+  if (st != KIN_OK) return st;
+  return sparse_decode_attn(dims, q, k_pages, v_pages, pt, seq_lens, sel_idx, sel_cnt, k_blocks,
+                            softmax_scale, out, lse, workspace, ws_bytes, dev_status, stream);
 }

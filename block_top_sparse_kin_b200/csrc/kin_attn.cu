@@ -115,18 +115,24 @@ __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kerne
   }
   if (it.ntiles == 0) return;  // a chunk index past this pair's chunks
 
-  // ---- this warp's tiles t = warp + W n; lane n holds tile n's source row and valid count
+  // ---- this warp's tiles t = warp + W n; lane n holds tile n's source
+  // offset (elements, into the contiguous cache or the page pool) and its
+  // valid row count
   const int tpb = p.bs / kTileTokens;
   const int n_w = warp < it.ntiles ? (it.ntiles - 1 - warp) / kAttnWarps + 1 : 0;
-  int my_row = 0, my_nvalid = 0;
+  int64_t my_off = 0;
+  int my_nvalid = 0;
   if (lane < n_w) {
     const int t = warp + kAttnWarps * lane;
     const int blk = __ldg(p.sel_idx + it.pair * p.k + it.j0 + t / tpb);
-    const bool bad = blk < 0 || blk >= it.nb;
+    const int sub = (t - (t / tpb) * tpb) * kTileTokens;
+    bool bad = blk < 0 || blk >= it.nb;
+    const int64_t off = bad ? -1 : kv_row_offset(p.pages, it.b, it.h, p.Hkv, p.Lcap, p.bs, blk, sub);
+    bad = off < 0;
     if (bad) set_status(p.dev_status, KIN_ERR_DEVICE_DATA);
-    const int row0 = blk * p.bs + (t - (t / tpb) * tpb) * kTileTokens;
+    const int row0 = blk * p.bs + sub;  // logical token index of the tile's first row
     my_nvalid = (bad || row0 >= it.L) ? 0 : min(kTileTokens, it.L - row0);
-    my_row = my_nvalid ? row0 : 0;
+    my_off = my_nvalid ? off : 0;
   }
 
   // Q fragments (B operand, "col" layout): head = lane/4, dims 16kk + 2(lane%4) (+8)
@@ -142,13 +148,12 @@ __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kerne
   }
 
   const uint32_t ring = smem_u32(smem) + (uint32_t)(warp * kStages * kStageBytes);
-  const __nv_bfloat16* kbase = p.k_cache + it.pair * (int64_t)p.Lcap * kHeadDim;
-  const __nv_bfloat16* vbase = p.v_cache + it.pair * (int64_t)p.Lcap * kHeadDim;
 
   // Issue tile n into its ring slot: lane l copies pieces l + 32 i (i < 8) of
   // the K tile and of the V tile; piece = (row r, 16-byte column cc).
   auto issue = [&](int n) {
-    const int row0 = __shfl_sync(0xffffffffu, my_row, n & 31);
+    const int64_t off0 = (int64_t)(((uint64_t)(uint32_t)__shfl_sync(0xffffffffu, (int)(my_off >> 32), n & 31) << 32) |
+                                   (uint32_t)__shfl_sync(0xffffffffu, (int)(uint32_t)my_off, n & 31));
     const int nv = __shfl_sync(0xffffffffu, my_nvalid, n & 31);
     if (n < n_w && nv > 0) {
       const uint32_t base = ring + (uint32_t)((n % kStages) * kStageBytes);
@@ -157,10 +162,10 @@ __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kerne
         const int piece = lane + 32 * i;
         const int r = piece >> 4, cc = piece & 15;
         const uint32_t off = (uint32_t)((cc >> 3) * kHalfBox + r * 128 + (((cc & 7) ^ (r & 7)) << 4));
-        const int64_t src = (int64_t)(row0 + (r < nv ? r : 0)) * kHeadDim + cc * 8;
+        const int64_t src = off0 + (int64_t)(r < nv ? r : 0) * kHeadDim + cc * 8;
         const uint32_t bytes = r < nv ? 16u : 0u;
-        cp_async16(base + off, kbase + src, bytes);
-        cp_async16(base + 2 * kHalfBox + off, vbase + src, bytes);
+        cp_async16(base + off, p.k_cache + src, bytes);
+        cp_async16(base + 2 * kHalfBox + off, p.v_cache + src, bytes);
       }
     }
     cp_async_commit();  // one group per tile, empty or not, keeps the accounting uniform

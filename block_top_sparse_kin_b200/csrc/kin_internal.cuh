@@ -107,12 +107,34 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// ---------------------------------------------------------- KV addressing
+// Where the K/V rows of a logical block live.  table == NULL: the contiguous
+// cache [B][Hkv][Lcap][D].  Otherwise a page pool [num_pages][Hkv][bs][D]
+// (the page is one KV block; a head's rows of a page are contiguous) and
+// table[b * max_blocks + i] is the page of sequence b's logical block i.
+struct PageTable {
+  const int32_t* table;
+  int max_blocks;
+  int num_pages;
+};
+
+// Element offset of row r (0 <= r < bs) of logical block blk of pair (b, h),
+// or -1 when the block's page index lies outside the pool.
+__device__ __forceinline__ int64_t kv_row_offset(const PageTable& pt, int b, int h, int Hkv, int Lcap,
+                                                 int bs, int blk, int r) {
+  if (!pt.table) return (((int64_t)b * Hkv + h) * Lcap + (int64_t)blk * bs + r) * kHeadDim;
+  const int page = __ldg(pt.table + (int64_t)b * pt.max_blocks + blk);
+  if (page < 0 || page >= pt.num_pages) return -1;
+  return (((int64_t)page * Hkv + h) * bs + r) * kHeadDim;
+}
+
 // ---------------------------------------------------------- launch params
 struct MeansBuildParams {
-  const __nv_bfloat16* k_cache;
+  const __nv_bfloat16* k_cache;  // contiguous cache or page pool (see PageTable)
   const int32_t* seq_lens;
   float* means;
   int32_t* dev_status;
+  PageTable pages;
   int B, Hkv, Lcap, bs, nbcap;
 };
 
@@ -124,6 +146,7 @@ struct MeansUpdateParams {
   const __nv_bfloat16* k_new;
   const __nv_bfloat16* v_new;
   int32_t* dev_status;
+  PageTable pages;
   int B, Hkv, Lcap, bs, nbcap, n_new;
 };
 
@@ -151,6 +174,7 @@ struct AttnParams {
   float* partials;      // workspace [B*Hkv][max_chunks][g][kPartStride]
   uint32_t* counters;   // workspace [B*Hkv], zero between calls
   int32_t* dev_status;
+  PageTable pages;
   int B, Hkv, Hq, g, bs, Lcap, k, chunk_blocks, max_chunks;
   float scale_log2;     // softmax_scale * log2(e)
 };

@@ -9,6 +9,9 @@
 //
 // Layout: one warp per block; lane l owns dims 4l..4l+3, so every cache row is
 // one coalesced 256-byte warp load and every mean one 512-byte warp store.
+// K/V rows are addressed through kv_row_offset, so the same kernels serve
+// the contiguous cache and the paged pool (a block's rows are contiguous in
+// both).
 #include "kin_internal.cuh"
 
 namespace kin {
@@ -40,7 +43,12 @@ __global__ void __launch_bounds__(256) means_build_kernel(MeansBuildParams p) {
   const int64_t pair = (int64_t)b * p.Hkv + h;
   const int t0 = i * p.bs;
   const int t1 = min(t0 + p.bs, L);
-  const uint2* src = reinterpret_cast<const uint2*>(p.k_cache + (pair * p.Lcap + t0) * kHeadDim) + lane;
+  const int64_t base = kv_row_offset(p.pages, b, h, p.Hkv, p.Lcap, p.bs, i, 0);  // the block's rows are contiguous
+  if (base < 0) {  // page index outside the pool: block skipped
+    if (lane == 0) set_status(p.dev_status, KIN_ERR_DEVICE_DATA);
+    return;
+  }
+  const uint2* src = reinterpret_cast<const uint2*>(p.k_cache + base) + lane;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   int t = t0;
   for (; t + 8 <= t1; t += 8) {  // 8 rows in flight per lane
@@ -76,15 +84,21 @@ __global__ void __launch_bounds__(kUpdThreads) means_update_kernel(MeansUpdatePa
     return;
   }
   const int L1 = L0 + n;
-  // 1. copy the new rows into the caches (16-byte chunks, 16 per row)
+  // 1. copy the new rows into the caches (16-byte chunks, 16 per row); a row
+  //    whose page index lies outside the pool is skipped and flagged
   const int64_t chunks = (int64_t)p.Hkv * n * (kHeadDim / 8);
   for (int64_t c = threadIdx.x; c < chunks; c += blockDim.x) {
     const int h = (int)(c / ((int64_t)n * 16));
     const int64_t rem = c - (int64_t)h * n * 16;
     const int r = (int)(rem / 16), q16 = (int)(rem % 16);
-    const int64_t pair = (int64_t)b * p.Hkv + h;
+    const int t = L0 + r;
+    const int64_t row = kv_row_offset(p.pages, b, h, p.Hkv, p.Lcap, p.bs, t / p.bs, t % p.bs);
+    if (row < 0) {
+      set_status(p.dev_status, KIN_ERR_DEVICE_DATA);
+      continue;
+    }
     const int64_t src = (((int64_t)b * p.Hkv + h) * n + r) * 16 + q16;
-    const int64_t dst = (pair * p.Lcap + L0 + r) * 16 + q16;
+    const int64_t dst = row / 8 + q16;
     reinterpret_cast<uint4*>(p.k_cache)[dst] = reinterpret_cast<const uint4*>(p.k_new)[src];
     reinterpret_cast<uint4*>(p.v_cache)[dst] = reinterpret_cast<const uint4*>(p.v_new)[src];
   }
@@ -101,14 +115,19 @@ __global__ void __launch_bounds__(kUpdThreads) means_update_kernel(MeansUpdatePa
     const int h = task / nblk, i = first + task % nblk;
     const int64_t pair = (int64_t)b * p.Hkv + h;
     const int t0 = i * p.bs, t1 = min(t0 + p.bs, L1);
-    const uint8_t* cache = reinterpret_cast<const uint8_t*>(p.k_cache + pair * p.Lcap * kHeadDim);
+    const int64_t base = kv_row_offset(p.pages, b, h, p.Hkv, p.Lcap, p.bs, i, 0);  // rows contiguous
+    if (base < 0) {  // page index outside the pool: this block's mean is left as it was
+      if (lane == 0) set_status(p.dev_status, KIN_ERR_DEVICE_DATA);
+      continue;
+    }
+    const uint8_t* cache = reinterpret_cast<const uint8_t*>(p.k_cache + base);  // row t0 of block i
     const uint8_t* fresh = reinterpret_cast<const uint8_t*>(p.k_new + pair * n * kHeadDim);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     for (int t = t0; t < t1; t += kUpdRows) {
       const int nrows = min(kUpdRows, t1 - t);
       for (int c = lane; c < nrows * 16; c += 32) {  // 16 pieces of 16 bytes per row
         const int r = t + (c >> 4), piece = c & 15;
-        const uint8_t* src = r < L0 ? cache + (int64_t)r * kRowBytes : fresh + (int64_t)(r - L0) * kRowBytes;
+        const uint8_t* src = r < L0 ? cache + (int64_t)(r - t0) * kRowBytes : fresh + (int64_t)(r - L0) * kRowBytes;
         cp_async16(rows_s + (uint32_t)(c * 16), src + piece * 16, 16u);
       }
       cp_async_commit();

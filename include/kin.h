@@ -148,6 +148,43 @@ kin_status kin_sparse_decode_attn(const kin_dims* dims, const void* q, const voi
                                   void* stream);
 
 /* ------------------------------------------------------------------------
+ * Paged KV cache.  Ragged, growing decode batches are served from a pool of
+ * fixed-size pages ("Kinetics: Rethinking Test-Time Scaling Law", response
+ * Q3: the FlashInfer backend partitions ragged lengths into pages).  Here a
+ * page is one KV block (page size = dims.block_size):
+ *     k_pages, v_pages  [num_pages][Hkv][bs][D]  bf16  (a head's rows of a
+ *                       page are contiguous: 4 KB at bs 16)
+ *     block_table       [B][NBcap] int32, NBcap = ceil(dims.max_seq_len / bs);
+ *                       block_table[b][i] is the page holding logical block
+ *                       i (tokens i*bs .. i*bs+bs-1) of sequence b.
+ * Only the entries of blocks a call touches are read: blocks below
+ * ceil(seq_len / bs) (and, for an append, the blocks the new tokens land
+ * in, which the caller must have mapped beforehand).  Block means stay in
+ * the logical layout [B][Hkv][NBcap][D], so kin_block_topk_select and its
+ * workspace serve both layouts unchanged, and every result equals the
+ * contiguous call's on the same logical cache, bit for bit.
+ * A page index outside [0, num_pages) is device-only bad data: the block (or
+ * tile, or appended row) is skipped and KIN_ERR_DEVICE_DATA is flagged.
+ * num_pages < 1 or a NULL table is KIN_ERR_INVALID_ARG.  Everything else,
+ * including dims.max_seq_len (the per-sequence capacity), is as in the
+ * contiguous calls above. */
+kin_status kin_block_means_build_paged(const kin_dims* dims, const void* k_pages, int32_t num_pages,
+                                       const int32_t* block_table, const int32_t* seq_lens,
+                                       float* block_means, int32_t* dev_status, void* stream);
+
+kin_status kin_block_means_update_paged(const kin_dims* dims, void* k_pages, void* v_pages,
+                                        int32_t num_pages, const int32_t* block_table, float* block_means,
+                                        int32_t* seq_lens, const void* k_new, const void* v_new,
+                                        int32_t n_new, int32_t* dev_status, void* stream);
+
+kin_status kin_sparse_decode_attn_paged(const kin_dims* dims, const void* q, const void* k_pages,
+                                        const void* v_pages, int32_t num_pages, const int32_t* block_table,
+                                        const int32_t* seq_lens, const int32_t* sel_idx,
+                                        const int32_t* sel_cnt, int32_t k_blocks, float softmax_scale,
+                                        void* out, float* lse, void* workspace, size_t ws_bytes,
+                                        int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------
  * Allocation-free variant of kin_block_topk_select (the pages describe no
  * counterpart; it exists for callers, not for the method).
  *

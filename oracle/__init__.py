@@ -181,3 +181,18 @@ def decode_pairs(*, Hkv, Hq, bs, seq_lens, q, Kc, Vc, means, k, scale, pairs, th
     if sc is not None:
         res["scores"] = sc
     return res
+
+
+def gather_paged(pages: np.ndarray, table_row: np.ndarray, L: int, bs: int, h: int) -> np.ndarray:
+    """Logical rows [L, D] of KV head h of one sequence held in a page pool.
+
+    pages [num_pages, Hkv, bs, D]; table_row [>= ceil(L / bs)]: token t lives
+    in page table_row[t // bs] at row t % bs.  A paged KV cache stores a
+    ragged batch in fixed-size pages ("Kinetics: Rethinking Test-Time Scaling
+    Law", response Q3); here the page is one KV block.  Plain indexing, no
+    arithmetic: attention over a paged cache is the oracle's attention over
+    the rows this returns.
+    """
+    nb = -(-L // bs)
+    blocks = [pages[int(table_row[i]), h] for i in range(nb)]
+    return np.concatenate(blocks, axis=0)[:L] if nb else pages[:0, h].reshape(0, pages.shape[-1])

@@ -187,3 +187,66 @@ def sample_pairs(w: ki.Workload, n: int):
     P = w.B * w.Hkv
     idx = sorted(set([0, P - 1] + [int(round(i * (P - 1) / max(n - 1, 1))) for i in range(n)]))
     return [(p // w.Hkv, p % w.Hkv) for p in idx]
+
+
+# ------------------------------------------------------------- paged KV cache
+@dataclass
+class Pages:
+    k: torch.Tensor          # [num_pages, Hkv, bs, D] bf16
+    v: torch.Tensor
+    table: torch.Tensor      # [B, nbcap] int32 (device); -1 where unmapped
+    table_host: np.ndarray
+    num_pages: int
+
+
+def to_pages(dc: DeviceCase, seed: int = 0, spare: int = 3) -> Pages:
+    """The case's (pre-append) contiguous cache copied into a shuffled page
+    pool: every block a sequence will hold after its append gets a page, in a
+    random order, plus `spare` unused pages; unused rows are NaN."""
+    w = dc.w
+    B, Hkv, cap, D = dc.k_cache.shape
+    bs, nbcap = w.bs, w.nbcap
+    nbs = [-(-int(L) // bs) for L in dc.lens_final]
+    total = sum(nbs)
+    P = total + spare
+    order = np.random.default_rng(seed).permutation(P)
+    table = np.full((B, nbcap), -1, np.int32)
+    j = 0
+    for b in range(B):
+        for i in range(nbs[b]):
+            table[b, i] = order[j]
+            j += 1
+    ib, ii = np.nonzero(table >= 0)
+    dst = torch.from_numpy(table[ib, ii].astype(np.int64)).cuda()
+    tb, ti = torch.from_numpy(ib).cuda(), torch.from_numpy(ii).cuda()
+    pools = []
+    for cache in (dc.k_cache, dc.v_cache):
+        padded = torch.nn.functional.pad(cache, (0, 0, 0, nbcap * bs - cap))
+        blocks = padded.view(B, Hkv, nbcap, bs, D)
+        pool = torch.full((P, Hkv, bs, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+        pool[dst] = blocks[tb, :, ti]
+        pools.append(pool)
+    return Pages(pools[0], pools[1], torch.from_numpy(table).cuda(), table, P)
+
+
+def gpu_step_paged(dc: DeviceCase, pg: Pages, k: int, seq_lens: torch.Tensor, means: torch.Tensor,
+                   ws: torch.Tensor | None = None) -> GpuResult:
+    """The paged path: means build (+ append), select, attention over pages."""
+    w = dc.w
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kin.kin_block_means_build_paged(dc.dims, pg.k, pg.table, seq_lens, means, st)
+    if w.n_append:
+        kin.kin_block_means_update_paged(dc.dims, pg.k, pg.v, pg.table, means, seq_lens, dc.k_new, dc.v_new,
+                                         w.n_append, st)
+    if ws is None:
+        ws = kin.alloc_workspace(dc.dims, k)
+    sel = torch.empty((w.B, w.Hkv, k), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((w.B, w.Hkv), dtype=torch.int32, device="cuda")
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
+    kin.kin_block_topk_select(dc.dims, dc.q, means, seq_lens, k, sel, cnt, ws, st)
+    kin.kin_sparse_decode_attn_paged(dc.dims, dc.q, pg.k, pg.v, pg.table, seq_lens, sel, cnt, k, 0.0, out, lse,
+                                     ws, st)
+    torch.cuda.synchronize()
+    return GpuResult(sel.cpu().numpy(), cnt.cpu().numpy(), out.float().cpu().numpy(), lse.cpu().numpy(),
+                     int(st.item()))

@@ -114,6 +114,36 @@ def test_means_calls_reject_before_launch(lib):
     assert lib.kin_block_means_build(ctypes.byref(dims(bs=8)), FAKE, FAKE, FAKE, None, None) == 1
 
 
+def test_paged_calls_reject_before_launch(lib):
+    d = dims()
+    bd = ctypes.byref(d)
+    # build: pool, table, page count, means
+    assert lib.kin_block_means_build_paged(bd, None, 4, FAKE, FAKE, FAKE, None, None) == 1
+    assert lib.kin_block_means_build_paged(bd, FAKE, 0, FAKE, FAKE, FAKE, None, None) == 1
+    assert lib.kin_block_means_build_paged(bd, FAKE, 4, None, FAKE, FAKE, None, None) == 1
+    assert lib.kin_block_means_build_paged(bd, ctypes.c_void_p((1 << 20) + 8), 4, FAKE, FAKE, FAKE, None,
+                                           None) == 1
+    assert lib.kin_block_means_build_paged(bd, FAKE, 4, FAKE, FAKE, None, None, None) == 1
+    # update: counts first (as the contiguous call), then the pool and table
+    up = lambda n, pool=FAKE, pages=4, table=FAKE: lib.kin_block_means_update_paged(
+        bd, pool, FAKE, pages, table, FAKE, FAKE, FAKE, FAKE, n, None, None)
+    assert up(-1) == 1
+    assert up(257) == 3
+    assert up(0, pool=None) == 0
+    assert up(1, pages=0) == 1
+    assert up(1, table=None) == 1
+    assert up(1, pool=None) == 1
+    # attention: pool and table, then the checks of the contiguous call
+    at = lambda pages=4, table=FAKE, k=8, ws=FAKE, n=1 << 30: lib.kin_sparse_decode_attn_paged(
+        bd, FAKE, FAKE, FAKE, pages, table, FAKE, FAKE, FAKE, k, 0.0, FAKE, None, ws, n, None, None)
+    assert at(pages=0) == 1
+    assert at(pages=-3) == 1
+    assert at(table=None) == 1
+    assert at(k=1) == 1
+    assert at(ws=None) == 2
+    assert at(n=64) == 2
+
+
 def test_binding_refuses_host_tensors(lib):
     import torch
     with pytest.raises(ValueError):

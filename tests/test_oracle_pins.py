@@ -263,3 +263,28 @@ def test_planted_block_is_selected_and_dominates():
     assert c == k and planted in sel
     out, _ = oracle.attend(q[:1], K, V, L, bs, sel, 1 / math.sqrt(D))
     np.testing.assert_allclose(out[0], f64(V[planted * bs:(planted + 1) * bs]).mean(axis=0), atol=1e-12)
+
+
+def test_gather_paged_follows_the_block_table():
+    """Token t of a paged sequence is row t % bs of page table[t // bs]: a
+    hand-made pool whose rows carry (page, row) markers, an identity layout,
+    and a shuffled pool that must give back the contiguous rows."""
+    bs, Hkv, D = 4, 2, 3
+    pool = np.zeros((5, Hkv, bs, D), np.int32)
+    for pg in range(5):
+        for h in range(Hkv):
+            for r in range(bs):
+                pool[pg, h, r] = (pg, h, r)
+    table = np.array([3, 0, 4], np.int32)
+    got = oracle.gather_paged(pool, table, 10, bs, 1)
+    assert got.shape == (10, D)
+    for t in range(10):
+        assert tuple(got[t]) == (table[t // bs], 1, t % bs)
+    rng = np.random.default_rng(3)
+    cont = rng.integers(0, 1 << 16, size=(Hkv, 12, D)).astype(np.uint16)  # 3 blocks of bs 4
+    ident = cont.reshape(Hkv, 3, bs, D).transpose(1, 0, 2, 3)
+    assert np.array_equal(oracle.gather_paged(ident, np.arange(3), 11, bs, 1), cont[1, :11])
+    perm = rng.permutation(6)[:3]
+    shuffled = np.zeros((6, Hkv, bs, D), np.uint16)
+    shuffled[perm] = ident
+    assert np.array_equal(oracle.gather_paged(shuffled, perm, 12, bs, 0), cont[0])
