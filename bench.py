@@ -40,6 +40,7 @@ import kin_inputs as ki  # noqa: E402
 DEFAULT_WORKLOAD = "qwen3_8b_32k"
 METRIC = "block-top-k decode attn query-heads/s"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 L2_FLUSH_BYTES = 256 << 20  # > 2x the 126 MB L2
 KERNEL_REPEATS = 4  # back-to-back calls per per-kernel timing graph
 
@@ -62,6 +63,35 @@ def algorithmic_bytes(w: ki.Workload, k: int, lens: np.ndarray):
     kv = int((w.Hkv * toks * w.D * 2 * 2).sum())
     attn_bytes = kv + q_bytes + w.B * w.Hq * w.D * 2 + idx_bytes
     return sel_bytes, attn_bytes
+
+
+def measured_bf16_peak():
+    """Dense bf16 FLOP/s: the measured burst figure, else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]) * 1e12, "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS * 1e12, "fallback"
+
+
+def eflops_report(w, k, lens, ms_per_step):
+    """The eFLOPs model's predicted step time (T = A/C + M/B) beside the
+    measured one, with the measured B200 peaks as C and B."""
+    from block_top_sparse_kin_b200 import eflops as ef
+    parts = ef.step_costs(w.B, w.Hkv, w.Hq, w.D, w.bs, lens, k, w.n_append)
+    tot = ef.Cost(0.0, 0.0)
+    for c in parts.values():
+        tot = tot + c
+    C, c_kind = measured_bf16_peak()
+    Bw, b_kind = measured_peak()
+    r = ef.eflops(tot, C, Bw * 1e9)
+    r["t_meas_us"] = ms_per_step * 1e3
+    r["meas_over_pred"] = r["t_meas_us"] / r["t_pred_us"]
+    r["C_flops"] = C
+    r["B_bytes_s"] = Bw * 1e9
+    r["peaks"] = f"C = dense bf16 ({c_kind}), B = HBM copy ({b_kind})"
+    return r
 
 
 def measured_peak():
@@ -521,6 +551,7 @@ def gpu_arm(args):
             },
             "e2e": {"value": e2e_value, "unit": "query-heads/s",
                     "h2d_bytes_per_step": int(q_pin.numel() * 2), "d2h_bytes_per_step": int(out_pin.numel() * 2)},
+            "eflops": eflops_report(w, k, st["lens_final"], ms_per_step),  # this rank's shard
             "clocks": clk.summary(),
             "wall_s_timed_region": wall,
             "device_status": status,
