@@ -46,7 +46,7 @@ KERNEL_REPEATS = 4  # back-to-back calls per per-kernel timing graph
 
 
 # ---------------------------------------------------------------- bytes model
-def algorithmic_bytes(w: ki.Workload, k: int, lens: np.ndarray):
+def algorithmic_bytes(w: ki.Workload, k: int, lens: np.ndarray, means_bytes: int = 4):
     """Algorithmic HBM bytes per launch: (select, attention).
 
     select: fp32 means of every block (skipped when k >= nb), q, indices.
@@ -54,7 +54,7 @@ def algorithmic_bytes(w: ki.Workload, k: int, lens: np.ndarray):
     """
     nb = -(-lens.astype(np.int64) // w.bs)
     scan = nb > k
-    means = int((w.Hkv * nb[scan] * w.D * 4).sum())
+    means = int((w.Hkv * nb[scan] * w.D * means_bytes).sum())
     q_bytes = w.B * w.Hq * w.D * 2
     idx_bytes = w.B * w.Hkv * k * 4
     sel_bytes = means + q_bytes + idx_bytes
@@ -75,11 +75,11 @@ def measured_bf16_peak():
         return FALLBACK_BF16_TFLOPS * 1e12, "fallback"
 
 
-def eflops_report(w, k, lens, ms_per_step):
+def eflops_report(w, k, lens, ms_per_step, means_bytes=4):
     """The eFLOPs model's predicted step time (T = A/C + M/B) beside the
     measured one, with the measured B200 peaks as C and B."""
     from block_top_sparse_kin_b200 import eflops as ef
-    parts = ef.step_costs(w.B, w.Hkv, w.Hq, w.D, w.bs, lens, k, w.n_append)
+    parts = ef.step_costs(w.B, w.Hkv, w.Hq, w.D, w.bs, lens, k, w.n_append, means_bytes)
     tot = ef.Cost(0.0, 0.0)
     for c in parts.values():
         tot = tot + c
@@ -261,7 +261,7 @@ def make_page_pool(st, seed: int):
     torch.cuda.empty_cache()
 
 
-def build_device_state(w: ki.Workload, k: int, paged: bool = False):
+def build_device_state(w: ki.Workload, k: int, paged: bool = False, means_bf16: bool = False):
     import torch
     import block_top_sparse_kin_b200 as kin
     lens_final, lens_pre, hh = ki.case_meta(w)
@@ -277,8 +277,12 @@ def build_device_state(w: ki.Workload, k: int, paged: bool = False):
     ki.kv_cache_device(w.seed, True, w.B, w.Hkv, w.cap, w.D, w.bs, st["seq"], hh_dev, False, kc)
     ki.kv_cache_device(w.seed, False, w.B, w.Hkv, w.cap, w.D, w.bs, st["seq"], hh_dev, False, vc)
     st["k_cache"], st["v_cache"] = kc, vc
-    st["means"] = torch.zeros((w.B, w.Hkv, w.nbcap, w.D), dtype=torch.float32, device="cuda")
-    kin.kin_block_means_build(dims, kc, st["seq"], st["means"])
+    st["means"] = torch.zeros((w.B, w.Hkv, w.nbcap, w.D), dtype=torch.bfloat16 if means_bf16 else torch.float32,
+                              device="cuda")
+    if means_bf16:
+        kin.kin_block_means_build_ex(dims, kc, st["seq"], st["means"])
+    else:
+        kin.kin_block_means_build(dims, kc, st["seq"], st["means"])
     if w.n_append:
         kn = np.empty((w.B, w.Hkv, w.n_append, w.D), np.uint16)
         vn = np.empty_like(kn)
@@ -303,28 +307,48 @@ def build_device_state(w: ki.Workload, k: int, paged: bool = False):
 
 def run_step(st, ev=None):
     """One decode step.  ev: optional list of 3 or 4 events to record between kernels."""
-    import block_top_sparse_kin_b200 as kin
-    w, dims, k = st["w"], st["dims"], st["k"]
+    w = st["w"]
     i = 0
     if ev is not None:
         ev[i].record(); i += 1
-    paged = "table" in st
     if w.n_append:
-        if paged:
-            kin.kin_block_means_update_paged(dims, st["k_pages"], st["v_pages"], st["table"], st["means"],
-                                             st["seq"], st["k_new"], st["v_new"], w.n_append, st["status"])
-        else:
-            kin.kin_block_means_update(dims, st["k_cache"], st["v_cache"], st["means"], st["seq"],
-                                       st["k_new"], st["v_new"], w.n_append, st["status"])
+        append(st)
         if ev is not None:
             ev[i].record(); i += 1
-    kin.kin_block_topk_select(dims, st["q"], st["means"], st["seq"], k, st["sel"], st["cnt"], st["ws"],
-                              st["status"])
+    select(st)
     if ev is not None:
         ev[i].record(); i += 1
     attend(st)
     if ev is not None:
         ev[i].record()
+
+
+def append(st):
+    """The step's append: n new tokens per sequence, touched block means refreshed."""
+    import block_top_sparse_kin_b200 as kin
+    w = st["w"]
+    paged = "table" in st
+    k_rows, v_rows = (st["k_pages"], st["v_pages"]) if paged else (st["k_cache"], st["v_cache"])
+    if str(st["means"].dtype) == "torch.bfloat16":
+        kin.kin_block_means_update_ex(st["dims"], k_rows, v_rows, st["means"], st["seq"], st["k_new"], st["v_new"],
+                                      w.n_append, block_table=st.get("table"), dev_status=st["status"])
+    elif paged:
+        kin.kin_block_means_update_paged(st["dims"], k_rows, v_rows, st["table"], st["means"], st["seq"],
+                                         st["k_new"], st["v_new"], w.n_append, st["status"])
+    else:
+        kin.kin_block_means_update(st["dims"], k_rows, v_rows, st["means"], st["seq"], st["k_new"], st["v_new"],
+                                   w.n_append, st["status"])
+
+
+def select(st):
+    """The step's block scoring and top-k (fp32 means, or bf16 through the extended call)."""
+    import block_top_sparse_kin_b200 as kin
+    if str(st["means"].dtype) == "torch.bfloat16":
+        kin.kin_block_topk_select_ex(st["dims"], st["q"], st["means"], st["seq"], st["k"], st["sel"], st["cnt"],
+                                     st["ws"], st["status"])
+    else:
+        kin.kin_block_topk_select(st["dims"], st["q"], st["means"], st["seq"], st["k"], st["sel"], st["cnt"],
+                                  st["ws"], st["status"])
 
 
 def attend(st):
@@ -353,7 +377,7 @@ def gpu_arm(args):
         w0 = w0.with_(B=args.batch, name=f"{w0.name}_b{args.batch}")
     k = args.k or w0.k
     w = shard_workload(w0, rank)
-    st = build_device_state(w, k, paged=args.paged)
+    st = build_device_state(w, k, paged=args.paged, means_bf16=args.means_bf16)
     flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
 
@@ -387,8 +411,7 @@ def gpu_arm(args):
     import block_top_sparse_kin_b200 as kin
 
     def call_select():
-        kin.kin_block_topk_select(st["dims"], st["q"], st["means"], st["seq"], k, st["sel"], st["cnt"],
-                                  st["ws"], st["status"])
+        select(st)
 
     def call_attn():
         attend(st)
@@ -428,13 +451,7 @@ def gpu_arm(args):
             with torch.cuda.graph(upd_graph, stream=cap):
                 reset_state(st)
                 upd_ev[0].record()
-                if "table" in st:
-                    kin.kin_block_means_update_paged(st["dims"], st["k_pages"], st["v_pages"], st["table"],
-                                                     st["means"], st["seq"], st["k_new"], st["v_new"],
-                                                     w.n_append, st["status"])
-                else:
-                    kin.kin_block_means_update(st["dims"], st["k_cache"], st["v_cache"], st["means"],
-                                               st["seq"], st["k_new"], st["v_new"], w.n_append, st["status"])
+                append(st)
                 upd_ev[1].record()
     torch.cuda.current_stream().wait_stream(cap)
     diag = [g for g in (sel_graph, attn_graph, upd_graph) if g is not None]
@@ -505,7 +522,7 @@ def gpu_arm(args):
     status = int(st["status"].item())
 
     if rank == 0:
-        sel_b, attn_b = algorithmic_bytes(w, k, st["lens_final"])
+        sel_b, attn_b = algorithmic_bytes(w, k, st["lens_final"], 2 if args.means_bf16 else 4)
         peak, peak_kind = measured_peak()
         sel_avg = statistics.mean(sel_ms)
         attn_avg = statistics.mean(attn_ms)
@@ -536,6 +553,7 @@ def gpu_arm(args):
                 "l2": "flushed before every step (256 MiB write + 256 MiB read, outside the timed events)",
                 "kv_layout": (f"paged: {st['num_pages']} pages of one {w.bs}-token block, shuffled pool + block table"
                               if args.paged else "contiguous [B][Hkv][Lcap][D]"),
+                "block_means": "bf16" if args.means_bf16 else "fp32",
             },
             "impl": "kin",
             "gpu_launches": launches_per_step * args.steps,  # in the timed region
@@ -551,7 +569,7 @@ def gpu_arm(args):
             },
             "e2e": {"value": e2e_value, "unit": "query-heads/s",
                     "h2d_bytes_per_step": int(q_pin.numel() * 2), "d2h_bytes_per_step": int(out_pin.numel() * 2)},
-            "eflops": eflops_report(w, k, st["lens_final"], ms_per_step),  # this rank's shard
+            "eflops": eflops_report(w, k, st["lens_final"], ms_per_step, 2 if args.means_bf16 else 4),
             "clocks": clk.summary(),
             "wall_s_timed_region": wall,
             "device_status": status,
@@ -671,6 +689,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-pairs", type=int, default=8, help="pairs per reference-arm step")
     ap.add_argument("--paged", action="store_true", help="KV cache in a shuffled page pool with a block table")
+    ap.add_argument("--means-bf16", action="store_true", help="bf16 block means (the extended calls)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "kin":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

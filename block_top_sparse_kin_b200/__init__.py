@@ -27,8 +27,10 @@ EXPORTED = (
     "kin_status_string", "kin_workspace_bytes", "kin_block_means_build",
     "kin_block_means_update", "kin_block_topk_select", "kin_sparse_decode_attn",
     "kin_block_topk_select_noalloc", "kin_block_means_build_paged", "kin_block_means_update_paged",
-    "kin_sparse_decode_attn_paged",
+    "kin_sparse_decode_attn_paged", "kin_block_means_build_ex", "kin_block_means_update_ex",
+    "kin_block_topk_select_ex",
 )
+KIN_MEANS_F32, KIN_MEANS_BF16 = 0, 1
 NOALLOC_SCRATCH_FLOATS = 1 << 21  # KIN_NOALLOC_SCRATCH_FLOATS in include/kin.h
 
 
@@ -93,6 +95,12 @@ def load_library(path: str = LIB_PATH):
     lib.kin_sparse_decode_attn_paged.argtypes = [dp, vp, vp, vp, i32, vp, vp, vp, vp, i32, f32, vp, vp, vp,
                                                  sz, vp, vp]
     lib.kin_sparse_decode_attn_paged.restype = ctypes.c_int
+    lib.kin_block_means_build_ex.argtypes = [dp, vp, i32, vp, vp, vp, i32, vp, vp]
+    lib.kin_block_means_build_ex.restype = ctypes.c_int
+    lib.kin_block_means_update_ex.argtypes = [dp, vp, vp, i32, vp, vp, i32, vp, vp, vp, i32, vp, vp]
+    lib.kin_block_means_update_ex.restype = ctypes.c_int
+    lib.kin_block_topk_select_ex.argtypes = [dp, vp, vp, i32, vp, i32, vp, vp, vp, sz, vp, vp]
+    lib.kin_block_topk_select_ex.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -232,3 +240,52 @@ def kin_sparse_decode_attn_paged(dims, q, k_pages, v_pages, block_table, seq_len
         workspace.numel() * workspace.element_size(),
         _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
     _check(rc, "kin_sparse_decode_attn_paged")
+
+
+# ------------------------------------------------ extended: bf16 block means
+# The means dtype follows the block_means tensor (float32 or bfloat16);
+# block_table None selects the contiguous cache.  See include/kin.h.
+
+def _means(block_means):
+    if block_means.dtype == torch.float32:
+        return _dev(block_means, "block_means", torch.float32), KIN_MEANS_F32
+    return _dev(block_means, "block_means", torch.bfloat16), KIN_MEANS_BF16
+
+
+def _layout(rows, block_table):
+    if block_table is None:
+        return 0, None
+    return int(rows.shape[0]), _dev(block_table, "block_table", torch.int32)
+
+
+def kin_block_means_build_ex(dims, k_rows, seq_lens, block_means, block_table=None, dev_status=None,
+                             stream=None):
+    pages, table = _layout(k_rows, block_table)
+    means, dtype = _means(block_means)
+    rc = load_library().kin_block_means_build_ex(
+        ctypes.byref(dims), _dev(k_rows, "k_rows", _BF16), pages, table, _dev(seq_lens, "seq_lens", torch.int32),
+        means, dtype, _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+    _check(rc, "kin_block_means_build_ex")
+
+
+def kin_block_means_update_ex(dims, k_rows, v_rows, block_means, seq_lens, k_new, v_new, n_new,
+                              block_table=None, dev_status=None, stream=None):
+    pages, table = _layout(k_rows, block_table)
+    means, dtype = _means(block_means)
+    rc = load_library().kin_block_means_update_ex(
+        ctypes.byref(dims), _dev(k_rows, "k_rows", _BF16), _dev(v_rows, "v_rows", _BF16), pages, table,
+        means, dtype, _dev(seq_lens, "seq_lens", torch.int32), _dev(k_new, "k_new", _BF16),
+        _dev(v_new, "v_new", _BF16), int(n_new), _dev(dev_status, "dev_status", torch.int32, nullable=True),
+        _stream(stream))
+    _check(rc, "kin_block_means_update_ex")
+
+
+def kin_block_topk_select_ex(dims, q, block_means, seq_lens, k_blocks, sel_idx, sel_cnt, workspace,
+                             dev_status=None, stream=None):
+    means, dtype = _means(block_means)
+    rc = load_library().kin_block_topk_select_ex(
+        ctypes.byref(dims), _dev(q, "q", _BF16), means, dtype, _dev(seq_lens, "seq_lens", torch.int32),
+        int(k_blocks), _dev(sel_idx, "sel_idx", torch.int32), _dev(sel_cnt, "sel_cnt", torch.int32),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+    _check(rc, "kin_block_topk_select_ex")

@@ -160,11 +160,12 @@ KIN_EXPORT size_t kin_workspace_bytes(const kin_dims* dims, int32_t k_blocks) {
 namespace {
 
 kin_status means_build(const kin_dims* dims, const void* k_rows, const PageTable& pt, const int32_t* seq_lens,
-                       float* block_means, int32_t* dev_status, void* stream) {
+                       void* block_means, int means_bf16, int32_t* dev_status, void* stream) {
   MeansBuildParams p;
   p.k_cache = static_cast<const __nv_bfloat16*>(k_rows);
   p.seq_lens = seq_lens;
   p.means = block_means;
+  p.means_bf16 = means_bf16;
   p.dev_status = dev_status;
   p.pages = pt;
   p.B = dims->batch;
@@ -176,12 +177,13 @@ kin_status means_build(const kin_dims* dims, const void* k_rows, const PageTable
 }
 
 kin_status means_update(const kin_dims* dims, void* k_rows, void* v_rows, const PageTable& pt,
-                        float* block_means, int32_t* seq_lens, const void* k_new, const void* v_new,
-                        int32_t n_new, int32_t* dev_status, void* stream) {
+                        void* block_means, int means_bf16, int32_t* seq_lens, const void* k_new,
+                        const void* v_new, int32_t n_new, int32_t* dev_status, void* stream) {
   MeansUpdateParams p;
   p.k_cache = static_cast<__nv_bfloat16*>(k_rows);
   p.v_cache = static_cast<__nv_bfloat16*>(v_rows);
   p.means = block_means;
+  p.means_bf16 = means_bf16;
   p.seq_lens = seq_lens;
   p.k_new = static_cast<const __nv_bfloat16*>(k_new);
   p.v_new = static_cast<const __nv_bfloat16*>(v_new);
@@ -202,7 +204,7 @@ kin_status check_update_count(const kin_dims* dims, int32_t n_new) {
   return KIN_OK;
 }
 
-kin_status check_update_args(const void* k_rows, const void* v_rows, const float* block_means,
+kin_status check_update_args(const void* k_rows, const void* v_rows, const void* block_means,
                              const int32_t* seq_lens, const void* k_new, const void* v_new) {
   if (!k_rows || !v_rows || !block_means || !seq_lens || !k_new || !v_new) return KIN_ERR_INVALID_ARG;
   if (!aligned16(k_rows) || !aligned16(v_rows) || !aligned16(block_means) || !aligned16(k_new) ||
@@ -220,7 +222,7 @@ KIN_EXPORT kin_status kin_block_means_build(const kin_dims* dims, const void* k_
   if (st != KIN_OK) return st;
   if (!k_cache || !seq_lens || !block_means) return KIN_ERR_INVALID_ARG;
   if (!aligned16(k_cache) || !aligned16(block_means)) return KIN_ERR_INVALID_ARG;
-  return means_build(dims, k_cache, contiguous(), seq_lens, block_means, dev_status, stream);
+  return means_build(dims, k_cache, contiguous(), seq_lens, block_means, 0, dev_status, stream);
 }
 
 KIN_EXPORT kin_status kin_block_means_build_paged(const kin_dims* dims, const void* k_pages, int32_t num_pages,
@@ -232,7 +234,7 @@ KIN_EXPORT kin_status kin_block_means_build_paged(const kin_dims* dims, const vo
   st = check_pages(*dims, k_pages, num_pages, block_table, &pt);
   if (st != KIN_OK) return st;
   if (!seq_lens || !block_means || !aligned16(block_means)) return KIN_ERR_INVALID_ARG;
-  return means_build(dims, k_pages, pt, seq_lens, block_means, dev_status, stream);
+  return means_build(dims, k_pages, pt, seq_lens, block_means, 0, dev_status, stream);
 }
 
 KIN_EXPORT kin_status kin_block_means_update(const kin_dims* dims, void* k_cache, void* v_cache,
@@ -245,7 +247,7 @@ KIN_EXPORT kin_status kin_block_means_update(const kin_dims* dims, void* k_cache
   if (st != KIN_OK || n_new == 0) return st;
   st = check_update_args(k_cache, v_cache, block_means, seq_lens, k_new, v_new);
   if (st != KIN_OK) return st;
-  return means_update(dims, k_cache, v_cache, contiguous(), block_means, seq_lens, k_new, v_new, n_new,
+  return means_update(dims, k_cache, v_cache, contiguous(), block_means, 0, seq_lens, k_new, v_new, n_new,
                       dev_status, stream);
 }
 
@@ -263,26 +265,26 @@ KIN_EXPORT kin_status kin_block_means_update_paged(const kin_dims* dims, void* k
   if (st != KIN_OK) return st;
   st = check_update_args(k_pages, v_pages, block_means, seq_lens, k_new, v_new);
   if (st != KIN_OK) return st;
-  return means_update(dims, k_pages, v_pages, pt, block_means, seq_lens, k_new, v_new, n_new, dev_status,
+  return means_update(dims, k_pages, v_pages, pt, block_means, 0, seq_lens, k_new, v_new, n_new, dev_status,
                       stream);
 }
 
-KIN_EXPORT kin_status kin_block_topk_select(const kin_dims* dims, const void* q, const float* block_means,
-                                            const int32_t* seq_lens, int32_t k_blocks, int32_t* sel_idx,
-                                            int32_t* sel_cnt, void* workspace, size_t ws_bytes,
-                                            int32_t* dev_status, void* stream) {
-  kin_status st = check_dims(dims);
-  if (st != KIN_OK) return st;
+namespace {
+
+kin_status topk_select(const kin_dims* dims, const void* q, const void* block_means, int means_bf16,
+                       const int32_t* seq_lens, int32_t k_blocks, int32_t* sel_idx, int32_t* sel_cnt,
+                       void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
   if (k_blocks < 2) return KIN_ERR_INVALID_ARG;
   if (!q || !block_means || !seq_lens || !sel_idx || !sel_cnt) return KIN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(block_means)) return KIN_ERR_INVALID_ARG;
   WsLayout w;
-  st = check_ws(*dims, k_blocks, workspace, ws_bytes, &w);
+  kin_status st = check_ws(*dims, k_blocks, workspace, ws_bytes, &w);
   if (st != KIN_OK) return st;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   SelectParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.means = block_means;
+  p.means_bf16 = means_bf16;
   p.seq_lens = seq_lens;
   p.sel_idx = sel_idx;
   p.sel_cnt = sel_cnt;
@@ -298,6 +300,81 @@ KIN_EXPORT kin_status kin_block_topk_select(const kin_dims* dims, const void* q,
   p.k = k_blocks;
   p.score_scale = 1.0f / std::sqrt((float)kHeadDim);
   return from_cuda(launch_select(p, static_cast<cudaStream_t>(stream)));
+}
+
+// means_dtype as a kernel flag (0 fp32, 1 bf16); -1 for an unknown value
+int means_flag(int32_t means_dtype) {
+  return means_dtype == KIN_MEANS_F32 ? 0 : means_dtype == KIN_MEANS_BF16 ? 1 : -1;
+}
+
+// A NULL table selects the contiguous cache (num_pages ignored).
+kin_status layout_of(const kin_dims& d, const void* k_rows, int32_t num_pages, const int32_t* block_table,
+                     PageTable* pt) {
+  if (!block_table) {
+    *pt = contiguous();
+    return KIN_OK;
+  }
+  return check_pages(d, k_rows, num_pages, block_table, pt);
+}
+
+}  // namespace
+
+KIN_EXPORT kin_status kin_block_topk_select(const kin_dims* dims, const void* q, const float* block_means,
+                                            const int32_t* seq_lens, int32_t k_blocks, int32_t* sel_idx,
+                                            int32_t* sel_cnt, void* workspace, size_t ws_bytes,
+                                            int32_t* dev_status, void* stream) {
+  kin_status st = check_dims(dims);
+  if (st != KIN_OK) return st;
+  return topk_select(dims, q, block_means, 0, seq_lens, k_blocks, sel_idx, sel_cnt, workspace, ws_bytes,
+                     dev_status, stream);
+}
+
+KIN_EXPORT kin_status kin_block_topk_select_ex(const kin_dims* dims, const void* q, const void* block_means,
+                                               int32_t means_dtype, const int32_t* seq_lens, int32_t k_blocks,
+                                               int32_t* sel_idx, int32_t* sel_cnt, void* workspace,
+                                               size_t ws_bytes, int32_t* dev_status, void* stream) {
+  kin_status st = check_dims(dims);
+  if (st != KIN_OK) return st;
+  const int bf = means_flag(means_dtype);
+  if (bf < 0) return KIN_ERR_INVALID_ARG;
+  return topk_select(dims, q, block_means, bf, seq_lens, k_blocks, sel_idx, sel_cnt, workspace, ws_bytes,
+                     dev_status, stream);
+}
+
+KIN_EXPORT kin_status kin_block_means_build_ex(const kin_dims* dims, const void* k_rows, int32_t num_pages,
+                                               const int32_t* block_table, const int32_t* seq_lens,
+                                               void* block_means, int32_t means_dtype, int32_t* dev_status,
+                                               void* stream) {
+  kin_status st = check_dims(dims);
+  if (st != KIN_OK) return st;
+  const int bf = means_flag(means_dtype);
+  if (bf < 0) return KIN_ERR_INVALID_ARG;
+  if (!k_rows || !seq_lens || !block_means) return KIN_ERR_INVALID_ARG;
+  if (!aligned16(k_rows) || !aligned16(block_means)) return KIN_ERR_INVALID_ARG;
+  PageTable pt;
+  st = layout_of(*dims, k_rows, num_pages, block_table, &pt);
+  if (st != KIN_OK) return st;
+  return means_build(dims, k_rows, pt, seq_lens, block_means, bf, dev_status, stream);
+}
+
+KIN_EXPORT kin_status kin_block_means_update_ex(const kin_dims* dims, void* k_rows, void* v_rows,
+                                                int32_t num_pages, const int32_t* block_table,
+                                                void* block_means, int32_t means_dtype, int32_t* seq_lens,
+                                                const void* k_new, const void* v_new, int32_t n_new,
+                                                int32_t* dev_status, void* stream) {
+  kin_status st = check_dims(dims);
+  if (st != KIN_OK) return st;
+  const int bf = means_flag(means_dtype);
+  if (bf < 0) return KIN_ERR_INVALID_ARG;
+  st = check_update_count(dims, n_new);
+  if (st != KIN_OK || n_new == 0) return st;
+  st = check_update_args(k_rows, v_rows, block_means, seq_lens, k_new, v_new);
+  if (st != KIN_OK) return st;
+  PageTable pt;
+  st = layout_of(*dims, k_rows, num_pages, block_table, &pt);
+  if (st != KIN_OK) return st;
+  return means_update(dims, k_rows, v_rows, pt, block_means, bf, seq_lens, k_new, v_new, n_new, dev_status,
+                      stream);
 }
 
 namespace {

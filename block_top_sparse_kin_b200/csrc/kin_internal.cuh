@@ -129,10 +129,24 @@ __device__ __forceinline__ int64_t kv_row_offset(const PageTable& pt, int b, int
 }
 
 // ---------------------------------------------------------- launch params
+// Block means are fp32 rows of D (the default), or bf16 rows (means_bf16:
+// each fp32 mean rounded to nearest even), [B][Hkv][nbcap][D] either way.
+__device__ __forceinline__ void store_mean_row(void* means, int means_bf16, int64_t row, int lane, float4 m) {
+  if (means_bf16) {
+    uint2 v;
+    v.x = pack_bf16x2(m.x, m.y);
+    v.y = pack_bf16x2(m.z, m.w);
+    reinterpret_cast<uint2*>(means)[row * (kHeadDim / 4) + lane] = v;
+  } else {
+    reinterpret_cast<float4*>(means)[row * (kHeadDim / 4) + lane] = m;
+  }
+}
+
 struct MeansBuildParams {
   const __nv_bfloat16* k_cache;  // contiguous cache or page pool (see PageTable)
   const int32_t* seq_lens;
-  float* means;
+  void* means;
+  int means_bf16;
   int32_t* dev_status;
   PageTable pages;
   int B, Hkv, Lcap, bs, nbcap;
@@ -141,7 +155,8 @@ struct MeansBuildParams {
 struct MeansUpdateParams {
   __nv_bfloat16* k_cache;
   __nv_bfloat16* v_cache;
-  float* means;
+  void* means;
+  int means_bf16;
   int32_t* seq_lens;
   const __nv_bfloat16* k_new;
   const __nv_bfloat16* v_new;
@@ -152,7 +167,8 @@ struct MeansUpdateParams {
 
 struct SelectParams {
   const __nv_bfloat16* q;
-  const float* means;
+  const void* means;
+  int means_bf16;
   const int32_t* seq_lens;
   int32_t* sel_idx;
   int32_t* sel_cnt;

@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(256) means_build_kernel(MeansBuildParams p) {
   const float n = (float)(t1 - t0);
   float4 m = make_float4(__fdiv_rn(acc[0], n), __fdiv_rn(acc[1], n), __fdiv_rn(acc[2], n),
                          __fdiv_rn(acc[3], n));
-  reinterpret_cast<float4*>(p.means + (pair * p.nbcap + i) * kHeadDim)[lane] = m;
+  store_mean_row(p.means, p.means_bf16, pair * p.nbcap + i, lane, m);
 }
 
 // grid (B), 256 threads.  One CTA owns a whole sequence so that the length
@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(kUpdThreads) means_update_kernel(MeansUpdatePa
     const float cnt = (float)(t1 - t0);
     float4 m = make_float4(__fdiv_rn(acc[0], cnt), __fdiv_rn(acc[1], cnt), __fdiv_rn(acc[2], cnt),
                            __fdiv_rn(acc[3], cnt));
-    reinterpret_cast<float4*>(p.means + (pair * p.nbcap + i) * kHeadDim)[lane] = m;
+    store_mean_row(p.means, p.means_bf16, pair * p.nbcap + i, lane, m);
   }
   __syncthreads();
   if (threadIdx.x == 0) p.seq_lens[b] = L1;

@@ -24,6 +24,8 @@
 // The top-k: the first block and the block holding the newest token are
 // always kept, ties go to the lower index, and the kept indices leave
 // ascending.
+#include <type_traits>
+
 #include "kin_internal.cuh"
 
 namespace kin {
@@ -601,14 +603,38 @@ __device__ __forceinline__ void pair_qsum(const SelectParams& p, int pair, int l
   }
 }
 
+// Mean rows as loaded (fp32: a float4 of 4 dims per lane; bf16: a uint2 of
+// 4 bf16 dims) and as used (4 floats).
+template <bool kBf16>
+struct MeanLane {
+  using Raw = typename std::conditional<kBf16, uint2, float4>::type;
+  static __device__ __forceinline__ Raw zero() {
+    if constexpr (kBf16) return make_uint2(0u, 0u);
+    else return make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  static __device__ __forceinline__ float4 widen(Raw r) {
+    if constexpr (kBf16) {
+      const float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&r.x));
+      const float2 b = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&r.y));
+      return make_float4(a.x, a.y, b.x, b.y);
+    } else {
+      return r;
+    }
+  }
+};
+
+// U rows per warp step: 8 fp32 rows or 16 bf16 rows, 4 KB in flight either way.
+template <bool kBf16, int U>
 __global__ void __launch_bounds__(kSelThreads, KIN_SEL_CTAS_PER_SM) select_scan_kernel(SelectParams p) {
+  using ML = MeanLane<kBf16>;
+  using Raw = typename ML::Raw;
   pdl_wait();  // means, lengths and q come from earlier work on the stream
   pdl_trigger_early();
   const int lane = threadIdx.x & 31;
   const int nwarps = gridDim.x * kSelWarps;
   const int gw = blockIdx.x * kSelWarps + (threadIdx.x >> 5);
-  const int nbp = (p.nbcap + kSelU - 1) / kSelU * kSelU;
-  const int steps = p.B * p.Hkv * (nbp / kSelU);
+  const int nbp = (p.nbcap + U - 1) / U * U;
+  const int steps = p.B * p.Hkv * (nbp / U);
   const int per = (steps + nwarps - 1) / nwarps;
   const int s0 = gw * per, s1 = min(s0 + per, steps);
   if (s0 >= s1) {
@@ -617,43 +643,42 @@ __global__ void __launch_bounds__(kSelThreads, KIN_SEL_CTAS_PER_SM) select_scan_
   }
 
   // step s covers slots s*U .. s*U+U-1 of pair (s*U) / nbp
-  int pair = (s0 * kSelU) / nbp;
-  int blk = s0 * kSelU - pair * nbp;
+  int pair = (s0 * U) / nbp;
+  int blk = s0 * U - pair * nbp;
   int nb = pair_nb(p, pair);
   float qs[4];
   pair_qsum(p, pair, lane, qs);
-  const float4* mrow = reinterpret_cast<const float4*>(p.means) + lane;
+  const Raw* mrow = reinterpret_cast<const Raw*>(p.means) + lane;
   auto row_ptr = [&](int pr, int bk) { return mrow + ((int64_t)pr * p.nbcap + bk) * (kHeadDim / 4); };
 
-  float4 cur[kSelU];
+  Raw cur[U];
 #pragma unroll
-  for (int u = 0; u < kSelU; ++u)
-    cur[u] = blk + u < nb ? __ldcs(row_ptr(pair, blk + u)) : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int u = 0; u < U; ++u) cur[u] = blk + u < nb ? __ldcs(row_ptr(pair, blk + u)) : ML::zero();
   for (int s = s0; s < s1; ++s) {
     // the next step's rows fly during this step's math
-    int npair = pair, nblk = blk + kSelU, nnb = nb;
+    int npair = pair, nblk = blk + U, nnb = nb;
     if (nblk >= nbp) {
       npair = pair + 1;
       nblk = 0;
       nnb = s + 1 < s1 ? pair_nb(p, npair) : 0;
     }
     const bool more = s + 1 < s1;
-    float4 nxt[kSelU];
+    Raw nxt[U];
 #pragma unroll
-    for (int u = 0; u < kSelU; ++u)
-      nxt[u] = more && nblk + u < nnb ? __ldcs(row_ptr(npair, nblk + u)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int u = 0; u < U; ++u) nxt[u] = more && nblk + u < nnb ? __ldcs(row_ptr(npair, nblk + u)) : ML::zero();
     if (blk < nb) {
-      float d[kSelU];
+      float d[U];
 #pragma unroll
-      for (int u = 0; u < kSelU; ++u) {
-        d[u] = qs[0] * cur[u].x;
-        d[u] = fmaf(qs[1], cur[u].y, d[u]);
-        d[u] = fmaf(qs[2], cur[u].z, d[u]);
-        d[u] = fmaf(qs[3], cur[u].w, d[u]);
+      for (int u = 0; u < U; ++u) {
+        const float4 m = ML::widen(cur[u]);
+        d[u] = qs[0] * m.x;
+        d[u] = fmaf(qs[1], m.y, d[u]);
+        d[u] = fmaf(qs[2], m.z, d[u]);
+        d[u] = fmaf(qs[3], m.w, d[u]);
       }
-      const float tot = warp_sum_rows<kSelU>(d, lane);
-      const int row = lane / (32 / kSelU);
-      if ((lane & (32 / kSelU - 1)) == 0 && blk + row < nb)
+      const float tot = warp_sum_rows<U>(d, lane);
+      const int row = lane / (32 / U);
+      if ((lane & (32 / U - 1)) == 0 && blk + row < nb)
         p.scores[(int64_t)pair * p.nbcap + blk + row] = tot * p.score_scale;
     }
     if (npair != pair && more) pair_qsum(p, npair, lane, qs);
@@ -661,7 +686,7 @@ __global__ void __launch_bounds__(kSelThreads, KIN_SEL_CTAS_PER_SM) select_scan_
     blk = nblk;
     nb = nnb;
 #pragma unroll
-    for (int u = 0; u < kSelU; ++u) cur[u] = nxt[u];
+    for (int u = 0; u < U; ++u) cur[u] = nxt[u];
   }
   pdl_trigger_late();
 }
@@ -725,10 +750,13 @@ cudaError_t launch_topk(const SelectParams& p, cudaStream_t s) {
 
 cudaError_t launch_select(const SelectParams& p, cudaStream_t s) {
   const int64_t rows = (int64_t)p.B * p.Hkv * p.nbcap;
-  const int64_t want = (rows + kSelWarps * kSelU * 4 - 1) / (kSelWarps * kSelU * 4);  // >= 4 steps per warp
+  const int u = p.means_bf16 ? 2 * kSelU : kSelU;
+  const int64_t want = (rows + kSelWarps * u * 4 - 1) / (kSelWarps * u * 4);  // >= 4 steps per warp
   const int64_t resident = (int64_t)device_sm_count() * KIN_SEL_CTAS_PER_SM;
   const int grid = (int)(want < resident ? (want > 0 ? want : 1) : resident);
-  cudaError_t e = launch_pdl(select_scan_kernel, dim3(grid), dim3(kSelThreads), 0, s, p);
+  cudaError_t e = p.means_bf16
+                      ? launch_pdl(select_scan_kernel<true, 2 * kSelU>, dim3(grid), dim3(kSelThreads), 0, s, p)
+                      : launch_pdl(select_scan_kernel<false, kSelU>, dim3(grid), dim3(kSelThreads), 0, s, p);
   if (e != cudaSuccess) return e;
   switch (topk_threads(p.nbcap, (int64_t)p.B * p.Hkv)) {
     case 256: return launch_topk<256>(p, s);

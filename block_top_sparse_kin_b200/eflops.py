@@ -39,9 +39,11 @@ class Cost:
         return Cost(self.flops + other.flops, self.bytes + other.bytes)
 
 
-def step_costs(B: int, Hkv: int, Hq: int, D: int, bs: int, lens, k: int, n_append: int = 0) -> dict:
+def step_costs(B: int, Hkv: int, Hq: int, D: int, bs: int, lens, k: int, n_append: int = 0,
+               means_bytes: int = 4) -> dict:
     """A and M of each part of one decode step.  lens: the lengths the
-    select and attention see (after the append)."""
+    select and attention see (after the append); means_bytes: 4 for fp32
+    block means, 2 for bf16."""
     g = Hq // Hkv
     lens = np.asarray(lens, dtype=np.int64)
     assert lens.shape == (B,)
@@ -51,7 +53,7 @@ def step_costs(B: int, Hkv: int, Hq: int, D: int, bs: int, lens, k: int, n_appen
     blocks_scanned = int((Hkv * nb[scanned]).sum())
     q_bytes = B * Hq * D * 2
     idx_bytes = B * Hkv * k * 4
-    select = Cost(2.0 * g * D * blocks_scanned, float(blocks_scanned * D * 4 + q_bytes + idx_bytes))
+    select = Cost(2.0 * g * D * blocks_scanned, float(blocks_scanned * D * means_bytes + q_bytes + idx_bytes))
     # attention over the kept tokens
     toks = np.where(scanned, (k - 1) * bs + (lens - (nb - 1) * bs), lens)
     kept = int((Hkv * toks).sum())
@@ -70,7 +72,7 @@ def step_costs(B: int, Hkv: int, Hq: int, D: int, bs: int, lens, k: int, n_appen
         upd_bytes = (new_rows * D * 2 * 2        # read k_new, v_new
                      + new_rows * D * 2 * 2      # write the K, V cache rows
                      + (rows - new_rows) * D * 2  # re-read the touched blocks' older K rows
-                     + touched * D * 4)          # write their means
+                     + touched * D * means_bytes)  # write their means
         parts["update"] = Cost(float(rows * D), float(upd_bytes))
     return parts
 

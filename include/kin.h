@@ -185,6 +185,36 @@ kin_status kin_sparse_decode_attn_paged(const kin_dims* dims, const void* q, con
                                         int32_t* dev_status, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Extended calls: block means in bf16, either KV layout.
+ *
+ * bf16 block means halve the bytes the select streams (a NEXT variant: the
+ * contiguous calls above keep fp32 means, whose scores stay within the
+ * method's 1e-4 near-tie band).  A bf16 mean is the fp32 mean of the calls
+ * above rounded to nearest even; scores are then computed in fp32 from the
+ * widened bf16 values.  block_means is [B][Hkv][NBcap][D] of the given
+ * dtype; the same buffer must be passed to the build/update and the select.
+ * block_table NULL selects the contiguous cache [B][Hkv][Lcap][D] (then
+ * num_pages is ignored); otherwise k_rows / v_rows are the page pool of the
+ * paged calls.  An unknown means_dtype is KIN_ERR_INVALID_ARG.  Otherwise
+ * arguments, semantics and errors are those of kin_block_means_build,
+ * kin_block_means_update (and their paged forms) and kin_block_topk_select. */
+typedef enum { KIN_MEANS_F32 = 0, KIN_MEANS_BF16 = 1 } kin_means_dtype;
+
+kin_status kin_block_means_build_ex(const kin_dims* dims, const void* k_rows, int32_t num_pages,
+                                    const int32_t* block_table, const int32_t* seq_lens, void* block_means,
+                                    int32_t means_dtype, int32_t* dev_status, void* stream);
+
+kin_status kin_block_means_update_ex(const kin_dims* dims, void* k_rows, void* v_rows, int32_t num_pages,
+                                     const int32_t* block_table, void* block_means, int32_t means_dtype,
+                                     int32_t* seq_lens, const void* k_new, const void* v_new, int32_t n_new,
+                                     int32_t* dev_status, void* stream);
+
+kin_status kin_block_topk_select_ex(const kin_dims* dims, const void* q, const void* block_means,
+                                    int32_t means_dtype, const int32_t* seq_lens, int32_t k_blocks,
+                                    int32_t* sel_idx, int32_t* sel_cnt, void* workspace, size_t ws_bytes,
+                                    int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------
  * Allocation-free variant of kin_block_topk_select (the pages describe no
  * counterpart; it exists for callers, not for the method).
  *

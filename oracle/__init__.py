@@ -196,3 +196,19 @@ def gather_paged(pages: np.ndarray, table_row: np.ndarray, L: int, bs: int, h: i
     nb = -(-L // bs)
     blocks = [pages[int(table_row[i]), h] for i in range(nb)]
     return np.concatenate(blocks, axis=0)[:L] if nb else pages[:0, h].reshape(0, pages.shape[-1])
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Values rounded to bfloat16 precision (8 significant bits, ties to even)
+    and returned as float64: x = m 2^e with 0.5 <= |m| < 1, m rounded to a
+    multiple of 2^-8.  The bf16-means variant of the select keeps each block
+    mean at this precision (block means of "Kinetics: Memory-Aware Test-Time
+    Scaling", Implementation, stored in half the bytes).  Inputs are finite
+    and within bf16's normal range."""
+    m, e = np.frexp(np.asarray(x, dtype=np.float64))
+    return np.ldexp(np.round(m * 256.0) / 256.0, e)
+
+
+def block_means_bf16(K: np.ndarray, L: int, bs: int) -> np.ndarray:
+    """block_means rounded to bf16 precision (fp64 array)."""
+    return round_bf16(block_means(K, L, bs))

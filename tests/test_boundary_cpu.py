@@ -144,6 +144,29 @@ def test_paged_calls_reject_before_launch(lib):
     assert at(n=64) == 2
 
 
+def test_extended_calls_reject_before_launch(lib):
+    d = dims()
+    bd = ctypes.byref(d)
+    sel = lambda dt=1, k=8, ws=FAKE: lib.kin_block_topk_select_ex(bd, FAKE, FAKE, dt, FAKE, k, FAKE, FAKE, ws,
+                                                                  1 << 30, None, None)
+    assert sel(dt=2) == 1
+    assert sel(dt=-1) == 1
+    assert sel(k=1) == 1
+    assert sel(ws=None) == 2
+    build = lambda dt=1, pool=FAKE, pages=0, table=None: lib.kin_block_means_build_ex(
+        bd, pool, pages, table, FAKE, FAKE, dt, None, None)
+    assert build(dt=7) == 1
+    assert build(pool=None) == 1
+    assert build(pages=0, table=FAKE) == 1        # a table needs a pool of >= 1 page
+    upd = lambda dt=1, n=1, pages=4, table=FAKE: lib.kin_block_means_update_ex(
+        bd, FAKE, FAKE, pages, table, FAKE, dt, FAKE, FAKE, FAKE, n, None, None)
+    assert upd(dt=3) == 1
+    assert upd(n=-1) == 1
+    assert upd(n=0) == 0
+    assert upd(n=257) == 3
+    assert upd(pages=0) == 1
+
+
 def test_binding_refuses_host_tensors(lib):
     import torch
     with pytest.raises(ValueError):

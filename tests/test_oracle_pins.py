@@ -288,3 +288,17 @@ def test_gather_paged_follows_the_block_table():
     shuffled = np.zeros((6, Hkv, bs, D), np.uint16)
     shuffled[perm] = ident
     assert np.array_equal(oracle.gather_paged(shuffled, perm, 12, bs, 0), cont[0])
+
+
+def test_round_bf16_matches_torch_conversion():
+    """bf16 rounding against torch's float32 -> bfloat16 conversion (round to
+    nearest even) on fp32 values, including exact ties and both signs."""
+    import torch
+    rng = np.random.default_rng(12)
+    x = np.concatenate([rng.normal(0, 1, 20000), rng.normal(0, 1e-3, 2000) * 1e3,
+                        [1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, -(1 + 2.0 ** -8), 0.0, 255.5, 3.0]]).astype(np.float32)
+    want = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(oracle.round_bf16(x.astype(np.float64)), want)
+    # ties go to even: 1 + 2^-8 sits halfway between 1 and 1 + 2^-7
+    assert oracle.round_bf16(np.array([1 + 2.0 ** -8]))[0] == 1.0
+    assert oracle.round_bf16(np.array([1 + 3 * 2.0 ** -8]))[0] == 1 + 2.0 ** -6
