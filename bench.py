@@ -65,6 +65,17 @@ def algorithmic_bytes(w: ki.Workload, k: int, lens: np.ndarray, means_bytes: int
     return sel_bytes, attn_bytes
 
 
+def token_algorithmic_bytes(w: ki.Workload, kt: int, lens: np.ndarray):
+    """Algorithmic HBM bytes of one token-level top-k step: every K row (the
+    logits pass), the kept V rows of every query head, q and the bf16 out.
+    The logits' round trip through workspace is reported as traffic, not
+    counted here."""
+    lens = lens.astype(np.int64)
+    k_rows = int((w.Hkv * lens).sum())
+    v_rows = int((w.Hq * np.minimum(kt, lens)).sum())
+    return (k_rows + v_rows) * w.D * 2 + 2 * w.B * w.Hq * w.D * 2
+
+
 def measured_bf16_peak():
     """Dense bf16 FLOP/s: the measured burst figure, else the fallback."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -75,11 +86,12 @@ def measured_bf16_peak():
         return FALLBACK_BF16_TFLOPS * 1e12, "fallback"
 
 
-def eflops_report(w, k, lens, ms_per_step, means_bytes=4):
+def eflops_report(w, k, lens, ms_per_step, means_bytes=4, token_kt=0):
     """The eFLOPs model's predicted step time (T = A/C + M/B) beside the
     measured one, with the measured B200 peaks as C and B."""
     from block_top_sparse_kin_b200 import eflops as ef
-    parts = ef.step_costs(w.B, w.Hkv, w.Hq, w.D, w.bs, lens, k, w.n_append, means_bytes)
+    parts = (ef.token_step_costs(w.B, w.Hkv, w.Hq, w.D, lens, token_kt) if token_kt else
+             ef.step_costs(w.B, w.Hkv, w.Hq, w.D, w.bs, lens, k, w.n_append, means_bytes))
     tot = ef.Cost(0.0, 0.0)
     for c in parts.values():
         tot = tot + c
@@ -315,6 +327,9 @@ def run_step(st, ev=None):
         append(st)
         if ev is not None:
             ev[i].record(); i += 1
+    if "token_kt" in st:
+        token_step(st)
+        return
     select(st)
     if ev is not None:
         ev[i].record(); i += 1
@@ -351,6 +366,13 @@ def select(st):
                                   st["ws"], st["status"])
 
 
+def token_step(st):
+    """Token-level top-k attention (logits of every token, top-k per query head, attention)."""
+    import block_top_sparse_kin_b200 as kin
+    kin.kin_token_topk_decode_attn(st["dims"], st["q"], st["k_cache"], st["v_cache"], st["seq"], st["token_kt"], 0.0,
+                                   st["out"], st["lse"], st["token_ws"], dev_status=st["status"])
+
+
 def attend(st):
     """The step's attention call, over the contiguous cache or the page pool."""
     import block_top_sparse_kin_b200 as kin
@@ -378,6 +400,12 @@ def gpu_arm(args):
     k = args.k or w0.k
     w = shard_workload(w0, rank)
     st = build_device_state(w, k, paged=args.paged, means_bf16=args.means_bf16)
+    if args.token_topk:
+        if args.paged:
+            raise SystemExit("--token-topk reads the contiguous cache")
+        import block_top_sparse_kin_b200 as kin_mod
+        st["token_kt"] = k * w.bs  # the block budget in tokens, per query head
+        st["token_ws"] = kin_mod.alloc_token_workspace(st["dims"], st["token_kt"])
     flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
 
@@ -388,7 +416,8 @@ def gpu_arm(args):
         flush_sink.copy_(flush_r.sum())
 
     flush_sink = torch.zeros((), dtype=torch.float32, device="cuda")
-    # select = scan + top-k kernels, then attention (+ the append update)
+    # block path: scan + top-k, then attention; token path: logits, top-k,
+    # attention; plus the append update
     launches_per_step = 4 if w.n_append else 3
 
     for _ in range(args.warmup):
@@ -410,11 +439,15 @@ def gpu_arm(args):
 
     import block_top_sparse_kin_b200 as kin
 
-    def call_select():
-        select(st)
-
-    def call_attn():
-        attend(st)
+    # the step's kernel families: (name, call, algorithmic bytes, source file)
+    means_bytes = 2 if args.means_bf16 else 4
+    if args.token_topk:
+        parts = [("token_topk_attn", lambda: token_step(st),
+                  token_algorithmic_bytes(w, st["token_kt"], st["lens_final"]), "kin_token.cu")]
+    else:
+        sel_b, attn_b = algorithmic_bytes(w, k, st["lens_final"], means_bytes)
+        parts = [("select", lambda: select(st), sel_b, "kin_select.cu"),
+                 ("attn", lambda: attend(st), attn_b, "kin_attn.cu")]
 
     # Per-kernel times for the roofline: a graph per kernel family holding
     # KERNEL_REPEATS back-to-back calls between two events.  The means and the
@@ -423,7 +456,7 @@ def gpu_arm(args):
     # spread over the calls, as in a decode pipeline.  The append update is
     # timed once per replay (its calls would move the lengths).
     step_ev = ext_events(2)
-    sel_ev, attn_ev = ext_events(2), ext_events(2)
+    part_ev = [ext_events(2) for _ in parts]
     upd_ev = ext_events(2)
     cap = torch.cuda.Stream()
     cap.wait_stream(torch.cuda.current_stream())
@@ -434,17 +467,15 @@ def gpu_arm(args):
             step_ev[0].record()
             run_step(st)
             step_ev[1].record()
-        sel_graph, attn_graph = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(sel_graph, stream=cap):
-            sel_ev[0].record()
-            for _ in range(KERNEL_REPEATS):
-                call_select()
-            sel_ev[1].record()
-        with torch.cuda.graph(attn_graph, stream=cap):
-            attn_ev[0].record()
-            for _ in range(KERNEL_REPEATS):
-                call_attn()
-            attn_ev[1].record()
+        part_graphs = []
+        for (_, call, _, _), ev in zip(parts, part_ev):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                ev[0].record()
+                for _ in range(KERNEL_REPEATS):
+                    call()
+                ev[1].record()
+            part_graphs.append(g)
         upd_graph = None
         if w.n_append:
             upd_graph = torch.cuda.CUDAGraph()
@@ -454,7 +485,7 @@ def gpu_arm(args):
                 append(st)
                 upd_ev[1].record()
     torch.cuda.current_stream().wait_stream(cap)
-    diag = [g for g in (sel_graph, attn_graph, upd_graph) if g is not None]
+    diag = part_graphs + ([upd_graph] if upd_graph is not None else [])
     for _ in range(args.warmup):
         flush_l2(0)
         graph.replay()
@@ -476,11 +507,11 @@ def gpu_arm(args):
         wall = time.perf_counter() - wall0
     if world > 1:
         dist.barrier()
-    sel_ms, attn_ms, upd_ms = [], [], []
+    part_ms = [[] for _ in parts]
+    upd_ms = []
     for s in range(args.steps):            # per-kernel timing pass (not in `value`)
-        for g, ev, out, reps in ((sel_graph, sel_ev, sel_ms, KERNEL_REPEATS),
-                                 (attn_graph, attn_ev, attn_ms, KERNEL_REPEATS),
-                                 (upd_graph, upd_ev, upd_ms, 1)):
+        for g, ev, out, reps in list(zip(part_graphs, part_ev, part_ms, [KERNEL_REPEATS] * len(parts))) + \
+                [(upd_graph, upd_ev, upd_ms, 1)]:
             if g is None:
                 continue
             flush_l2(s)
@@ -522,16 +553,12 @@ def gpu_arm(args):
     status = int(st["status"].item())
 
     if rank == 0:
-        sel_b, attn_b = algorithmic_bytes(w, k, st["lens_final"], 2 if args.means_bf16 else 4)
         peak, peak_kind = measured_peak()
-        sel_avg = statistics.mean(sel_ms)
-        attn_avg = statistics.mean(attn_ms)
-        attn_gbs = attn_b / (attn_avg * 1e-3) / 1e9
-        sel_gbs = sel_b / (sel_avg * 1e-3) / 1e9
-        step_gbs = (sel_b + attn_b) / (ms_per_step * 1e-3) / 1e9
-        dominant = "attn" if attn_avg >= sel_avg else "select"
-        dom_file = "kin_attn.cu" if dominant == "attn" else "kin_select.cu"
-        dom_bytes, dom_ms, dom_gbs = (attn_b, attn_avg, attn_gbs) if dominant == "attn" else (sel_b, sel_avg, sel_gbs)
+        avg = {name: statistics.mean(ms) for (name, _, _, _), ms in zip(parts, part_ms)}
+        gbs = {name: nbytes / (avg[name] * 1e-3) / 1e9 for name, _, nbytes, _ in parts}
+        step_gbs = sum(nbytes for _, _, nbytes, _ in parts) / (ms_per_step * 1e-3) / 1e9
+        dominant, _, dom_bytes, dom_file = max(parts, key=lambda pt: avg[pt[0]])
+        dom_gbs = gbs[dominant]
         line = {
             "metric": METRIC,
             "value": value,
@@ -554,12 +581,13 @@ def gpu_arm(args):
                 "kv_layout": (f"paged: {st['num_pages']} pages of one {w.bs}-token block, shuffled pool + block table"
                               if args.paged else "contiguous [B][Hkv][Lcap][D]"),
                 "block_means": "bf16" if args.means_bf16 else "fp32",
+                **({"attention": f"token-level top-k, {st['token_kt']} tokens per query head"} if args.token_topk else {}),
             },
             "impl": "kin",
             "gpu_launches": launches_per_step * args.steps,  # in the timed region
-            "kernel_ms": {"select": sel_avg, "attn": attn_avg, **({"update": statistics.mean(upd_ms)} if upd_ms else {})},
-            "hbm_gbs": {"select": sel_gbs, "attn": attn_gbs, "step": step_gbs},
-            "hbm_frac": {"select": sel_gbs / peak, "attn": attn_gbs / peak, "step": step_gbs / peak,
+            "kernel_ms": {**avg, **({"update": statistics.mean(upd_ms)} if upd_ms else {})},
+            "hbm_gbs": {**gbs, "step": step_gbs},
+            "hbm_frac": {**{n: v / peak for n, v in gbs.items()}, "step": step_gbs / peak,
                          "peak_gbs": peak, "peak_kind": peak_kind},
             "roofline": {
                 "kernel": dominant, "bound": "hbm", "achieved": dom_gbs, "peak": peak, "unit": "GB/s",
@@ -569,12 +597,13 @@ def gpu_arm(args):
             },
             "e2e": {"value": e2e_value, "unit": "query-heads/s",
                     "h2d_bytes_per_step": int(q_pin.numel() * 2), "d2h_bytes_per_step": int(out_pin.numel() * 2)},
-            "eflops": eflops_report(w, k, st["lens_final"], ms_per_step, 2 if args.means_bf16 else 4),
+            "eflops": eflops_report(w, k, st["lens_final"], ms_per_step, means_bytes,
+                                    st.get("token_kt", 0)),
             "clocks": clk.summary(),
             "wall_s_timed_region": wall,
             "device_status": status,
         }
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and not args.token_topk:
             line["cpu_baseline"] = cpu_baseline(w0, k, budget_s=args.cpu_seconds)
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -690,6 +719,8 @@ def main():
     ap.add_argument("--ref-pairs", type=int, default=8, help="pairs per reference-arm step")
     ap.add_argument("--paged", action="store_true", help="KV cache in a shuffled page pool with a block table")
     ap.add_argument("--means-bf16", action="store_true", help="bf16 block means (the extended calls)")
+    ap.add_argument("--token-topk", action="store_true",
+                    help="token-level top-k attention instead of the block path (budget = k blocks x bs tokens)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "kin":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

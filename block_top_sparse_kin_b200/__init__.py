@@ -28,7 +28,7 @@ EXPORTED = (
     "kin_block_means_update", "kin_block_topk_select", "kin_sparse_decode_attn",
     "kin_block_topk_select_noalloc", "kin_block_means_build_paged", "kin_block_means_update_paged",
     "kin_sparse_decode_attn_paged", "kin_block_means_build_ex", "kin_block_means_update_ex",
-    "kin_block_topk_select_ex",
+    "kin_block_topk_select_ex", "kin_token_topk_workspace_bytes", "kin_token_topk_decode_attn",
 )
 KIN_MEANS_F32, KIN_MEANS_BF16 = 0, 1
 NOALLOC_SCRATCH_FLOATS = 1 << 21  # KIN_NOALLOC_SCRATCH_FLOATS in include/kin.h
@@ -101,6 +101,10 @@ def load_library(path: str = LIB_PATH):
     lib.kin_block_means_update_ex.restype = ctypes.c_int
     lib.kin_block_topk_select_ex.argtypes = [dp, vp, vp, i32, vp, i32, vp, vp, vp, sz, vp, vp]
     lib.kin_block_topk_select_ex.restype = ctypes.c_int
+    lib.kin_token_topk_workspace_bytes.argtypes = [dp, i32]
+    lib.kin_token_topk_workspace_bytes.restype = sz
+    lib.kin_token_topk_decode_attn.argtypes = [dp, vp, vp, vp, vp, i32, f32, vp, vp, vp, vp, sz, vp, vp]
+    lib.kin_token_topk_decode_attn.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -289,3 +293,28 @@ def kin_block_topk_select_ex(dims, q, block_means, seq_lens, k_blocks, sel_idx, 
         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
     _check(rc, "kin_block_topk_select_ex")
+
+
+# --------------------------------------------------- token-level top-k attention
+
+def kin_token_topk_workspace_bytes(dims: kin_dims, k_tokens: int) -> int:
+    return int(load_library().kin_token_topk_workspace_bytes(ctypes.byref(dims), k_tokens))
+
+
+def alloc_token_workspace(dims: kin_dims, k_tokens: int, device="cuda") -> torch.Tensor:
+    n = kin_token_topk_workspace_bytes(dims, k_tokens)
+    if n == 0:
+        raise KinError(1, "kin_token_topk_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def kin_token_topk_decode_attn(dims, q, k_cache, v_cache, seq_lens, k_tokens, softmax_scale, out, lse, workspace,
+                               sel_tokens=None, dev_status=None, stream=None):
+    rc = load_library().kin_token_topk_decode_attn(
+        ctypes.byref(dims), _dev(q, "q", _BF16), _dev(k_cache, "k_cache", _BF16), _dev(v_cache, "v_cache", _BF16),
+        _dev(seq_lens, "seq_lens", torch.int32), int(k_tokens), float(softmax_scale), _dev(out, "out", _BF16),
+        _dev(lse, "lse", torch.float32, nullable=True),
+        _dev(sel_tokens, "sel_tokens", torch.int32, nullable=True), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(),
+        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+    _check(rc, "kin_token_topk_decode_attn")

@@ -8,7 +8,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libkin.so")
-SOURCES = ["kin_api.cu", "kin_means.cu", "kin_select.cu", "kin_attn.cu", "kin_noalloc.cu"]
+SOURCES = ["kin_api.cu", "kin_means.cu", "kin_select.cu", "kin_attn.cu", "kin_noalloc.cu", "kin_token.cu"]
 
 
 def nvcc_command(out: str = LIB, ptxas_verbose: bool = False, defines=()) -> list:

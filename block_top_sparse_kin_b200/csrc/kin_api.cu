@@ -448,3 +448,77 @@ KIN_EXPORT kin_status kin_sparse_decode_attn_paged(const kin_dims* dims, const v
   return sparse_decode_attn(dims, q, k_pages, v_pages, pt, seq_lens, sel_idx, sel_cnt, k_blocks,
                             softmax_scale, out, lse, workspace, ws_bytes, dev_status, stream);
 }
+
+// ------------------------------------------------------------ token top-k
+namespace {
+
+constexpr int kTokenKeyCap = 32768;  // the token top-k keeps keys in shared memory up to this length
+
+struct TokenWs {
+  size_t logits, keys, sel, cnt, total;
+};
+
+TokenWs token_ws_layout(const kin_dims& d, int kt) {
+  const size_t rows = (size_t)d.batch * d.num_q_heads;
+  TokenWs w;
+  size_t off = 0;
+  w.logits = off;
+  off = align_up(off + rows * (size_t)d.max_seq_len * sizeof(float));
+  w.keys = off;
+  if (d.max_seq_len > kTokenKeyCap) off = align_up(off + rows * (size_t)d.max_seq_len * sizeof(uint32_t));
+  w.sel = off;
+  off = align_up(off + rows * (size_t)kt * sizeof(int32_t));
+  w.cnt = off;
+  off = align_up(off + rows * sizeof(int32_t));
+  w.total = off;
+  return w;
+}
+
+}  // namespace
+
+KIN_EXPORT size_t kin_token_topk_workspace_bytes(const kin_dims* dims, int32_t k_tokens) {
+  if (check_dims(dims) != KIN_OK || k_tokens < 1) return 0;
+  return token_ws_layout(*dims, k_tokens).total;
+}
+
+KIN_EXPORT kin_status kin_token_topk_decode_attn(const kin_dims* dims, const void* q, const void* k_cache,
+                                                 const void* v_cache, const int32_t* seq_lens, int32_t k_tokens,
+                                                 float softmax_scale, void* out, float* lse, int32_t* sel_tokens,
+                                                 void* workspace, size_t ws_bytes, int32_t* dev_status,
+                                                 void* stream) {
+  kin_status st = check_dims(dims);
+  if (st != KIN_OK) return st;
+  if (k_tokens < 1) return KIN_ERR_INVALID_ARG;
+  if (!q || !k_cache || !v_cache || !seq_lens || !out) return KIN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return KIN_ERR_INVALID_ARG;
+  if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale)) return KIN_ERR_INVALID_ARG;
+  if ((int64_t)dims->batch * dims->num_q_heads * dims->max_seq_len >= (int64_t)1 << 31) return KIN_ERR_CAPACITY;
+  const TokenWs w = token_ws_layout(*dims, k_tokens);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0 || ws_bytes < w.total)
+    return KIN_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  TokenParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
+  p.v_cache = static_cast<const __nv_bfloat16*>(v_cache);
+  p.seq_lens = seq_lens;
+  p.logits = reinterpret_cast<float*>(ws + w.logits);
+  p.key_scratch = reinterpret_cast<uint32_t*>(ws + w.keys);
+  p.sel = sel_tokens ? sel_tokens : reinterpret_cast<int32_t*>(ws + w.sel);
+  p.cnt = reinterpret_cast<int32_t*>(ws + w.cnt);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.dev_status = dev_status;
+  p.B = dims->batch;
+  p.Hkv = dims->num_kv_heads;
+  p.Hq = dims->num_q_heads;
+  p.g = dims->num_q_heads / dims->num_kv_heads;
+  p.Lcap = dims->max_seq_len;
+  p.kt = k_tokens;
+  p.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)kHeadDim);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_token_logits(p, s);
+  if (e == cudaSuccess) e = launch_token_topk(p, s);
+  if (e == cudaSuccess) e = launch_token_attn(p, s);
+  return from_cuda(e);
+}

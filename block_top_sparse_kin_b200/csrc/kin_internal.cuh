@@ -195,6 +195,24 @@ struct AttnParams {
   float scale_log2;     // softmax_scale * log2(e)
 };
 
+// Token-level top-k attention: every logit of every query head, a top-k of
+// tokens per head, attention over the kept tokens.
+struct TokenParams {
+  const __nv_bfloat16* q;        // [B][Hq][D]
+  const __nv_bfloat16* k_cache;  // [B][Hkv][Lcap][D]
+  const __nv_bfloat16* v_cache;
+  const int32_t* seq_lens;
+  float* logits;                 // workspace [B][Hq][Lcap]: scale * q . K_t
+  uint32_t* key_scratch;         // workspace [B][Hq][Lcap] when Lcap exceeds the shared-memory key cap
+  int32_t* sel;                  // [B][Hq][kt] kept token indices, ascending, -1 padded
+  int32_t* cnt;                  // [B][Hq]
+  __nv_bfloat16* out;            // [B][Hq][D]
+  float* lse;                    // [B][Hq] or NULL
+  int32_t* dev_status;
+  int B, Hkv, Hq, g, Lcap, kt;
+  float scale;                   // softmax scale (natural log base)
+};
+
 // Launch with programmatic stream serialization (see pdl_wait).
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
@@ -223,5 +241,8 @@ cudaError_t launch_means_build(const MeansBuildParams& p, cudaStream_t s);
 cudaError_t launch_means_update(const MeansUpdateParams& p, cudaStream_t s);
 cudaError_t launch_select(const SelectParams& p, cudaStream_t s);
 cudaError_t launch_attn(const AttnParams& p, int num_items, cudaStream_t s);
+cudaError_t launch_token_logits(const TokenParams& p, cudaStream_t s);
+cudaError_t launch_token_topk(const TokenParams& p, cudaStream_t s);
+cudaError_t launch_token_attn(const TokenParams& p, cudaStream_t s);
 
 }  // namespace kin

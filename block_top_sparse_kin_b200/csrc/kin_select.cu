@@ -79,6 +79,15 @@ constexpr int kMaxKPT = 8;      // keys per thread on the register path
 constexpr int kHistWords = 256 + 32;
 __device__ __forceinline__ int hidx(int bin) { return bin + (bin >> 3); }
 
+// The candidates of a top-k over nb keys: indices lo..hi compete for kr
+// slots; every other index below nb is forced (always kept).  Block select:
+// lo = 1, hi = nb - 2, kr = k - 2 (the first and the newest block forced).
+// Token select: lo = 0, hi = nb - 1, kr = k (nothing forced).
+struct Cands {
+  int lo, hi, kr;
+  __device__ __forceinline__ bool has(int i) const { return i >= lo && i <= hi; }
+};
+
 template <int NT>
 struct TopkSmem {
   static constexpr int NW = NT / 32;
@@ -153,7 +162,7 @@ __device__ __forceinline__ void warp_find_bin(const int* hist, int kr, int& bin,
 // On return every key above `prefix` under `mask` is kept, and the first kr
 // keys equal to it under the mask (by index).
 template <int NT>
-__device__ __forceinline__ void radix_threshold(const uint32_t* keys, int nb, TopkSmem<NT>& sm,
+__device__ __forceinline__ void radix_threshold(const uint32_t* keys, int nb, const Cands& cd, TopkSmem<NT>& sm,
                                                 uint32_t& prefix, uint32_t& mask, int& kr) {
   const int tid = threadIdx.x, lane = tid & 31;
   prefix = 0u;
@@ -170,7 +179,7 @@ __device__ __forceinline__ void radix_threshold(const uint32_t* keys, int nb, To
         for (int base = 0; base < nb; base += NT) {  // uniform trip count per warp
           const int i = base + tid;
           const uint32_t key = i < nb ? keys[i] : 0u;
-          const bool match = i >= 1 && i <= nb - 2 && (key & mask) == prefix;
+          const bool match = cd.has(i) && (key & mask) == prefix;
           if (match) atomicAdd(&hist[hidx((key >> shift) & 0xFFu)], 1);
           if (use_list) {  // one list reservation per warp, lanes take slots in order
             const unsigned m = __ballot_sync(0xffffffffu, match);
@@ -186,7 +195,7 @@ __device__ __forceinline__ void radix_threshold(const uint32_t* keys, int nb, To
           if ((key & mask) == prefix) atomicAdd(&hist[hidx((key >> shift) & 0xFFu)], 1);
         }
       } else {
-        for (int i = 1 + tid; i < nb - 1; i += NT) {
+        for (int i = cd.lo + tid; i <= cd.hi; i += NT) {
           const uint32_t key = keys[i];
           if ((key & mask) == prefix) atomicAdd(&hist[hidx((key >> shift) & 0xFFu)], 1);
         }
@@ -222,7 +231,7 @@ __device__ __forceinline__ void radix_threshold(const uint32_t* keys, int nb, To
 // greater / equal keys, one barrier publishes the counts, and a second pass
 // writes the taken indices in order (so ties go to lower indices).
 template <int NT>
-__device__ __forceinline__ void emit_selection(const uint32_t* keys, int nb, int k, uint32_t prefix,
+__device__ __forceinline__ void emit_selection(const uint32_t* keys, int nb, const Cands& cd, int k, uint32_t prefix,
                                                uint32_t mask, int kr, int32_t* sel, TopkSmem<NT>& sm,
                                                int32_t* dev_status) {
   constexpr int NW = NT / 32;
@@ -235,7 +244,7 @@ __device__ __forceinline__ void emit_selection(const uint32_t* keys, int nb, int
     const int i = base + lane;
     const bool in = i < w1;
     const uint32_t key = in ? (keys[i] & mask) : 0u;
-    const bool cand = in && i >= 1 && i <= nb - 2;
+    const bool cand = in && cd.has(i);
     n_forced += __popc(__ballot_sync(0xffffffffu, in && !cand));
     n_gt += __popc(__ballot_sync(0xffffffffu, cand && key > prefix));
     n_eq += __popc(__ballot_sync(0xffffffffu, cand && key == prefix));
@@ -258,7 +267,7 @@ __device__ __forceinline__ void emit_selection(const uint32_t* keys, int nb, int
     const int i = base + lane;
     const bool in = i < w1;
     const uint32_t key = in ? (keys[i] & mask) : 0u;
-    const bool cand = in && i >= 1 && i <= nb - 2;
+    const bool cand = in && cd.has(i);
     const bool eq = cand && key == prefix;
     const unsigned eq_mask = __ballot_sync(0xffffffffu, eq);
     const bool take = (in && !cand) || (cand && key > prefix) || (eq && eq_rank + __popc(eq_mask & lt) < kr);
@@ -309,7 +318,7 @@ __device__ __forceinline__ void rank_boundary_bin(int c, int need, TopkSmem<NT>&
 // is too crowded: the caller then runs the radix search.  Expects
 // sm.hist[0] zero.
 template <int NT>
-__device__ __forceinline__ bool linear_threshold(const uint32_t* keys, int nb, int kr, uint32_t kmin,
+__device__ __forceinline__ bool linear_threshold(const uint32_t* keys, const Cands& cd, int kr, uint32_t kmin,
                                                  uint32_t kmax, TopkSmem<NT>& sm, uint32_t& thresh,
                                                  int& take) {
   const float lo = key_float(kmin), hi = key_float(kmax);
@@ -318,15 +327,15 @@ __device__ __forceinline__ bool linear_threshold(const uint32_t* keys, int nb, i
   if (!(isfinite(lo) && isfinite(hi) && range > 0.f && isfinite(range) && isfinite(inv))) return false;
   const int tid = threadIdx.x, lane = tid & 31;
   auto bin_of = [&](uint32_t key) { return min((int)((key_float(key) - lo) * inv), 255); };
-  for (int i = 1 + tid; i <= nb - 2; i += NT) atomicAdd(&sm.hist[0][hidx(bin_of(keys[i]))], 1);
+  for (int i = cd.lo + tid; i <= cd.hi; i += NT) atomicAdd(&sm.hist[0][hidx(bin_of(keys[i]))], 1);
   if (tid == 0) sm.list_n = 0;
   __syncthreads();
   int bstar, above, c;
   warp_find_bin(sm.hist[0], kr, bstar, above, c);  // every warp, same result
   if (c > kRankCap) return false;
-  for (int base = 1; base <= nb - 2; base += NT) {  // uniform trip count per warp
+  for (int base = cd.lo; base <= cd.hi; base += NT) {  // uniform trip count per warp
     const int i = base + tid;
-    const bool in = i <= nb - 2;
+    const bool in = i <= cd.hi;
     const uint32_t key = in ? keys[i] : 0u;
     const bool match = in && bin_of(key) == bstar;
     const unsigned m = __ballot_sync(0xffffffffu, match);
@@ -346,28 +355,28 @@ __device__ __forceinline__ bool linear_threshold(const uint32_t* keys, int nb, i
 // written ascending to sel[0..k).  kmin / kmax: the smallest and largest
 // candidate key.  Expects sm.hist[0] and sm.hist[1] zero.
 template <int NT>
-__device__ __forceinline__ void select_from_keys(const uint32_t* keys, int nb, int k, uint32_t kmin,
-                                                 uint32_t kmax, int32_t* sel, TopkSmem<NT>& sm,
+__device__ __forceinline__ void select_from_keys(const uint32_t* keys, int nb, const Cands& cd, int k,
+                                                 uint32_t kmin, uint32_t kmax, int32_t* sel, TopkSmem<NT>& sm,
                                                  int32_t* dev_status) {
-  uint32_t prefix = 0xFFFFFFFFu, mask = 0xFFFFFFFFu;  // budget of two: no candidate passes
-  int kr = k - 2;
-  if (kr > 0 && !linear_threshold(keys, nb, kr, kmin, kmax, sm, prefix, kr)) {
+  uint32_t prefix = 0xFFFFFFFFu, mask = 0xFFFFFFFFu;  // kr == 0: no candidate passes
+  int kr = cd.kr;
+  if (kr > 0 && !linear_threshold(keys, cd, kr, kmin, kmax, sm, prefix, kr)) {
     __syncthreads();  // every warp is done with the bin histogram
     zero_hist(sm, 0);
     __syncthreads();
-    for (int i = 1 + threadIdx.x; i <= nb - 2; i += NT) atomicAdd(&sm.hist[0][hidx(keys[i] >> 24)], 1);
+    for (int i = cd.lo + threadIdx.x; i <= cd.hi; i += NT) atomicAdd(&sm.hist[0][hidx(keys[i] >> 24)], 1);
     __syncthreads();
-    kr = k - 2;
-    radix_threshold(keys, nb, sm, prefix, mask, kr);
+    kr = cd.kr;
+    radix_threshold(keys, nb, cd, sm, prefix, mask, kr);
   }
-  emit_selection(keys, nb, k, prefix, mask, kr, sel, sm, dev_status);
+  emit_selection(keys, nb, cd, k, prefix, mask, kr, sel, sm, dev_status);
 }
 
 // Loads a pair's nb scores (written by the scan kernel: read from L2) as
 // keys into keys[] (shared memory, or the score row itself), returns the
 // smallest and largest candidate key, and zeroes both histograms.
 template <int NT>
-__device__ __forceinline__ void load_keys(const uint32_t* sc, uint32_t* keys, int nb, TopkSmem<NT>& sm,
+__device__ __forceinline__ void load_keys(const uint32_t* sc, uint32_t* keys, int nb, const Cands& cd, TopkSmem<NT>& sm,
                                           uint32_t& kmin, uint32_t& kmax) {
   constexpr int NW = NT / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -386,7 +395,7 @@ __device__ __forceinline__ void load_keys(const uint32_t* sc, uint32_t* keys, in
       if (i < nb) {
         const uint32_t key = key_of_bits(v[u]);
         keys[i] = key;
-        if (i >= 1 && i <= nb - 2) {
+        if (cd.has(i)) {
           lo = min(lo, key);
           hi = max(hi, key);
         }
@@ -411,16 +420,17 @@ __device__ __forceinline__ void load_keys(const uint32_t* sc, uint32_t* keys, in
   }
 }
 
-// The top-k of one pair with any nb, keys in memory: shared memory when
-// nb <= key_cap, else the pair's own score row (which nothing else reads
-// afterwards).
+// The top-k of one row of nb scores with any nb, keys in memory: shared
+// memory when nb <= key_cap, else gkeys (nb words of global scratch, which
+// may be the score row itself when nothing reads it afterwards).
 template <int NT>
-__device__ __forceinline__ void topk_memory(const uint32_t* row, int nb, int k, int32_t* sel, uint32_t* skey,
-                                            int key_cap, TopkSmem<NT>& sm, int32_t* dev_status) {
-  uint32_t* keys = nb <= key_cap ? skey : const_cast<uint32_t*>(row);
+__device__ __forceinline__ void topk_memory(const uint32_t* row, int nb, const Cands& cd, int k, int32_t* sel,
+                                            uint32_t* skey, int key_cap, uint32_t* gkeys, TopkSmem<NT>& sm,
+                                            int32_t* dev_status) {
+  uint32_t* keys = nb <= key_cap ? skey : gkeys;
   uint32_t kmin, kmax;
-  load_keys(row, keys, nb, sm, kmin, kmax);
-  select_from_keys(keys, nb, k, kmin, kmax, sel, sm, dev_status);
+  load_keys(row, keys, nb, cd, sm, kmin, kmax);
+  select_from_keys(keys, nb, cd, k, kmin, kmax, sel, sm, dev_status);
 }
 
 // The top-k of one pair with nb <= KPT * NT blocks, keys held in registers:
@@ -433,7 +443,7 @@ __device__ __forceinline__ void topk_memory(const uint32_t* row, int nb, int k, 
 // packed counts, every warp scans them, and every thread writes its taken
 // indices at their final positions.
 template <int NT, int KPT>
-__device__ __forceinline__ void topk_regs(const uint32_t* row, int nb, int k, int32_t* sel, uint32_t* skey,
+__device__ __forceinline__ void topk_regs(const uint32_t* row, int nb, const Cands& cd, int k, int32_t* sel, uint32_t* skey,
                                           TopkSmem<NT>& sm, int32_t* dev_status) {
   constexpr int NW = NT / 32;
   constexpr int kPerLane = KPT * NW / 32;  // slots per lane in the emit's scan
@@ -450,7 +460,7 @@ __device__ __forceinline__ void topk_regs(const uint32_t* row, int nb, int k, in
   for (int u = 0; u < KPT; ++u) {
     const int i = u * NT + tid;
     key[u] = key_of_bits(key[u]);
-    if (i >= 1 && i <= nb - 2) {
+    if (cd.has(i)) {
       lo = min(lo, key[u]);
       hi = max(hi, key[u]);
     }
@@ -471,8 +481,8 @@ __device__ __forceinline__ void topk_regs(const uint32_t* row, int nb, int k, in
     kmax = max(kmax, sm.wmax[w]);
   }
 
-  const int kr = k - 2;
-  uint32_t T = 0xFFFFFFFFu;  // budget of two: no candidate is above T, none equal is taken
+  const int kr = cd.kr;
+  uint32_t T = 0xFFFFFFFFu;  // kr == 0: no candidate is above T, none equal is taken
   int take = 0;
   if (kr > 0) {
     const float flo = key_float(kmin), fhi = key_float(kmax);
@@ -485,7 +495,7 @@ __device__ __forceinline__ void topk_regs(const uint32_t* row, int nb, int k, in
 #pragma unroll
       for (int u = 0; u < KPT; ++u) {
         const int i = u * NT + tid;
-        if (i >= 1 && i <= nb - 2) atomicAdd(&sm.hist[0][hidx(bin_of(key[u]))], 1);
+        if (cd.has(i)) atomicAdd(&sm.hist[0][hidx(bin_of(key[u]))], 1);
       }
       __syncthreads();
       warp_find_bin(sm.hist[0], kr, bstar, above, c);  // every warp, same result
@@ -501,18 +511,18 @@ __device__ __forceinline__ void topk_regs(const uint32_t* row, int nb, int k, in
       zero_hist(sm, 0);
       zero_hist(sm, 1);
       __syncthreads();
-      for (int i = 1 + tid; i <= nb - 2; i += NT) atomicAdd(&sm.hist[0][hidx(skey[i] >> 24)], 1);
+      for (int i = cd.lo + tid; i <= cd.hi; i += NT) atomicAdd(&sm.hist[0][hidx(skey[i] >> 24)], 1);
       __syncthreads();
       uint32_t prefix, mask;
       int kr2 = kr;
-      radix_threshold(skey, nb, sm, prefix, mask, kr2);
-      emit_selection(skey, nb, k, prefix, mask, kr2, sel, sm, dev_status);
+      radix_threshold(skey, nb, cd, sm, prefix, mask, kr2);
+      emit_selection(skey, nb, cd, k, prefix, mask, kr2, sel, sm, dev_status);
       return;
     }
 #pragma unroll
     for (int u = 0; u < KPT; ++u) {
       const int i = u * NT + tid;
-      const bool match = i >= 1 && i <= nb - 2 && bin_of(key[u]) == bstar;
+      const bool match = cd.has(i) && bin_of(key[u]) == bstar;
       const unsigned m = __ballot_sync(0xffffffffu, match);
       int slot = 0;
       if (lane == 0 && m) slot = atomicAdd(&sm.list_n, __popc(m));
@@ -529,7 +539,7 @@ __device__ __forceinline__ void topk_regs(const uint32_t* row, int nb, int k, in
   const unsigned lt = (1u << lane) - 1u;
   auto flags = [&](int u, bool& g, bool& e) {
     const int i = u * NT + tid;
-    const bool cand = i >= 1 && i <= nb - 2;
+    const bool cand = cd.has(i);
     g = (i < nb && !cand) || (cand && key[u] > T);
     e = cand && key[u] == T;
   };
@@ -722,10 +732,58 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_topk_kernel(SelectParams
     return;
   }
   const uint32_t* row = reinterpret_cast<const uint32_t*>(p.scores + pair * p.nbcap);
-  if (nb <= 4 * NT) topk_regs<NT, 4>(row, nb, k, sel, skey, sm, p.dev_status);
-  else if (nb <= 8 * NT) topk_regs<NT, 8>(row, nb, k, sel, skey, sm, p.dev_status);
-  else topk_memory<NT>(row, nb, k, sel, skey, p.nbcap, sm, p.dev_status);
+  const Cands cd{1, nb - 2, k - 2};  // blocks 0 and nb - 1 forced
+  if (nb <= 4 * NT) topk_regs<NT, 4>(row, nb, cd, k, sel, skey, sm, p.dev_status);
+  else if (nb <= 8 * NT) topk_regs<NT, 8>(row, nb, cd, k, sel, skey, sm, p.dev_status);
+  else topk_memory<NT>(row, nb, cd, k, sel, skey, p.nbcap, const_cast<uint32_t*>(row), sm, p.dev_status);
   if (tid == 0) p.sel_cnt[pair] = k;
+}
+
+// ---- token-level top-k: one 1024-thread CTA per (sequence, query head)
+// keeps the k tokens with the largest logits (ties to the lower index,
+// nothing forced), ascending, -1 padded; every token when k >= L.
+constexpr int kTokTopkThreads = 1024;
+constexpr int kTokKeyCap = 32768;  // keys kept in shared memory up to this many tokens
+
+__global__ void __launch_bounds__(kTokTopkThreads, 1) token_topk_kernel(TokenParams p) {
+  extern __shared__ uint32_t skey[];  // [min(Lcap, kTokKeyCap)]
+  __shared__ TopkSmem<kTokTopkThreads> sm;
+  const int tid = threadIdx.x;
+  pdl_wait();  // the logits come from the logits kernel
+  pdl_trigger_early();
+  const int64_t row_id = blockIdx.x;  // b * Hq + query head
+  const int b = (int)(row_id / p.Hq);
+  const int k = p.kt;
+  int32_t* sel = p.sel + row_id * k;
+  const int L = __ldg(p.seq_lens + b);
+  if (L < 1 || L > p.Lcap) {
+    for (int i = tid; i < k; i += kTokTopkThreads) sel[i] = -1;
+    if (tid == 0) {
+      p.cnt[row_id] = 0;
+      set_status(p.dev_status, KIN_ERR_DEVICE_DATA);
+    }
+    return;
+  }
+  if (L <= k) {
+    for (int i = tid; i < k; i += kTokTopkThreads) sel[i] = i < L ? i : -1;
+    if (tid == 0) p.cnt[row_id] = L;
+    return;
+  }
+  const uint32_t* row = reinterpret_cast<const uint32_t*>(p.logits + row_id * p.Lcap);
+  const Cands cd{0, L - 1, k};
+  if (L <= 4 * kTokTopkThreads) topk_regs<kTokTopkThreads, 4>(row, L, cd, k, sel, skey, sm, p.dev_status);
+  else if (L <= 8 * kTokTopkThreads) topk_regs<kTokTopkThreads, 8>(row, L, cd, k, sel, skey, sm, p.dev_status);
+  else
+    topk_memory<kTokTopkThreads>(row, L, cd, k, sel, skey, kTokKeyCap, p.key_scratch + row_id * p.Lcap, sm,
+                                 p.dev_status);
+  if (tid == 0) p.cnt[row_id] = k;
+}
+
+cudaError_t launch_token_topk(const TokenParams& p, cudaStream_t s) {
+  const size_t smem = (size_t)(p.Lcap < kTokKeyCap ? p.Lcap : kTokKeyCap) * sizeof(uint32_t);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(token_topk_kernel), 5, smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(token_topk_kernel, dim3(p.B * p.Hq), dim3(kTokTopkThreads), smem, s, p);
 }
 
 // Threads per top-k CTA: enough for 4 keys per thread (up to 4096 blocks),

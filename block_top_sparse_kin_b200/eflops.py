@@ -77,6 +77,18 @@ def step_costs(B: int, Hkv: int, Hq: int, D: int, bs: int, lens, k: int, n_appen
     return parts
 
 
+def token_step_costs(B: int, Hkv: int, Hq: int, D: int, lens, k_tokens: int) -> dict:
+    """A and M of token-level top-k attention: every logit of every query
+    head (2 D FLOPs per token and head, every K row read), then p.V over the
+    k kept tokens of each head (2 D FLOPs, one V row each)."""
+    lens = np.asarray(lens, dtype=np.int64)
+    kept = np.minimum(k_tokens, lens)
+    q_out = 2 * B * Hq * D * 2
+    logits = Cost(2.0 * D * Hq * float(lens.sum()), float(Hkv * lens.sum() * D * 2))
+    attn = Cost(2.0 * D * Hq * float(kept.sum()), float(Hq * kept.sum() * D * 2 + q_out))
+    return {"logits": logits, "attn": attn}
+
+
 def eflops(cost: Cost, peak_flops: float, bandwidth: float) -> dict:
     """eFLOPs = A + I M with I = C / B, and the predicted time T = eFLOPs / C
     (= A/C + M/B)."""

@@ -215,6 +215,31 @@ kin_status kin_block_topk_select_ex(const kin_dims* dims, const void* q, const v
                                     int32_t* dev_status, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Token-level top-k attention (the variant the block method is compared
+ * with: "Kinetics: Rethinking Test-Time Scaling Law", response Q2, Fig. 8's
+ * TopK attention; TopK attention keeps the keys and values with the highest
+ * attention scores).  For query head j of sequence b, over the tokens
+ * t < seq_lens[b] of the contiguous cache:
+ *   z_t = softmax_scale * q[b][j] . K_t            (every token: a dense K pass)
+ *   S   = the k_tokens tokens with the largest z_t (ties to the lower index,
+ *         nothing forced; every token when k_tokens >= seq_lens[b])
+ *   out[b][j] = sum_{t in S} e^{z_t - max z} V_t / sum_{t in S} e^{z_t - max z}
+ *   lse[b][j] = max z + ln sum_{t in S} e^{z_t - max z}      (max over S)
+ * Each query head selects its own tokens (a GQA group does not share them).
+ * sel_tokens ([B][Hq][k_tokens] int32, ascending, -1 padded) receives S when
+ * not NULL.  softmax_scale <= 0 selects 1/sqrt(D); lse may be NULL.  A bad
+ * length gets out = 0, lse = -inf and flags KIN_ERR_DEVICE_DATA.  Scratch:
+ * kin_token_topk_workspace_bytes (256-byte aligned; no zeroing needed; the
+ * fp32 logits of every token of every query head live there).  k_tokens < 1
+ * is KIN_ERR_INVALID_ARG; B * Hq * max_seq_len must stay below 2^31. */
+size_t kin_token_topk_workspace_bytes(const kin_dims* dims, int32_t k_tokens);
+
+kin_status kin_token_topk_decode_attn(const kin_dims* dims, const void* q, const void* k_cache,
+                                      const void* v_cache, const int32_t* seq_lens, int32_t k_tokens,
+                                      float softmax_scale, void* out, float* lse, int32_t* sel_tokens,
+                                      void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------
  * Allocation-free variant of kin_block_topk_select (the pages describe no
  * counterpart; it exists for callers, not for the method).
  *

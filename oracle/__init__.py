@@ -212,3 +212,37 @@ def round_bf16(x: np.ndarray) -> np.ndarray:
 def block_means_bf16(K: np.ndarray, L: int, bs: int) -> np.ndarray:
     """block_means rounded to bf16 precision (fp64 array)."""
     return round_bf16(block_means(K, L, bs))
+
+
+def token_topk_attend(q_group: np.ndarray, K: np.ndarray, V: np.ndarray, L: int, k_tokens: int, scale: float):
+    """Token-level TopK attention for each query head of one group, in fp64:
+    the logits z_t = scale q_j . K_t of every token t < L, the k_tokens tokens
+    with the largest z_t (ties to the lower index; every token when
+    k_tokens >= L), then softmax over those tokens and the weighted sum of
+    their V rows.  TopK attention keeps the keys and values with the highest
+    attention scores ("Kinetics: Rethinking Test-Time Scaling Law", response
+    Q2, Fig. 8's variant; MagicPIG's abstract on the same pages).
+    q_group [g, D], K, V [>= L, D] as bf16 bits.  Returns (sel [g, min(k, L)]
+    ascending, out [g, D], lse [g], z [g, L])."""
+    q = bf16_bits_to_f64(q_group)
+    Kf = bf16_bits_to_f64(np.asarray(K)[:L])
+    Vf = bf16_bits_to_f64(np.asarray(V)[:L])
+    z = scale * (q @ Kf.T)                         # [g, L]
+    n = min(k_tokens, L)
+    sels, outs, lses = [], [], []
+    for j in range(z.shape[0]):
+        order = np.lexsort((np.arange(L), -z[j]))  # z descending, index ascending
+        s = np.sort(order[:n])
+        zs = z[j, s]
+        m = zs.max()
+        w = np.exp(zs - m)
+        outs.append((w[:, None] * Vf[s]).sum(axis=0) / w.sum())
+        lses.append(m + np.log(w.sum()))
+        sels.append(s)
+    return np.array(sels), np.array(outs), np.array(lses), z
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) widened exactly to fp64."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)

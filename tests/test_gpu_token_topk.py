@@ -1,0 +1,105 @@
+"""Token-level top-k attention on the GPU (kin_token_topk_decode_attn)
+against the fp64 oracle on the same bf16 inputs.
+
+Kept token sets must match the oracle's except for swaps between tokens
+whose oracle logits lie within delta = 1e-4 max(|tau_k|, |tau_k+1|, eps) of
+the k-th / (k+1)-th largest logit (eps: the logits' natural magnitude, the
+mean over tokens of scale sum_d |q_d| |K_td|); outputs are then compared
+with the oracle recomputed on the GPU's set (max |err| <= 2e-2, mean
+<= 2e-3; lse within 1e-3 + 1e-4 |lse|)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import block_top_sparse_kin_b200 as kin
+import kin_inputs as ki
+import oracle
+from kin_testlib import D, make_device_case
+
+pytestmark = pytest.mark.gpu
+W = ki.Workload
+TIE_REL = 1e-4
+
+
+def run_token(dc, kt):
+    w = dc.w
+    ws = kin.alloc_token_workspace(dc.dims, kt)
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
+    sel = torch.full((w.B, w.Hq, kt), -7, dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kin.kin_token_topk_decode_attn(dc.dims, dc.q, dc.k_cache, dc.v_cache, dc.seq_lens, kt, 0.0, out, lse, ws,
+                                   sel_tokens=sel, dev_status=st)
+    torch.cuda.synchronize()
+    return sel.cpu().numpy(), out.float().cpu().numpy(), lse.cpu().numpy(), int(st.item())
+
+
+def check_head(dc, b, j, kt, sel, out, lse):
+    w = dc.w
+    h = j // w.g
+    L = int(dc.lens_final[b])
+    K, V = ki.pair_rows(w, dc.hh, b, h, L)
+    q = dc.q_host[b, j:j + 1]
+    scale = 1 / math.sqrt(D)
+    rsel, rout, rlse, z = oracle.token_topk_attend(q, K, V, L, kt, scale)
+    n = min(kt, L)
+    gsel = sel[b, j]
+    assert np.all(gsel[n:] == -1), (b, j)
+    g = gsel[:n]
+    assert np.all(np.diff(g) > 0), (b, j, "not ascending")
+    if not np.array_equal(g, rsel[0]):
+        zs = np.sort(z[0])[::-1]
+        tau_k, tau_k1 = zs[n - 1], zs[n] if n < L else zs[n - 1]
+        eps = scale * (np.abs(oracle.bf16_bits_to_f64(q[0])) @ np.abs(oracle.bf16_bits_to_f64(K[:L])).T).mean()
+        delta = TIE_REL * max(abs(tau_k), abs(tau_k1), eps)
+        for t in set(g.tolist()) ^ set(rsel[0].tolist()):
+            assert min(abs(z[0, t] - tau_k), abs(z[0, t] - tau_k1)) <= delta, (b, j, t)
+        # outputs against the oracle on the GPU's set
+        zz = z[0, g]
+        m = zz.max()
+        wts = np.exp(zz - m)
+        rout = ((wts[:, None] * oracle.bf16_bits_to_f64(V[g])).sum(0) / wts.sum())[None]
+        rlse = np.array([m + np.log(wts.sum())])
+    err = np.abs(out[b, j].astype(np.float64) - rout[0])
+    assert err.max() <= 2e-2 and err.mean() <= 2e-3, (b, j, err.max(), err.mean())
+    assert abs(lse[b, j] - rlse[0]) <= 1e-3 + 1e-4 * abs(rlse[0]), (b, j, lse[b, j], rlse[0])
+
+
+@pytest.mark.parametrize("w,kt", [
+    (W("tok_g4", 2, 2, 8, D, 16, 700, 1000, 8, 90, Lcap=1024), 96),
+    (W("tok_g1_ragged", 3, 1, 1, D, 16, 20, 600, 8, 91, Lcap=640), 50),
+    (W("tok_g8_long", 1, 1, 8, D, 16, 0, 0, 8, 92, Lcap=9000, lens=(8999,)), 700),
+    (W("tok_dense_and_len1", 3, 1, 2, D, 16, 0, 0, 8, 93, Lcap=128, lens=(100, 1, 33)), 64),
+    (W("tok_k1", 2, 2, 4, D, 16, 50, 300, 8, 94, Lcap=320), 1),
+], ids=lambda x: x.name if hasattr(x, "name") else str(x))
+def test_token_topk_every_head(w, kt):
+    dc = make_device_case(w)
+    sel, out, lse, status = run_token(dc, kt)
+    assert status == 0
+    for b in range(w.B):
+        for j in range(w.Hq):
+            check_head(dc, b, j, kt, sel, out, lse)
+
+
+def test_token_topk_bad_length_is_flagged():
+    w = W("tok_bad", 2, 1, 2, D, 16, 0, 0, 8, 95, Lcap=128, lens=(100, 60))
+    dc = make_device_case(w)
+    dc.seq_lens[1] = 500
+    sel, out, lse, status = run_token(dc, 16)
+    assert status == 5
+    assert np.all(out[1] == 0) and np.all(np.isneginf(lse[1])) and np.all(sel[1] == -1)
+    check_head(dc, 0, 0, 16, sel, out, lse)
+
+
+def test_token_topk_32k_workload_sampled():
+    """The 32K decode batch with a token budget equal to the block budget
+    (256 blocks x 16 tokens = 4096 tokens per query head), sampled heads."""
+    w = ki.WORKLOADS["qwen3_8b_32k"]
+    dc = make_device_case(w)
+    kt = w.k * w.bs
+    sel, out, lse, status = run_token(dc, kt)
+    assert status == 0
+    for b, j in [(0, 0), (7, 13), (19, 30), (31, 31)]:
+        check_head(dc, b, j, kt, sel, out, lse)

@@ -302,3 +302,59 @@ def test_round_bf16_matches_torch_conversion():
     # ties go to even: 1 + 2^-8 sits halfway between 1 and 1 + 2^-7
     assert oracle.round_bf16(np.array([1 + 2.0 ** -8]))[0] == 1.0
     assert oracle.round_bf16(np.array([1 + 3 * 2.0 ** -8]))[0] == 1 + 2.0 ** -6
+
+
+def _bits(x):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_token_topk_full_budget_is_dense_attention():
+    import torch
+    rng = np.random.default_rng(21)
+    g, L, D = 3, 57, 128
+    q = _bits(rng.normal(size=(g, D)))
+    K = _bits(rng.normal(size=(L + 5, D)))
+    V = _bits(rng.normal(size=(L + 5, D)))
+    scale = 1 / np.sqrt(D)
+    sel, out, lse, _ = oracle.token_topk_attend(q, K, V, L, L + 3, scale)
+    assert np.array_equal(sel, np.tile(np.arange(L), (g, 1)))
+    qt = torch.from_numpy(oracle.bf16_bits_to_f64(q))[:, None, None, :]
+    kt = torch.from_numpy(oracle.bf16_bits_to_f64(K[:L]))[None, None]
+    vt = torch.from_numpy(oracle.bf16_bits_to_f64(V[:L]))[None, None]
+    want = torch.nn.functional.scaled_dot_product_attention(qt, kt.expand(g, 1, L, D), vt.expand(g, 1, L, D))
+    assert np.allclose(out, want[:, 0, 0].numpy(), atol=1e-12, rtol=0)
+    logits = (qt[:, 0, 0] @ kt[0, 0].T) * scale
+    assert np.allclose(lse, torch.logsumexp(logits, dim=-1).numpy(), atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("trial", range(20))
+def test_token_topk_keeps_the_best_set(trial):
+    """Brute force over every token subset of the budget's size: the kept set
+    maximises the summed logit and is the lexicographically smallest such set
+    (ties to the lower index); dyadic logits make ties exact."""
+    rng = np.random.default_rng(100 + trial)
+    L, D = int(rng.integers(3, 11)), 128
+    n = int(rng.integers(1, L))
+    q = np.zeros((1, D), np.float32)
+    q[0, 0] = 1.0
+    K = np.zeros((L, D), np.float32)
+    K[:, 0] = rng.integers(-3, 4, size=L) * 0.5
+    sel, _, _, z = oracle.token_topk_attend(_bits(q), _bits(K), _bits(K), L, n, 1.0)
+    best = max(itertools.combinations(range(L), n), key=lambda s: (sum(z[0, list(s)]), [-i for i in s]))
+    assert list(sel[0]) == list(best)
+
+
+def test_token_topk_weights_are_softmax_of_kept_logits_only():
+    from scipy.special import logsumexp, softmax
+    rng = np.random.default_rng(7)
+    L, D, n = 40, 128, 9
+    q = _bits(rng.normal(size=(1, D)))
+    K = _bits(rng.normal(size=(L, D)))
+    V = _bits(np.eye(L, D, dtype=np.float32))      # one-hot rows: out exposes the weights (L <= D)
+    sel, out, lse, z = oracle.token_topk_attend(q, K, V, L, n, 0.2)
+    w = np.zeros(L)
+    w[sel[0]] = softmax(z[0, sel[0]])
+    assert np.allclose(out[0, :L], w, atol=1e-14)
+    assert np.all(out[0, :L][np.setdiff1d(np.arange(L), sel[0])] == 0)
+    assert np.isclose(lse[0], logsumexp(z[0, sel[0]]), atol=1e-12)
