@@ -65,6 +65,34 @@ def algorithmic_bytes(w: ki.Workload, k: int, lens: np.ndarray, means_bytes: int
     return sel_bytes, attn_bytes
 
 
+def shared_algorithmic_bytes(w: ki.Workload, k: int, st, means_bytes: int = 4):
+    """Algorithmic bytes when groups of samples share their prompt's pages
+    and per-page means, each shared item read once: (select) the distinct
+    mean rows (page, head) of the scanned sequences; (attention) the
+    distinct kept K/V blocks (page, head) of each group, a full shared page
+    counted once, plus q, out and indices.  Uses the step's selection."""
+    lens = st["lens_final"].astype(np.int64)
+    table = st["table_host"]
+    sel = st["sel"].cpu().numpy()
+    cnt = st["cnt"].cpu().numpy()
+    nb = -(-lens // w.bs)
+    scanned = nb > k
+    pages = set()
+    for b in np.nonzero(scanned)[0]:
+        pages.update(table[b, :nb[b]].tolist())
+    q_bytes = w.B * w.Hq * w.D * 2
+    idx_bytes = w.B * w.Hkv * k * 4
+    sel_bytes = len(pages) * w.Hkv * w.D * means_bytes + q_bytes + idx_bytes
+    kept = {}  # (page, head) -> valid tokens
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            for blk in sel[b, h, :cnt[b, h]]:
+                key = (int(table[b, blk]), h)
+                kept[key] = max(kept.get(key, 0), int(min(w.bs, lens[b] - blk * w.bs)))
+    attn_bytes = sum(kept.values()) * w.D * 2 * 2 + q_bytes + w.B * w.Hq * w.D * 2 + idx_bytes
+    return sel_bytes, attn_bytes
+
+
 def token_algorithmic_bytes(w: ki.Workload, kt: int, lens: np.ndarray):
     """Algorithmic HBM bytes of one token-level top-k step: every K row (the
     logits pass), the kept V rows of every query head, q and the bf16 out.
@@ -237,25 +265,45 @@ def shard_workload(w: ki.Workload, rank: int) -> ki.Workload:
     return w.with_(seed=w.seed + 1000 * rank) if rank else w
 
 
-def make_page_pool(st, seed: int):
+SHARED_GEN_TOKENS = 2048  # tokens each Best-of-N sample generated after the shared prompt
+
+
+def make_page_pool(st, seed: int, share_n: int = 1, shuffle: bool = True):
     """Moves the contiguous K/V caches into a shuffled page pool (page = one
     KV block, [num_pages, Hkv, bs, D]) with a block table [B, nbcap]: every
     block a sequence holds after the step's append gets a page, in random
-    order.  Frees the contiguous caches."""
+    order.  share_n > 1: consecutive groups of share_n sequences are samples
+    of one prompt; the prompt's blocks (all but the last SHARED_GEN_TOKENS
+    tokens of the group's shortest sequence, whole blocks) map to the pages
+    of the group's first sample.  shuffle=False keeps the pages in the order
+    the sequences fill them (as a prefill allocator would).  Frees the
+    contiguous caches."""
     import torch
     w = st["w"]
     B, Hkv, cap, D = st["k_cache"].shape
     bs, nbcap = w.bs, w.nbcap
-    nbs = [-(-int(L) // bs) for L in st["lens_final"]]
-    P = sum(nbs)
-    order = np.random.default_rng(seed).permutation(P)
-    table = np.full((B, nbcap), -1, np.int32)
-    j = 0
+    lens = st["lens_final"]
+    nbs = [-(-int(L) // bs) for L in lens]
+    owner = []
+    table = np.full((B, nbcap), -1, np.int64)
     for b in range(B):
-        table[b, :nbs[b]] = order[j:j + nbs[b]]
-        j += nbs[b]
-    ib, ii = np.nonzero(table >= 0)
-    dst = torch.from_numpy(table[ib, ii].astype(np.int64)).cuda()
+        first = b - b % share_n
+        shared = 0
+        if share_n > 1:
+            group_min = int(min(lens[first:first + share_n]) - w.n_append)
+            shared = max(0, (group_min - SHARED_GEN_TOKENS) // bs)
+        for i in range(nbs[b]):
+            if i < shared and b != first:
+                table[b, i] = table[first, i]
+            else:
+                table[b, i] = len(owner)
+                owner.append((b, i))
+    P = len(owner)
+    order = np.random.default_rng(seed).permutation(P) if shuffle else np.arange(P)
+    table = np.where(table >= 0, order[np.maximum(table, 0)], -1).astype(np.int32)
+    ib = np.array([o[0] for o in owner])
+    ii = np.array([o[1] for o in owner])
+    dst = torch.from_numpy(order.astype(np.int64)).cuda()
     tb, ti = torch.from_numpy(ib).cuda(), torch.from_numpy(ii).cuda()
     for name in ("k_cache", "v_cache"):
         cache = st.pop(name)
@@ -269,11 +317,13 @@ def make_page_pool(st, seed: int):
         st[name.replace("cache", "pages")] = pool
         del cache, blocks
     st["table"] = torch.from_numpy(table).cuda()
+    st["table_host"] = table
     st["num_pages"] = P
     torch.cuda.empty_cache()
 
 
-def build_device_state(w: ki.Workload, k: int, paged: bool = False, means_bf16: bool = False):
+def build_device_state(w: ki.Workload, k: int, paged: bool = False, means_bf16: bool = False, share_n: int = 1,
+                       shuffle_pages: bool = True):
     import torch
     import block_top_sparse_kin_b200 as kin
     lens_final, lens_pre, hh = ki.case_meta(w)
@@ -311,8 +361,15 @@ def build_device_state(w: ki.Workload, k: int, paged: bool = False, means_bf16: 
     st["lse"] = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
     st["status"] = torch.zeros(1, dtype=torch.int32, device="cuda")
     st["ws"] = kin.alloc_workspace(dims, k)
-    if paged:
-        make_page_pool(st, w.seed)
+    if paged or share_n > 1:
+        make_page_pool(st, w.seed, share_n, shuffle_pages)
+    if share_n > 1:  # block means per page: the shared prompt's means exist once
+        st["means"] = torch.zeros((st["num_pages"], w.Hkv, w.D),
+                                  dtype=torch.bfloat16 if means_bf16 else torch.float32, device="cuda")
+        st["seq"].copy_(st["seq_pre"])
+        kin.kin_block_means_build_ex(dims, st["k_pages"], st["seq"], st["means"], block_table=st["table"],
+                                     per_page=True)
+        st["page_means"] = True
     torch.cuda.synchronize()
     return st
 
@@ -344,9 +401,10 @@ def append(st):
     w = st["w"]
     paged = "table" in st
     k_rows, v_rows = (st["k_pages"], st["v_pages"]) if paged else (st["k_cache"], st["v_cache"])
-    if str(st["means"].dtype) == "torch.bfloat16":
+    if "page_means" in st or str(st["means"].dtype) == "torch.bfloat16":
         kin.kin_block_means_update_ex(st["dims"], k_rows, v_rows, st["means"], st["seq"], st["k_new"], st["v_new"],
-                                      w.n_append, block_table=st.get("table"), dev_status=st["status"])
+                                      w.n_append, block_table=st.get("table"), dev_status=st["status"],
+                                      per_page="page_means" in st)
     elif paged:
         kin.kin_block_means_update_paged(st["dims"], k_rows, v_rows, st["table"], st["means"], st["seq"],
                                          st["k_new"], st["v_new"], w.n_append, st["status"])
@@ -358,7 +416,10 @@ def append(st):
 def select(st):
     """The step's block scoring and top-k (fp32 means, or bf16 through the extended call)."""
     import block_top_sparse_kin_b200 as kin
-    if str(st["means"].dtype) == "torch.bfloat16":
+    if "page_means" in st:
+        kin.kin_block_topk_select_paged(st["dims"], st["q"], st["means"], st["table"], st["seq"], st["k"], st["sel"],
+                                        st["cnt"], st["ws"], st["status"])
+    elif str(st["means"].dtype) == "torch.bfloat16":
         kin.kin_block_topk_select_ex(st["dims"], st["q"], st["means"], st["seq"], st["k"], st["sel"], st["cnt"],
                                      st["ws"], st["status"])
     else:
@@ -399,9 +460,10 @@ def gpu_arm(args):
         w0 = w0.with_(B=args.batch, name=f"{w0.name}_b{args.batch}")
     k = args.k or w0.k
     w = shard_workload(w0, rank)
-    st = build_device_state(w, k, paged=args.paged, means_bf16=args.means_bf16)
+    st = build_device_state(w, k, paged=args.paged, means_bf16=args.means_bf16, share_n=args.shared_prefix,
+                            shuffle_pages=args.page_order == "shuffled")
     if args.token_topk:
-        if args.paged:
+        if args.paged or args.shared_prefix > 1:
             raise SystemExit("--token-topk reads the contiguous cache")
         import block_top_sparse_kin_b200 as kin_mod
         st["token_kt"] = k * w.bs  # the block budget in tokens, per query head
@@ -445,7 +507,10 @@ def gpu_arm(args):
         parts = [("token_topk_attn", lambda: token_step(st),
                   token_algorithmic_bytes(w, st["token_kt"], st["lens_final"]), "kin_token.cu")]
     else:
-        sel_b, attn_b = algorithmic_bytes(w, k, st["lens_final"], means_bytes)
+        if args.shared_prefix > 1:  # shared items counted once (the step's selection, from warm-up)
+            sel_b, attn_b = shared_algorithmic_bytes(w, k, st, means_bytes)
+        else:
+            sel_b, attn_b = algorithmic_bytes(w, k, st["lens_final"], means_bytes)
         parts = [("select", lambda: select(st), sel_b, "kin_select.cu"),
                  ("attn", lambda: attend(st), attn_b, "kin_attn.cu")]
 
@@ -578,8 +643,11 @@ def gpu_arm(args):
                 "top_k_blocks": k, "append_tokens": w0.n_append,
                 "global_batch": w0.B * world, "parallelism": f"dp{world}",
                 "l2": "flushed before every step (256 MiB write + 256 MiB read, outside the timed events)",
-                "kv_layout": (f"paged: {st['num_pages']} pages of one {w.bs}-token block, shuffled pool + block table"
-                              if args.paged else "contiguous [B][Hkv][Lcap][D]"),
+                "kv_layout": (f"paged: {st['num_pages']} pages of one {w.bs}-token block, {args.page_order} pool"
+                              f" + block table"
+                              + (f"; groups of {args.shared_prefix} samples share their prompt's pages and"
+                                 f" per-page means" if args.shared_prefix > 1 else "")
+                              if "table" in st else "contiguous [B][Hkv][Lcap][D]"),
                 "block_means": "bf16" if args.means_bf16 else "fp32",
                 **({"attention": f"token-level top-k, {st['token_kt']} tokens per query head"} if args.token_topk else {}),
             },
@@ -719,6 +787,10 @@ def main():
     ap.add_argument("--ref-pairs", type=int, default=8, help="pairs per reference-arm step")
     ap.add_argument("--paged", action="store_true", help="KV cache in a shuffled page pool with a block table")
     ap.add_argument("--means-bf16", action="store_true", help="bf16 block means (the extended calls)")
+    ap.add_argument("--page-order", default="shuffled", choices=["shuffled", "sequential"],
+                    help="page pool order for --paged / --shared-prefix")
+    ap.add_argument("--shared-prefix", type=int, default=1,
+                    help="groups of N samples share a prompt (paged, block means per page)")
     ap.add_argument("--token-topk", action="store_true",
                     help="token-level top-k attention instead of the block path (budget = k blocks x bs tokens)")
     args = ap.parse_args()

@@ -29,8 +29,10 @@ EXPORTED = (
     "kin_block_topk_select_noalloc", "kin_block_means_build_paged", "kin_block_means_update_paged",
     "kin_sparse_decode_attn_paged", "kin_block_means_build_ex", "kin_block_means_update_ex",
     "kin_block_topk_select_ex", "kin_token_topk_workspace_bytes", "kin_token_topk_decode_attn",
+    "kin_block_topk_select_paged",
 )
 KIN_MEANS_F32, KIN_MEANS_BF16 = 0, 1
+KIN_MEANS_PER_PAGE = 0x100
 NOALLOC_SCRATCH_FLOATS = 1 << 21  # KIN_NOALLOC_SCRATCH_FLOATS in include/kin.h
 
 
@@ -105,6 +107,8 @@ def load_library(path: str = LIB_PATH):
     lib.kin_token_topk_workspace_bytes.restype = sz
     lib.kin_token_topk_decode_attn.argtypes = [dp, vp, vp, vp, vp, i32, f32, vp, vp, vp, vp, sz, vp, vp]
     lib.kin_token_topk_decode_attn.restype = ctypes.c_int
+    lib.kin_block_topk_select_paged.argtypes = [dp, vp, vp, i32, i32, vp, vp, i32, vp, vp, vp, sz, vp, vp]
+    lib.kin_block_topk_select_paged.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -263,9 +267,11 @@ def _layout(rows, block_table):
 
 
 def kin_block_means_build_ex(dims, k_rows, seq_lens, block_means, block_table=None, dev_status=None,
-                             stream=None):
+                             stream=None, per_page=False):
+    """per_page: block_means is [num_pages, Hkv, D] (one mean per page; needs block_table)."""
     pages, table = _layout(k_rows, block_table)
     means, dtype = _means(block_means)
+    dtype |= KIN_MEANS_PER_PAGE if per_page else 0
     rc = load_library().kin_block_means_build_ex(
         ctypes.byref(dims), _dev(k_rows, "k_rows", _BF16), pages, table, _dev(seq_lens, "seq_lens", torch.int32),
         means, dtype, _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
@@ -273,9 +279,10 @@ def kin_block_means_build_ex(dims, k_rows, seq_lens, block_means, block_table=No
 
 
 def kin_block_means_update_ex(dims, k_rows, v_rows, block_means, seq_lens, k_new, v_new, n_new,
-                              block_table=None, dev_status=None, stream=None):
+                              block_table=None, dev_status=None, stream=None, per_page=False):
     pages, table = _layout(k_rows, block_table)
     means, dtype = _means(block_means)
+    dtype |= KIN_MEANS_PER_PAGE if per_page else 0
     rc = load_library().kin_block_means_update_ex(
         ctypes.byref(dims), _dev(k_rows, "k_rows", _BF16), _dev(v_rows, "v_rows", _BF16), pages, table,
         means, dtype, _dev(seq_lens, "seq_lens", torch.int32), _dev(k_new, "k_new", _BF16),
@@ -318,3 +325,17 @@ def kin_token_topk_decode_attn(dims, q, k_cache, v_cache, seq_lens, k_tokens, so
         workspace.numel() * workspace.element_size(),
         _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
     _check(rc, "kin_token_topk_decode_attn")
+
+
+def kin_block_topk_select_paged(dims, q, page_means, block_table, seq_lens, k_blocks, sel_idx, sel_cnt, workspace,
+                                dev_status=None, stream=None):
+    """The select over per-page block means [num_pages, Hkv, D] (fp32 or bf16),
+    found through block_table: the shared-prompt layout (see include/kin.h)."""
+    means, dtype = _means(page_means)
+    rc = load_library().kin_block_topk_select_paged(
+        ctypes.byref(dims), _dev(q, "q", _BF16), means, dtype, int(page_means.shape[0]),
+        _dev(block_table, "block_table", torch.int32), _dev(seq_lens, "seq_lens", torch.int32), int(k_blocks),
+        _dev(sel_idx, "sel_idx", torch.int32), _dev(sel_cnt, "sel_cnt", torch.int32), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(),
+        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+    _check(rc, "kin_block_topk_select_paged")

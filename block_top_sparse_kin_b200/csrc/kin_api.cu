@@ -160,8 +160,9 @@ KIN_EXPORT size_t kin_workspace_bytes(const kin_dims* dims, int32_t k_blocks) {
 namespace {
 
 kin_status means_build(const kin_dims* dims, const void* k_rows, const PageTable& pt, const int32_t* seq_lens,
-                       void* block_means, int means_bf16, int32_t* dev_status, void* stream) {
+                       void* block_means, int means_bf16, int32_t* dev_status, void* stream, int per_page = 0) {
   MeansBuildParams p;
+  p.means_per_page = per_page;
   p.k_cache = static_cast<const __nv_bfloat16*>(k_rows);
   p.seq_lens = seq_lens;
   p.means = block_means;
@@ -178,8 +179,9 @@ kin_status means_build(const kin_dims* dims, const void* k_rows, const PageTable
 
 kin_status means_update(const kin_dims* dims, void* k_rows, void* v_rows, const PageTable& pt,
                         void* block_means, int means_bf16, int32_t* seq_lens, const void* k_new,
-                        const void* v_new, int32_t n_new, int32_t* dev_status, void* stream) {
+                        const void* v_new, int32_t n_new, int32_t* dev_status, void* stream, int per_page = 0) {
   MeansUpdateParams p;
+  p.means_per_page = per_page;
   p.k_cache = static_cast<__nv_bfloat16*>(k_rows);
   p.v_cache = static_cast<__nv_bfloat16*>(v_rows);
   p.means = block_means;
@@ -273,7 +275,8 @@ namespace {
 
 kin_status topk_select(const kin_dims* dims, const void* q, const void* block_means, int means_bf16,
                        const int32_t* seq_lens, int32_t k_blocks, int32_t* sel_idx, int32_t* sel_cnt,
-                       void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
+                       void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream,
+                       const PageTable* mpages = nullptr) {
   if (k_blocks < 2) return KIN_ERR_INVALID_ARG;
   if (!q || !block_means || !seq_lens || !sel_idx || !sel_cnt) return KIN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(block_means)) return KIN_ERR_INVALID_ARG;
@@ -285,6 +288,7 @@ kin_status topk_select(const kin_dims* dims, const void* q, const void* block_me
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.means = block_means;
   p.means_bf16 = means_bf16;
+  p.mpages = mpages ? *mpages : contiguous();
   p.seq_lens = seq_lens;
   p.sel_idx = sel_idx;
   p.sel_cnt = sel_cnt;
@@ -304,8 +308,10 @@ kin_status topk_select(const kin_dims* dims, const void* q, const void* block_me
 
 // means_dtype as a kernel flag (0 fp32, 1 bf16); -1 for an unknown value
 int means_flag(int32_t means_dtype) {
-  return means_dtype == KIN_MEANS_F32 ? 0 : means_dtype == KIN_MEANS_BF16 ? 1 : -1;
+  const int32_t t = means_dtype & ~KIN_MEANS_PER_PAGE;
+  return t == KIN_MEANS_F32 ? 0 : t == KIN_MEANS_BF16 ? 1 : -1;
 }
+int per_page_flag(int32_t means_dtype) { return (means_dtype & KIN_MEANS_PER_PAGE) ? 1 : 0; }
 
 // A NULL table selects the contiguous cache (num_pages ignored).
 kin_status layout_of(const kin_dims& d, const void* k_rows, int32_t num_pages, const int32_t* block_table,
@@ -336,9 +342,26 @@ KIN_EXPORT kin_status kin_block_topk_select_ex(const kin_dims* dims, const void*
   kin_status st = check_dims(dims);
   if (st != KIN_OK) return st;
   const int bf = means_flag(means_dtype);
-  if (bf < 0) return KIN_ERR_INVALID_ARG;
+  if (bf < 0 || per_page_flag(means_dtype)) return KIN_ERR_INVALID_ARG;  // per-page means need the table
   return topk_select(dims, q, block_means, bf, seq_lens, k_blocks, sel_idx, sel_cnt, workspace, ws_bytes,
                      dev_status, stream);
+}
+
+KIN_EXPORT kin_status kin_block_topk_select_paged(const kin_dims* dims, const void* q, const void* page_means,
+                                                  int32_t means_dtype, int32_t num_pages,
+                                                  const int32_t* block_table, const int32_t* seq_lens,
+                                                  int32_t k_blocks, int32_t* sel_idx, int32_t* sel_cnt,
+                                                  void* workspace, size_t ws_bytes, int32_t* dev_status,
+                                                  void* stream) {
+  kin_status st = check_dims(dims);
+  if (st != KIN_OK) return st;
+  const int bf = means_flag(means_dtype);
+  if (bf < 0) return KIN_ERR_INVALID_ARG;
+  PageTable pt;
+  st = check_pages(*dims, page_means, num_pages, block_table, &pt);
+  if (st != KIN_OK) return st;
+  return topk_select(dims, q, page_means, bf, seq_lens, k_blocks, sel_idx, sel_cnt, workspace, ws_bytes,
+                     dev_status, stream, &pt);
 }
 
 KIN_EXPORT kin_status kin_block_means_build_ex(const kin_dims* dims, const void* k_rows, int32_t num_pages,
@@ -354,7 +377,9 @@ KIN_EXPORT kin_status kin_block_means_build_ex(const kin_dims* dims, const void*
   PageTable pt;
   st = layout_of(*dims, k_rows, num_pages, block_table, &pt);
   if (st != KIN_OK) return st;
-  return means_build(dims, k_rows, pt, seq_lens, block_means, bf, dev_status, stream);
+  const int pp = per_page_flag(means_dtype);
+  if (pp && !block_table) return KIN_ERR_INVALID_ARG;
+  return means_build(dims, k_rows, pt, seq_lens, block_means, bf, dev_status, stream, pp);
 }
 
 KIN_EXPORT kin_status kin_block_means_update_ex(const kin_dims* dims, void* k_rows, void* v_rows,
@@ -373,8 +398,10 @@ KIN_EXPORT kin_status kin_block_means_update_ex(const kin_dims* dims, void* k_ro
   PageTable pt;
   st = layout_of(*dims, k_rows, num_pages, block_table, &pt);
   if (st != KIN_OK) return st;
+  const int pp = per_page_flag(means_dtype);
+  if (pp && !block_table) return KIN_ERR_INVALID_ARG;
   return means_update(dims, k_rows, v_rows, pt, block_means, bf, seq_lens, k_new, v_new, n_new, dev_status,
-                      stream);
+                      stream, pp);
 }
 
 namespace {

@@ -142,11 +142,24 @@ __device__ __forceinline__ void store_mean_row(void* means, int means_bf16, int6
   }
 }
 
+// Row of block i of pair (b, h) in the block-means array: logical
+// [B][Hkv][nbcap][D], or per page [num_pages][Hkv][D] (means_per_page: the
+// mean of a page's rows, shared by every sequence whose table maps a block
+// to that page).  -1 for a page index outside the pool.
+__device__ __forceinline__ int64_t means_row_index(const PageTable& pt, int means_per_page, int b, int h, int Hkv,
+                                                   int nbcap, int i) {
+  if (!means_per_page) return ((int64_t)b * Hkv + h) * nbcap + i;
+  const int page = __ldg(pt.table + (int64_t)b * pt.max_blocks + i);
+  if (page < 0 || page >= pt.num_pages) return -1;
+  return (int64_t)page * Hkv + h;
+}
+
 struct MeansBuildParams {
   const __nv_bfloat16* k_cache;  // contiguous cache or page pool (see PageTable)
   const int32_t* seq_lens;
   void* means;
   int means_bf16;
+  int means_per_page;            // means [num_pages][Hkv][D] (needs a page table)
   int32_t* dev_status;
   PageTable pages;
   int B, Hkv, Lcap, bs, nbcap;
@@ -157,6 +170,7 @@ struct MeansUpdateParams {
   __nv_bfloat16* v_cache;
   void* means;
   int means_bf16;
+  int means_per_page;
   int32_t* seq_lens;
   const __nv_bfloat16* k_new;
   const __nv_bfloat16* v_new;
@@ -169,6 +183,7 @@ struct SelectParams {
   const __nv_bfloat16* q;
   const void* means;
   int means_bf16;
+  PageTable mpages;     // table != NULL: means per page [num_pages][Hkv][D], found through the table
   const int32_t* seq_lens;
   int32_t* sel_idx;
   int32_t* sel_cnt;

@@ -40,7 +40,6 @@ __global__ void __launch_bounds__(256) means_build_kernel(MeansBuildParams p) {
   const int i = blockIdx.x * 8 + warp;
   const int nb = (L + p.bs - 1) / p.bs;
   if (i >= nb) return;
-  const int64_t pair = (int64_t)b * p.Hkv + h;
   const int t0 = i * p.bs;
   const int t1 = min(t0 + p.bs, L);
   const int64_t base = kv_row_offset(p.pages, b, h, p.Hkv, p.Lcap, p.bs, i, 0);  // the block's rows are contiguous
@@ -62,7 +61,8 @@ __global__ void __launch_bounds__(256) means_build_kernel(MeansBuildParams p) {
   const float n = (float)(t1 - t0);
   float4 m = make_float4(__fdiv_rn(acc[0], n), __fdiv_rn(acc[1], n), __fdiv_rn(acc[2], n),
                          __fdiv_rn(acc[3], n));
-  store_mean_row(p.means, p.means_bf16, pair * p.nbcap + i, lane, m);
+  const int64_t mrow = means_row_index(p.pages, p.means_per_page, b, h, p.Hkv, p.nbcap, i);
+  if (mrow >= 0) store_mean_row(p.means, p.means_bf16, mrow, lane, m);
 }
 
 // grid (B), 256 threads.  One CTA owns a whole sequence so that the length
@@ -139,7 +139,8 @@ __global__ void __launch_bounds__(kUpdThreads) means_update_kernel(MeansUpdatePa
     const float cnt = (float)(t1 - t0);
     float4 m = make_float4(__fdiv_rn(acc[0], cnt), __fdiv_rn(acc[1], cnt), __fdiv_rn(acc[2], cnt),
                            __fdiv_rn(acc[3], cnt));
-    store_mean_row(p.means, p.means_bf16, pair * p.nbcap + i, lane, m);
+    const int64_t mrow = means_row_index(p.pages, p.means_per_page, b, h, p.Hkv, p.nbcap, i);
+    if (mrow >= 0) store_mean_row(p.means, p.means_bf16, mrow, lane, m);
   }
   __syncthreads();
   if (threadIdx.x == 0) p.seq_lens[b] = L1;

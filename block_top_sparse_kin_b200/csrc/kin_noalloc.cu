@@ -85,6 +85,9 @@ KIN_EXPORT kin_status kin_block_topk_select_noalloc(const kin_dims* dims, const 
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.means = block_means;
   p.means_bf16 = 0;
+  p.mpages.table = nullptr;  // logical means
+  p.mpages.max_blocks = 0;
+  p.mpages.num_pages = 0;
   p.seq_lens = seq_lens;
   p.sel_idx = sel_idx;
   p.sel_cnt = sel_cnt;

@@ -701,6 +701,150 @@ __global__ void __launch_bounds__(kSelThreads, KIN_SEL_CTAS_PER_SM) select_scan_
   pdl_trigger_late();
 }
 
+// The scan over block means stored per page (the shared-prompt layout),
+// found through the page table.  Rows are scattered, so a warp splits into
+// 4 groups of 8 lanes, each group owning one mean row at a time: lane x of a
+// group holds the 4-dim partials of lanes x, x+8, x+16 and x+24 of the
+// contiguous kernel's layout (4 coalesced loads), every lane of a group
+// fetches its row's page index itself (no address shuffles), and the row
+// total is formed by the same pairing tree as warp_sum_rows (xor 16 and 8
+// inside the lane, xor 4, 2, 1 across the group), so the scores equal the
+// contiguous kernel's bit for bit.  RG row groups per lane per step keep
+// 4 KB of means in flight per warp; the page indices of the next step are
+// loaded one step ahead of its rows.
+template <bool kBf16>
+__global__ void __launch_bounds__(kSelThreads, KIN_SEL_CTAS_PER_SM) select_scan_paged_kernel(SelectParams p) {
+  using ML = MeanLane<kBf16>;
+  using Raw = typename ML::Raw;
+  constexpr int RG = kBf16 ? 4 : 2;  // rows per lane per step
+  constexpr int U = 4 * RG;          // rows per warp per step
+  pdl_wait();
+  pdl_trigger_early();
+  const int lane = threadIdx.x & 31, grp = lane >> 3, x = lane & 7;
+  const int nwarps = gridDim.x * kSelWarps;
+  const int gw = blockIdx.x * kSelWarps + (threadIdx.x >> 5);
+  const int nbp = (p.nbcap + U - 1) / U * U;
+  const int steps = p.B * p.Hkv * (nbp / U);
+  const int per = (steps + nwarps - 1) / nwarps;
+  const int s0 = gw * per, s1 = min(s0 + per, steps);
+  if (s0 >= s1) {
+    pdl_trigger_late();
+    return;
+  }
+  // lane row j of a step is block blk + grp + 4 j
+  auto load_pages = [&](int pr, int bk, int nbr, int (&pg)[RG]) {
+#pragma unroll
+    for (int j = 0; j < RG; ++j) {
+      const int r = bk + grp + 4 * j;
+      pg[j] = -1;
+      if (r < nbr) {
+        const int v = __ldg(p.mpages.table + (int64_t)(pr / p.Hkv) * p.mpages.max_blocks + r);
+        if (v < 0 || v >= p.mpages.num_pages) {
+          if (x == 0) set_status(p.dev_status, KIN_ERR_DEVICE_DATA);
+        } else {
+          pg[j] = v;
+        }
+      }
+    }
+  };
+  const Raw* mbase = reinterpret_cast<const Raw*>(p.means) + x;
+  auto load_rows = [&](int pr, const int (&pg)[RG], Raw (&v)[RG][4]) {
+    const int h = pr % p.Hkv;
+#pragma unroll
+    for (int j = 0; j < RG; ++j) {
+      const Raw* row = mbase + ((int64_t)(pg[j] < 0 ? 0 : pg[j]) * p.Hkv + h) * (kHeadDim / 4);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) v[j][c] = pg[j] >= 0 ? __ldcs(row + 8 * c) : ML::zero();
+    }
+  };
+  // the group-summed query of a pair, at the 4 x 4 dims this lane scores
+  auto load_q = [&](int pr, float4 (&qs)[4]) {
+    const int b = pr / p.Hkv, h = pr - b * p.Hkv;
+    const __nv_bfloat16* qg = p.q + ((int64_t)b * p.Hq + (int64_t)h * p.g) * kHeadDim;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) qs[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int jh = 0; jh < p.g; ++jh) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint2 raw = __ldg(reinterpret_cast<const uint2*>(qg + jh * kHeadDim) + x + 8 * c);
+        const float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&raw.x));
+        const float2 bb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&raw.y));
+        qs[c].x += a.x;
+        qs[c].y += a.y;
+        qs[c].z += bb.x;
+        qs[c].w += bb.y;
+      }
+    }
+  };
+  auto advance = [&](int& pr, int& bk) {
+    bk += U;
+    if (bk >= nbp) {
+      ++pr;
+      bk = 0;
+    }
+  };
+
+  int pair = (s0 * U) / nbp;
+  int blk = s0 * U - pair * nbp;
+  int nb = pair_nb(p, pair);
+  float4 qs[4];
+  load_q(pair, qs);
+  int pg[RG];
+  load_pages(pair, blk, nb, pg);
+  Raw cur[RG][4];
+  load_rows(pair, pg, cur);
+  int npair = pair, nblk = blk;
+  advance(npair, nblk);
+  int nnb = s0 + 1 < s1 ? (npair == pair ? nb : pair_nb(p, npair)) : 0;
+  int npg[RG];
+  load_pages(npair, nblk, nnb, npg);
+  for (int s = s0; s < s1; ++s) {
+    const bool more = s + 1 < s1;
+    Raw nxt[RG][4];
+    load_rows(npair, npg, nxt);  // rows with no page (beyond nb, or none) load nothing
+    int n2pair = npair, n2blk = nblk;
+    advance(n2pair, n2blk);
+    const int n2nb = s + 2 < s1 ? (n2pair == npair ? nnb : pair_nb(p, n2pair)) : 0;
+    int n2pg[RG];
+    load_pages(n2pair, n2blk, n2nb, n2pg);
+    if (blk < nb) {
+#pragma unroll
+      for (int j = 0; j < RG; ++j) {
+        float d[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float4 m = ML::widen(cur[j][c]);
+          d[c] = qs[c].x * m.x;
+          d[c] = fmaf(qs[c].y, m.y, d[c]);
+          d[c] = fmaf(qs[c].z, m.z, d[c]);
+          d[c] = fmaf(qs[c].w, m.w, d[c]);
+        }
+        // lanes x (c 0), x+8 (c 1), x+16 (c 2), x+24 (c 3): pair xor 16, then xor 8
+        float t = (d[0] + d[2]) + (d[1] + d[3]);
+        t += __shfl_xor_sync(0xffffffffu, t, 4);
+        t += __shfl_xor_sync(0xffffffffu, t, 2);
+        t += __shfl_xor_sync(0xffffffffu, t, 1);
+        const int r = blk + grp + 4 * j;
+        if (x == 0 && r < nb) p.scores[(int64_t)pair * p.nbcap + r] = t * p.score_scale;
+      }
+    }
+    if (npair != pair && more) load_q(npair, qs);
+    pair = npair;
+    blk = nblk;
+    nb = nnb;
+    npair = n2pair;
+    nblk = n2blk;
+    nnb = n2nb;
+#pragma unroll
+    for (int j = 0; j < RG; ++j) {
+      npg[j] = n2pg[j];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) cur[j][c] = nxt[j][c];
+    }
+  }
+  pdl_trigger_late();
+}
+
 
 // ---- kernel 2: one CTA of NT threads per pair: dense shortcut, bad-length
 // flag, or the exact top-k over the scores the scan left in workspace
@@ -812,9 +956,14 @@ cudaError_t launch_select(const SelectParams& p, cudaStream_t s) {
   const int64_t want = (rows + kSelWarps * u * 4 - 1) / (kSelWarps * u * 4);  // >= 4 steps per warp
   const int64_t resident = (int64_t)device_sm_count() * KIN_SEL_CTAS_PER_SM;
   const int grid = (int)(want < resident ? (want > 0 ? want : 1) : resident);
-  cudaError_t e = p.means_bf16
-                      ? launch_pdl(select_scan_kernel<true, 2 * kSelU>, dim3(grid), dim3(kSelThreads), 0, s, p)
-                      : launch_pdl(select_scan_kernel<false, kSelU>, dim3(grid), dim3(kSelThreads), 0, s, p);
+  const dim3 gd(grid), bd(kSelThreads);
+  cudaError_t e;
+  if (p.mpages.table)
+    e = p.means_bf16 ? launch_pdl(select_scan_paged_kernel<true>, gd, bd, 0, s, p)
+                     : launch_pdl(select_scan_paged_kernel<false>, gd, bd, 0, s, p);
+  else
+    e = p.means_bf16 ? launch_pdl(select_scan_kernel<true, 2 * kSelU>, gd, bd, 0, s, p)
+                     : launch_pdl(select_scan_kernel<false, kSelU>, gd, bd, 0, s, p);
   if (e != cudaSuccess) return e;
   switch (topk_threads(p.nbcap, (int64_t)p.B * p.Hkv)) {
     case 256: return launch_topk<256>(p, s);

@@ -199,6 +199,10 @@ kin_status kin_sparse_decode_attn_paged(const kin_dims* dims, const void* q, con
  * arguments, semantics and errors are those of kin_block_means_build,
  * kin_block_means_update (and their paged forms) and kin_block_topk_select. */
 typedef enum { KIN_MEANS_F32 = 0, KIN_MEANS_BF16 = 1 } kin_means_dtype;
+/* OR-ed into means_dtype of the build/update calls (with a block table):
+ * block means per page, [num_pages][Hkv][D], read by
+ * kin_block_topk_select_paged below. */
+#define KIN_MEANS_PER_PAGE 0x100
 
 kin_status kin_block_means_build_ex(const kin_dims* dims, const void* k_rows, int32_t num_pages,
                                     const int32_t* block_table, const int32_t* seq_lens, void* block_means,
@@ -213,6 +217,29 @@ kin_status kin_block_topk_select_ex(const kin_dims* dims, const void* q, const v
                                     int32_t means_dtype, const int32_t* seq_lens, int32_t k_blocks,
                                     int32_t* sel_idx, int32_t* sel_cnt, void* workspace, size_t ws_bytes,
                                     int32_t* dev_status, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Shared-prompt (Best-of-N) reuse.  N samples of one prompt share the
+ * prompt's KV, which is read once for all of them ("Kinetics: Rethinking
+ * Test-Time Scaling Law", response W3: prompt sharing lets different
+ * requests access the same KV memory at decoding time).  With the paged
+ * calls, each sample's block table maps the prompt's blocks to the same
+ * pages; with block means per page (KIN_MEANS_PER_PAGE in the build/update
+ * calls), the prompt's means are stored once too.  This select reads the
+ * per-page means through the table:
+ *   page_means  [num_pages][Hkv][D], fp32 or bf16 (means_dtype, without the
+ *               per-page flag); block i of (b, h) is page_means[block_table
+ *               [b][i]][h].
+ * A page shared by several sequences must hold full blocks (bs valid rows)
+ * in each of them, so its mean is the same for all.  Results equal those
+ * of the select over logical means of the same blocks, bit for bit.  A page
+ * index outside the pool zeroes that block's score and flags
+ * KIN_ERR_DEVICE_DATA.  Other arguments and errors: kin_block_topk_select. */
+kin_status kin_block_topk_select_paged(const kin_dims* dims, const void* q, const void* page_means,
+                                       int32_t means_dtype, int32_t num_pages, const int32_t* block_table,
+                                       const int32_t* seq_lens, int32_t k_blocks, int32_t* sel_idx,
+                                       int32_t* sel_cnt, void* workspace, size_t ws_bytes, int32_t* dev_status,
+                                       void* stream);
 
 /* ------------------------------------------------------------------------
  * Token-level top-k attention (the variant the block method is compared
