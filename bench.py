@@ -720,7 +720,7 @@ class OracleSample:
 
     def describe(self, passes, seconds):
         return (f"{self.n} of {self.P} (batch, kv-head) pairs of {self.w.name} (k={self.k}), {passes} "
-                f"passes in {seconds:.1f} s; scores + top-k + attention in fp64, block means precomputed")
+                f"passes in {seconds:.3f} s; scores + top-k + attention in fp64, block means precomputed")
 
 
 def cpu_baseline(w: ki.Workload, k: int, budget_s: float = 12.0, max_pairs: int = 32):
