@@ -35,10 +35,10 @@ int nbcap_of(const kin_dims& d) { return (d.max_seq_len + d.block_size - 1) / d.
 int pairs_of(const kin_dims& d) { return d.batch * d.num_kv_heads; }
 
 #ifndef KIN_ATTN_CHUNK_TOKENS
-#define KIN_ATTN_CHUNK_TOKENS 512
+#define KIN_ATTN_CHUNK_TOKENS 768
 #endif
 
-// Kept blocks per attention CTA: KIN_ATTN_CHUNK_TOKENS tokens (512 -> 256 KB
+// Kept blocks per attention CTA: KIN_ATTN_CHUNK_TOKENS tokens (768 -> 384 KB
 // of K+V), fewer when the grid would hold fewer than 2 CTAs per SM.
 int attn_chunk_blocks(const kin_dims& d, int k) {
   const int k_eff = k < nbcap_of(d) ? k : nbcap_of(d);
