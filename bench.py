@@ -199,18 +199,24 @@ class ClockSampler:
             self.error = repr(e)
         return self
 
-    def _run(self):
+    def poll(self):
+        """One sample now (the timed loop also calls this after every step)."""
+        if self.handle is None:
+            return
         nv = self.nv
-        while not self.stop.is_set():
+        try:
+            mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
             try:
-                mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
-                try:
-                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
-                except AttributeError:
-                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.handle)
-                self.samples.append((mhz, rs))
-            except Exception:
-                pass
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+            except AttributeError:
+                rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.handle)
+            self.samples.append((mhz, rs))
+        except Exception:
+            pass
+
+    def _run(self):
+        while not self.stop.is_set():
+            self.poll()
             time.sleep(0.001)
 
     def __exit__(self, *a):
@@ -569,6 +575,7 @@ def gpu_arm(args):
             graph.replay()
             torch.cuda.synchronize()
             per_step.append(step_ev[0].elapsed_time(step_ev[1]))
+            clk.poll()                     # the clock right after each step (outside the events)
         wall = time.perf_counter() - wall0
     if world > 1:
         dist.barrier()
