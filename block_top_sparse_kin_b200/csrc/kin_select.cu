@@ -24,6 +24,14 @@
 // The top-k: the first block and the block holding the newest token are
 // always kept, ties go to the lower index, and the kept indices leave
 // ascending.
+//
+// Variants served by the same code: bf16 block means (the scan templated on
+// the means type, 16 rows per warp step); block means stored per page of a
+// paged cache (select_scan_paged_kernel: 8-lane groups own one scattered
+// row each, with the same summation tree, so the scores are bit-identical);
+// and the token-level top-k of every query head's logits
+// (token_topk_kernel: the same threshold search over an explicit candidate
+// range with nothing forced).
 #include <type_traits>
 
 #include "kin_internal.cuh"
