@@ -85,9 +85,14 @@ def test_crafted_scores_exercise_both_threshold_searches():
             np.where(rng.random(nb) < 0.05, 50.0 + rng.random(nb), 2.0 + 1e-2 * (np.arange(nb) // 3)),
             # negative scores only
             -1.0 - rng.random(nb),
+            # one outlier widens the bins, so the boundary bin holds nearly
+            # every block (too many to rank pairwise: the radix search runs),
+            # with ties of two around the threshold
+            np.where(np.arange(nb) == 5, 1e3,
+                     np.where(np.arange(nb) == 9, 0.0, 1.0 + 1e-3 * (np.arange(nb) // 2))),
         ]
         vals.append(pairs)
-    dims, q, means, lens_t, means_h, q_bits = _crafted_case(2, 4, g, bs, lens, vals)
+    dims, q, means, lens_t, means_h, q_bits = _crafted_case(2, 5, g, bs, lens, vals)
     ref = _oracle_sel(means_h, q_bits, lens, bs, g, k)
     sel_f, cnt_f, st_f = _select(dims, q, means, lens_t, k)
     sel_n, cnt_n, st_n = _select(dims, q, means, lens_t, k, noalloc=True)
