@@ -14,9 +14,11 @@
 //     m16n8k16 per tile (tokens = M, the GQA group = N), fp32 logits to
 //     workspace.
 //  2. token_topk_kernel (kin_select.cu): the exact top-k per query head.
-//  3. token_attn_kernel: one CTA per query head gathers the kept V rows
-//     (one coalesced 256-byte warp load per row, 8 rows in flight per lane)
-//     and sums them weighted by exp(z_t - max z) in fp32.
+//  3. token_attn_kernel: one 4-warp CTA per query head stages the kept
+//     indices and logits in shared memory (segments of 2048, running
+//     maximum), gathers the kept V rows (one coalesced 256-byte warp load
+//     per row, 16 rows in flight per lane) and sums them weighted by
+//     exp(z_t - max z) in fp32.
 #include "kin_internal.cuh"
 
 namespace kin {
@@ -121,12 +123,22 @@ __global__ void __launch_bounds__(kTokThreads) token_logits_kernel(TokenParams p
   cp_async_wait<0>();
 }
 
-constexpr int kTokAttnWarps = 8;
+constexpr int kTokAttnWarps = 4;
 constexpr int kTokAttnThreads = kTokAttnWarps * 32;
+constexpr int kTokSeg = 2048;                               // kept tokens staged per segment
+constexpr int kTokSegPerThread = kTokSeg / kTokAttnThreads;  // 16
+constexpr int kTokVRows = 16;                               // V rows in flight per lane
 
 // one CTA per (sequence, query head): out = sum_t e^(z_t - M) V_t / sum_t e^(z_t - M)
-// over the kept tokens, lse = M + ln sum_t e^(z_t - M)
-__global__ void __launch_bounds__(kTokAttnThreads) token_attn_kernel(TokenParams p) {
+// over the kept tokens, lse = M + ln sum_t e^(z_t - M).  The kept tokens are
+// taken in segments of kTokSeg: each thread fetches its 16 indices, then
+// their 16 logits, all in flight together, into shared memory; the running
+// maximum M is raised to the segment's and the partial sums rescaled; then
+// warp w streams its quarter of the segment's V rows, 16 rows in flight per
+// lane (lane l owns dims 4l .. 4l + 3).
+__global__ void __launch_bounds__(kTokAttnThreads, 7) token_attn_kernel(TokenParams p) {
+  __shared__ int s_t[kTokSeg];
+  __shared__ float s_z[kTokSeg];
   __shared__ __align__(16) float s_acc[kTokAttnWarps][kHeadDim];
   __shared__ float s_red[kTokAttnWarps];
   __shared__ float s_l[kTokAttnWarps];
@@ -144,53 +156,74 @@ __global__ void __launch_bounds__(kTokAttnThreads) token_attn_kernel(TokenParams
   }
   const int32_t* sel = p.sel + row_id * p.kt;
   const float* z = p.logits + row_id * p.Lcap;
-  // pass 1: the largest kept logit
-  float mx = kTokNegInf;
-  for (int i = tid; i < cnt; i += kTokAttnThreads) mx = fmaxf(mx, z[__ldg(sel + i)]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if (lane == 0) s_red[warp] = mx;
-  __syncthreads();
-  float M = s_red[0];
-#pragma unroll
-  for (int w = 1; w < kTokAttnWarps; ++w) M = fmaxf(M, s_red[w]);
-  const float ml2 = M * 1.4426950408889634f;
-
-  // pass 2: warp w takes kept tokens [w per, (w + 1) per) in batches of 32:
-  // lane l fetches token l's index and weight, then the warp streams the
-  // batch's V rows 8 at a time (lane l owns dims 4l .. 4l + 3)
   const uint2* vbase = reinterpret_cast<const uint2*>(p.v_cache + ((int64_t)b * p.Hkv + h) * p.Lcap * kHeadDim) + lane;
-  const int per = (cnt + kTokAttnWarps - 1) / kTokAttnWarps;
-  const int i0 = warp * per, i1 = min(i0 + per, cnt);
+  constexpr float kLog2e = 1.4426950408889634f;
+  float M = kTokNegInf;  // running maximum over the segments so far (CTA-uniform)
   float acc[4] = {0.f, 0.f, 0.f, 0.f}, lsum = 0.f;
-  for (int base = i0; base < i1; base += 32) {
-    const int i = base + lane;
-    const int t = i < i1 ? __ldg(sel + i) : 0;
-    const float e = i < i1 ? exp2f(z[t] * 1.4426950408889634f - ml2) : 0.f;
-    lsum += e;
-    const int nb = min(32, i1 - base);
-    for (int u0 = 0; u0 < nb; u0 += 8) {
-      uint2 v[8];
-      float w8[8];
+  for (int s0 = 0; s0 < cnt; s0 += kTokSeg) {
+    const int ns = min(kTokSeg, cnt - s0);
+    // stage the segment's indices and logits; its maximum
+    int tv[kTokSegPerThread];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int src = (u0 + u) & 31;
-        const int tt = __shfl_sync(0xffffffffu, t, src);
-        w8[u] = __shfl_sync(0xffffffffu, e, src);
-        v[u] = u0 + u < nb ? __ldg(vbase + (int64_t)tt * (kHeadDim / 4)) : make_uint2(0u, 0u);
+    for (int r = 0; r < kTokSegPerThread; ++r) {
+      const int i = r * kTokAttnThreads + tid;
+      tv[r] = i < ns ? __ldg(sel + s0 + i) : 0;
+    }
+    float mx = kTokNegInf;
+#pragma unroll
+    for (int r = 0; r < kTokSegPerThread; ++r) {
+      const int i = r * kTokAttnThreads + tid;
+      if (i < ns) {
+        const float zi = z[tv[r]];
+        s_t[i] = tv[r];
+        s_z[i] = zi;
+        mx = fmaxf(mx, zi);
       }
+    }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (u0 + u < nb) {
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) s_red[warp] = mx;
+    __syncthreads();
+    float Mn = M;
+#pragma unroll
+    for (int w = 0; w < kTokAttnWarps; ++w) Mn = fmaxf(Mn, s_red[w]);
+    if (Mn > M) {  // rescale what the earlier segments summed
+      const float sc = M == kTokNegInf ? 0.f : exp2f((M - Mn) * kLog2e);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[c] *= sc;
+      lsum *= sc;
+      M = Mn;
+    }
+    const float ml2 = M * kLog2e;
+    // warp w: segment rows [r0, r1), in batches of 32 (lane l: row r0 + 32 q + l's index and weight)
+    const int per = (ns + kTokAttnWarps - 1) / kTokAttnWarps;
+    const int r0 = min(warp * per, ns), r1 = min(r0 + per, ns);
+    for (int base = r0; base < r1; base += 32) {
+      const int i = base + lane;
+      const int t = i < r1 ? s_t[i] : 0;
+      const float e = i < r1 ? exp2f(s_z[i] * kLog2e - ml2) : 0.f;
+      lsum += e;
+      const int nb = min(32, r1 - base);
+      for (int u0 = 0; u0 < nb; u0 += kTokVRows) {
+        uint2 v[kTokVRows];
+#pragma unroll
+        for (int u = 0; u < kTokVRows; ++u) {
+          const int tt = __shfl_sync(0xffffffffu, t, (u0 + u) & 31);
+          v[u] = u0 + u < nb ? __ldg(vbase + (int64_t)tt * (kHeadDim / 4)) : make_uint2(0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < kTokVRows; ++u) {
+          const float wu = __shfl_sync(0xffffffffu, e, (u0 + u) & 31);  // 0 past the batch's end
           const float2 lo = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&v[u].x));
           const float2 hi = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&v[u].y));
-          acc[0] = fmaf(w8[u], lo.x, acc[0]);
-          acc[1] = fmaf(w8[u], lo.y, acc[1]);
-          acc[2] = fmaf(w8[u], hi.x, acc[2]);
-          acc[3] = fmaf(w8[u], hi.y, acc[3]);
+          acc[0] = fmaf(wu, lo.x, acc[0]);
+          acc[1] = fmaf(wu, lo.y, acc[1]);
+          acc[2] = fmaf(wu, hi.x, acc[2]);
+          acc[3] = fmaf(wu, hi.y, acc[3]);
         }
       }
     }
+    __syncthreads();  // the next segment overwrites s_t, s_z and s_red
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);

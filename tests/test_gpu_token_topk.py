@@ -73,6 +73,8 @@ def check_head(dc, b, j, kt, sel, out, lse):
     (W("tok_g8_long", 1, 1, 8, D, 16, 0, 0, 8, 92, Lcap=9000, lens=(8999,)), 700),
     (W("tok_dense_and_len1", 3, 1, 2, D, 16, 0, 0, 8, 93, Lcap=128, lens=(100, 1, 33)), 64),
     (W("tok_k1", 2, 2, 4, D, 16, 50, 300, 8, 94, Lcap=320), 1),
+    # kept tokens over three segments of the attention kernel (2048, 2048, 404)
+    (W("tok_g2_segments", 1, 2, 4, D, 16, 0, 0, 8, 96, Lcap=6000, lens=(5999,)), 4500),
 ], ids=lambda x: x.name if hasattr(x, "name") else str(x))
 def test_token_topk_every_head(w, kt):
     dc = make_device_case(w)
