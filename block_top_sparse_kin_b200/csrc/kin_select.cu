@@ -20,7 +20,10 @@
 //     pair's scores into order-preserving uint32 keys, finds the exact
 //     threshold (equal-width score bins, then a pairwise rank of the
 //     boundary bin; a radix search over the key bits when the range is
-//     crowded or degenerate) and writes the kept indices.
+//     crowded or degenerate) and writes the kept indices.  Rows too long
+//     for registers keep their keys in shared memory (or a scratch row):
+//     there the bin pass is fused with the emit's per-lane bit masks, and a
+//     crowded boundary bin is ranked through its 256 sub-bins.
 // The top-k: the first block and the block holding the newest token are
 // always kept, ties go to the lower index, and the kept indices leave
 // ascending.
@@ -80,7 +83,8 @@ __device__ __forceinline__ float warp_sum_rows(float (&v)[U], int lane) {
 // threshold is found by a search over 256 equal-width score bins, with a
 // radix search over the key bits for crowded or degenerate ranges.
 constexpr int kListCap = 4096;  // radix: candidates kept after the first pass
-constexpr int kRankCap = 512;   // equal-width bins: boundary-bin keys ranked pairwise
+constexpr int kRankCap = 512;   // equal-width bins: boundary-bin keys listed (ranked pairwise, or by sub-bins)
+constexpr int kDirectRank = 64;  // boundary bins up to this size are ranked without sub-bins
 constexpr int kMaxKPT = 8;      // keys per thread on the register path
 // 256-bin histograms padded by one word per 8 bins, so a lane reading 8
 // consecutive bins (stride 9 words between lanes) hits 32 distinct banks
@@ -101,8 +105,8 @@ struct TopkSmem {
   static constexpr int NW = NT / 32;
   int hist[2][kHistWords];   // histograms (equal-width bins, or radix digits double-buffered), hidx-padded
   uint32_t list[kListCap];   // radix: candidate indices; equal-width bins: boundary-bin keys
-  int list_n;
-  int warp_cnt[3][NW];       // per-warp counts: forced, > T, == T
+  int list_n, list_n2;
+  int warp_cnt[2][NW];       // emit: per-warp counts of keys taken outright, and equal to the threshold
   uint32_t wmin[NW], wmax[NW];
   int digit, above, bin;
   uint32_t thresh;
@@ -232,76 +236,179 @@ __device__ __forceinline__ void radix_threshold(const uint32_t* keys, int nb, co
   }
 }
 
+// One round of the emit, every warp's range holding at most 1024 keys: lane
+// l's masks cover the 32 keys from i0 (bit b = key i0 + b): gm those taken
+// outright, em those equal to the threshold, of which the first kr (by
+// index, over the whole row) are taken.  One barrier publishes the warp
+// totals; warp scans give every lane its output position; each lane writes
+// its taken indices in bit order.  Checks that exactly k were taken.
+template <int NT>
+__device__ __forceinline__ void emit_round(unsigned gm, unsigned em, int i0, int k, int kr, int32_t* sel,
+                                           TopkSmem<NT>& sm, int32_t* dev_status) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int ng = __popc(gm), ne = __popc(em);
+  int ig = ng, ie = ne;  // inclusive scans over the warp's lanes
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int tg = __shfl_up_sync(0xffffffffu, ig, o), te = __shfl_up_sync(0xffffffffu, ie, o);
+    if (lane >= o) {
+      ig += tg;
+      ie += te;
+    }
+  }
+  if (lane == 31) {
+    sm.warp_cnt[0][warp] = ig;
+    sm.warp_cnt[1][warp] = ie;
+  }
+  __syncthreads();
+  int sg = lane < NW ? sm.warp_cnt[0][lane] : 0, se = lane < NW ? sm.warp_cnt[1][lane] : 0;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {  // inclusive scans over the warps
+    const int tg = __shfl_up_sync(0xffffffffu, sg, o), te = __shfl_up_sync(0xffffffffu, se, o);
+    if (lane >= o) {
+      sg += tg;
+      se += te;
+    }
+  }
+  const int gb = (warp ? __shfl_sync(0xffffffffu, sg, warp - 1) : 0) + ig - ng;  // before this lane's first key
+  const int eb = (warp ? __shfl_sync(0xffffffffu, se, warp - 1) : 0) + ie - ne;
+  unsigned take = gm;
+  for (int keep = min(max(kr - eb, 0), ne); keep > 0; --keep) {  // its first equal keys still wanted
+    take |= em & (0u - em);
+    em &= em - 1u;
+  }
+  int pos = gb + min(eb, kr);
+  while (take) {
+    const int b = __ffs(take) - 1;
+    take &= take - 1u;
+    if (pos < k) sel[pos] = i0 + b;  // never write past the pair's row
+    ++pos;
+  }
+  const int g_all = __shfl_sync(0xffffffffu, sg, 31), e_all = __shfl_sync(0xffffffffu, se, 31);
+  if (threadIdx.x == 0 && g_all + min(e_all, kr) != k) set_status(dev_status, KIN_ERR_DEVICE_DATA);
+}
+
 // Writes the kept blocks ascending to sel[0..k): the forced blocks 0 and
 // nb-1, every candidate whose key under `mask` is above `prefix`, and the
 // first kr candidates (by index) whose key under the mask equals it.  Warp w
-// owns a contiguous index range; one pass of ballots counts its forced /
-// greater / equal keys, one barrier publishes the counts, and a second pass
-// writes the taken indices in order (so ties go to lower indices).
+// owns a contiguous index range in rounds of 1024 keys; in a round, lane l
+// owns the 32 consecutive keys from 32 l and reads them in a rotated order
+// (step j: key (j + l) mod 32), so the warp's 32 reads hit 32 distinct
+// banks, into two 32-bit masks (taken outright; equal to the threshold).
+// One round per warp goes straight to emit_round; longer ranges count every
+// round first, publish the warp totals, then rebuild each round's masks and
+// write (ties go to lower indices).
 template <int NT>
 __device__ __forceinline__ void emit_selection(const uint32_t* keys, int nb, const Cands& cd, int k, uint32_t prefix,
                                                uint32_t mask, int kr, int32_t* sel, TopkSmem<NT>& sm,
                                                int32_t* dev_status) {
   constexpr int NW = NT / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int span = ((nb + NW - 1) / NW + 31) & ~31;  // per-warp range, whole batches
+  const int span = ((nb + NW - 1) / NW + 1023) & ~1023;  // per-warp range, whole rounds
   const int w0 = min(warp * span, nb), w1 = min(w0 + span, nb);
-  const unsigned lt = (1u << lane) - 1u;
-  int n_forced = 0, n_gt = 0, n_eq = 0;
-  for (int base = w0; base < w1; base += 32) {
-    const int i = base + lane;
-    const bool in = i < w1;
-    const uint32_t key = in ? (keys[i] & mask) : 0u;
-    const bool cand = in && cd.has(i);
-    n_forced += __popc(__ballot_sync(0xffffffffu, in && !cand));
-    n_gt += __popc(__ballot_sync(0xffffffffu, cand && key > prefix));
-    n_eq += __popc(__ballot_sync(0xffffffffu, cand && key == prefix));
+  auto chunk_masks = [&](int c0, unsigned& gm, unsigned& em) {
+    gm = 0u;
+    em = 0u;
+    if (c0 + 32 <= w1 && c0 >= cd.lo && c0 + 31 <= cd.hi) {  // 32 candidates
+#pragma unroll 8
+      for (int j = 0; j < 32; ++j) {
+        const int b = (j + lane) & 31;
+        const uint32_t key = keys[c0 + b] & mask;
+        gm |= (unsigned)(key > prefix) << b;
+        em |= (unsigned)(key == prefix) << b;
+      }
+    } else if (c0 < w1) {
+      for (int j = 0; j < 32; ++j) {
+        const int b = (j + lane) & 31;
+        const int i = c0 + b;
+        if (i < w1) {
+          const uint32_t key = keys[i] & mask;
+          const bool cand = cd.has(i);
+          gm |= (unsigned)(!cand || key > prefix) << b;
+          em |= (unsigned)(cand && key == prefix) << b;
+        }
+      }
+    }
+  };
+  if (span <= 1024) {  // CTA-uniform
+    unsigned gm, em;
+    chunk_masks(w0 + 32 * lane, gm, em);
+    emit_round(gm, em, w0 + 32 * lane, k, kr, sel, sm, dev_status);
+    return;
   }
+  int n_g = 0, n_e = 0;
+  for (int c = w0; c < w1; c += 1024) {
+    unsigned gm, em;
+    chunk_masks(c + 32 * lane, gm, em);
+    n_g += __popc(gm);
+    n_e += __popc(em);
+  }
+  n_g = __reduce_add_sync(0xffffffffu, n_g);
+  n_e = __reduce_add_sync(0xffffffffu, n_e);
   if (lane == 0) {
-    sm.warp_cnt[0][warp] = n_forced;
-    sm.warp_cnt[1][warp] = n_gt;
-    sm.warp_cnt[2][warp] = n_eq;
+    sm.warp_cnt[0][warp] = n_g;
+    sm.warp_cnt[1][warp] = n_e;
   }
   __syncthreads();
-  int eq_base = 0, out_base = 0;
-  for (int w = 0; w < warp; ++w) {
-    const int e = sm.warp_cnt[2][w];
-    const int eq_take = min(max(kr - eq_base, 0), e);  // equal keys warp w takes
-    out_base += sm.warp_cnt[0][w] + sm.warp_cnt[1][w] + eq_take;
-    eq_base += e;
-  }
-  int pos = out_base, eq_rank = eq_base;
-  for (int base = w0; base < w1; base += 32) {
-    const int i = base + lane;
-    const bool in = i < w1;
-    const uint32_t key = in ? (keys[i] & mask) : 0u;
-    const bool cand = in && cd.has(i);
-    const bool eq = cand && key == prefix;
-    const unsigned eq_mask = __ballot_sync(0xffffffffu, eq);
-    const bool take = (in && !cand) || (cand && key > prefix) || (eq && eq_rank + __popc(eq_mask & lt) < kr);
-    const unsigned take_mask = __ballot_sync(0xffffffffu, take);
-    if (take) {
-      const int o = pos + __popc(take_mask & lt);
-      if (o < k) sel[o] = i;  // never write past the pair's row
+  // keys before this warp: lane l holds warps 0..l inclusive
+  int sg = lane < NW ? sm.warp_cnt[0][lane] : 0, se = lane < NW ? sm.warp_cnt[1][lane] : 0;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int tg = __shfl_up_sync(0xffffffffu, sg, o), te = __shfl_up_sync(0xffffffffu, se, o);
+    if (lane >= o) {
+      sg += tg;
+      se += te;
     }
-    pos += __popc(take_mask);
-    eq_rank += __popc(eq_mask);
   }
-  // self-check: exactly k blocks were emitted (the last warp ends at k)
-  if (warp == NW - 1 && lane == 0 && pos != k) set_status(dev_status, KIN_ERR_DEVICE_DATA);
+  int g_run = warp ? __shfl_sync(0xffffffffu, sg, warp - 1) : 0;
+  int e_run = warp ? __shfl_sync(0xffffffffu, se, warp - 1) : 0;
+  for (int c = w0; c < w1; c += 1024) {
+    unsigned gm, em;
+    chunk_masks(c + 32 * lane, gm, em);
+    const int ng = __popc(gm), ne = __popc(em);
+    int ig = ng, ie = ne;  // inclusive scans over the lanes
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int tg = __shfl_up_sync(0xffffffffu, ig, o), te = __shfl_up_sync(0xffffffffu, ie, o);
+      if (lane >= o) {
+        ig += tg;
+        ie += te;
+      }
+    }
+    const int gb = g_run + ig - ng, eb = e_run + ie - ne;  // keys before this lane's first
+    unsigned take = gm;
+    for (int keep = min(max(kr - eb, 0), ne); keep > 0; --keep) {
+      take |= em & (0u - em);
+      em &= em - 1u;
+    }
+    int pos = gb + min(eb, kr);
+    const int i0 = c + 32 * lane;
+    while (take) {
+      const int b = __ffs(take) - 1;
+      take &= take - 1u;
+      if (pos < k) sel[pos] = i0 + b;
+      ++pos;
+    }
+    g_run += __shfl_sync(0xffffffffu, ig, 31);
+    e_run += __shfl_sync(0xffffffffu, ie, 31);
+  }
+  // self-check: exactly k blocks were emitted
+  if (warp == NW - 1 && lane == 0 && g_run + min(e_run, kr) != k) set_status(dev_status, KIN_ERR_DEVICE_DATA);
 }
 
-// Ranks the boundary bin's c keys (sm.list[0..c)) pairwise: the need-th
-// largest, with multiplicity, is the threshold T, and need - #{keys > T} of
-// the keys equal to T are kept.  Every thread that finds it writes the same
-// values.  Ends with a barrier.
+// Ranks the c keys sm.list[off..off+c) pairwise: the need-th largest, with
+// multiplicity, is the threshold T, and need - #{keys > T} of the keys equal
+// to T are kept.  Every thread that finds it writes the same values.  Ends
+// with a barrier.
 template <int NT>
-__device__ __forceinline__ void rank_boundary_bin(int c, int need, TopkSmem<NT>& sm) {
+__device__ __forceinline__ void rank_keys(int off, int c, int need, TopkSmem<NT>& sm) {
+  const uint32_t* list = sm.list + off;
   for (int j = threadIdx.x; j < c; j += NT) {
-    const uint32_t kj = sm.list[j];
+    const uint32_t kj = list[j];
     int gt = 0, ge = 0;
     for (int i = 0; i < c; ++i) {
-      const uint32_t ki = sm.list[i];
+      const uint32_t ki = list[i];
       gt += ki > kj;
       ge += ki >= kj;
     }
@@ -311,6 +418,133 @@ __device__ __forceinline__ void rank_boundary_bin(int c, int need, TopkSmem<NT>&
     }
   }
   __syncthreads();
+}
+
+// The boundary bin's c keys (sm.list[0..c)) ranked pairwise.
+template <int NT>
+__device__ __forceinline__ void rank_boundary_bin(int c, int need, TopkSmem<NT>& sm) {
+  rank_keys(0, c, need, sm);
+}
+
+// Sub-bin (0..255) of a key whose scaled score x = (s - s_min) * (256 /
+// (s_max - s_min)) fell in equal-width bin `bin`: the fraction of x above the
+// bin's lower edge, cut into 256 equal parts.  Non-decreasing in x (the
+// subtraction of a constant and the scaling by 2^8 are correctly rounded),
+// with explicitly rounded operations so that no call site fuses them.
+__device__ __forceinline__ int sub_bin(float x, int bin) {
+  const float f = __fmul_rn(__fsub_rn(x, (float)bin), 256.f);
+  return min(max((int)f, 0), 255);
+}
+
+// The equal-width-bin search fused with the emit, for rows whose emit ranges
+// are one round per warp (nb <= 1024 warps): the bin histogram (any order),
+// then one pass in the emit's ownership (lane l of warp w: the 32 keys from
+// w0 + 32 l, rotated reads) that sets, per lane, the mask of keys taken
+// outright (forced, or in a bin above the boundary bin) and the mask of keys
+// in the boundary bin, and lists the latter's keys (one reservation per
+// warp).  A boundary bin of more than kDirectRank keys also histograms its
+// keys' 256 sub-bins (sm.hist[1]) while listing them, and only the sub-bin
+// holding the threshold is copied out and ranked pairwise (keys in higher
+// sub-bins are larger); a smaller bin is ranked whole.  Then only the
+// boundary-bin bits are revisited to split them into above / equal to the
+// threshold, and emit_round writes.  Returns false (CTA-uniform, nothing
+// written) when the range is empty or not finite, or the boundary bin holds
+// more than kRankCap keys.  Expects sm.hist[0] and sm.hist[1] zero.
+template <int NT>
+__device__ __forceinline__ bool linear_select(const uint32_t* keys, int nb, const Cands& cd, int k, uint32_t kmin,
+                                              uint32_t kmax, int32_t* sel, TopkSmem<NT>& sm, int32_t* dev_status) {
+  constexpr int NW = NT / 32;
+  const int kr = cd.kr;
+  const float lo = key_float(kmin), hi = key_float(kmax);
+  const float range = hi - lo;
+  const float inv = 256.f / range;
+  if (!(isfinite(lo) && isfinite(hi) && range > 0.f && isfinite(range) && isfinite(inv))) return false;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  auto scaled = [&](uint32_t key) { return __fmul_rn(__fsub_rn(key_float(key), lo), inv); };
+  auto bin_of = [&](uint32_t key) { return min((int)scaled(key), 255); };
+  for (int i = cd.lo + tid; i <= cd.hi; i += NT) atomicAdd(&sm.hist[0][hidx(bin_of(keys[i]))], 1);
+  if (tid == 0) sm.list_n = sm.list_n2 = 0;
+  __syncthreads();
+  int bstar, above, c;
+  warp_find_bin(sm.hist[0], kr, bstar, above, c);  // every warp, same result
+  if (c > kRankCap) return false;
+  const bool two_level = c > kDirectRank;
+  auto sub_of = [&](uint32_t key) { return sub_bin(scaled(key), bstar); };
+  const int span = ((nb + NW - 1) / NW + 1023) & ~1023;  // 1024: one round
+  const int w0 = min(warp * span, nb), w1 = min(w0 + span, nb);
+  const int c0 = w0 + 32 * lane;
+  unsigned gm = 0u, bm = 0u;
+  if (c0 + 32 <= w1 && c0 >= cd.lo && c0 + 31 <= cd.hi) {  // 32 candidates
+#pragma unroll 8
+    for (int j = 0; j < 32; ++j) {
+      const int b = (j + lane) & 31;
+      const int bin = bin_of(keys[c0 + b]);
+      gm |= (unsigned)(bin > bstar) << b;
+      bm |= (unsigned)(bin == bstar) << b;
+    }
+  } else if (c0 < w1) {
+    for (int j = 0; j < 32; ++j) {
+      const int b = (j + lane) & 31;
+      const int i = c0 + b;
+      if (i < w1) {
+        if (!cd.has(i)) {
+          gm |= 1u << b;  // forced
+        } else {
+          const int bin = bin_of(keys[i]);
+          gm |= (unsigned)(bin > bstar) << b;
+          bm |= (unsigned)(bin == bstar) << b;
+        }
+      }
+    }
+  }
+  {  // list the boundary bin's keys: one reservation per warp, lanes in order
+    const int nbm = __popc(bm);
+    int incl = nbm;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    int slot = 0;
+    if (lane == 31 && incl) slot = atomicAdd(&sm.list_n, incl);
+    slot = __shfl_sync(0xffffffffu, slot, 31) + incl - nbm;
+    for (unsigned m = bm; m; m &= m - 1u, ++slot) {
+      const uint32_t key = keys[c0 + __ffs(m) - 1];
+      if (slot < kListCap) sm.list[slot] = key;
+      if (two_level) atomicAdd(&sm.hist[1][hidx(sub_of(key))], 1);
+    }
+  }
+  __syncthreads();
+  if (two_level) {
+    int sb, above2, c2;
+    warp_find_bin(sm.hist[1], kr - above, sb, above2, c2);  // every warp, same result
+    for (int base = 0; base < c; base += NT) {  // copy the sub-bin's keys to list[c..c+c2)
+      const int j = base + tid;
+      const uint32_t key = j < c ? sm.list[j] : 0u;
+      const bool match = j < c && sub_of(key) == sb;
+      const unsigned m = __ballot_sync(0xffffffffu, match);
+      if (m) {
+        int slot = 0;
+        if (lane == 0) slot = atomicAdd(&sm.list_n2, __popc(m));
+        slot = c + __shfl_sync(0xffffffffu, slot, 0) + __popc(m & ((1u << lane) - 1u));
+        if (match && slot < kListCap) sm.list[slot] = key;
+      }
+    }
+    __syncthreads();
+    rank_keys(c, c2, kr - above - above2, sm);
+  } else {
+    rank_keys(0, c, kr - above, sm);
+  }
+  const uint32_t T = sm.thresh;
+  unsigned em = 0u;
+  for (unsigned m = bm; m; m &= m - 1u) {
+    const int b = __ffs(m) - 1;
+    const uint32_t key = keys[c0 + b];
+    gm |= (unsigned)(key > T) << b;
+    em |= (unsigned)(key == T) << b;
+  }
+  emit_round(gm, em, c0, k, sm.thresh_take, sel, sm, dev_status);
+  return true;
 }
 
 // One-pass threshold search for score distributions without extreme
@@ -347,10 +581,12 @@ __device__ __forceinline__ bool linear_threshold(const uint32_t* keys, const Can
     const uint32_t key = in ? keys[i] : 0u;
     const bool match = in && bin_of(key) == bstar;
     const unsigned m = __ballot_sync(0xffffffffu, match);
-    int slot = 0;
-    if (lane == 0 && m) slot = atomicAdd(&sm.list_n, __popc(m));
-    slot = __shfl_sync(0xffffffffu, slot, 0);
-    if (match) sm.list[slot + __popc(m & ((1u << lane) - 1u))] = key;
+    if (m) {  // warp-uniform: one list reservation per warp, lanes take slots in order
+      int slot = 0;
+      if (lane == 0) slot = atomicAdd(&sm.list_n, __popc(m));
+      slot = __shfl_sync(0xffffffffu, slot, 0);
+      if (match) sm.list[slot + __popc(m & ((1u << lane) - 1u))] = key;
+    }
   }
   __syncthreads();
   rank_boundary_bin(c, kr - above, sm);
@@ -366,9 +602,16 @@ template <int NT>
 __device__ __forceinline__ void select_from_keys(const uint32_t* keys, int nb, const Cands& cd, int k,
                                                  uint32_t kmin, uint32_t kmax, int32_t* sel, TopkSmem<NT>& sm,
                                                  int32_t* dev_status) {
+  constexpr int NW = NT / 32;
   uint32_t prefix = 0xFFFFFFFFu, mask = 0xFFFFFFFFu;  // kr == 0: no candidate passes
   int kr = cd.kr;
-  if (kr > 0 && !linear_threshold(keys, cd, kr, kmin, kmax, sm, prefix, kr)) {
+  if (kr > 0) {
+    if (nb <= 1024 * NW) {
+      if (linear_select(keys, nb, cd, k, kmin, kmax, sel, sm, dev_status)) return;
+    } else if (linear_threshold(keys, cd, kr, kmin, kmax, sm, prefix, kr)) {
+      emit_selection(keys, nb, cd, k, prefix, mask, kr, sel, sm, dev_status);
+      return;
+    }
     __syncthreads();  // every warp is done with the bin histogram
     zero_hist(sm, 0);
     __syncthreads();
@@ -382,15 +625,51 @@ __device__ __forceinline__ void select_from_keys(const uint32_t* keys, int nb, c
 
 // Loads a pair's nb scores (written by the scan kernel: read from L2) as
 // keys into keys[] (shared memory, or the score row itself), returns the
-// smallest and largest candidate key, and zeroes both histograms.
+// smallest and largest candidate key, and zeroes both histograms.  With both
+// rows 16-byte aligned, whole groups of 4 scores move as 16-byte loads and
+// stores, 8 per thread in flight; the rest one score at a time.
 template <int NT>
 __device__ __forceinline__ void load_keys(const uint32_t* sc, uint32_t* keys, int nb, const Cands& cd, TopkSmem<NT>& sm,
                                           uint32_t& kmin, uint32_t& kmax) {
   constexpr int NW = NT / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int kBatch = 8;
   uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-  for (int base = 0; base < nb; base += kBatch * NT) {
+  int done = 0;
+  if (((reinterpret_cast<uintptr_t>(sc) | reinterpret_cast<uintptr_t>(keys)) & 15) == 0) {
+    constexpr int kVec = 8;
+    const int nv = nb >> 2;
+    const uint4* sc4 = reinterpret_cast<const uint4*>(sc);
+    uint4* keys4 = reinterpret_cast<uint4*>(keys);
+    for (int base = 0; base < nv; base += kVec * NT) {
+      uint4 v[kVec];
+#pragma unroll
+      for (int u = 0; u < kVec; ++u) {
+        const int j = base + u * NT + tid;
+        v[u] = j < nv ? __ldcg(sc4 + j) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kVec; ++u) {
+        const int j = base + u * NT + tid;
+        if (j < nv) {
+          const uint4 kk = make_uint4(key_of_bits(v[u].x), key_of_bits(v[u].y), key_of_bits(v[u].z), key_of_bits(v[u].w));
+          keys4[j] = kk;
+          const int i = 4 * j;
+          if (i >= cd.lo && i + 3 <= cd.hi) {
+            lo = min(lo, min(min(kk.x, kk.y), min(kk.z, kk.w)));
+            hi = max(hi, max(max(kk.x, kk.y), max(kk.z, kk.w)));
+          } else {
+            if (cd.has(i)) { lo = min(lo, kk.x); hi = max(hi, kk.x); }
+            if (cd.has(i + 1)) { lo = min(lo, kk.y); hi = max(hi, kk.y); }
+            if (cd.has(i + 2)) { lo = min(lo, kk.z); hi = max(hi, kk.z); }
+            if (cd.has(i + 3)) { lo = min(lo, kk.w); hi = max(hi, kk.w); }
+          }
+        }
+      }
+    }
+    done = nv << 2;
+  }
+  constexpr int kBatch = 8;
+  for (int base = done; base < nb; base += kBatch * NT) {
     uint32_t v[kBatch];
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
@@ -532,10 +811,12 @@ __device__ __forceinline__ void topk_regs(const uint32_t* row, int nb, const Can
       const int i = u * NT + tid;
       const bool match = cd.has(i) && bin_of(key[u]) == bstar;
       const unsigned m = __ballot_sync(0xffffffffu, match);
-      int slot = 0;
-      if (lane == 0 && m) slot = atomicAdd(&sm.list_n, __popc(m));
-      slot = __shfl_sync(0xffffffffu, slot, 0);
-      if (match) sm.list[slot + __popc(m & ((1u << lane) - 1u))] = key[u];
+      if (m) {  // warp-uniform
+        int slot = 0;
+        if (lane == 0) slot = atomicAdd(&sm.list_n, __popc(m));
+        slot = __shfl_sync(0xffffffffu, slot, 0);
+        if (match) sm.list[slot + __popc(m & ((1u << lane) - 1u))] = key[u];
+      }
     }
     __syncthreads();
     rank_boundary_bin(c, kr - above, sm);

@@ -103,6 +103,30 @@ def test_crafted_scores_exercise_both_threshold_searches():
         assert list(sel_f[b, h]) == list(rsel), (b, h)
 
 
+def test_long_row_boundary_bin_ranked_through_sub_bins():
+    """A pair of 9000 blocks (keys in shared memory): one outlier widens the
+    bins, the rest climb steeply (v = 0.1 + 39 (i/9000)^4, in ties of two), so
+    the boundary bin holds ~280 keys and the threshold is found through its
+    sub-bins, one tie pair per sub-bin, with the budget taking one key of the
+    deciding pair (the lower index); a second pair with the same blocks
+    reversed puts the ties' lower index on the other side."""
+    bs, g, k, nb = 16, 4, 601, 9000
+    i = np.arange(nb)
+    v = 0.1 + 39.0 * ((i // 2) * 2 / nb) ** 4
+    v = np.where(i == 5, 1e3, np.where(i == 9, 0.0, v))
+    vals = [[v, v[::-1].copy()]]
+    lens = [nb * bs]
+    dims, q, means, lens_t, means_h, q_bits = _crafted_case(1, 2, g, bs, lens, vals)
+    ref = _oracle_sel(means_h, q_bits, lens, bs, g, k)
+    sel_f, cnt_f, st_f = _select(dims, q, means, lens_t, k)
+    sel_n, cnt_n, st_n = _select(dims, q, means, lens_t, k, noalloc=True)
+    assert st_f == 0 and st_n == 0
+    assert np.array_equal(sel_f, sel_n) and np.array_equal(cnt_f, cnt_n)
+    for (b, h), (rsel, rcnt) in ref.items():
+        assert cnt_f[b, h] == rcnt == k
+        assert list(sel_f[b, h]) == list(rsel), (b, h)
+
+
 def test_large_batch_with_dense_scanned_and_bad_lengths():
     """1030 sequences, dense and scanned mixed; sampled pairs against the
     oracle, then one bad length in the middle, flagged and emptied."""
