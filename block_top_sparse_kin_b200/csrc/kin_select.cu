@@ -82,10 +82,10 @@ __device__ __forceinline__ float warp_sum_rows(float (&v)[U], int lane) {
 // per pair.  Scores become order-preserving uint32 keys (float_key); the
 // threshold is found by a search over 256 equal-width score bins, with a
 // radix search over the key bits for crowded or degenerate ranges.
-constexpr int kListCap = 4096;  // radix: candidates kept after the first pass
-constexpr int kRankCap = 512;   // equal-width bins: boundary-bin keys listed (ranked pairwise, or by sub-bins)
-constexpr int kDirectRank = 64;  // boundary bins up to this size are ranked without sub-bins
-constexpr int kMaxKPT = 8;      // keys per thread on the register path
+constexpr int kListCap = 4096;   // radix: candidates kept after the first pass
+constexpr int kRankCap = 512;    // equal-width bins: most boundary-bin keys listed
+constexpr int kDirectRank = 64;  // keys in memory: larger boundary bins are ranked through sub-bins
+constexpr int kMaxKPT = 8;       // keys per thread on the register path
 // 256-bin histograms padded by one word per 8 bins, so a lane reading 8
 // consecutive bins (stride 9 words between lanes) hits 32 distinct banks
 constexpr int kHistWords = 256 + 32;
@@ -104,7 +104,7 @@ template <int NT>
 struct TopkSmem {
   static constexpr int NW = NT / 32;
   int hist[2][kHistWords];   // histograms (equal-width bins, or radix digits double-buffered), hidx-padded
-  uint32_t list[kListCap];   // radix: candidate indices; equal-width bins: boundary-bin keys
+  uint32_t list[kListCap];   // radix: candidate indices; equal-width bins: boundary-bin keys (then the deciding sub-bin's)
   int list_n, list_n2;
   int warp_cnt[2][NW];       // emit: per-warp counts of keys taken outright, and equal to the threshold
   uint32_t wmin[NW], wmax[NW];
@@ -548,7 +548,9 @@ __device__ __forceinline__ bool linear_select(const uint32_t* keys, int nb, cons
 }
 
 // One-pass threshold search for score distributions without extreme
-// outliers, over keys in memory.  The candidates' scores are cut into 256
+// outliers, over keys in memory, for rows longer than 1024 keys per warp
+// (shorter rows take linear_select, which shares its binning and fuses the
+// emit).  The candidates' scores are cut into 256
 // equal-width bins between the smallest (kmin) and largest (kmax) candidate
 // key; the bin of a score, trunc((s - s_min) * (256 / (s_max - s_min))), is a
 // non-decreasing function of s (a correctly rounded subtract and multiply,
