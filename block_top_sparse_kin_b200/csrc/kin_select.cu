@@ -451,8 +451,9 @@ __device__ __forceinline__ int sub_bin(float x, int bin) {
 // written) when the range is empty or not finite, or the boundary bin holds
 // more than kRankCap keys.  Expects sm.hist[0] and sm.hist[1] zero.
 template <int NT>
-__device__ __forceinline__ bool linear_select(const uint32_t* keys, int nb, const Cands& cd, int k, uint32_t kmin,
-                                              uint32_t kmax, int32_t* sel, TopkSmem<NT>& sm, int32_t* dev_status) {
+__device__ __forceinline__ bool linear_select(const uint32_t* keys, uint8_t* bins, int nb, const Cands& cd, int k,
+                                              uint32_t kmin, uint32_t kmax, int32_t* sel, TopkSmem<NT>& sm,
+                                              int32_t* dev_status) {
   constexpr int NW = NT / 32;
   const int kr = cd.kr;
   const float lo = key_float(kmin), hi = key_float(kmax);
@@ -462,7 +463,11 @@ __device__ __forceinline__ bool linear_select(const uint32_t* keys, int nb, cons
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   auto scaled = [&](uint32_t key) { return __fmul_rn(__fsub_rn(key_float(key), lo), inv); };
   auto bin_of = [&](uint32_t key) { return min((int)scaled(key), 255); };
-  for (int i = cd.lo + tid; i <= cd.hi; i += NT) atomicAdd(&sm.hist[0][hidx(bin_of(keys[i]))], 1);
+  for (int i = cd.lo + tid; i <= cd.hi; i += NT) {
+    const int bin = bin_of(keys[i]);
+    bins[i] = (uint8_t)bin;
+    atomicAdd(&sm.hist[0][hidx(bin)], 1);
+  }
   if (tid == 0) sm.list_n = sm.list_n2 = 0;
   __syncthreads();
   int bstar, above, c;
@@ -475,12 +480,20 @@ __device__ __forceinline__ bool linear_select(const uint32_t* keys, int nb, cons
   const int c0 = w0 + 32 * lane;
   unsigned gm = 0u, bm = 0u;
   if (c0 + 32 <= w1 && c0 >= cd.lo && c0 + 31 <= cd.hi) {  // 32 candidates
-#pragma unroll 8
-    for (int j = 0; j < 32; ++j) {
-      const int b = (j + lane) & 31;
-      const int bin = bin_of(keys[c0 + b]);
-      gm |= (unsigned)(bin > bstar) << b;
-      bm |= (unsigned)(bin == bstar) << b;
+    // the chunk's 32 bins as 8 words, 4 compared at once; word r holds keys
+    // c0 + 4r .. c0 + 4r + 3 (byte e: key c0 + 4r + e).  Lane l takes word
+    // (j + l / 4) mod 8 at step j: 32 distinct banks.  A compare gives 0xFF
+    // per true byte; (m & 0x01010101) * 0x01020408 gathers the four flags
+    // into bits 24..27 (byte e's flag to bit 24 + e, no carries).
+    const uint32_t b4 = 0x01010101u * (uint32_t)bstar;
+    const uint32_t* binw = reinterpret_cast<const uint32_t*>(bins + c0);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int r = (j + (lane >> 2)) & 7;
+      const uint32_t w = binw[r];
+      const uint32_t gt = __vcmpgtu4(w, b4), eq = __vcmpeq4(w, b4);
+      gm |= (((gt & 0x01010101u) * 0x01020408u) >> 24) << (4 * r);
+      bm |= (((eq & 0x01010101u) * 0x01020408u) >> 24) << (4 * r);
     }
   } else if (c0 < w1) {
     for (int j = 0; j < 32; ++j) {
@@ -490,7 +503,7 @@ __device__ __forceinline__ bool linear_select(const uint32_t* keys, int nb, cons
         if (!cd.has(i)) {
           gm |= 1u << b;  // forced
         } else {
-          const int bin = bin_of(keys[i]);
+          const int bin = bins[i];
           gm |= (unsigned)(bin > bstar) << b;
           bm |= (unsigned)(bin == bstar) << b;
         }
@@ -599,17 +612,18 @@ __device__ __forceinline__ bool linear_threshold(const uint32_t* keys, const Can
 
 // Exact top-(k-2) over keys[1..nb-2] plus the forced blocks 0 and nb-1,
 // written ascending to sel[0..k).  kmin / kmax: the smallest and largest
-// candidate key.  Expects sm.hist[0] and sm.hist[1] zero.
+// candidate key; bins: nb bytes of shared memory for the keys' bins, or
+// null.  Expects sm.hist[0] and sm.hist[1] zero.
 template <int NT>
-__device__ __forceinline__ void select_from_keys(const uint32_t* keys, int nb, const Cands& cd, int k,
+__device__ __forceinline__ void select_from_keys(const uint32_t* keys, uint8_t* bins, int nb, const Cands& cd, int k,
                                                  uint32_t kmin, uint32_t kmax, int32_t* sel, TopkSmem<NT>& sm,
                                                  int32_t* dev_status) {
   constexpr int NW = NT / 32;
   uint32_t prefix = 0xFFFFFFFFu, mask = 0xFFFFFFFFu;  // kr == 0: no candidate passes
   int kr = cd.kr;
   if (kr > 0) {
-    if (nb <= 1024 * NW) {
-      if (linear_select(keys, nb, cd, k, kmin, kmax, sel, sm, dev_status)) return;
+    if (bins && nb <= 1024 * NW) {
+      if (linear_select(keys, bins, nb, cd, k, kmin, kmax, sel, sm, dev_status)) return;
     } else if (linear_threshold(keys, cd, kr, kmin, kmax, sm, prefix, kr)) {
       emit_selection(keys, nb, cd, k, prefix, mask, kr, sel, sm, dev_status);
       return;
@@ -710,16 +724,19 @@ __device__ __forceinline__ void load_keys(const uint32_t* sc, uint32_t* keys, in
 }
 
 // The top-k of one row of nb scores with any nb, keys in memory: shared
-// memory when nb <= key_cap, else gkeys (nb words of global scratch, which
-// may be the score row itself when nothing reads it afterwards).
+// memory when nb <= key_cap (skey holds key_cap words, then key_cap bytes
+// for the keys' bins), else gkeys (nb words of global scratch, which may be
+// the score row itself when nothing reads it afterwards).
 template <int NT>
 __device__ __forceinline__ void topk_memory(const uint32_t* row, int nb, const Cands& cd, int k, int32_t* sel,
                                             uint32_t* skey, int key_cap, uint32_t* gkeys, TopkSmem<NT>& sm,
                                             int32_t* dev_status) {
-  uint32_t* keys = nb <= key_cap ? skey : gkeys;
+  const bool in_smem = nb <= key_cap;
+  uint32_t* keys = in_smem ? skey : gkeys;
+  uint8_t* bins = in_smem ? reinterpret_cast<uint8_t*>(skey + key_cap) : nullptr;
   uint32_t kmin, kmax;
   load_keys(row, keys, nb, cd, sm, kmin, kmax);
-  select_from_keys(keys, nb, cd, k, kmin, kmax, sel, sm, dev_status);
+  select_from_keys(keys, bins, nb, cd, k, kmin, kmax, sel, sm, dev_status);
 }
 
 // The top-k of one pair with nb <= KPT * NT blocks, keys held in registers:
@@ -1142,7 +1159,7 @@ __global__ void __launch_bounds__(kSelThreads, KIN_SEL_CTAS_PER_SM) select_scan_
 // (L2-resident), in registers when nb <= 8 NT.
 template <int NT>
 __global__ void __launch_bounds__(NT, 1024 / NT) select_topk_kernel(SelectParams p) {
-  extern __shared__ uint32_t skey[];  // [nbcap]
+  extern __shared__ uint32_t skey[];  // [nbcap] keys (rows beyond 8 NT blocks: then nbcap bytes of bins)
   __shared__ TopkSmem<NT> sm;
   const int tid = threadIdx.x;
   pdl_wait();  // scores come from the scan kernel
@@ -1181,7 +1198,7 @@ constexpr int kTokTopkThreads = 1024;
 constexpr int kTokKeyCap = 32768;  // keys kept in shared memory up to this many tokens
 
 __global__ void __launch_bounds__(kTokTopkThreads, 1) token_topk_kernel(TokenParams p) {
-  extern __shared__ uint32_t skey[];  // [min(Lcap, kTokKeyCap)]
+  extern __shared__ uint32_t skey[];  // [min(Lcap, kTokKeyCap)] keys, then as many bytes of bins
   __shared__ TopkSmem<kTokTopkThreads> sm;
   const int tid = threadIdx.x;
   pdl_wait();  // the logits come from the logits kernel
@@ -1209,13 +1226,14 @@ __global__ void __launch_bounds__(kTokTopkThreads, 1) token_topk_kernel(TokenPar
   if (L <= 4 * kTokTopkThreads) topk_regs<kTokTopkThreads, 4>(row, L, cd, k, sel, skey, sm, p.dev_status);
   else if (L <= 8 * kTokTopkThreads) topk_regs<kTokTopkThreads, 8>(row, L, cd, k, sel, skey, sm, p.dev_status);
   else
-    topk_memory<kTokTopkThreads>(row, L, cd, k, sel, skey, kTokKeyCap, p.key_scratch + row_id * p.Lcap, sm,
+    topk_memory<kTokTopkThreads>(row, L, cd, k, sel, skey, min(p.Lcap, kTokKeyCap), p.key_scratch + row_id * p.Lcap, sm,
                                  p.dev_status);
   if (tid == 0) p.cnt[row_id] = k;
 }
 
 cudaError_t launch_token_topk(const TokenParams& p, cudaStream_t s) {
-  const size_t smem = (size_t)(p.Lcap < kTokKeyCap ? p.Lcap : kTokKeyCap) * sizeof(uint32_t);
+  const size_t cap = (size_t)(p.Lcap < kTokKeyCap ? p.Lcap : kTokKeyCap);
+  const size_t smem = cap * sizeof(uint32_t) + ((cap + 3) & ~size_t(3));  // keys, then their bins
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(token_topk_kernel), 5, smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(token_topk_kernel, dim3(p.B * p.Hq), dim3(kTokTopkThreads), smem, s, p);
@@ -1232,7 +1250,8 @@ int topk_threads(int nbcap, int64_t pairs) {
 
 template <int NT>
 cudaError_t launch_topk(const SelectParams& p, cudaStream_t s) {
-  const size_t smem = (size_t)p.nbcap * sizeof(uint32_t);
+  // keys (when they do not fit in registers: then also their bins)
+  const size_t smem = (size_t)p.nbcap * sizeof(uint32_t) + (p.nbcap > 8 * NT ? ((size_t)p.nbcap + 3) & ~size_t(3) : 0);
   if (smem > 16 * 1024) {
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(select_topk_kernel<NT>),
                                       NT == 256 ? 0 : NT == 512 ? 2 : 3, smem);

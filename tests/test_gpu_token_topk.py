@@ -75,6 +75,9 @@ def check_head(dc, b, j, kt, sel, out, lse):
     (W("tok_k1", 2, 2, 4, D, 16, 50, 300, 8, 94, Lcap=320), 1),
     # kept tokens over three segments of the attention kernel (2048, 2048, 404)
     (W("tok_g2_segments", 1, 2, 4, D, 16, 0, 0, 8, 96, Lcap=6000, lens=(5999,)), 4500),
+    # rows longer than the 32768 keys kept in shared memory: keys in the
+    # workspace scratch row, the emit in two rounds per warp
+    (W("tok_long_scratch", 1, 1, 2, D, 16, 0, 0, 8, 97, Lcap=40000, lens=(39999,)), 3000),
 ], ids=lambda x: x.name if hasattr(x, "name") else str(x))
 def test_token_topk_every_head(w, kt):
     dc = make_device_case(w)
