@@ -167,6 +167,43 @@ def test_extended_calls_reject_before_launch(lib):
     assert upd(pages=0) == 1
 
 
+def test_token_and_page_means_calls_reject_before_launch(lib):
+    d = dims()
+    bd = ctypes.byref(d)
+    # token workspace: logits + kept indices + counts; a key scratch row only past 32768 tokens
+    assert kin.kin_token_topk_workspace_bytes(d, 0) == 0
+    assert kin.kin_token_topk_workspace_bytes(dims(D=64), 8) == 0
+    rows, L = 2 * 8, 256
+    n8 = kin.kin_token_topk_workspace_bytes(d, 8)
+    assert n8 >= rows * L * 4 + rows * 8 * 4 + rows * 4 and n8 % 256 == 0
+    assert kin.kin_token_topk_workspace_bytes(d, 64) >= n8 + rows * 56 * 4
+    at_cap = kin.kin_token_topk_workspace_bytes(kin.make_dims(1, 1, 2, 128, 16, 32768), 8)
+    past_cap = kin.kin_token_topk_workspace_bytes(kin.make_dims(1, 1, 2, 128, 16, 32769), 8)
+    assert at_cap < 2 * 32768 * 8 and past_cap >= 2 * 32769 * 8
+    tok = lambda k=8, q=FAKE, scale=0.0, ws=FAKE, n=1 << 30, dd=bd: lib.kin_token_topk_decode_attn(
+        dd, q, FAKE, FAKE, FAKE, k, scale, FAKE, None, None, ws, n, None, None)
+    assert tok(k=0) == 1
+    assert tok(q=None) == 1
+    assert tok(q=ctypes.c_void_p((1 << 20) + 2)) == 1
+    assert tok(scale=float("nan")) == 1
+    assert tok(scale=float("inf")) == 1
+    assert tok(ws=None) == 2
+    assert tok(ws=ctypes.c_void_p((1 << 20) + 16)) == 2
+    assert tok(n=64) == 2
+    rows_cap = kin.make_dims(64, 8, 64, 128, 16, 1 << 19)   # B * Hq * Lcap = 2^31
+    assert tok(dd=ctypes.byref(rows_cap)) == 3
+    # the select over means stored per page
+    sp = lambda dt=0, pages=4, table=FAKE, pool=FAKE, k=8, ws=FAKE: lib.kin_block_topk_select_paged(
+        bd, FAKE, pool, dt, pages, table, FAKE, k, FAKE, FAKE, ws, 1 << 30, None, None)
+    assert sp(dt=2) == 1
+    assert sp(pages=0) == 1
+    assert sp(table=None) == 1
+    assert sp(pool=None) == 1
+    assert sp(pool=ctypes.c_void_p((1 << 20) + 8)) == 1
+    assert sp(k=1) == 1
+    assert sp(ws=None) == 2
+
+
 def test_binding_refuses_host_tensors(lib):
     import torch
     with pytest.raises(ValueError):
