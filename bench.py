@@ -7,10 +7,14 @@ an append first run kin_block_means_update.  The block means and KV cache are
 resident decode state built before timing.
 
 Metric: query-heads/s = B * Hq / t_step (whole job: summed over ranks, time =
-max over ranks).  Timing: CUDA events on the launching stream, one event pair
-per kernel per step, L2 flushed (a 256 MiB write then a 256 MiB read, outside
-the events) before every step; W warm-up steps; barrier + synchronize around
-the K timed steps.
+max over ranks).  Timing: the step is captured once as a CUDA graph and
+replayed, with two timing events inside it around the step's kernels (CUDA
+events on the launching stream); L2 flushed (a 256 MiB write then a 256 MiB
+read, outside the events) before every step; W warm-up steps; barrier +
+synchronize around the K timed steps.  Per-kernel times (for the roofline)
+come from one graph per kernel family holding back-to-back calls; the e2e
+figure runs the step eagerly through the public calls with pinned host
+copies of q in and out inside the events.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--k K]
   python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
