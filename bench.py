@@ -13,7 +13,7 @@ events on the launching stream); L2 flushed (a 256 MiB write then a 256 MiB
 read, outside the events) before every step; W warm-up steps; barrier +
 synchronize around the K timed steps.  Per-kernel times (for the roofline)
 come from one graph per kernel family holding back-to-back calls; the e2e
-figure runs the step eagerly through the public calls with pinned host
+figure runs the step eagerly through the public calls, with the copy of q
 copies of q in and out inside the events.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--k K]
