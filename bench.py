@@ -14,7 +14,7 @@ read, outside the events) before every step; W warm-up steps; barrier +
 synchronize around the K timed steps.  Per-kernel times (for the roofline)
 come from one graph per kernel family holding back-to-back calls; the e2e
 figure runs the step eagerly through the public calls, with the copy of q
-copies of q in and out inside the events.
+from pinned host memory and of the output back to it inside the events.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--k K]
   python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
