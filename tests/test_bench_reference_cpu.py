@@ -1,0 +1,38 @@
+"""The benchmark's reference arm on the CPU: it times the oracle as it stands
+on the host cores and prints one JSON line with the contract's keys; under a
+multi-rank launch only rank 0 works and prints."""
+import json
+import os
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _run(env_extra):
+    env = dict(os.environ, **env_extra)
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1", "--warmup", "1",
+           "--ref-pairs", "2"]
+    return subprocess.run(cmd, capture_output=True, text=True, timeout=600, env=env, check=True).stdout
+
+
+def test_reference_arm_prints_the_contract_line():
+    lines = [l for l in _run({}).splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["unit"] == "query-heads/s" and d["higher_is_better"] is True
+    assert d["value"] > 0 and d["steps"] == 1 and d["warmup"] == 1
+    assert d["config"]["workload"] == "qwen3_8b_32k"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and "2 of 256" in cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "query-heads/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    # the metric's time per full step follows from the rate
+    assert abs(d["ms_per_step"] - 32 * 32 / d["value"] * 1e3) < 1e-6 * d["ms_per_step"]
+
+
+def test_reference_arm_is_silent_on_other_ranks():
+    assert _run({"RANK": "1", "WORLD_SIZE": "2"}).strip() == ""
