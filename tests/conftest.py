@@ -25,3 +25,22 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """How often a GPU top-k set differed from the oracle's and was accepted
+    as a near tie (kin_tiecheck), per test that compared selections."""
+    mod = sys.modules.get("kin_tiecheck")
+    if mod is None or not mod.TALLY:
+        return
+    tally = {k: v for k, v in mod.TALLY.items() if "test_tiecheck" not in k}
+    if not tally:
+        return
+    tr = terminalreporter
+    tr.write_sep("-", "top-k sets compared with the oracle / accepted near ties")
+    total = [0, 0]
+    for name, (n, d) in sorted(tally.items()):
+        tr.write_line(f"{name}: {n} compared, {d} near-tie")
+        total[0] += n
+        total[1] += d
+    tr.write_line(f"all: {total[0]} compared, {total[1]} near-tie")

@@ -9,7 +9,7 @@ import torch
 
 import block_top_sparse_kin_b200 as kin
 import kin_inputs as ki
-from kin_testlib import D, GpuResult, check_pair, make_device_case, sample_pairs, to_pages
+from kin_testlib import D, GpuResult, all_pairs, check_pair, check_pairs, make_device_case, to_pages
 
 pytestmark = pytest.mark.gpu
 W = ki.Workload
@@ -85,11 +85,10 @@ def test_bf16_means_paged_equals_contiguous():
     assert np.array_equal(g_c.sel, g_p.sel) and np.array_equal(g_c.out, g_p.out)
 
 
-def test_bf16_means_32k_workload_sampled():
+def test_bf16_means_32k_workload_every_pair():
     w = ki.WORKLOADS["qwen3_8b_32k"]
     dc = make_device_case(w)
     means, _, gr = step_bf16(dc, w.k)
     assert gr.status == 0
     gm = means.float().cpu().numpy()
-    for b, h in sample_pairs(w, 6):
-        check_pair(dc, gr, b, h, w.k, gpu_means=gm, bf16_means=True)
+    check_pairs(dc, [(w.k, gr)], all_pairs(w), gpu_means=gm, bf16_means=True)

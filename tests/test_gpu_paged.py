@@ -13,7 +13,7 @@ import torch
 import block_top_sparse_kin_b200 as kin
 import kin_inputs as ki
 import oracle
-from kin_testlib import (D, check_pair, gpu_step, gpu_step_paged, make_device_case, sample_pairs,
+from kin_testlib import (D, all_pairs, check_pair, check_pairs, gpu_step, gpu_step_paged, make_device_case,
                          to_pages)
 
 pytestmark = pytest.mark.gpu
@@ -106,8 +106,7 @@ def test_paged_bad_page_index_is_flagged_and_skipped():
 
 def test_paged_ragged_workload_full_size():
     """The ragged 64-sequence workload at full size over a shuffled pool:
-    bit-identical to the contiguous cache, sampled pairs against the oracle."""
+    bit-identical to the contiguous cache, every pair against the oracle."""
     w = ki.WORKLOADS["qwen3_14b_ragged"]
     dc, pg, gr = _compare_with_contiguous(w, seed=11)
-    for b, h in sample_pairs(w, 6):
-        check_pair(dc, gr, b, h, w.k)
+    check_pairs(dc, [(w.k, gr)], all_pairs(w))

@@ -13,7 +13,8 @@ import torch
 import block_top_sparse_kin_b200 as kin
 import kin_inputs as ki
 import oracle
-from kin_testlib import D, TIE_REL, make_device_case
+from kin_testlib import D, make_device_case
+from kin_tiecheck import check_topk_set
 
 pytestmark = pytest.mark.gpu
 W = ki.Workload
@@ -92,15 +93,13 @@ def oracle_check(dc, kpool, vpool, table_host, b, h, k, sel, cnt, out, lse):
     c = int(cnt[b, h])
     assert c == rcnt
     g = sel[b, h, :c]
-    if not np.array_equal(g, rsel[:rcnt]):
-        nb = means.shape[0]
-        cand = np.sort(scores[1:nb - 1])[::-1]
-        tau_k, tau_k1 = cand[c - 3], cand[c - 2] if c - 2 < len(cand) else cand[c - 3]
-        qf = ki.bf16_to_f32(qg).astype(np.float64)
-        eps = (np.abs(qf).sum(axis=0) @ np.abs(means).T).mean() / math.sqrt(D)
-        delta = TIE_REL * max(abs(tau_k), abs(tau_k1), eps)
-        for i in set(g.tolist()) ^ set(rsel[:rcnt].tolist()):
-            assert min(abs(scores[i] - tau_k), abs(scores[i] - tau_k1)) <= delta, (b, h, i)
+    nb = means.shape[0]
+    forced = {0, nb - 1}
+    assert np.all(np.diff(g) > 0) and forced <= set(g.tolist()), (b, h)
+    qf = ki.bf16_to_f32(qg).astype(np.float64)
+    eps = (np.abs(qf).sum(axis=0) @ np.abs(means).T).mean() / math.sqrt(D)
+    check_topk_set(scores, np.arange(1, nb - 1), [i for i in rsel[:rcnt] if i not in forced],
+                   [i for i in g if i not in forced], eps, what=(b, h))
     o_ref, lse_ref = oracle.attend(qg, K, V, L, w.bs, g, 1 / math.sqrt(D))
     err = np.abs(out[b, h * w.g:(h + 1) * w.g].astype(np.float64) - o_ref)
     assert err.max() <= 2e-2 and err.mean() <= 2e-3, (b, h, err.max())

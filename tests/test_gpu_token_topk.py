@@ -1,13 +1,16 @@
 """Token-level top-k attention on the GPU (kin_token_topk_decode_attn)
 against the fp64 oracle on the same bf16 inputs.
 
-Kept token sets must match the oracle's except for swaps between tokens
-whose oracle logits lie within delta = 1e-4 max(|tau_k|, |tau_k+1|, eps) of
-the k-th / (k+1)-th largest logit (eps: the logits' natural magnitude, the
-mean over tokens of scale sum_d |q_d| |K_td|); outputs are then compared
+Kept token sets must equal the oracle's, except where the oracle's k-th and
+(k+1)-th largest logits are within delta = 1e-4 max(|tau_k|, |tau_k+1|, eps)
+of each other (eps: the logits' natural magnitude, the mean over tokens of
+scale sum_d |q_d| |K_td|); there the GPU set may differ only as a top set of
+logits perturbed by at most delta (kin_tiecheck).  Outputs are then compared
 with the oracle recomputed on the GPU's set (max |err| <= 2e-2, mean
 <= 2e-3; lse within 1e-3 + 1e-4 |lse|)."""
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 import pytest
@@ -16,11 +19,11 @@ import torch
 import block_top_sparse_kin_b200 as kin
 import kin_inputs as ki
 import oracle
-from kin_testlib import D, make_device_case
+from kin_testlib import D, all_pairs, make_device_case
+from kin_tiecheck import check_topk_set
 
 pytestmark = pytest.mark.gpu
 W = ki.Workload
-TIE_REL = 1e-4
 
 
 def run_token(dc, kt):
@@ -36,11 +39,13 @@ def run_token(dc, kt):
     return sel.cpu().numpy(), out.float().cpu().numpy(), lse.cpu().numpy(), int(st.item())
 
 
-def check_head(dc, b, j, kt, sel, out, lse):
+def check_head(dc, b, j, kt, sel, out, lse, rows=None):
+    """One query head against the oracle; rows: its pair's (K, V) when the
+    caller regenerated them already."""
     w = dc.w
     h = j // w.g
     L = int(dc.lens_final[b])
-    K, V = ki.pair_rows(w, dc.hh, b, h, L)
+    K, V = rows if rows is not None else ki.pair_rows(w, dc.hh, b, h, L)
     q = dc.q_host[b, j:j + 1]
     scale = 1 / math.sqrt(D)
     rsel, rout, rlse, z = oracle.token_topk_attend(q, K, V, L, kt, scale)
@@ -49,13 +54,9 @@ def check_head(dc, b, j, kt, sel, out, lse):
     assert np.all(gsel[n:] == -1), (b, j)
     g = gsel[:n]
     assert np.all(np.diff(g) > 0), (b, j, "not ascending")
+    scale_eps = scale * (np.abs(oracle.bf16_bits_to_f64(q[0])) @ np.abs(oracle.bf16_bits_to_f64(K[:L])).T).mean()
+    check_topk_set(z[0], np.arange(L), rsel[0], g, scale_eps, what=(b, j))
     if not np.array_equal(g, rsel[0]):
-        zs = np.sort(z[0])[::-1]
-        tau_k, tau_k1 = zs[n - 1], zs[n] if n < L else zs[n - 1]
-        eps = scale * (np.abs(oracle.bf16_bits_to_f64(q[0])) @ np.abs(oracle.bf16_bits_to_f64(K[:L])).T).mean()
-        delta = TIE_REL * max(abs(tau_k), abs(tau_k1), eps)
-        for t in set(g.tolist()) ^ set(rsel[0].tolist()):
-            assert min(abs(z[0, t] - tau_k), abs(z[0, t] - tau_k1)) <= delta, (b, j, t)
         # outputs against the oracle on the GPU's set
         zz = z[0, g]
         m = zz.max()
@@ -98,13 +99,23 @@ def test_token_topk_bad_length_is_flagged():
     check_head(dc, 0, 0, 16, sel, out, lse)
 
 
-def test_token_topk_32k_workload_sampled():
+def test_token_topk_32k_workload_every_head():
     """The 32K decode batch with a token budget equal to the block budget
-    (256 blocks x 16 tokens = 4096 tokens per query head), sampled heads."""
+    (256 blocks x 16 tokens = 4096 tokens per query head), every head
+    against the oracle (host threads, one K/V regeneration per pair)."""
     w = ki.WORKLOADS["qwen3_8b_32k"]
     dc = make_device_case(w)
     kt = w.k * w.bs
     sel, out, lse, status = run_token(dc, kt)
     assert status == 0
-    for b, j in [(0, 0), (7, 13), (19, 30), (31, 31)]:
-        check_head(dc, b, j, kt, sel, out, lse)
+    del dc.k_cache, dc.v_cache
+    torch.cuda.empty_cache()
+
+    def pair(bh):
+        b, h = bh
+        rows = ki.pair_rows(w, dc.hh, b, h, int(dc.lens_final[b]))
+        for j in range(h * w.g, (h + 1) * w.g):
+            check_head(dc, b, j, kt, sel, out, lse, rows)
+
+    with ThreadPoolExecutor(max(1, os.cpu_count() or 1)) as ex:
+        list(ex.map(pair, all_pairs(w)))
