@@ -33,6 +33,7 @@ import subprocess
 import sys
 import threading
 import time
+from dataclasses import dataclass
 
 import numpy as np
 
@@ -239,29 +240,73 @@ class ClockSampler:
 
 # --------------------------------------------------------------- GPU arm
 def setup_dist(args):
+    """One process per GPU.  Under a launcher (WORLD_SIZE > 1) the ranks join
+    one process group: NCCL on GPU hosts (gloo where no GPU is visible, which
+    only the host-side tests use); it carries the barriers around the timed
+    region and the max-over-ranks reduction, never data of the decode path."""
     import torch
     import torch.distributed as dist
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
-        torch.cuda.set_device(local)
         from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
-    else:
+        if torch.cuda.is_available():
+            if local >= torch.cuda.device_count():
+                raise SystemExit(f"rank {rank}: LOCAL_RANK {local} but only {torch.cuda.device_count()} GPUs visible")
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=timedelta(seconds=120))
+    elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return rank, world, local
 
 
-def reduce_max(x: float, device) -> float:
+def _reduce_device():
+    import torch.distributed as dist
+    return "cuda" if dist.get_backend() == "nccl" else "cpu"
+
+
+def reduce_max(x: float, device=None) -> float:
     """Max of a per-rank number over all ranks (identity on one rank)."""
+    return reduce_max_list([x], device)[0]
+
+
+def reduce_max_list(xs, device=None):
+    """Element-wise max over all ranks of a list of per-rank numbers, in one
+    collective (identity on one rank)."""
     import torch
     import torch.distributed as dist
     if not dist.is_initialized() or dist.get_world_size() == 1:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device=device)
+        return [float(x) for x in xs]
+    t = torch.tensor([float(x) for x in xs], dtype=torch.float64, device=device or _reduce_device())
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return [float(v) for v in t.cpu().tolist()]
+
+
+def launch_ranks(args):
+    """--gpus N.  Under a launcher, WORLD_SIZE must equal N (else exit 2).
+    Without one, N > 1 runs this same command under torch.distributed.run
+    with N ranks, one per GPU, on this node, and returns its exit code;
+    None means this process is the (only) rank and runs the arm itself."""
+    env_world = os.environ.get("WORLD_SIZE")
+    if args.gpus < 1:
+        raise SystemExit(2)
+    if env_world is not None:
+        if int(env_world) != args.gpus:
+            print(f"bench.py: --gpus {args.gpus} disagrees with WORLD_SIZE={env_world}", file=sys.stderr)
+            raise SystemExit(2)
+        return None
+    if args.gpus == 1:
+        return None
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", sys.argv[0], *sys.argv[1:]]
+    return subprocess.call(cmd)
 
 
 def whole_job_value(world: int, qh_per_step: int, steps: int, max_total_ms: float) -> float:
@@ -461,10 +506,45 @@ def reset_state(st):
         st["seq"].copy_(st["seq_pre"])
 
 
+@dataclass
+class RankRecord:
+    """What one rank measured; report() reduces it over ranks.  Times in ms."""
+    w0: ki.Workload                # the workload as named (every rank's shard has its shape)
+    w: ki.Workload                 # this rank's shard
+    k: int
+    lens_final: np.ndarray
+    per_step: list                 # device time of every timed step
+    parts: list                    # [(name, algorithmic bytes per launch, source file)]
+    part_ms: dict                  # name -> per-launch times
+    upd_ms: list                   # the append update, per call (workloads with an append)
+    e2e_ms: list                   # every e2e step (copies included)
+    e2e: dict                      # how the e2e leg ran: mode, h2d/d2h bytes per step
+    clocks: dict
+    wall: float                    # host seconds around the timed loop
+    status: int
+    launches_per_step: int
+    kv_layout: str
+    token_kt: int = 0
+
+
 def gpu_arm(args):
-    import torch
     import torch.distributed as dist
     rank, world, local = setup_dist(args)
+    try:
+        rec = measure_rank(args, rank, world, local)
+        report(args, rank, world, rec)
+    finally:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+def measure_rank(args, rank, world, local) -> RankRecord:
+    """Builds this rank's decode state on its GPU and times the step; the
+    ranks meet only at the barriers around the timed regions."""
+    import torch
+    import torch.distributed as dist
+    import block_top_sparse_kin_b200 as kin
     w0 = ki.WORKLOADS[args.workload]
     if args.batch:
         w0 = w0.with_(B=args.batch, name=f"{w0.name}_b{args.batch}")
@@ -475,11 +555,11 @@ def gpu_arm(args):
     if args.token_topk:
         if args.paged or args.shared_prefix > 1:
             raise SystemExit("--token-topk reads the contiguous cache")
-        import block_top_sparse_kin_b200 as kin_mod
         st["token_kt"] = k * w.bs  # the block budget in tokens, per query head
-        st["token_ws"] = kin_mod.alloc_token_workspace(st["dims"], st["token_kt"])
+        st["token_ws"] = kin.alloc_token_workspace(st["dims"], st["token_kt"])
     flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    flush_sink = torch.zeros((), dtype=torch.float32, device="cuda")
 
     def flush_l2(i):
         """Write a buffer larger than L2, then read another one, so a timed
@@ -487,7 +567,10 @@ def gpu_arm(args):
         flush_w.fill_(i & 0xFF)
         flush_sink.copy_(flush_r.sum())
 
-    flush_sink = torch.zeros((), dtype=torch.float32, device="cuda")
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
     # block path: scan + top-k, then attention; token path: logits, top-k,
     # attention; plus the append update
     launches_per_step = 4 if w.n_append else 3
@@ -508,8 +591,6 @@ def gpu_arm(args):
     # host synchronize, also outside the events) before the next replay.
     def ext_events(n):
         return [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n)]
-
-    import block_top_sparse_kin_b200 as kin
 
     # the step's kernel families: (name, call, algorithmic bytes, source file)
     means_bytes = 2 if args.means_bf16 else 4
@@ -568,8 +649,7 @@ def gpu_arm(args):
             flush_l2(0)
             g.replay()
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    barrier()
     torch.cuda.synchronize()
     per_step = []
     with ClockSampler(local) as clk:
@@ -581,122 +661,198 @@ def gpu_arm(args):
             per_step.append(step_ev[0].elapsed_time(step_ev[1]))
             clk.poll()                     # the clock right after each step (outside the events)
         wall = time.perf_counter() - wall0
-    if world > 1:
-        dist.barrier()
-    part_ms = [[] for _ in parts]
+    barrier()
+    part_ms = {name: [] for name, _, _, _ in parts}
     upd_ms = []
     for s in range(args.steps):            # per-kernel timing pass (not in `value`)
-        for g, ev, out, reps in list(zip(part_graphs, part_ev, part_ms, [KERNEL_REPEATS] * len(parts))) + \
-                [(upd_graph, upd_ev, upd_ms, 1)]:
-            if g is None:
-                continue
+        for (name, _, _, _), g, ev in zip(parts, part_graphs, part_ev):
             flush_l2(s)
             g.replay()
             torch.cuda.synchronize()
-            out.append(ev[0].elapsed_time(ev[1]) / reps)
+            part_ms[name].append(ev[0].elapsed_time(ev[1]) / KERNEL_REPEATS)
+        if upd_graph is not None:
+            flush_l2(s)
+            upd_graph.replay()
+            torch.cuda.synchronize()
+            upd_ms.append(upd_ev[0].elapsed_time(upd_ev[1]))
     reset_state(st)
     run_step(st)                           # leave the state as one step leaves it
     torch.cuda.synchronize()
-    total_ms = reduce_max(sum(per_step), "cuda")
-    ms_per_step = total_ms / args.steps
-    qh_per_step = w.B * w.Hq
-    value = whole_job_value(world, qh_per_step, args.steps, total_ms)
+    del graph, part_graphs, upd_graph, diag
 
-    # ---- e2e: the same step through the public API with host buffers:
-    # pinned q -> device, step, device out -> pinned host, all on one stream.
-    q_pin = torch.from_numpy(st["q_host"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    e2e_ms, e2e = e2e_leg(args, st, flush_l2, barrier)
+    return RankRecord(
+        w0=w0, w=w, k=k, lens_final=st["lens_final"], per_step=per_step,
+        parts=[(name, nbytes, src) for name, _, nbytes, src in parts], part_ms=part_ms, upd_ms=upd_ms,
+        e2e_ms=e2e_ms, e2e=e2e, clocks=clk.summary(), wall=wall, status=int(st["status"].item()),
+        launches_per_step=launches_per_step, token_kt=st.get("token_kt", 0),
+        kv_layout=(f"paged: {st['num_pages']} pages of one {w.bs}-token block, {args.page_order} pool"
+                   f" + block table"
+                   + (f"; groups of {args.shared_prefix} samples share their prompt's pages and"
+                      f" per-page means" if args.shared_prefix > 1 else "")
+                   if "table" in st else "contiguous [B][Hkv][Lcap][D]"))
+
+
+def e2e_leg(args, st, flush_l2, barrier):
+    """The step as a decode loop runs it from host buffers: the step's inputs
+    (q, and the appended K/V rows where the workload appends) copied from
+    pinned host memory, the step's kernels, and the output copied back to
+    pinned host memory, all captured once in one CUDA graph and replayed.
+    Each step is timed by CUDA events recorded on the stream around the
+    replay (so the graph's launch edge on the device is inside), L2 flushed
+    before.  Returns the per-step times and what was copied."""
+    import torch
+    w = st["w"]
+    h2d = [(st["q"], torch.from_numpy(st["q_host"].view(np.int16)).view(torch.bfloat16).pin_memory())]
+    if w.n_append:
+        for name in ("k_new", "v_new"):
+            h2d.append((st[name], st[name].cpu().pin_memory()))
     out_pin = torch.empty(st["out"].shape, dtype=torch.bfloat16).pin_memory()
-    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    for _ in range(args.warmup):
-        reset_state(st)
-        st["q"].copy_(q_pin, non_blocking=True)
-        run_step(st)
-        out_pin.copy_(st["out"], non_blocking=True)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    for s in range(args.steps):
-        reset_state(st)
-        flush_l2(s)
-        e2e_ev[s][0].record()
-        st["q"].copy_(q_pin, non_blocking=True)
-        run_step(st)
-        out_pin.copy_(st["out"], non_blocking=True)
-        e2e_ev[s][1].record()
-    torch.cuda.synchronize()
-    e2e_ms = reduce_max(sum(a.elapsed_time(b) for a, b in e2e_ev), "cuda")
-    e2e_value = whole_job_value(world, qh_per_step, args.steps, e2e_ms)
-    status = int(st["status"].item())
 
-    if rank == 0:
-        peak, peak_kind = measured_peak()
-        avg = {name: statistics.mean(ms) for (name, _, _, _), ms in zip(parts, part_ms)}
-        gbs = {name: nbytes / (avg[name] * 1e-3) / 1e9 for name, _, nbytes, _ in parts}
-        step_gbs = sum(nbytes for _, _, nbytes, _ in parts) / (ms_per_step * 1e-3) / 1e9
-        dominant, _, dom_bytes, dom_file = max(parts, key=lambda pt: avg[pt[0]])
-        dom_gbs = gbs[dominant]
-        line = {
-            "metric": METRIC,
-            "value": value,
-            "unit": "query-heads/s",
-            "n_gpus": world,
-            "steps": args.steps,
-            "warmup": args.warmup,
-            "ms_per_step": ms_per_step,
-            "higher_is_better": True,
-            "scaling": "weak",
-            "vs_baseline": None,
-            "dtype": "bf16",
-            "data": "synthetic (seeded Philox N(0,1) q/K/V, 5% heavy-hitter key-bias blocks)",
-            "config": {
-                "workload": w0.name, "batch": w0.B, "kv_heads": w0.Hkv, "q_heads": w0.Hq,
-                "head_dim": w0.D, "context": [w0.Lmin, w0.Lmax], "block_size": w0.bs,
-                "top_k_blocks": k, "append_tokens": w0.n_append,
-                "global_batch": w0.B * world, "parallelism": f"dp{world}",
-                "l2": "flushed before every step (256 MiB write + 256 MiB read, outside the timed events)",
-                "kv_layout": (f"paged: {st['num_pages']} pages of one {w.bs}-token block, {args.page_order} pool"
-                              f" + block table"
-                              + (f"; groups of {args.shared_prefix} samples share their prompt's pages and"
-                                 f" per-page means" if args.shared_prefix > 1 else "")
-                              if "table" in st else "contiguous [B][Hkv][Lcap][D]"),
-                "block_means": "bf16" if args.means_bf16 else "fp32",
-                **({"attention": f"token-level top-k, {st['token_kt']} tokens per query head"} if args.token_topk else {}),
-            },
-            "impl": "kin",
-            "gpu_launches": launches_per_step * args.steps,  # in the timed region
-            "kernel_ms": {**avg, **({"update": statistics.mean(upd_ms)} if upd_ms else {})},
-            "hbm_gbs": {**gbs, "step": step_gbs},
-            "hbm_frac": {**{n: v / peak for n, v in gbs.items()}, "step": step_gbs / peak,
-                         "peak_gbs": peak, "peak_kind": peak_kind},
-            "roofline": {
-                "kernel": dominant, "bound": "hbm", "achieved": dom_gbs, "peak": peak, "unit": "GB/s",
-                "frac": dom_gbs / peak, "peak_kind": peak_kind,
-                "algorithmic_bytes_per_launch": dom_bytes,
-                "traffic": profiled_traffic(dom_file, w0.name, k),
-            },
-            "e2e": {"value": e2e_value, "unit": "query-heads/s",
-                    "h2d_bytes_per_step": int(q_pin.numel() * 2), "d2h_bytes_per_step": int(out_pin.numel() * 2)},
-            "eflops": eflops_report(w, k, st["lens_final"], ms_per_step, means_bytes,
-                                    st.get("token_kt", 0)),
-            "clocks": clk.summary(),
-            "wall_s_timed_region": wall,
-            "device_status": status,
-        }
-        if world == 1 and not args.no_cpu_baseline and not args.token_topk:
-            line["cpu_baseline"] = cpu_baseline(w0, k, budget_s=args.cpu_seconds)
-        print(json.dumps(line), flush=True)
+    def body():
+        reset_state(st)
+        for dev, host in h2d:
+            dev.copy_(host, non_blocking=True)
+        run_step(st)
+        out_pin.copy_(st["out"], non_blocking=True)
+
+    for _ in range(args.warmup):
+        body()
+    torch.cuda.synchronize()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cap):
+            body()
+    torch.cuda.current_stream().wait_stream(cap)
+    for _ in range(args.warmup):
+        flush_l2(0)
+        graph.replay()
+    torch.cuda.synchronize()
+    barrier()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    stream = torch.cuda.current_stream()
+    for s in range(args.steps):
+        flush_l2(s)
+        ev[s][0].record(stream)
+        graph.replay()
+        ev[s][1].record(stream)
+    torch.cuda.synchronize()
+    times = [a.elapsed_time(b) for a, b in ev]
+    # the copies really carried this step's data: the host copy of out is the device's
+    if not torch.equal(out_pin.view(torch.int16), st["out"].cpu().view(torch.int16)):
+        raise RuntimeError("e2e: the output copied to the host differs from the device output")
+    del graph
+    return times, {"mode": "graph replay: h2d copies + step + d2h copy",
+                   "h2d_bytes_per_step": int(sum(host.numel() * host.element_size() for _, host in h2d)),
+                   "d2h_bytes_per_step": int(out_pin.numel() * out_pin.element_size())}
+
+
+L2_NOTE = ("GPU arm: L2 flushed before every step (256 MiB write + 256 MiB read, outside the timed events); "
+           "oracle arm: host cores")
+
+
+def workload_config(w0: ki.Workload, k: int, world: int, kv_layout: str = "contiguous [B][Hkv][Lcap][D]",
+                    means_bf16: bool = False, token_kt: int = 0) -> dict:
+    """The JSON line's config: the workload as named, the same in both arms."""
+    return {
+        "workload": w0.name, "batch": w0.B, "kv_heads": w0.Hkv, "q_heads": w0.Hq,
+        "head_dim": w0.D, "context": [w0.Lmin, w0.Lmax], "block_size": w0.bs,
+        "top_k_blocks": k, "append_tokens": w0.n_append,
+        "global_batch": w0.B * world, "parallelism": f"dp{world}",
+        "l2": L2_NOTE,
+        "kv_layout": kv_layout,
+        "block_means": "bf16" if means_bf16 else "fp32",
+        **({"attention": f"token-level top-k, {token_kt} tokens per query head"} if token_kt else {}),
+    }
+
+
+def report(args, rank, world, rec: RankRecord):
+    """Reduces the ranks' records (max over ranks) and prints the JSON line
+    on rank 0."""
+    import torch.distributed as dist
+    names = [name for name, _, _ in rec.parts]
+    means = [statistics.mean(rec.part_ms[n]) for n in names]
+    upd = statistics.mean(rec.upd_ms) if rec.upd_ms else 0.0
+    red = reduce_max_list([sum(rec.per_step), sum(rec.e2e_ms), rec.wall, upd, *means])
+    total_ms, e2e_total, wall, upd = red[:4]
+    avg = dict(zip(names, red[4:]))
+    clocks_all = [rec.clocks]
     if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+        clocks_all = [None] * world
+        dist.all_gather_object(clocks_all, rec.clocks)
+        status = reduce_max(float(rec.status))
+    else:
+        status = rec.status
+    if rank != 0:
+        return
+    w0, w, k = rec.w0, rec.w, rec.k
+    steps = len(rec.per_step)
+    ms_per_step = total_ms / steps
+    qh_per_step = w.B * w.Hq
+    value = whole_job_value(world, qh_per_step, steps, total_ms)
+    e2e_value = whole_job_value(world, qh_per_step, len(rec.e2e_ms), e2e_total)
+    peak, peak_kind = measured_peak()
+    gbs = {name: nbytes / (avg[name] * 1e-3) / 1e9 for name, nbytes, _ in rec.parts}
+    step_gbs = sum(nbytes for _, nbytes, _ in rec.parts) / (ms_per_step * 1e-3) / 1e9
+    dominant, dom_bytes, dom_file = max(rec.parts, key=lambda pt: avg[pt[0]])
+    dom_gbs = gbs[dominant]
+    clocks = dict(rec.clocks)
+    if world > 1:
+        clocks["per_rank"] = clocks_all
+        clocks["reasons"] = sorted(set(r for c in clocks_all for r in (c or {}).get("reasons", [])))
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "query-heads/s",
+        "n_gpus": world,
+        "steps": steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded Philox N(0,1) q/K/V, 5% heavy-hitter key-bias blocks)",
+        "config": workload_config(w0, k, world, rec.kv_layout, args.means_bf16, rec.token_kt),
+        "impl": "kin",
+        "gpu_launches": rec.launches_per_step * steps,  # in the timed region
+        "kernel_ms": {**avg, **({"update": upd} if rec.upd_ms else {})},
+        "hbm_gbs": {**gbs, "step": step_gbs},
+        "hbm_frac": {**{n: v / peak for n, v in gbs.items()}, "step": step_gbs / peak,
+                     "peak_gbs": peak, "peak_kind": peak_kind},
+        "roofline": {
+            "kernel": dominant, "bound": "hbm", "achieved": dom_gbs, "peak": peak, "unit": "GB/s",
+            "frac": dom_gbs / peak, "peak_kind": peak_kind,
+            "algorithmic_bytes_per_launch": dom_bytes,
+            "traffic": profiled_traffic(dom_file, w0.name, k),
+        },
+        "e2e": {"value": e2e_value, "unit": "query-heads/s", **rec.e2e},
+        "eflops": eflops_report(w, k, rec.lens_final, ms_per_step, 2 if args.means_bf16 else 4, rec.token_kt),
+        "clocks": clocks,
+        "wall_s_timed_region": wall,
+        "device_status": int(status),
+    }
+    if world == 1 and not args.no_cpu_baseline and not rec.token_kt:
+        line["cpu_baseline"] = cpu_baseline(w0, k, budget_s=args.cpu_seconds)
+    print(json.dumps(line), flush=True)
 
 
 # ---------------------------------------------------------- oracle (CPU) arm
+def sample_pairs_default() -> int:
+    """Pairs in the oracle's timing sample: two per host thread, at least 32,
+    so every thread stays busy through a pass."""
+    return max(32, 2 * (os.cpu_count() or 1))
+
+
 class OracleSample:
     """A bounded sample of (batch, kv-head) pairs of a workload, prepared on
     the host for the fp64 oracle: K/V rows regenerated from the seeded
     generator and block means precomputed (resident state, as on the GPU)."""
 
     def __init__(self, w: ki.Workload, k: int, max_pairs: int):
+        from concurrent.futures import ThreadPoolExecutor
         import oracle
         self.oracle = oracle
         self.w, self.k = w, k
@@ -713,14 +869,18 @@ class OracleSample:
         self.means = np.zeros((self.n, 1, nbcap, w.D))
         self.qs = np.zeros((self.n, w.g, w.D), np.uint16)
         self.lens = np.zeros(self.n, np.int32)
-        for i, p in enumerate(pairs):
-            b, h = divmod(p, w.Hkv)
+        self.threads = os.cpu_count() or 1
+
+        def fill(i):  # the generator and the oracle are C calls that release the GIL
+            b, h = divmod(pairs[i], w.Hkv)
             L = int(lens_final[b])
             self.Kc[i, 0, :L], self.Vc[i, 0, :L] = ki.pair_rows(w, hh, b, h, L)
             self.means[i, 0, :-(-L // w.bs)] = oracle.block_means(self.Kc[i, 0], L, w.bs)
             self.qs[i] = q_all[b, h * w.g:(h + 1) * w.g]
             self.lens[i] = L
-        self.threads = os.cpu_count() or 1
+
+        with ThreadPoolExecutor(self.threads) as ex:
+            list(ex.map(fill, range(self.n)))
 
     def run_pass(self):
         w = self.w
@@ -731,13 +891,14 @@ class OracleSample:
 
     def describe(self, passes, seconds):
         return (f"{self.n} of {self.P} (batch, kv-head) pairs of {self.w.name} (k={self.k}), {passes} "
-                f"passes in {seconds:.3f} s; scores + top-k + attention in fp64, block means precomputed")
+                f"passes in {seconds:.3f} s on {self.threads} threads; scores + top-k + attention in fp64, "
+                f"block means precomputed")
 
 
-def cpu_baseline(w: ki.Workload, k: int, budget_s: float = 12.0, max_pairs: int = 32):
+def cpu_baseline(w: ki.Workload, k: int, budget_s: float = 12.0, max_pairs: int = 0):
     """The oracle (as it stands) on the host cores: whole passes over the
     sample until `budget_s` has elapsed; query-heads/s."""
-    smp = OracleSample(w, k, max_pairs)
+    smp = OracleSample(w, k, max_pairs or sample_pairs_default())
     t0 = time.perf_counter()
     passes, qh = 0, 0
     while True:
@@ -752,14 +913,16 @@ def cpu_baseline(w: ki.Workload, k: int, budget_s: float = 12.0, max_pairs: int 
 
 def reference_arm(args):
     """The oracle as the reference arm: each step is one pass over a bounded
-    sample of the workload's pairs, timed on the host clock."""
+    sample of the workload's pairs (the CPU baseline's sample by default),
+    timed on the host clock.  ms_per_step is the time of that sampled pass,
+    not of the whole batch; value (query-heads/s) is the sample's rate."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     w = ki.WORKLOADS[args.workload]
     k = args.k or w.k
     t0 = time.perf_counter()
-    smp = OracleSample(w, k, max_pairs=args.ref_pairs)
+    smp = OracleSample(w, k, max_pairs=args.ref_pairs or sample_pairs_default())
     for _ in range(args.warmup):
         smp.run_pass()
     el, qh = 0.0, 0
@@ -771,10 +934,10 @@ def reference_arm(args):
     line = {
         "metric": METRIC, "value": value, "unit": "query-heads/s",
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": w.B * w.Hq / value * 1e3, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "batch": w.B, "kv_heads": w.Hkv, "q_heads": w.Hq, "head_dim": w.D,
-                   "context": [w.Lmin, w.Lmax], "block_size": w.bs, "top_k_blocks": k},
+        "config": workload_config(w, k, int(os.environ.get("WORLD_SIZE", "1"))),
+        "step": f"one pass over {smp.n} sampled (batch, kv-head) pairs ({smp.n * w.g} query heads)",
         "impl": "reference",
         "cpu_baseline": {"value": value, "unit": "query-heads/s", "cores": smp.threads, "kind": "oracle",
                          "sample": smp.describe(args.steps, el)},
@@ -784,7 +947,7 @@ def reference_arm(args):
     print(json.dumps(line), flush=True)
 
 
-def main():
+def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
@@ -795,7 +958,8 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ref-pairs", type=int, default=8, help="pairs per reference-arm step")
+    ap.add_argument("--ref-pairs", type=int, default=0,
+                    help="(batch, kv-head) pairs per reference-arm step (default: the CPU baseline's sample)")
     ap.add_argument("--paged", action="store_true", help="KV cache in a shuffled page pool with a block table")
     ap.add_argument("--means-bf16", action="store_true", help="bf16 block means (the extended calls)")
     ap.add_argument("--page-order", default="shuffled", choices=["shuffled", "sequential"],
@@ -804,14 +968,18 @@ def main():
                     help="groups of N samples share a prompt (paged, block means per page)")
     ap.add_argument("--token-topk", action="store_true",
                     help="token-level top-k attention instead of the block path (budget = k blocks x bs tokens)")
-    args = ap.parse_args()
+    args = ap.parse_args(argv)
+    rc = launch_ranks(args)
+    if rc is not None:  # this process launched the ranks
+        return rc
     if args.warmup < 3 and args.impl == "kin":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         reference_arm(args)
     else:
         gpu_arm(args)
+    return 0
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main())

@@ -1,6 +1,7 @@
 """The benchmark's reference arm on the CPU: it times the oracle as it stands
-on the host cores and prints one JSON line with the contract's keys; under a
-multi-rank launch only rank 0 works and prints."""
+on the host cores and prints one JSON line with the contract's keys; its
+step is one pass over the sampled pairs, whose time fits inside the run;
+under a multi-rank launch only rank 0 works and prints."""
 import json
 import os
 import subprocess
@@ -9,10 +10,10 @@ import sys
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _run(env_extra):
+def _run(env_extra, *extra):
     env = dict(os.environ, **env_extra)
     cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1", "--warmup", "1",
-           "--ref-pairs", "2"]
+           "--ref-pairs", "2", *extra]
     return subprocess.run(cmd, capture_output=True, text=True, timeout=600, env=env, check=True).stdout
 
 
@@ -30,9 +31,20 @@ def test_reference_arm_prints_the_contract_line():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and "2 of 256" in cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "query-heads/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
-    # the metric's time per full step follows from the rate
-    assert abs(d["ms_per_step"] - 32 * 32 / d["value"] * 1e3) < 1e-6 * d["ms_per_step"]
+    # a step is one pass over the sampled pairs (2 pairs x 4 query heads), and
+    # its time follows from the rate; the claimed time fits inside the run
+    assert "2 sampled" in d["step"]
+    import bench
+    assert d["config"] == bench.workload_config(bench.ki.WORKLOADS["qwen3_8b_32k"], 256, 1)
+    assert abs(d["ms_per_step"] - 2 * 4 / d["value"] * 1e3) < 1e-6 * d["ms_per_step"]
+    assert d["steps"] * d["ms_per_step"] / 1e3 <= d["wall_s"]
 
 
 def test_reference_arm_is_silent_on_other_ranks():
-    assert _run({"RANK": "1", "WORLD_SIZE": "2"}).strip() == ""
+    assert _run({"RANK": "1", "WORLD_SIZE": "2"}, "--gpus", "2").strip() == ""
+
+
+def test_default_sample_keeps_every_host_thread_busy():
+    import bench
+    assert bench.sample_pairs_default() >= 2 * (os.cpu_count() or 1)
+    assert bench.sample_pairs_default() >= 32
