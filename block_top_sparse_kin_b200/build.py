@@ -20,7 +20,7 @@ def nvcc_command(out: str = LIB, ptxas_verbose: bool = False, defines=()) -> lis
     if ptxas_verbose:
         cmd += ["-Xptxas", "-v"]
     cmd += [f"-D{d}" for d in defines]
-    cmd += [os.path.join(CSRC, s) for s in SOURCES] + ["-o", out]
+    cmd += [os.path.join(CSRC, s) for s in SOURCES] + ["-o", out, "-ldl"]
     return cmd
 
 

@@ -15,21 +15,6 @@ constexpr int kTargetSMs = 148;  // B200 SM count, used only to shape grids
 constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-kin_status check_dims(const kin_dims* d) {
-  if (!d) return KIN_ERR_INVALID_ARG;
-  if (d->batch < 1 || d->num_kv_heads < 1 || d->num_q_heads < 1 || d->max_seq_len < 1)
-    return KIN_ERR_INVALID_ARG;
-  if (d->num_q_heads % d->num_kv_heads != 0) return KIN_ERR_INVALID_ARG;
-  if (d->head_dim != kHeadDim) return KIN_ERR_INVALID_ARG;
-  const int bs = d->block_size;
-  if (bs != 16 && bs != 32 && bs != 64 && bs != 128) return KIN_ERR_INVALID_ARG;
-  if (d->num_q_heads / d->num_kv_heads > kMaxGroup) return KIN_ERR_CAPACITY;
-  if ((d->max_seq_len + bs - 1) / bs > kMaxBlocksPerSeq) return KIN_ERR_CAPACITY;
-  if ((int64_t)d->batch * d->num_kv_heads * d->max_seq_len >= (int64_t)1 << 31) return KIN_ERR_CAPACITY;
-  return KIN_OK;
-}
 
 int nbcap_of(const kin_dims& d) { return (d.max_seq_len + d.block_size - 1) / d.block_size; }
 int pairs_of(const kin_dims& d) { return d.batch * d.num_kv_heads; }
@@ -106,6 +91,22 @@ kin_status check_pages(const kin_dims& d, const void* pool, int32_t num_pages, c
 }  // namespace
 
 namespace kin {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+kin_status check_dims(const kin_dims* d) {
+  if (!d) return KIN_ERR_INVALID_ARG;
+  if (d->batch < 1 || d->num_kv_heads < 1 || d->num_q_heads < 1 || d->max_seq_len < 1)
+    return KIN_ERR_INVALID_ARG;
+  if (d->num_q_heads % d->num_kv_heads != 0) return KIN_ERR_INVALID_ARG;
+  if (d->head_dim != kHeadDim) return KIN_ERR_INVALID_ARG;
+  const int bs = d->block_size;
+  if (bs != 16 && bs != 32 && bs != 64 && bs != 128) return KIN_ERR_INVALID_ARG;
+  if (d->num_q_heads / d->num_kv_heads > kMaxGroup) return KIN_ERR_CAPACITY;
+  if ((d->max_seq_len + bs - 1) / bs > kMaxBlocksPerSeq) return KIN_ERR_CAPACITY;
+  if ((int64_t)d->batch * d->num_kv_heads * d->max_seq_len >= (int64_t)1 << 31) return KIN_ERR_CAPACITY;
+  return KIN_OK;
+}
 
 constexpr int kMaxDevices = 64;
 
@@ -220,6 +221,7 @@ kin_status check_update_args(const void* k_rows, const void* v_rows, const void*
 KIN_EXPORT kin_status kin_block_means_build(const kin_dims* dims, const void* k_cache,
                                             const int32_t* seq_lens, float* block_means,
                                             int32_t* dev_status, void* stream) {
+  KIN_NVTX_RANGE();
   kin_status st = check_dims(dims);
   if (st != KIN_OK) return st;
   if (!k_cache || !seq_lens || !block_means) return KIN_ERR_INVALID_ARG;
@@ -230,6 +232,7 @@ KIN_EXPORT kin_status kin_block_means_build(const kin_dims* dims, const void* k_
 KIN_EXPORT kin_status kin_block_means_build_paged(const kin_dims* dims, const void* k_pages, int32_t num_pages,
                                                   const int32_t* block_table, const int32_t* seq_lens,
                                                   float* block_means, int32_t* dev_status, void* stream) {
+  KIN_NVTX_RANGE();
   kin_status st = check_dims(dims);
   if (st != KIN_OK) return st;
   PageTable pt;
@@ -243,6 +246,7 @@ KIN_EXPORT kin_status kin_block_means_update(const kin_dims* dims, void* k_cache
                                              float* block_means, int32_t* seq_lens,
                                              const void* k_new, const void* v_new, int32_t n_new,
                                              int32_t* dev_status, void* stream) {
+  KIN_NVTX_RANGE();
   kin_status st = check_dims(dims);
   if (st != KIN_OK) return st;
   st = check_update_count(dims, n_new);
@@ -258,6 +262,7 @@ KIN_EXPORT kin_status kin_block_means_update_paged(const kin_dims* dims, void* k
                                                    float* block_means, int32_t* seq_lens, const void* k_new,
                                                    const void* v_new, int32_t n_new, int32_t* dev_status,
                                                    void* stream) {
+  KIN_NVTX_RANGE();
   kin_status st = check_dims(dims);
   if (st != KIN_OK) return st;
   st = check_update_count(dims, n_new);
@@ -329,6 +334,7 @@ KIN_EXPORT kin_status kin_block_topk_select(const kin_dims* dims, const void* q,
                                             const int32_t* seq_lens, int32_t k_blocks, int32_t* sel_idx,
                                             int32_t* sel_cnt, void* workspace, size_t ws_bytes,
                                             int32_t* dev_status, void* stream) {
+  KIN_NVTX_RANGE();
   kin_status st = check_dims(dims);
   if (st != KIN_OK) return st;
   return topk_select(dims, q, block_means, 0, seq_lens, k_blocks, sel_idx, sel_cnt, workspace, ws_bytes,
@@ -339,6 +345,7 @@ KIN_EXPORT kin_status kin_block_topk_select_ex(const kin_dims* dims, const void*
                                                int32_t means_dtype, const int32_t* seq_lens, int32_t k_blocks,
                                                int32_t* sel_idx, int32_t* sel_cnt, void* workspace,
                                                size_t ws_bytes, int32_t* dev_status, void* stream) {
+  KIN_NVTX_RANGE();
   kin_status st = check_dims(dims);
   if (st != KIN_OK) return st;
   const int bf = means_flag(means_dtype);
@@ -353,6 +360,7 @@ KIN_EXPORT kin_status kin_block_topk_select_paged(const kin_dims* dims, const vo
                                                   int32_t k_blocks, int32_t* sel_idx, int32_t* sel_cnt,
                                                   void* workspace, size_t ws_bytes, int32_t* dev_status,
                                                   void* stream) {
+  KIN_NVTX_RANGE();
   kin_status st = check_dims(dims);
   if (st != KIN_OK) return st;
   const int bf = means_flag(means_dtype);
@@ -368,6 +376,7 @@ KIN_EXPORT kin_status kin_block_means_build_ex(const kin_dims* dims, const void*
                                                const int32_t* block_table, const int32_t* seq_lens,
                                                void* block_means, int32_t means_dtype, int32_t* dev_status,
                                                void* stream) {
+  KIN_NVTX_RANGE();
   kin_status st = check_dims(dims);
   if (st != KIN_OK) return st;
   const int bf = means_flag(means_dtype);
@@ -387,6 +396,7 @@ KIN_EXPORT kin_status kin_block_means_update_ex(const kin_dims* dims, void* k_ro
                                                 void* block_means, int32_t means_dtype, int32_t* seq_lens,
                                                 const void* k_new, const void* v_new, int32_t n_new,
                                                 int32_t* dev_status, void* stream) {
+  KIN_NVTX_RANGE();
   kin_status st = check_dims(dims);
   if (st != KIN_OK) return st;
   const int bf = means_flag(means_dtype);
@@ -454,6 +464,7 @@ KIN_EXPORT kin_status kin_sparse_decode_attn(const kin_dims* dims, const void* q
                                              int32_t k_blocks, float softmax_scale, void* out, float* lse,
                                              void* workspace, size_t ws_bytes, int32_t* dev_status,
                                              void* stream) {
+  KIN_NVTX_RANGE();
   kin_status st = check_dims(dims);
   if (st != KIN_OK) return st;
   return sparse_decode_attn(dims, q, k_cache, v_cache, contiguous(), seq_lens, sel_idx, sel_cnt, k_blocks,
@@ -467,6 +478,7 @@ KIN_EXPORT kin_status kin_sparse_decode_attn_paged(const kin_dims* dims, const v
                                                    int32_t k_blocks, float softmax_scale, void* out,
                                                    float* lse, void* workspace, size_t ws_bytes,
                                                    int32_t* dev_status, void* stream) {
+  KIN_NVTX_RANGE();
   kin_status st = check_dims(dims);
   if (st != KIN_OK) return st;
   PageTable pt;
@@ -513,6 +525,7 @@ KIN_EXPORT kin_status kin_token_topk_decode_attn(const kin_dims* dims, const voi
                                                  float softmax_scale, void* out, float* lse, int32_t* sel_tokens,
                                                  void* workspace, size_t ws_bytes, int32_t* dev_status,
                                                  void* stream) {
+  KIN_NVTX_RANGE();
   kin_status st = check_dims(dims);
   if (st != KIN_OK) return st;
   if (k_tokens < 1) return KIN_ERR_INVALID_ARG;

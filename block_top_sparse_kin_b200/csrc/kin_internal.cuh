@@ -8,7 +8,35 @@
 
 #include "../../include/kin.h"
 
+// NVTX ranges around every launching kin_* call (header-only NVTX3; a no-op
+// unless a profiler is attached).  -DKIN_NVTX=0 compiles them out.
+#ifndef KIN_NVTX
+#define KIN_NVTX 1
+#endif
+#if KIN_NVTX
+#include <nvtx3/nvToolsExt.h>
+#endif
+
 namespace kin {
+
+// Scoped NVTX range named after the entry point (host code).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) {
+#if KIN_NVTX
+    nvtxRangePushA(name);
+#else
+    (void)name;
+#endif
+  }
+  ~NvtxRange() {
+#if KIN_NVTX
+    nvtxRangePop();
+#endif
+  }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define KIN_NVTX_RANGE() ::kin::NvtxRange kin_nvtx_range_(__func__)
 
 constexpr int kHeadDim = 128;
 constexpr int kMaxGroup = 8;
@@ -244,6 +272,11 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
+
+// Host-side argument checks shared by every entry point: the problem
+// dimensions every kernel supports, and 16-byte alignment of a pointer.
+kin_status check_dims(const kin_dims* d);
+bool aligned16(const void* p);
 
 // Per-device facts the launchers need, cached after the first query (a
 // device's SM count never changes; racing first calls store the same value).

@@ -46,20 +46,6 @@ float* scratch_on_current_device(cudaError_t* err) {
   return static_cast<float*>(ptr);
 }
 
-kin_status check_dims_noalloc(const kin_dims* d) {
-  if (!d) return KIN_ERR_INVALID_ARG;
-  if (d->batch < 1 || d->num_kv_heads < 1 || d->num_q_heads < 1 || d->max_seq_len < 1)
-    return KIN_ERR_INVALID_ARG;
-  if (d->num_q_heads % d->num_kv_heads != 0) return KIN_ERR_INVALID_ARG;
-  if (d->head_dim != kHeadDim) return KIN_ERR_INVALID_ARG;
-  const int bs = d->block_size;
-  if (bs != 16 && bs != 32 && bs != 64 && bs != 128) return KIN_ERR_INVALID_ARG;
-  if (d->num_q_heads / d->num_kv_heads > kMaxGroup) return KIN_ERR_CAPACITY;
-  if ((d->max_seq_len + bs - 1) / bs > kMaxBlocksPerSeq) return KIN_ERR_CAPACITY;
-  if ((int64_t)d->batch * d->num_kv_heads * d->max_seq_len >= (int64_t)1 << 31) return KIN_ERR_CAPACITY;
-  return KIN_OK;
-}
-
 }  // namespace
 
 KIN_EXPORT kin_status kin_block_topk_select_noalloc(const kin_dims* dims, const void* q,
@@ -67,12 +53,12 @@ KIN_EXPORT kin_status kin_block_topk_select_noalloc(const kin_dims* dims, const 
                                                     int32_t k_blocks, int32_t* sel_idx,
                                                     int32_t* sel_cnt, int32_t* dev_status,
                                                     void* stream) {
-  kin_status st = check_dims_noalloc(dims);
+  KIN_NVTX_RANGE();
+  kin_status st = check_dims(dims);
   if (st != KIN_OK) return st;
   if (k_blocks < 2) return KIN_ERR_INVALID_ARG;
   if (!q || !block_means || !seq_lens || !sel_idx || !sel_cnt) return KIN_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(q) & 15u) || (reinterpret_cast<uintptr_t>(block_means) & 15u))
-    return KIN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(block_means)) return KIN_ERR_INVALID_ARG;
   const int bs = dims->block_size;
   const int nbcap = (dims->max_seq_len + bs - 1) / bs;
   const int64_t need = (int64_t)dims->batch * dims->num_kv_heads * nbcap;  // one score per block

@@ -43,6 +43,10 @@
  *  - No C++ exception crosses this boundary; the library keeps no state
  *    between calls other than what the caller's buffers hold (except the
  *    scratch array of kin_block_topk_select_noalloc, described there).
+ *  - Every call that launches kernels opens an NVTX range named after the
+ *    call for its host-side duration (NVTX3, header-only: it costs nothing
+ *    measurable unless a profiler is attached; built with -DKIN_NVTX=0 the
+ *    ranges are compiled out).
  *  - Limits: head_dim == 128; Hq % Hkv == 0 with 1 <= Hq/Hkv <= 8;
  *    block_size in {16, 32, 64, 128}; ceil(Lcap / bs) <= 32768;
  *    B * Hkv * Lcap < 2^31.

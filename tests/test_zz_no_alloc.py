@@ -54,6 +54,27 @@ def test_noalloc_select_matches_workspace_select_on_consecutive_calls():
         assert np.array_equal(sel, ref[0])
 
 
+def test_noalloc_select_takes_no_device_memory():
+    """After a first call on the device (which looks up the scratch array),
+    further calls leave the device's free memory unchanged: the call itself
+    allocates nothing.  Outputs are allocated before the measurement."""
+    w = ki.Workload("noalloc_mem", 2, 2, 8, D, 16, 900, 2000, 12, 33, Lcap=2048)
+    dc = make_device_case(w)
+    kin.kin_block_means_build(dc.dims, dc.k_cache, dc.seq_lens, dc.means)
+    sel = torch.empty((w.B, w.Hkv, w.k), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((w.B, w.Hkv), dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kin.kin_block_topk_select_noalloc(dc.dims, dc.q, dc.means, dc.seq_lens, w.k, sel, cnt, st)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        kin.kin_block_topk_select_noalloc(dc.dims, dc.q, dc.means, dc.seq_lens, w.k, sel, cnt, st)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert int(st.item()) == 0
+    assert free1 == free0
+
+
 def test_noalloc_select_rejects_problems_beyond_its_scratch():
     # B * Hkv * ceil(Lcap / bs) = 64 * 8 * 8192 > 2^21 scores
     dims = kin.make_dims(64, 8, 32, D, 16, 8192 * 16)
