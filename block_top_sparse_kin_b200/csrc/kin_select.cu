@@ -26,7 +26,8 @@
 //     crowded boundary bin is ranked through its 256 sub-bins.
 // The top-k: the first block and the block holding the newest token are
 // always kept, ties go to the lower index, and the kept indices leave
-// ascending.
+// ascending.  A budget that covers every block the dims allow (k >= nbcap)
+// skips both: select_dense_kernel writes the selections directly.
 //
 // Variants served by the same code: bf16 block means (the scan templated on
 // the means type, 16 rows per warp step); block means stored per page of a
@@ -1260,11 +1261,39 @@ cudaError_t launch_topk(const SelectParams& p, cudaStream_t s) {
   return launch_pdl(select_topk_kernel<NT>, dim3(p.B * p.Hkv), dim3(NT), smem, s, p);
 }
 
+// The selection when the budget covers every block of every sequence the
+// dims allow (k >= nbcap): nothing to score.  Every block is kept (sel_cnt
+// nb), or sel_cnt 0 and a row of -1 for a length outside [1, Lcap]
+// (flagged), one thread per output entry.
+__global__ void __launch_bounds__(256) select_dense_kernel(SelectParams p) {
+  pdl_wait();
+  pdl_trigger_early();
+  const int64_t total = (int64_t)p.B * p.Hkv * p.k;
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t pair = idx / p.k;
+    const int j = (int)(idx - pair * p.k);
+    const int L = __ldg(p.seq_lens + pair / p.Hkv);
+    const bool bad = L < 1 || L > p.Lcap;
+    const int nb = bad ? 0 : (L + p.bs - 1) / p.bs;
+    p.sel_idx[idx] = j < nb ? j : -1;
+    if (j == 0) {
+      p.sel_cnt[pair] = nb;
+      if (bad) set_status(p.dev_status, KIN_ERR_DEVICE_DATA);
+    }
+  }
+}
+
 cudaError_t launch_select(const SelectParams& p, cudaStream_t s) {
+  const int64_t resident = (int64_t)device_sm_count() * KIN_SEL_CTAS_PER_SM;
+  if (p.k >= p.nbcap) {  // every sequence's blocks fit the budget
+    const int64_t want = ((int64_t)p.B * p.Hkv * p.k + 255) / 256;
+    const int grid = (int)(want < 4 * resident ? want : 4 * resident);
+    return launch_pdl(select_dense_kernel, dim3(grid), dim3(256), 0, s, p);
+  }
   const int64_t rows = (int64_t)p.B * p.Hkv * p.nbcap;
   const int u = p.means_bf16 ? 2 * kSelU : kSelU;
   const int64_t want = (rows + kSelWarps * u * 4 - 1) / (kSelWarps * u * 4);  // >= 4 steps per warp
-  const int64_t resident = (int64_t)device_sm_count() * KIN_SEL_CTAS_PER_SM;
   const int grid = (int)(want < resident ? (want > 0 ? want : 1) : resident);
   const dim3 gd(grid), bd(kSelThreads);
   cudaError_t e;

@@ -104,6 +104,27 @@ def test_bad_device_lengths_are_flagged_not_fatal():
     assert np.array_equal(gr.out[0], gr0.out[0])
 
 
+def test_budget_covering_every_block_with_a_bad_length():
+    """k >= ceil(Lcap / bs): the select writes every block of each sequence
+    without scoring (no sequence can hold more blocks than the budget); a
+    length outside [1, Lcap] gets sel_cnt 0, a row of -1 and the status;
+    the outputs of the good sequences equal dense attention (oracle)."""
+    w = W("dense_only", 3, 2, 4, D, 16, 0, 0, 8, 25, Lcap=100, lens=(100, 37, 1))
+    dc = make_device_case(w)
+    gr = gpu_step(dc, w.k)
+    assert gr.status == 0
+    for b in range(w.B):
+        nb = -(-int(dc.lens_final[b]) // w.bs)
+        for h in range(w.Hkv):
+            assert list(gr.sel[b, h]) == list(range(nb)) + [-1] * (w.k - nb)
+            check_pair(dc, gr, b, h, w.k)
+    dc.seq_lens.copy_(torch.tensor([100, 0, 1], dtype=torch.int32))
+    bad = gpu_step(dc, w.k, build_means=False)
+    assert bad.status == 5
+    assert np.all(bad.cnt[1] == 0) and np.all(bad.sel[1] == -1)
+    assert np.array_equal(bad.sel[[0, 2]], gr.sel[[0, 2]]) and np.array_equal(bad.out[0], gr.out[0])
+
+
 def test_bad_block_index_is_flagged_and_skipped():
     w = W("badidx", 1, 1, 4, D, 16, 0, 0, 4, 24, Lcap=256, lens=(200,))
     dc = make_device_case(w)
