@@ -361,6 +361,15 @@ __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kerne
     cp_async_commit();
     cp_async_wait<0>();
     __syncthreads();
+    // the staged records are dead in memory: drop their L2 lines without a
+    // write-back (only lines wholly inside this batch's records, so no other
+    // pair's records are touched; the next call rewrites them before reading)
+    {
+      const uintptr_t lo = reinterpret_cast<uintptr_t>(s4), hi = lo + (uintptr_t)n4 * 16u;
+      const uintptr_t first = (lo + 127u) & ~uintptr_t(127);
+      const int nlines = hi > first ? (int)((hi - first) >> 7) : 0;
+      for (int i = tid; i < nlines; i += kAttnThreads) discard_l2_line(reinterpret_cast<const void*>(first + 128u * i));
+    }
     if (tid < g) {  // head j: batch maximum, rescale of the running sums, chunk weights
       const int j = tid;
       float Mb = kNegInf;
