@@ -104,6 +104,19 @@ __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kerne
   const int g = p.g;
   pdl_wait();  // the selection comes from the select kernels
   pdl_trigger_early();
+  // Lane l's tile of this warp (tile warp + W l of the chunk): its block
+  // index is requested before the pair's length and count, whose round trip
+  // it would otherwise follow (a chunk holds at most chunk_blocks blocks,
+  // all inside the pair's row of k; entries past the count are checked below).
+  const int tpb = p.bs / kTileTokens;
+  int blk_spec = -1;
+  {
+    const int64_t pair0 = blockIdx.x / p.max_chunks;
+    const int c0 = (int)(blockIdx.x - pair0 * p.max_chunks);
+    const int t = warp + kAttnWarps * lane;
+    const int j = c0 * p.chunk_blocks + t / tpb;
+    if (t < p.chunk_blocks * tpb && j < p.k) blk_spec = __ldg(p.sel_idx + pair0 * p.k + j);
+  }
   const ItemInfo it = item_info(p, blockIdx.x);
   const int64_t qh0 = (int64_t)it.b * p.Hq + (int64_t)it.h * g;
   if (it.cnt <= 0) {  // nothing selected (flagged upstream): out = 0, lse = -inf
@@ -118,13 +131,12 @@ __global__ void __launch_bounds__(kAttnThreads, KIN_ATTN_CTAS_PER_SM) attn_kerne
   // ---- this warp's tiles t = warp + W n; lane n holds tile n's source
   // offset (elements, into the contiguous cache or the page pool) and its
   // valid row count
-  const int tpb = p.bs / kTileTokens;
   const int n_w = warp < it.ntiles ? (it.ntiles - 1 - warp) / kAttnWarps + 1 : 0;
   int64_t my_off = 0;
   int my_nvalid = 0;
   if (lane < n_w) {
     const int t = warp + kAttnWarps * lane;
-    const int blk = __ldg(p.sel_idx + it.pair * p.k + it.j0 + t / tpb);
+    const int blk = blk_spec;
     const int sub = (t - (t / tpb) * tpb) * kTileTokens;
     bool bad = blk < 0 || blk >= it.nb;
     const int64_t off = bad ? -1 : kv_row_offset(p.pages, it.b, it.h, p.Hkv, p.Lcap, p.bs, blk, sub);
