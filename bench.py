@@ -309,6 +309,12 @@ def launch_ranks(args):
     return subprocess.call(cmd)
 
 
+def step_percentiles(step_ms) -> dict:
+    """p10 / p50 / p90 of the timed steps (each step's max over ranks), in us."""
+    p10, p50, p90 = np.percentile(np.asarray(step_ms, dtype=np.float64) * 1e3, [10, 50, 90])
+    return {"p10": float(p10), "p50": float(p50), "p90": float(p90)}
+
+
 def whole_job_value(world: int, qh_per_step: int, steps: int, max_total_ms: float) -> float:
     """Query heads decoded by all ranks per second of the slowest rank's time."""
     return world * qh_per_step * steps / (max_total_ms / 1e3)
@@ -775,9 +781,12 @@ def report(args, rank, world, rec: RankRecord):
     names = [name for name, _, _ in rec.parts]
     means = [statistics.mean(rec.part_ms[n]) for n in names]
     upd = statistics.mean(rec.upd_ms) if rec.upd_ms else 0.0
-    red = reduce_max_list([sum(rec.per_step), sum(rec.e2e_ms), rec.wall, upd, *means])
+    # one collective: totals, per-kernel means, then every step's time (the
+    # step's max over ranks, for its percentiles)
+    red = reduce_max_list([sum(rec.per_step), sum(rec.e2e_ms), rec.wall, upd, *means, *rec.per_step])
     total_ms, e2e_total, wall, upd = red[:4]
-    avg = dict(zip(names, red[4:]))
+    avg = dict(zip(names, red[4:4 + len(names)]))
+    step_max_ms = red[4 + len(names):]
     clocks_all = [rec.clocks]
     if world > 1:
         clocks_all = [None] * world
@@ -810,6 +819,7 @@ def report(args, rank, world, rec: RankRecord):
         "steps": steps,
         "warmup": args.warmup,
         "ms_per_step": ms_per_step,
+        "step_us": step_percentiles(step_max_ms),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -925,16 +935,18 @@ def reference_arm(args):
     smp = OracleSample(w, k, max_pairs=args.ref_pairs or sample_pairs_default())
     for _ in range(args.warmup):
         smp.run_pass()
-    el, qh = 0.0, 0
+    el, qh, pass_ms = 0.0, 0, []
     for _ in range(args.steps):
         a = time.perf_counter()
         qh += smp.run_pass()
-        el += time.perf_counter() - a
+        pass_ms.append((time.perf_counter() - a) * 1e3)
+        el += pass_ms[-1] / 1e3
     value = qh / el
     line = {
         "metric": METRIC, "value": value, "unit": "query-heads/s",
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": el / args.steps * 1e3, "step_us": step_percentiles(pass_ms),
+        "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w, k, int(os.environ.get("WORLD_SIZE", "1"))),
         "step": f"one pass over {smp.n} sampled (batch, kv-head) pairs ({smp.n * w.g} query heads)",

@@ -38,6 +38,8 @@ def test_reference_arm_prints_the_contract_line():
     assert d["config"] == bench.workload_config(bench.ki.WORKLOADS["qwen3_8b_32k"], 256, 1)
     assert abs(d["ms_per_step"] - 2 * 4 / d["value"] * 1e3) < 1e-6 * d["ms_per_step"]
     assert d["steps"] * d["ms_per_step"] / 1e3 <= d["wall_s"]
+    p = d["step_us"]
+    assert 0 < p["p10"] <= p["p50"] <= p["p90"] <= d["wall_s"] * 1e6
 
 
 def test_reference_arm_is_silent_on_other_ranks():

@@ -65,9 +65,9 @@ def test_single_rank_reduce_is_identity():
 
 
 # A wrapper that runs bench.py's own entry point with the per-rank GPU
-# measurement replaced by a CPU stub (rank r takes 10 + 5 r ms per step), so
-# the launcher, the process group, the max-over-ranks reduction and the JSON
-# line are exercised on CPU ranks.
+# measurement replaced by a CPU stub (three steps: rank 0 takes 5, 25 and
+# 5 ms, rank 1 15 ms each), so the launcher, the process group, the
+# max-over-ranks reduction and the JSON line are exercised on CPU ranks.
 _STUB = """
 import sys
 sys.path.insert(0, {root!r})
@@ -82,7 +82,7 @@ def fake_measure(args, rank, world, local):
     lens, _, _ = ki.case_meta(w)
     dist.barrier()
     return bench.RankRecord(
-        w0=w0, w=w, k=w0.k, lens_final=lens, per_step=[10.0 + 5.0 * rank] * args.steps,
+        w0=w0, w=w, k=w0.k, lens_final=lens, per_step=[5.0, 25.0, 5.0] if rank == 0 else [15.0] * 3,
         parts=[("select", 269e6, "kin_select.cu"), ("attn", 538e6, "kin_attn.cu")],
         part_ms={{"select": [0.04 + 0.01 * rank], "attn": [0.09]}}, upd_ms=[],
         e2e_ms=[12.0 + rank] * args.steps, e2e={{"mode": "stub", "h2d_bytes_per_step": 1, "d2h_bytes_per_step": 1}},
@@ -119,6 +119,8 @@ def test_bench_gpus_flag_launches_ranks_and_reports_the_slowest(tmp_path):
     d = json.loads(lines[0])
     assert d["n_gpus"] == 2 and d["config"]["global_batch"] == 64 and d["config"]["parallelism"] == "dp2"
     assert d["ms_per_step"] == pytest.approx(15.0)                       # the slower rank's time
+    # percentiles of each step's max over ranks: 15, 25, 15 ms
+    assert d["step_us"] == pytest.approx({"p10": 15e3, "p50": 15e3, "p90": 23e3})
     assert d["value"] == pytest.approx(2 * 32 * 32 * 3 / 0.045)          # both ranks' heads / max time
     assert d["e2e"]["value"] == pytest.approx(2 * 32 * 32 * 3 / 0.039)
     assert d["kernel_ms"]["select"] == pytest.approx(0.05)              # max over ranks
