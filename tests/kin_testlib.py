@@ -89,8 +89,10 @@ class GpuResult:
     status: int
 
 
-def gpu_step(dc: DeviceCase, k: int, ws: torch.Tensor | None = None, build_means: bool = True) -> GpuResult:
-    """Means (build, then append if the workload has one), select, attend."""
+def gpu_step(dc: DeviceCase, k: int, ws: torch.Tensor | None = None, build_means: bool = True,
+             scale: float = 0.0) -> GpuResult:
+    """Means (build, then append if the workload has one), select, attend
+    (softmax scale: 0 = the default 1/sqrt(D))."""
     w = dc.w
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     if build_means:
@@ -105,7 +107,7 @@ def gpu_step(dc: DeviceCase, k: int, ws: torch.Tensor | None = None, build_means
     out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
     kin.kin_block_topk_select(dc.dims, dc.q, dc.means, dc.seq_lens, k, sel, cnt, ws, st)
-    kin.kin_sparse_decode_attn(dc.dims, dc.q, dc.k_cache, dc.v_cache, dc.seq_lens, sel, cnt, k, 0.0,
+    kin.kin_sparse_decode_attn(dc.dims, dc.q, dc.k_cache, dc.v_cache, dc.seq_lens, sel, cnt, k, scale,
                                out, lse, ws, st)
     torch.cuda.synchronize()
     return GpuResult(sel.cpu().numpy(), cnt.cpu().numpy(), out.float().cpu().numpy(),
@@ -164,8 +166,9 @@ def check_selection(dc: DeviceCase, b: int, h: int, k: int, ref: PairRef, gsel: 
 
 
 def check_pair(dc: DeviceCase, gr: GpuResult, b: int, h: int, k: int, gpu_means: np.ndarray | None = None,
-               bf16_means: bool = False, rows=None):
-    """Full parity of one (b, h): means, selection, outputs, lse.  With
+               bf16_means: bool = False, rows=None, scale: float = 0.0):
+    """Full parity of one (b, h): means, selection, outputs, lse (softmax
+    scale as passed to the attention: 0 = the default 1/sqrt(D)).  With
     bf16_means the oracle scores blocks from its means rounded to bf16, and
     GPU means may differ from them by one bf16 step (the GPU rounds its fp32
     mean, the oracle its fp64 mean)."""
@@ -184,7 +187,7 @@ def check_pair(dc: DeviceCase, gr: GpuResult, b: int, h: int, k: int, gpu_means:
     same = check_selection(dc, b, h, k, ref, gr.sel[b, h], int(gr.cnt[b, h]))
     blocks = gr.sel[b, h, :gr.cnt[b, h]] if not same else ref.sel[:ref.cnt]
     qg = dc.q_host[b, h * w.g:(h + 1) * w.g]
-    o_ref, lse_ref = oracle.attend(qg, ref.K, ref.V, ref.L, w.bs, blocks, 1 / math.sqrt(D))
+    o_ref, lse_ref = oracle.attend(qg, ref.K, ref.V, ref.L, w.bs, blocks, scale if scale > 0 else 1 / math.sqrt(D))
     o_gpu = gr.out[b, h * w.g:(h + 1) * w.g].astype(np.float64)
     err = np.abs(o_gpu - o_ref)
     assert err.max() <= OUT_MAX_ABS and err.mean() <= OUT_MEAN_ABS, (b, h, err.max(), err.mean())

@@ -35,6 +35,44 @@ def test_edge_shapes_every_pair(w):
             check_pair(dc, gr, b, h, w.k, gpu_means=means)
 
 
+@pytest.mark.parametrize("mult", [0.5, 2.0, math.sqrt(D)], ids=["half", "double", "one"])
+def test_explicit_softmax_scale(mult):
+    """A softmax scale passed explicitly (mult / sqrt(D); sqrt(D) gives 1.0,
+    a peaked softmax): out and lse against the oracle at the same scale, on
+    pairs of three chunks (so the merge runs); the selection does not
+    depend on it."""
+    w = W("scale", 3, 2, 8, D, 16, 1500, 3000, 100, 50, Lcap=3072)
+    dc = make_device_case(w)
+    scale = mult / math.sqrt(D)
+    gr = gpu_step(dc, w.k, scale=scale)
+    assert gr.status == 0
+    default = gpu_step(dc, w.k, build_means=False)
+    assert np.array_equal(gr.sel, default.sel) and np.array_equal(gr.cnt, default.cnt)
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            check_pair(dc, gr, b, h, w.k, scale=scale)
+
+
+def test_attention_without_lse_output():
+    """lse is optional: with a null lse the outputs (a 2-block sequence and
+    long ones whose pairs span many chunks, merged in the kernel) equal
+    those of a call that writes lse, bit for bit."""
+    w = W("no_lse", 3, 2, 8, D, 16, 0, 0, 100, 51, Lcap=3072, lens=(20, 908, 3072))
+    dc = make_device_case(w)
+    gr = gpu_step(dc, w.k)
+    assert gr.status == 0
+    sel = torch.from_numpy(gr.sel).cuda()
+    cnt = torch.from_numpy(gr.cnt).cuda()
+    out = torch.empty((w.B, w.Hq, D), dtype=torch.bfloat16, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = kin.alloc_workspace(dc.dims, w.k)
+    kin.kin_sparse_decode_attn(dc.dims, dc.q, dc.k_cache, dc.v_cache, dc.seq_lens, sel, cnt, w.k, 0.0,
+                               out, None, ws, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert np.array_equal(out.float().cpu().numpy(), gr.out)
+
+
 def test_long_block_list_with_all_equal_scores():
     """16384 blocks whose scores all tie: the top-k cannot keep a compact
     candidate list and must still pick blocks 0..k-2 and the last one."""

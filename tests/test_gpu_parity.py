@@ -90,6 +90,38 @@ def test_workspace_reuse_is_deterministic():
     assert torch.count_nonzero(ws[:n]) == 0
 
 
+def test_one_workspace_serves_every_budget_in_turn():
+    """One zeroed workspace of the largest size the budgets need, used by a
+    select and an attention per budget back to back on one stream (no
+    re-zeroing, one synchronize at the end; the budgets split the pairs into
+    different chunk counts and the last one is dense): every budget's
+    results equal a fresh workspace's bit for bit, and the completion
+    counters end at zero."""
+    w = W("ws_budgets", 4, 2, 8, D, 16, 2000, 4000, 8, 26, Lcap=4096)
+    dc = make_device_case(w)
+    ks = (2, 8, 31, 73, 200, 256)
+    fresh = [gpu_step(dc, k, build_means=i == 0) for i, k in enumerate(ks)]
+    ws = torch.zeros(max(kin.kin_workspace_bytes(dc.dims, k) for k in ks), dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    runs = []
+    for k in ks:
+        sel = torch.empty((w.B, w.Hkv, k), dtype=torch.int32, device="cuda")
+        cnt = torch.empty((w.B, w.Hkv), dtype=torch.int32, device="cuda")
+        out = torch.empty((w.B, w.Hq, D), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
+        kin.kin_block_topk_select(dc.dims, dc.q, dc.means, dc.seq_lens, k, sel, cnt, ws, st)
+        kin.kin_sparse_decode_attn(dc.dims, dc.q, dc.k_cache, dc.v_cache, dc.seq_lens, sel, cnt, k, 0.0,
+                                   out, lse, ws, st)
+        runs.append((sel, cnt, out, lse))
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for k, f, (sel, cnt, out, lse) in zip(ks, fresh, runs):
+        assert np.array_equal(sel.cpu().numpy(), f.sel) and np.array_equal(cnt.cpu().numpy(), f.cnt), k
+        assert np.array_equal(out.float().cpu().numpy(), f.out) and np.array_equal(lse.cpu().numpy(), f.lse), k
+    n = (w.B * w.Hkv * 4 + 255) // 256 * 256
+    assert torch.count_nonzero(ws[:n]) == 0
+
+
 def test_bad_device_lengths_are_flagged_not_fatal():
     w = W("bad", 3, 1, 4, D, 16, 0, 0, 4, 23, Lcap=128, lens=(100, 50, 80))
     dc = make_device_case(w)

@@ -26,28 +26,29 @@ pytestmark = pytest.mark.gpu
 W = ki.Workload
 
 
-def run_token(dc, kt):
+def run_token(dc, kt, scale=0.0):
     w = dc.w
     ws = kin.alloc_token_workspace(dc.dims, kt)
     out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
     sel = torch.full((w.B, w.Hq, kt), -7, dtype=torch.int32, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    kin.kin_token_topk_decode_attn(dc.dims, dc.q, dc.k_cache, dc.v_cache, dc.seq_lens, kt, 0.0, out, lse, ws,
+    kin.kin_token_topk_decode_attn(dc.dims, dc.q, dc.k_cache, dc.v_cache, dc.seq_lens, kt, scale, out, lse, ws,
                                    sel_tokens=sel, dev_status=st)
     torch.cuda.synchronize()
     return sel.cpu().numpy(), out.float().cpu().numpy(), lse.cpu().numpy(), int(st.item())
 
 
-def check_head(dc, b, j, kt, sel, out, lse, rows=None):
+def check_head(dc, b, j, kt, sel, out, lse, rows=None, scale=0.0):
     """One query head against the oracle; rows: its pair's (K, V) when the
-    caller regenerated them already."""
+    caller regenerated them already; scale as passed to the GPU (0 = the
+    default 1/sqrt(D))."""
     w = dc.w
     h = j // w.g
     L = int(dc.lens_final[b])
     K, V = rows if rows is not None else ki.pair_rows(w, dc.hh, b, h, L)
     q = dc.q_host[b, j:j + 1]
-    scale = 1 / math.sqrt(D)
+    scale = scale if scale > 0 else 1 / math.sqrt(D)
     rsel, rout, rlse, z = oracle.token_topk_attend(q, K, V, L, kt, scale)
     n = min(kt, L)
     gsel = sel[b, j]
@@ -87,6 +88,21 @@ def test_token_topk_every_head(w, kt):
     for b in range(w.B):
         for j in range(w.Hq):
             check_head(dc, b, j, kt, sel, out, lse)
+
+
+@pytest.mark.parametrize("scale", [0.03, 0.5])
+def test_token_topk_explicit_scale(scale):
+    """An explicit softmax scale: kept tokens, out and lse against the
+    oracle at that scale (the logits are rounded after scaling, so the set
+    is checked by the near-tie rule at that scale, not against the default
+    scale's set)."""
+    w = W("tok_scale", 2, 2, 8, D, 16, 700, 1000, 8, 98, Lcap=1024)
+    dc = make_device_case(w)
+    sel, out, lse, status = run_token(dc, 96, scale)
+    assert status == 0
+    for b in range(w.B):
+        for j in range(w.Hq):
+            check_head(dc, b, j, 96, sel, out, lse, scale=scale)
 
 
 def test_token_topk_bad_length_is_flagged():
