@@ -39,7 +39,9 @@
  *  - Data that only the device can see (a sequence length outside
  *    [1, Lcap], a block index outside [0, nb)) makes the kernel skip that
  *    item and write the status code into *dev_status (first error wins) when
- *    dev_status is not NULL.  Kernels never trap; every wait is bounded.
+ *    dev_status is not NULL.  Kernels never trap and never wait on other
+ *    CTAs or kernels: a split-K merge is run by the last chunk to arrive
+ *    (counted with an atomic), so nothing spins.
  *  - No C++ exception crosses this boundary; the library keeps no state
  *    between calls other than what the caller's buffers hold (except the
  *    scratch array of kin_block_topk_select_noalloc, described there).
@@ -68,7 +70,7 @@ typedef enum {
   KIN_ERR_CAPACITY = 3,     /* a size beyond a documented limit */
   KIN_ERR_CUDA = 4,         /* a CUDA runtime/driver call or launch failed */
   KIN_ERR_DEVICE_DATA = 5,  /* (device) bad seq_len / block index: item skipped */
-  KIN_ERR_TIMEOUT = 6       /* (device) a bounded wait expired: item skipped */
+  KIN_ERR_TIMEOUT = 6       /* reserved for a bounded device wait; no kernel waits today */
 } kin_status;
 
 typedef struct {
