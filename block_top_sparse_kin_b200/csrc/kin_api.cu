@@ -1,6 +1,8 @@
 // kin_api.cu -- the extern "C" boundary of libkin.so: argument checks,
 // workspace layout, launch-shape heuristics, TMA descriptors and launches.
 // Semantics of every call are documented in include/kin.h.
+#include <atomic>
+#include <mutex>
 #include <cmath>
 
 #include "kin_internal.cuh"
@@ -111,31 +113,42 @@ kin_status check_dims(const kin_dims* d) {
 constexpr int kMaxDevices = 64;
 
 int device_sm_count() {
-  static int cache[kMaxDevices] = {0};
+  // per device, written once with the same value by whichever thread gets there first
+  static std::atomic<int> cache[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return kTargetSMs;
-  if (dev >= kMaxDevices) {
-    int n = 0;
-    return cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? n : kTargetSMs;
+  int n = dev < kMaxDevices ? cache[dev].load(std::memory_order_relaxed) : 0;
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) return kTargetSMs;
+    if (dev < kMaxDevices) cache[dev].store(n, std::memory_order_relaxed);
   }
-  if (cache[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return kTargetSMs;
-    cache[dev] = n;
-  }
-  return cache[dev];
+  return n;
 }
 
 cudaError_t ensure_smem_limit(const void* kernel, int slot, size_t bytes) {
-  // slot: a small per-kernel index; the cache remembers the largest limit set
-  static size_t done[8][kMaxDevices] = {{0}};
+  // slot: a small per-kernel index.  The kernel's limit only ever grows: it
+  // is read and raised under one lock, so a thread never lowers it under
+  // another thread's launch, and the cache (the limit last seen, per slot and
+  // device) never exceeds the limit in force.
+  static std::atomic<size_t> done[8][kMaxDevices];
+  static std::mutex mu;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < kMaxDevices && slot >= 0 && slot < 8 && done[slot][dev] >= bytes) return cudaSuccess;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  if (e == cudaSuccess && dev < kMaxDevices && slot >= 0 && slot < 8) done[slot][dev] = bytes;
-  return e;
+  const bool cached = dev >= 0 && dev < kMaxDevices && slot >= 0 && slot < 8;
+  if (cached && done[slot][dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+  std::lock_guard<std::mutex> lock(mu);
+  cudaFuncAttributes attr;
+  e = cudaFuncGetAttributes(&attr, kernel);
+  if (e != cudaSuccess) return e;
+  size_t limit = attr.maxDynamicSharedSizeBytes > 0 ? (size_t)attr.maxDynamicSharedSizeBytes : 0;
+  if (limit < bytes) {
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return e;
+    limit = bytes;
+  }
+  if (cached) done[slot][dev].store(limit, std::memory_order_release);
+  return cudaSuccess;
 }
 
 }  // namespace kin

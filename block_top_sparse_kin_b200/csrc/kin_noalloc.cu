@@ -20,6 +20,7 @@
 // the array needs to start at zero: every score the top-k reads is written by
 // the scan of the same call.  All calls share the one array, so calls whose
 // kernels overlap on a GPU (two streams, or two threads) race on it.
+#include <atomic>
 #include "kin_internal.cuh"
 
 #define KIN_EXPORT extern "C" __attribute__((visibility("default")))
@@ -34,15 +35,20 @@ constexpr int kMaxDevicesNoAlloc = 64;
 
 // Device address of g_select_scratch on the current device (nullptr on error).
 float* scratch_on_current_device(cudaError_t* err) {
-  static float* cache[kMaxDevicesNoAlloc] = {nullptr};
+  // per device, written once with the same address by whichever thread gets there first
+  static std::atomic<float*> cache[kMaxDevicesNoAlloc];
   int dev = 0;
   *err = cudaGetDevice(&dev);
   if (*err != cudaSuccess) return nullptr;
-  if (dev >= 0 && dev < kMaxDevicesNoAlloc && cache[dev]) return cache[dev];
+  const bool cached = dev >= 0 && dev < kMaxDevicesNoAlloc;
+  if (cached) {
+    float* c = cache[dev].load(std::memory_order_relaxed);
+    if (c) return c;
+  }
   void* ptr = nullptr;
   *err = cudaGetSymbolAddress(&ptr, g_select_scratch);
   if (*err != cudaSuccess || !ptr) return nullptr;
-  if (dev >= 0 && dev < kMaxDevicesNoAlloc) cache[dev] = static_cast<float*>(ptr);
+  if (cached) cache[dev].store(static_cast<float*>(ptr), std::memory_order_relaxed);
   return static_cast<float*>(ptr);
 }
 

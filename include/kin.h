@@ -44,7 +44,10 @@
  *    (counted with an atomic), so nothing spins.
  *  - No C++ exception crosses this boundary; the library keeps no state
  *    between calls other than what the caller's buffers hold (except the
- *    scratch array of kin_block_topk_select_noalloc, described there).
+ *    scratch array of kin_block_topk_select_noalloc, described there, and
+ *    per-device caches of device properties and kernel shared-memory
+ *    limits, kept with atomics and a lock).  Calls may come from several
+ *    host threads at once, each with its own buffers and workspace.
  *  - Every call that launches kernels opens an NVTX range named after the
  *    call for its host-side duration (NVTX3, header-only: it costs nothing
  *    measurable unless a profiler is attached; built with -DKIN_NVTX=0 the

@@ -3,6 +3,10 @@ appends, very long block lists (the top-k path without a candidate list),
 a multi-step decode loop (append -> select -> attend, checked every step),
 and a whole step captured in a CUDA graph (as the benchmark replays it)."""
 import math
+import os
+import subprocess
+import sys
+import textwrap
 
 import numpy as np
 import pytest
@@ -175,3 +179,67 @@ def test_step_captured_in_a_cuda_graph_matches_eager():
         for a, b in zip(eager, graphed):
             assert torch.equal(a, b)
     assert int(st.item()) == 0
+
+
+_THREADS = textwrap.dedent("""
+    import sys, threading
+    sys.path.insert(0, {root!r})
+    sys.path.insert(0, {tests!r})
+    import numpy as np, torch
+    import block_top_sparse_kin_b200 as kin
+    import kin_inputs as ki
+    from kin_testlib import make_device_case
+    W = ki.Workload
+    # two shapes whose top-k kernels need different dynamic shared memory
+    cases = [make_device_case(W("thr_a", 1, 1, 4, 128, 16, 0, 0, 8, 60, Lcap=9000, lens=(8999,))),
+             make_device_case(W("thr_b", 1, 1, 2, 128, 16, 0, 0, 8, 61, Lcap=40000, lens=(39999,)))]
+    torch.cuda.synchronize()
+
+    def run(dc, kt, stream):
+        w = dc.w
+        with torch.cuda.stream(stream):
+            ws = kin.alloc_token_workspace(dc.dims, kt)
+            out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
+            lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
+            sel = torch.empty((w.B, w.Hq, kt), dtype=torch.int32, device="cuda")
+            st = torch.zeros(1, dtype=torch.int32, device="cuda")
+            kin.kin_token_topk_decode_attn(dc.dims, dc.q, dc.k_cache, dc.v_cache, dc.seq_lens, kt, 0.0, out, lse,
+                                           ws, sel_tokens=sel, dev_status=st)
+        stream.synchronize()
+        return int(st.item()), sel.cpu().numpy(), out.view(torch.int16).cpu().numpy(), lse.cpu().numpy()
+
+    n = 8
+    gate = threading.Barrier(n)
+    res, errs = [None] * n, []
+
+    def worker(i):
+        s = torch.cuda.Stream()
+        try:
+            gate.wait()
+            res[i] = run(cases[i % 2], 700, s)
+        except Exception as e:
+            errs.append(repr(e))
+
+    th = [threading.Thread(target=worker, args=(i,)) for i in range(n)]
+    for t in th: t.start()
+    for t in th: t.join()
+    assert not errs, errs
+    ref = [run(cases[j], 700, torch.cuda.current_stream()) for j in range(2)]
+    for i, r in enumerate(res):
+        assert r[0] == 0, (i, r[0])
+        for a, b in zip(r[1:], ref[i % 2][1:]):
+            assert np.array_equal(a, b), i
+    print("threads ok")
+""")
+
+
+def test_concurrent_first_calls_from_host_threads():
+    """Eight host threads, released together in a fresh process (so the
+    library's per-device caches are cold), each on its own stream with its
+    own buffers, on two shapes whose top-k kernels need different dynamic
+    shared memory: every call succeeds and every result equals a serial
+    run's, bit for bit."""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    script = _THREADS.format(root=root, tests=os.path.join(root, "tests"))
+    r = subprocess.run([sys.executable, "-c", script], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and "threads ok" in r.stdout, (r.stdout[-2000:], r.stderr[-3000:])
