@@ -113,18 +113,58 @@ def load_library(path: str = LIB_PATH):
     return lib
 
 
-def _dev(t: Optional[torch.Tensor], name: str, dtype=None, nullable=False):
+def _dev(t: Optional[torch.Tensor], name: str, dtype=None, nullable=False, count: Optional[int] = None):
+    """The device pointer of t after checking that it is a contiguous CUDA
+    tensor on the current device, of an accepted dtype and, when count is
+    given, of at least count elements (what the library reads or writes
+    through it): a short tensor is refused here, on the host, because the C
+    ABI receives bare pointers and could not see it."""
     if t is None:
         if nullable:
             return None
         raise ValueError(f"{name} is required")
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device}; the calls run on the current device "
+                         f"cuda:{torch.cuda.current_device()}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
         raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if count is not None and t.numel() < count:
+        raise ValueError(f"{name} holds {t.numel()} elements; the dims need {count}")
     return ctypes.c_void_p(t.data_ptr())
+
+
+class _Counts:
+    """Element counts of every buffer a call touches, from the dims (all
+    None when the dims are invalid: the call then returns the library's
+    own status for them)."""
+
+    def __init__(self, dims: kin_dims):
+        ok = load_library().kin_workspace_bytes(ctypes.byref(dims), 2) > 0
+        B, Hkv, Hq, D = dims.batch, dims.num_kv_heads, dims.num_q_heads, dims.head_dim
+        bs, L = dims.block_size, dims.max_seq_len
+        nbcap = -(-L // bs) if ok else 0
+        self.ok = ok
+        self.q = B * Hq * D if ok else None            # q, out
+        self.lse = B * Hq if ok else None
+        self.cache = B * Hkv * L * D if ok else None   # k_cache, v_cache
+        self.means = B * Hkv * nbcap * D if ok else None
+        self.table = B * nbcap if ok else None
+        self.lens = B if ok else None
+        self.pairs = B * Hkv if ok else None           # sel_cnt
+        self.page = Hkv * bs * D if ok else None       # one page of a pool
+        self.page_mean = Hkv * D if ok else None       # one per-page mean
+        self.bkd = B * Hkv * D if ok else None         # one appended row per (b, h)
+
+    def times(self, n, per):
+        return None if per is None else int(n) * per
+
+
+def _status(dev_status):
+    return _dev(dev_status, "dev_status", torch.int32, nullable=True, count=1)
 
 
 def _stream(stream) -> ctypes.c_void_p:
@@ -158,44 +198,49 @@ def alloc_workspace(dims: kin_dims, k_blocks: int, device="cuda") -> torch.Tenso
 
 
 def kin_block_means_build(dims, k_cache, seq_lens, block_means, dev_status=None, stream=None):
+    c = _Counts(dims)
     rc = load_library().kin_block_means_build(
-        ctypes.byref(dims), _dev(k_cache, "k_cache", _BF16), _dev(seq_lens, "seq_lens", torch.int32),
-        _dev(block_means, "block_means", torch.float32),
-        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+        ctypes.byref(dims), _dev(k_cache, "k_cache", _BF16, count=c.cache),
+        _dev(seq_lens, "seq_lens", torch.int32, count=c.lens),
+        _dev(block_means, "block_means", torch.float32, count=c.means), _status(dev_status), _stream(stream))
     _check(rc, "kin_block_means_build")
 
 
 def kin_block_means_update(dims, k_cache, v_cache, block_means, seq_lens, k_new, v_new, n_new,
                            dev_status=None, stream=None):
+    c = _Counts(dims)
+    new_rows = c.times(max(int(n_new), 0), c.bkd)
     rc = load_library().kin_block_means_update(
-        ctypes.byref(dims), _dev(k_cache, "k_cache", _BF16), _dev(v_cache, "v_cache", _BF16),
-        _dev(block_means, "block_means", torch.float32), _dev(seq_lens, "seq_lens", torch.int32),
-        _dev(k_new, "k_new", _BF16), _dev(v_new, "v_new", _BF16), int(n_new),
-        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+        ctypes.byref(dims), _dev(k_cache, "k_cache", _BF16, count=c.cache),
+        _dev(v_cache, "v_cache", _BF16, count=c.cache), _dev(block_means, "block_means", torch.float32, count=c.means),
+        _dev(seq_lens, "seq_lens", torch.int32, count=c.lens), _dev(k_new, "k_new", _BF16, count=new_rows),
+        _dev(v_new, "v_new", _BF16, count=new_rows), int(n_new), _status(dev_status), _stream(stream))
     _check(rc, "kin_block_means_update")
 
 
 def kin_block_topk_select(dims, q, block_means, seq_lens, k_blocks, sel_idx, sel_cnt, workspace,
                           dev_status=None, stream=None):
+    c = _Counts(dims)
     rc = load_library().kin_block_topk_select(
-        ctypes.byref(dims), _dev(q, "q", _BF16), _dev(block_means, "block_means", torch.float32),
-        _dev(seq_lens, "seq_lens", torch.int32), int(k_blocks), _dev(sel_idx, "sel_idx", torch.int32),
-        _dev(sel_cnt, "sel_cnt", torch.int32), _dev(workspace, "workspace"),
-        workspace.numel() * workspace.element_size(),
-        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+        ctypes.byref(dims), _dev(q, "q", _BF16, count=c.q), _dev(block_means, "block_means", torch.float32, count=c.means),
+        _dev(seq_lens, "seq_lens", torch.int32, count=c.lens), int(k_blocks),
+        _dev(sel_idx, "sel_idx", torch.int32, count=c.times(max(int(k_blocks), 0), c.pairs)),
+        _dev(sel_cnt, "sel_cnt", torch.int32, count=c.pairs), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _status(dev_status), _stream(stream))
     _check(rc, "kin_block_topk_select")
 
 
 def kin_sparse_decode_attn(dims, q, k_cache, v_cache, seq_lens, sel_idx, sel_cnt, k_blocks,
                            softmax_scale, out, lse, workspace, dev_status=None, stream=None):
+    c = _Counts(dims)
     rc = load_library().kin_sparse_decode_attn(
-        ctypes.byref(dims), _dev(q, "q", _BF16), _dev(k_cache, "k_cache", _BF16),
-        _dev(v_cache, "v_cache", _BF16), _dev(seq_lens, "seq_lens", torch.int32),
-        _dev(sel_idx, "sel_idx", torch.int32), _dev(sel_cnt, "sel_cnt", torch.int32),
-        int(k_blocks), float(softmax_scale), _dev(out, "out", _BF16),
-        _dev(lse, "lse", torch.float32, nullable=True), _dev(workspace, "workspace"),
-        workspace.numel() * workspace.element_size(),
-        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+        ctypes.byref(dims), _dev(q, "q", _BF16, count=c.q), _dev(k_cache, "k_cache", _BF16, count=c.cache),
+        _dev(v_cache, "v_cache", _BF16, count=c.cache), _dev(seq_lens, "seq_lens", torch.int32, count=c.lens),
+        _dev(sel_idx, "sel_idx", torch.int32, count=c.times(max(int(k_blocks), 0), c.pairs)),
+        _dev(sel_cnt, "sel_cnt", torch.int32, count=c.pairs), int(k_blocks), float(softmax_scale),
+        _dev(out, "out", _BF16, count=c.q), _dev(lse, "lse", torch.float32, nullable=True, count=c.lse),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _status(dev_status),
+        _stream(stream))
     _check(rc, "kin_sparse_decode_attn")
 
 
@@ -204,11 +249,12 @@ def kin_block_topk_select_noalloc(dims, q, block_means, seq_lens, k_blocks, sel_
     """kin_block_topk_select without a workspace, for callers that may not
     allocate device memory: the scratch lives in a fixed array inside
     libkin.so (see include/kin.h for its limit and its sharing rules)."""
+    c = _Counts(dims)
     rc = load_library().kin_block_topk_select_noalloc(
-        ctypes.byref(dims), _dev(q, "q", _BF16), _dev(block_means, "block_means", torch.float32),
-        _dev(seq_lens, "seq_lens", torch.int32), int(k_blocks), _dev(sel_idx, "sel_idx", torch.int32),
-        _dev(sel_cnt, "sel_cnt", torch.int32),
-        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+        ctypes.byref(dims), _dev(q, "q", _BF16, count=c.q), _dev(block_means, "block_means", torch.float32, count=c.means),
+        _dev(seq_lens, "seq_lens", torch.int32, count=c.lens), int(k_blocks),
+        _dev(sel_idx, "sel_idx", torch.int32, count=c.times(max(int(k_blocks), 0), c.pairs)),
+        _dev(sel_cnt, "sel_cnt", torch.int32, count=c.pairs), _status(dev_status), _stream(stream))
     _check(rc, "kin_block_topk_select_noalloc")
 
 
@@ -218,35 +264,45 @@ def kin_block_topk_select_noalloc(dims, q, block_means, seq_lens, k_blocks, sel_
 
 def kin_block_means_build_paged(dims, k_pages, block_table, seq_lens, block_means, dev_status=None,
                                 stream=None):
+    c = _Counts(dims)
+    pages = int(k_pages.shape[0])
     rc = load_library().kin_block_means_build_paged(
-        ctypes.byref(dims), _dev(k_pages, "k_pages", _BF16), int(k_pages.shape[0]),
-        _dev(block_table, "block_table", torch.int32), _dev(seq_lens, "seq_lens", torch.int32),
-        _dev(block_means, "block_means", torch.float32),
-        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+        ctypes.byref(dims), _dev(k_pages, "k_pages", _BF16, count=c.times(pages, c.page)), pages,
+        _dev(block_table, "block_table", torch.int32, count=c.table),
+        _dev(seq_lens, "seq_lens", torch.int32, count=c.lens),
+        _dev(block_means, "block_means", torch.float32, count=c.means), _status(dev_status), _stream(stream))
     _check(rc, "kin_block_means_build_paged")
 
 
 def kin_block_means_update_paged(dims, k_pages, v_pages, block_table, block_means, seq_lens, k_new, v_new,
                                  n_new, dev_status=None, stream=None):
+    c = _Counts(dims)
+    pages = int(k_pages.shape[0])
+    new_rows = c.times(max(int(n_new), 0), c.bkd)
     rc = load_library().kin_block_means_update_paged(
-        ctypes.byref(dims), _dev(k_pages, "k_pages", _BF16), _dev(v_pages, "v_pages", _BF16),
-        int(k_pages.shape[0]), _dev(block_table, "block_table", torch.int32),
-        _dev(block_means, "block_means", torch.float32), _dev(seq_lens, "seq_lens", torch.int32),
-        _dev(k_new, "k_new", _BF16), _dev(v_new, "v_new", _BF16), int(n_new),
-        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+        ctypes.byref(dims), _dev(k_pages, "k_pages", _BF16, count=c.times(pages, c.page)),
+        _dev(v_pages, "v_pages", _BF16, count=c.times(pages, c.page)), pages,
+        _dev(block_table, "block_table", torch.int32, count=c.table),
+        _dev(block_means, "block_means", torch.float32, count=c.means),
+        _dev(seq_lens, "seq_lens", torch.int32, count=c.lens), _dev(k_new, "k_new", _BF16, count=new_rows),
+        _dev(v_new, "v_new", _BF16, count=new_rows), int(n_new), _status(dev_status), _stream(stream))
     _check(rc, "kin_block_means_update_paged")
 
 
 def kin_sparse_decode_attn_paged(dims, q, k_pages, v_pages, block_table, seq_lens, sel_idx, sel_cnt, k_blocks,
                                  softmax_scale, out, lse, workspace, dev_status=None, stream=None):
+    c = _Counts(dims)
+    pages = int(k_pages.shape[0])
     rc = load_library().kin_sparse_decode_attn_paged(
-        ctypes.byref(dims), _dev(q, "q", _BF16), _dev(k_pages, "k_pages", _BF16),
-        _dev(v_pages, "v_pages", _BF16), int(k_pages.shape[0]), _dev(block_table, "block_table", torch.int32),
-        _dev(seq_lens, "seq_lens", torch.int32), _dev(sel_idx, "sel_idx", torch.int32),
-        _dev(sel_cnt, "sel_cnt", torch.int32), int(k_blocks), float(softmax_scale), _dev(out, "out", _BF16),
-        _dev(lse, "lse", torch.float32, nullable=True), _dev(workspace, "workspace"),
-        workspace.numel() * workspace.element_size(),
-        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+        ctypes.byref(dims), _dev(q, "q", _BF16, count=c.q), _dev(k_pages, "k_pages", _BF16, count=c.times(pages, c.page)),
+        _dev(v_pages, "v_pages", _BF16, count=c.times(pages, c.page)), pages,
+        _dev(block_table, "block_table", torch.int32, count=c.table),
+        _dev(seq_lens, "seq_lens", torch.int32, count=c.lens),
+        _dev(sel_idx, "sel_idx", torch.int32, count=c.times(max(int(k_blocks), 0), c.pairs)),
+        _dev(sel_cnt, "sel_cnt", torch.int32, count=c.pairs), int(k_blocks), float(softmax_scale),
+        _dev(out, "out", _BF16, count=c.q), _dev(lse, "lse", torch.float32, nullable=True, count=c.lse),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _status(dev_status),
+        _stream(stream))
     _check(rc, "kin_sparse_decode_attn_paged")
 
 
@@ -254,51 +310,59 @@ def kin_sparse_decode_attn_paged(dims, q, k_pages, v_pages, block_table, seq_len
 # The means dtype follows the block_means tensor (float32 or bfloat16);
 # block_table None selects the contiguous cache.  See include/kin.h.
 
-def _means(block_means):
-    if block_means.dtype == torch.float32:
-        return _dev(block_means, "block_means", torch.float32), KIN_MEANS_F32
-    return _dev(block_means, "block_means", torch.bfloat16), KIN_MEANS_BF16
+def _means(block_means, count=None, name="block_means"):
+    if block_means is not None and block_means.dtype == torch.float32:
+        return _dev(block_means, name, torch.float32, count=count), KIN_MEANS_F32
+    return _dev(block_means, name, torch.bfloat16, count=count), KIN_MEANS_BF16
 
 
-def _layout(rows, block_table):
+def _layout(rows, block_table, c: _Counts):
+    """(num_pages, table pointer, rows per K/V tensor): the contiguous cache
+    without a table, else the page pool it indexes."""
     if block_table is None:
-        return 0, None
-    return int(rows.shape[0]), _dev(block_table, "block_table", torch.int32)
+        return 0, None, c.cache
+    pages = int(rows.shape[0])
+    return pages, _dev(block_table, "block_table", torch.int32, count=c.table), c.times(pages, c.page)
 
 
 def kin_block_means_build_ex(dims, k_rows, seq_lens, block_means, block_table=None, dev_status=None,
                              stream=None, per_page=False):
     """per_page: block_means is [num_pages, Hkv, D] (one mean per page; needs block_table)."""
-    pages, table = _layout(k_rows, block_table)
-    means, dtype = _means(block_means)
+    c = _Counts(dims)
+    pages, table, rows = _layout(k_rows, block_table, c)
+    means, dtype = _means(block_means, c.times(pages, c.page_mean) if per_page else c.means)
     dtype |= KIN_MEANS_PER_PAGE if per_page else 0
     rc = load_library().kin_block_means_build_ex(
-        ctypes.byref(dims), _dev(k_rows, "k_rows", _BF16), pages, table, _dev(seq_lens, "seq_lens", torch.int32),
-        means, dtype, _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+        ctypes.byref(dims), _dev(k_rows, "k_rows", _BF16, count=rows), pages, table,
+        _dev(seq_lens, "seq_lens", torch.int32, count=c.lens), means, dtype, _status(dev_status), _stream(stream))
     _check(rc, "kin_block_means_build_ex")
 
 
 def kin_block_means_update_ex(dims, k_rows, v_rows, block_means, seq_lens, k_new, v_new, n_new,
                               block_table=None, dev_status=None, stream=None, per_page=False):
-    pages, table = _layout(k_rows, block_table)
-    means, dtype = _means(block_means)
+    c = _Counts(dims)
+    pages, table, rows = _layout(k_rows, block_table, c)
+    means, dtype = _means(block_means, c.times(pages, c.page_mean) if per_page else c.means)
     dtype |= KIN_MEANS_PER_PAGE if per_page else 0
+    new_rows = c.times(max(int(n_new), 0), c.bkd)
     rc = load_library().kin_block_means_update_ex(
-        ctypes.byref(dims), _dev(k_rows, "k_rows", _BF16), _dev(v_rows, "v_rows", _BF16), pages, table,
-        means, dtype, _dev(seq_lens, "seq_lens", torch.int32), _dev(k_new, "k_new", _BF16),
-        _dev(v_new, "v_new", _BF16), int(n_new), _dev(dev_status, "dev_status", torch.int32, nullable=True),
-        _stream(stream))
+        ctypes.byref(dims), _dev(k_rows, "k_rows", _BF16, count=rows), _dev(v_rows, "v_rows", _BF16, count=rows),
+        pages, table, means, dtype, _dev(seq_lens, "seq_lens", torch.int32, count=c.lens),
+        _dev(k_new, "k_new", _BF16, count=new_rows), _dev(v_new, "v_new", _BF16, count=new_rows), int(n_new),
+        _status(dev_status), _stream(stream))
     _check(rc, "kin_block_means_update_ex")
 
 
 def kin_block_topk_select_ex(dims, q, block_means, seq_lens, k_blocks, sel_idx, sel_cnt, workspace,
                              dev_status=None, stream=None):
-    means, dtype = _means(block_means)
+    c = _Counts(dims)
+    means, dtype = _means(block_means, c.means)
     rc = load_library().kin_block_topk_select_ex(
-        ctypes.byref(dims), _dev(q, "q", _BF16), means, dtype, _dev(seq_lens, "seq_lens", torch.int32),
-        int(k_blocks), _dev(sel_idx, "sel_idx", torch.int32), _dev(sel_cnt, "sel_cnt", torch.int32),
-        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
-        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+        ctypes.byref(dims), _dev(q, "q", _BF16, count=c.q), means, dtype,
+        _dev(seq_lens, "seq_lens", torch.int32, count=c.lens), int(k_blocks),
+        _dev(sel_idx, "sel_idx", torch.int32, count=c.times(max(int(k_blocks), 0), c.pairs)),
+        _dev(sel_cnt, "sel_cnt", torch.int32, count=c.pairs), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _status(dev_status), _stream(stream))
     _check(rc, "kin_block_topk_select_ex")
 
 
@@ -317,13 +381,15 @@ def alloc_token_workspace(dims: kin_dims, k_tokens: int, device="cuda") -> torch
 
 def kin_token_topk_decode_attn(dims, q, k_cache, v_cache, seq_lens, k_tokens, softmax_scale, out, lse, workspace,
                                sel_tokens=None, dev_status=None, stream=None):
+    c = _Counts(dims)
     rc = load_library().kin_token_topk_decode_attn(
-        ctypes.byref(dims), _dev(q, "q", _BF16), _dev(k_cache, "k_cache", _BF16), _dev(v_cache, "v_cache", _BF16),
-        _dev(seq_lens, "seq_lens", torch.int32), int(k_tokens), float(softmax_scale), _dev(out, "out", _BF16),
-        _dev(lse, "lse", torch.float32, nullable=True),
-        _dev(sel_tokens, "sel_tokens", torch.int32, nullable=True), _dev(workspace, "workspace"),
-        workspace.numel() * workspace.element_size(),
-        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+        ctypes.byref(dims), _dev(q, "q", _BF16, count=c.q), _dev(k_cache, "k_cache", _BF16, count=c.cache),
+        _dev(v_cache, "v_cache", _BF16, count=c.cache), _dev(seq_lens, "seq_lens", torch.int32, count=c.lens),
+        int(k_tokens), float(softmax_scale), _dev(out, "out", _BF16, count=c.q),
+        _dev(lse, "lse", torch.float32, nullable=True, count=c.lse),
+        _dev(sel_tokens, "sel_tokens", torch.int32, nullable=True, count=c.times(max(int(k_tokens), 0), c.lse)),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _status(dev_status),
+        _stream(stream))
     _check(rc, "kin_token_topk_decode_attn")
 
 
@@ -331,11 +397,14 @@ def kin_block_topk_select_paged(dims, q, page_means, block_table, seq_lens, k_bl
                                 dev_status=None, stream=None):
     """The select over per-page block means [num_pages, Hkv, D] (fp32 or bf16),
     found through block_table: the shared-prompt layout (see include/kin.h)."""
-    means, dtype = _means(page_means)
+    c = _Counts(dims)
+    pages = int(page_means.shape[0])
+    means, dtype = _means(page_means, c.times(pages, c.page_mean), "page_means")
     rc = load_library().kin_block_topk_select_paged(
-        ctypes.byref(dims), _dev(q, "q", _BF16), means, dtype, int(page_means.shape[0]),
-        _dev(block_table, "block_table", torch.int32), _dev(seq_lens, "seq_lens", torch.int32), int(k_blocks),
-        _dev(sel_idx, "sel_idx", torch.int32), _dev(sel_cnt, "sel_cnt", torch.int32), _dev(workspace, "workspace"),
-        workspace.numel() * workspace.element_size(),
-        _dev(dev_status, "dev_status", torch.int32, nullable=True), _stream(stream))
+        ctypes.byref(dims), _dev(q, "q", _BF16, count=c.q), means, dtype, pages,
+        _dev(block_table, "block_table", torch.int32, count=c.table),
+        _dev(seq_lens, "seq_lens", torch.int32, count=c.lens), int(k_blocks),
+        _dev(sel_idx, "sel_idx", torch.int32, count=c.times(max(int(k_blocks), 0), c.pairs)),
+        _dev(sel_cnt, "sel_cnt", torch.int32, count=c.pairs), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _status(dev_status), _stream(stream))
     _check(rc, "kin_block_topk_select_paged")

@@ -196,6 +196,43 @@ def test_host_validation_errors():
     assert e.value.status == 3
 
 
+def test_binding_refuses_short_or_foreign_tensors():
+    """The C ABI receives bare pointers, so the binding checks every tensor
+    against the dims before the call: a buffer shorter than the dims imply,
+    a host tensor or a non-contiguous view raises ValueError and nothing is
+    launched (the outputs keep their contents)."""
+    dims = kin.make_dims(2, 2, 8, D, 16, 256)
+    lens = torch.full((2,), 200, dtype=torch.int32, device="cuda")
+    q = torch.zeros((2, 8, D), dtype=torch.bfloat16, device="cuda")
+    means = torch.zeros((2, 2, 16, D), dtype=torch.float32, device="cuda")
+    sel = torch.full((2, 2, 4), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.full((2, 2), -7, dtype=torch.int32, device="cuda")
+    ws = kin.alloc_workspace(dims, 4)
+    bad = {
+        "q": (q[:1], means, sel, cnt, lens),
+        "block_means": (q, means[:, :, :15].contiguous(), sel, cnt, lens),
+        "sel_idx": (q, means, sel[:, :, :3].contiguous(), cnt, lens),
+        "sel_cnt": (q, means, sel, cnt[:1], lens),
+        "seq_lens": (q, means, sel, cnt, lens[:1]),
+    }
+    for name, (qq, mm, ss, cc, ll) in bad.items():
+        with pytest.raises(ValueError, match=name):
+            kin.kin_block_topk_select(dims, qq, mm, ll, 4, ss, cc, ws)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        kin.kin_block_topk_select(dims, q.cpu(), means, lens, 4, sel, cnt, ws)
+    with pytest.raises(ValueError, match="contiguous"):
+        kin.kin_block_topk_select(dims, q, means, lens, 4, sel.transpose(0, 1), cnt, ws)
+    out = torch.zeros((2, 8, D), dtype=torch.bfloat16, device="cuda")
+    k_cache = torch.zeros((2, 2, 256, D), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError, match="v_cache"):
+        kin.kin_sparse_decode_attn(dims, q, k_cache, k_cache[:1], lens, sel, cnt, 4, 0.0, out, None, ws)
+    with pytest.raises(ValueError, match="lse"):
+        kin.kin_sparse_decode_attn(dims, q, k_cache, k_cache, lens, sel, cnt, 4, 0.0, out,
+                                   torch.zeros(3, device="cuda"), ws)
+    torch.cuda.synchronize()
+    assert torch.all(sel == -7) and torch.all(cnt == -7)
+
+
 # ------------------------------------------------------- full-size workloads
 def _full(name, ks=None):
     """A decode workload at full size, in the benchmark's launch shapes:
