@@ -79,3 +79,58 @@ def test_pins_catch_planted_mistake(name, orig, bad, tmp_path):
 
 def test_unmodified_oracle_passes_the_same_pins():
     assert _run_pins() == []
+
+
+# The oracle's Python parts (token top-k, paged gather, bf16 rounding): the
+# same check, with the mistake planted in a copy of the function's source
+# that replaces it for the duration of the test.
+PY_MUTANTS = [
+    ("token_ties_to_higher_index", "token_topk_attend",
+     "np.lexsort((np.arange(L), -z[j]))", "np.lexsort((-np.arange(L), -z[j]))"),
+    ("token_keeps_smallest_logits", "token_topk_attend",
+     "np.lexsort((np.arange(L), -z[j]))", "np.lexsort((np.arange(L), z[j]))"),
+    ("token_drops_scale", "token_topk_attend", "z = scale * (q @ Kf.T)", "z = q @ Kf.T"),
+    ("token_kept_set_not_ascending", "token_topk_attend", "s = np.sort(order[:n])", "s = order[:n]"),
+    ("token_normalises_over_every_token", "token_topk_attend",
+     "/ w.sum())", "/ np.exp(z[j] - m).sum())"),
+    ("token_lse_over_every_token", "token_topk_attend",
+     "lses.append(m + np.log(w.sum()))", "lses.append(m + np.log(np.exp(z[j] - m).sum()))"),
+    ("paged_ignores_the_table", "gather_paged", "pages[int(table_row[i]), h]", "pages[i, h]"),
+    ("paged_reads_head_zero", "gather_paged", "pages[int(table_row[i]), h]", "pages[int(table_row[i]), 0]"),
+    ("bf16_truncates", "round_bf16", "np.round(m * 256.0)", "np.floor(m * 256.0)"),
+    ("bf16_seven_bits", "round_bf16", "np.round(m * 256.0) / 256.0", "np.round(m * 128.0) / 128.0"),
+]
+
+
+def _run_py_pins():
+    checks = [
+        ("token_dense", pins.test_token_topk_full_budget_is_dense_attention),
+        ("token_brute_force", lambda: [pins.test_token_topk_keeps_the_best_set(t) for t in range(20)]),
+        ("token_weights", pins.test_token_topk_weights_are_softmax_of_kept_logits_only),
+        ("paged", pins.test_gather_paged_follows_the_block_table),
+        ("bf16", pins.test_round_bf16_matches_torch_conversion),
+    ]
+    failed = []
+    for name, fn in checks:
+        try:
+            fn()
+        except AssertionError:
+            failed.append(name)
+    return failed
+
+
+@pytest.mark.parametrize("name,func,orig,bad", PY_MUTANTS, ids=[m[0] for m in PY_MUTANTS])
+def test_python_pins_catch_planted_mistake(name, func, orig, bad, monkeypatch):
+    import inspect
+    import textwrap
+    src = textwrap.dedent(inspect.getsource(getattr(oracle, func)))
+    assert src.count(orig) == 1, (name, "the original text must occur once")
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(orig, bad), f"<mutant {name}>", "exec"), ns)
+    monkeypatch.setattr(oracle, func, ns[func])
+    failed = _run_py_pins()
+    assert failed, f"planted mistake {name!r} passed every pin"
+
+
+def test_unmodified_python_oracle_passes_the_same_pins():
+    assert _run_py_pins() == []
