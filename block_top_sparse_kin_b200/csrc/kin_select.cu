@@ -1202,8 +1202,7 @@ __global__ void __launch_bounds__(kTokTopkThreads, 1) token_topk_kernel(TokenPar
   extern __shared__ uint32_t skey[];  // [min(Lcap, kTokKeyCap)] keys, then as many bytes of bins
   __shared__ TopkSmem<kTokTopkThreads> sm;
   const int tid = threadIdx.x;
-  pdl_wait();  // the logits come from the logits kernel
-  pdl_trigger_early();
+  pdl_wait();  // the logits come from the logits kernel (no early trigger: see token_logits_kernel)
   const int64_t row_id = blockIdx.x;  // b * Hq + query head
   const int b = (int)(row_id / p.Hq);
   const int k = p.kt;
