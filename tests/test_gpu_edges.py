@@ -77,6 +77,23 @@ def test_attention_without_lse_output():
     assert np.array_equal(out.float().cpu().numpy(), gr.out)
 
 
+@pytest.mark.parametrize("k", [300, 32767])
+def test_maximum_block_count(k):
+    """The largest block count a sequence may have (ceil(Lcap / bs) = 32768
+    at bs 16: 524288 tokens): the top-k over 32768 keys in shared memory,
+    and a budget one block short of the whole sequence, whose 683 chunks per
+    pair the attention merges in many staged batches; every pair against
+    the oracle."""
+    L = 32768 * 16
+    w = W("max_blocks", 1, 2, 8, D, 16, 0, 0, k, 52, Lcap=L, lens=(L,))
+    dc = make_device_case(w)
+    gr = gpu_step(dc, k)
+    assert gr.status == 0
+    assert np.all(gr.cnt == k)
+    for h in range(w.Hkv):
+        check_pair(dc, gr, 0, h, k)
+
+
 def test_long_block_list_with_all_equal_scores():
     """16384 blocks whose scores all tie: the top-k cannot keep a compact
     candidate list and must still pick blocks 0..k-2 and the last one."""
