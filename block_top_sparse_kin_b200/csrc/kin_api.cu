@@ -1,5 +1,5 @@
 // kin_api.cu -- the extern "C" boundary of libkin.so: argument checks,
-// workspace layout, launch-shape heuristics, TMA descriptors and launches.
+// workspace layout, launch-shape heuristics and launches.
 // Semantics of every call are documented in include/kin.h.
 #include <atomic>
 #include <mutex>
