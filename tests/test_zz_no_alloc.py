@@ -75,6 +75,44 @@ def test_noalloc_select_takes_no_device_memory():
     assert free1 == free0
 
 
+def test_noalloc_select_at_its_scratch_capacity():
+    """B * Hkv * ceil(Lcap / bs) exactly KIN_NOALLOC_SCRATCH_FLOATS (64 x 8 x
+    4096 = 2^21 scores, so the last pair's row ends at the array's end), on
+    seeded random means and ragged lengths that include full sequences: the
+    same selection as the workspace select, bit for bit.  One block more of
+    capacity is refused by the entry point before anything is launched."""
+    import ctypes
+    B, Hkv, Hq, bs, Lcap, k = 64, 8, 32, 16, 4096 * 16, 300
+    assert B * Hkv * (Lcap // bs) == kin.NOALLOC_SCRATCH_FLOATS
+    dims = kin.make_dims(B, Hkv, Hq, D, bs, Lcap)
+    g = torch.Generator(device="cuda").manual_seed(33)
+    means = torch.randn((B, Hkv, Lcap // bs, D), generator=g, device="cuda", dtype=torch.float32)
+    q = torch.randn((B, Hq, D), generator=g, device="cuda", dtype=torch.float32).to(torch.bfloat16)
+    lens = torch.randint(1, Lcap + 1, (B,), generator=g, device="cuda", dtype=torch.int32)
+    lens[:4] = Lcap
+    ws = kin.alloc_workspace(dims, k)
+    out = []
+    for noalloc in (False, True):
+        sel = torch.full((B, Hkv, k), -7, dtype=torch.int32, device="cuda")
+        cnt = torch.full((B, Hkv), -7, dtype=torch.int32, device="cuda")
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        if noalloc:
+            kin.kin_block_topk_select_noalloc(dims, q, means, lens, k, sel, cnt, st)
+        else:
+            kin.kin_block_topk_select(dims, q, means, lens, k, sel, cnt, ws, st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        out.append((sel.cpu().numpy(), cnt.cpu().numpy()))
+    assert np.array_equal(out[0][1], out[1][1]) and np.array_equal(out[0][0], out[1][0])
+    nb = -(-lens.cpu().numpy() // bs)
+    assert np.array_equal(out[1][1], np.minimum(nb, k)[:, None].repeat(Hkv, 1))
+    over = kin.make_dims(B, Hkv, Hq, D, bs, Lcap + 1)  # 4097 blocks per sequence
+    p = [ctypes.c_void_p(x.data_ptr()) for x in (q, means, lens, ws, ws)]
+    rc = kin.load_library().kin_block_topk_select_noalloc(ctypes.byref(over), p[0], p[1], p[2], k, p[3], p[4],
+                                                          None, None)
+    assert rc == 3
+
+
 def test_noalloc_select_rejects_problems_beyond_its_scratch():
     # B * Hkv * ceil(Lcap / bs) = 64 * 8 * 8192 > 2^21 scores
     # (the C entry point itself, with small stand-in buffers: it refuses before
