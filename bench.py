@@ -384,7 +384,7 @@ def make_page_pool(st, seed: int, share_n: int = 1, shuffle: bool = True):
 
 
 def build_device_state(w: ki.Workload, k: int, paged: bool = False, means_bf16: bool = False, share_n: int = 1,
-                       shuffle_pages: bool = True):
+                       shuffle_pages: bool = True, means_dual: bool = False):
     import torch
     import block_top_sparse_kin_b200 as kin
     lens_final, lens_pre, hh = ki.case_meta(w)
@@ -400,9 +400,12 @@ def build_device_state(w: ki.Workload, k: int, paged: bool = False, means_bf16: 
     ki.kv_cache_device(w.seed, True, w.B, w.Hkv, w.cap, w.D, w.bs, st["seq"], hh_dev, False, kc)
     ki.kv_cache_device(w.seed, False, w.B, w.Hkv, w.cap, w.D, w.bs, st["seq"], hh_dev, False, vc)
     st["k_cache"], st["v_cache"] = kc, vc
-    st["means"] = torch.zeros((w.B, w.Hkv, w.nbcap, w.D), dtype=torch.bfloat16 if means_bf16 else torch.float32,
-                              device="cuda")
-    if means_bf16:
+    if means_dual:  # fp32 means, their bf16 rounding and the row norms in one buffer
+        st["means"] = kin.alloc_dual_means(dims)
+    else:
+        st["means"] = torch.zeros((w.B, w.Hkv, w.nbcap, w.D), dtype=torch.bfloat16 if means_bf16 else torch.float32,
+                                  device="cuda")
+    if means_bf16 or means_dual:
         kin.kin_block_means_build_ex(dims, kc, st["seq"], st["means"])
     else:
         kin.kin_block_means_build(dims, kc, st["seq"], st["means"])
@@ -462,7 +465,7 @@ def append(st):
     w = st["w"]
     paged = "table" in st
     k_rows, v_rows = (st["k_pages"], st["v_pages"]) if paged else (st["k_cache"], st["v_cache"])
-    if "page_means" in st or str(st["means"].dtype) == "torch.bfloat16":
+    if "page_means" in st or str(st["means"].dtype) in ("torch.bfloat16", "torch.uint8"):
         kin.kin_block_means_update_ex(st["dims"], k_rows, v_rows, st["means"], st["seq"], st["k_new"], st["v_new"],
                                       w.n_append, block_table=st.get("table"), dev_status=st["status"],
                                       per_page="page_means" in st)
@@ -475,12 +478,12 @@ def append(st):
 
 
 def select(st):
-    """The step's block scoring and top-k (fp32 means, or bf16 through the extended call)."""
+    """The step's block scoring and top-k (fp32 means, or bf16 or dual means through the extended call)."""
     import block_top_sparse_kin_b200 as kin
     if "page_means" in st:
         kin.kin_block_topk_select_paged(st["dims"], st["q"], st["means"], st["table"], st["seq"], st["k"], st["sel"],
                                         st["cnt"], st["ws"], st["status"])
-    elif str(st["means"].dtype) == "torch.bfloat16":
+    elif str(st["means"].dtype) in ("torch.bfloat16", "torch.uint8"):
         kin.kin_block_topk_select_ex(st["dims"], st["q"], st["means"], st["seq"], st["k"], st["sel"], st["cnt"],
                                      st["ws"], st["status"])
     else:
@@ -556,7 +559,8 @@ def measure_rank(args, rank, world, local) -> RankRecord:
         w0 = w0.with_(B=args.batch, name=f"{w0.name}_b{args.batch}")
     k = args.k or w0.k
     w = shard_workload(w0, rank)
-    st = build_device_state(w, k, paged=args.paged, means_bf16=args.means_bf16, share_n=args.shared_prefix,
+    st = build_device_state(w, k, paged=args.paged, means_bf16=args.means_bf16,
+                            means_dual=means_kind(args) == "dual", share_n=args.shared_prefix,
                             shuffle_pages=args.page_order == "shuffled")
     if args.token_topk:
         if args.paged or args.shared_prefix > 1:
@@ -599,7 +603,7 @@ def measure_rank(args, rank, world, local) -> RankRecord:
         return [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n)]
 
     # the step's kernel families: (name, call, algorithmic bytes, source file)
-    means_bytes = 2 if args.means_bf16 else 4
+    means_bytes = means_bytes_per_dim(args)
     if args.token_topk:
         parts = [("token_topk_attn", lambda: token_step(st),
                   token_algorithmic_bytes(w, st["token_kt"], st["lens_final"]), "kin_token.cu")]
@@ -759,8 +763,34 @@ L2_NOTE = ("GPU arm: L2 flushed before every step (256 MiB write + 256 MiB read,
            "oracle arm: host cores")
 
 
+MEANS_KINDS = {
+    "fp32": "fp32",
+    "bf16": "bf16",
+    "dual": "dual: the fp32 selection, read from a bf16 copy (fp32 + bf16 means + row norms)",
+}
+
+
+def means_kind(args) -> str:
+    """fp32 (--means-fp32, and always for per-page shared-prompt means), bf16
+    (--means-bf16), else dual: the fp32 selection read from a bf16 copy."""
+    if getattr(args, "means_bf16", False) and getattr(args, "means_fp32", False):
+        raise SystemExit("--means-bf16 and --means-fp32 exclude each other")
+    if getattr(args, "means_bf16", False):
+        return "bf16"
+    if getattr(args, "means_fp32", False) or getattr(args, "shared_prefix", 1) > 1:
+        return "fp32"
+    return "dual"
+
+
+def means_bytes_per_dim(args) -> float:
+    """Block-mean bytes the select streams per head dim: fp32 4, bf16 2, dual
+    2 + the row norm's 4 bytes spread over the 128 dims (the fp32 rows it
+    rescores are counted as traffic, not here)."""
+    return {"fp32": 4.0, "bf16": 2.0, "dual": 2.0 + 4.0 / 128}[means_kind(args)]
+
+
 def workload_config(w0: ki.Workload, k: int, world: int, kv_layout: str = "contiguous [B][Hkv][Lcap][D]",
-                    means_bf16: bool = False, token_kt: int = 0) -> dict:
+                    means: str = "fp32", token_kt: int = 0) -> dict:
     """The JSON line's config: the workload as named, the same in both arms."""
     return {
         "workload": w0.name, "batch": w0.B, "kv_heads": w0.Hkv, "q_heads": w0.Hq,
@@ -769,7 +799,7 @@ def workload_config(w0: ki.Workload, k: int, world: int, kv_layout: str = "conti
         "global_batch": w0.B * world, "parallelism": f"dp{world}",
         "l2": L2_NOTE,
         "kv_layout": kv_layout,
-        "block_means": "bf16" if means_bf16 else "fp32",
+        "block_means": MEANS_KINDS[means],
         **({"attention": f"token-level top-k, {token_kt} tokens per query head"} if token_kt else {}),
     }
 
@@ -825,7 +855,7 @@ def report(args, rank, world, rec: RankRecord):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded Philox N(0,1) q/K/V, 5% heavy-hitter key-bias blocks)",
-        "config": workload_config(w0, k, world, rec.kv_layout, args.means_bf16, rec.token_kt),
+        "config": workload_config(w0, k, world, rec.kv_layout, means_kind(args), rec.token_kt),
         "impl": "kin",
         "gpu_launches": rec.launches_per_step * steps,  # in the timed region
         "kernel_ms": {**avg, **({"update": upd} if rec.upd_ms else {})},
@@ -839,7 +869,7 @@ def report(args, rank, world, rec: RankRecord):
             "traffic": profiled_traffic(dom_file, w0.name, k),
         },
         "e2e": {"value": e2e_value, "unit": "query-heads/s", **rec.e2e},
-        "eflops": eflops_report(w, k, rec.lens_final, ms_per_step, 2 if args.means_bf16 else 4, rec.token_kt),
+        "eflops": eflops_report(w, k, rec.lens_final, ms_per_step, means_bytes_per_dim(args), rec.token_kt),
         "clocks": clocks,
         "wall_s_timed_region": wall,
         "device_status": int(status),
@@ -948,7 +978,7 @@ def reference_arm(args):
         "ms_per_step": el / args.steps * 1e3, "step_us": step_percentiles(pass_ms),
         "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w, k, int(os.environ.get("WORLD_SIZE", "1"))),
+        "config": workload_config(w, k, int(os.environ.get("WORLD_SIZE", "1")), means=means_kind(args)),
         "step": f"one pass over {smp.n} sampled (batch, kv-head) pairs ({smp.n * w.g} query heads)",
         "impl": "reference",
         "cpu_baseline": {"value": value, "unit": "query-heads/s", "cores": smp.threads, "kind": "oracle",
@@ -974,6 +1004,9 @@ def main(argv=None):
                     help="(batch, kv-head) pairs per reference-arm step (default: the CPU baseline's sample)")
     ap.add_argument("--paged", action="store_true", help="KV cache in a shuffled page pool with a block table")
     ap.add_argument("--means-bf16", action="store_true", help="bf16 block means (the extended calls)")
+    ap.add_argument("--means-fp32", action="store_true",
+                    help="fp32 block means only: the plain select, which scans them in full (the default keeps dual "
+                         "means and returns the same selection from a bf16 copy; see kin.h KIN_MEANS_DUAL)")
     ap.add_argument("--page-order", default="shuffled", choices=["shuffled", "sequential"],
                     help="page pool order for --paged / --shared-prefix")
     ap.add_argument("--shared-prefix", type=int, default=1,

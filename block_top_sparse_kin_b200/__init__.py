@@ -29,9 +29,9 @@ EXPORTED = (
     "kin_block_topk_select_noalloc", "kin_block_means_build_paged", "kin_block_means_update_paged",
     "kin_sparse_decode_attn_paged", "kin_block_means_build_ex", "kin_block_means_update_ex",
     "kin_block_topk_select_ex", "kin_token_topk_workspace_bytes", "kin_token_topk_decode_attn",
-    "kin_block_topk_select_paged",
+    "kin_block_topk_select_paged", "kin_dual_means_bytes",
 )
-KIN_MEANS_F32, KIN_MEANS_BF16 = 0, 1
+KIN_MEANS_F32, KIN_MEANS_BF16, KIN_MEANS_DUAL = 0, 1, 2
 KIN_MEANS_PER_PAGE = 0x100
 NOALLOC_SCRATCH_FLOATS = 1 << 21  # KIN_NOALLOC_SCRATCH_FLOATS in include/kin.h
 
@@ -109,6 +109,8 @@ def load_library(path: str = LIB_PATH):
     lib.kin_token_topk_decode_attn.restype = ctypes.c_int
     lib.kin_block_topk_select_paged.argtypes = [dp, vp, vp, i32, i32, vp, vp, i32, vp, vp, vp, sz, vp, vp]
     lib.kin_block_topk_select_paged.restype = ctypes.c_int
+    lib.kin_dual_means_bytes.argtypes = [dp]
+    lib.kin_dual_means_bytes.restype = sz
     _lib = lib
     return lib
 
@@ -310,10 +312,31 @@ def kin_sparse_decode_attn_paged(dims, q, k_pages, v_pages, block_table, seq_len
 # The means dtype follows the block_means tensor (float32 or bfloat16);
 # block_table None selects the contiguous cache.  See include/kin.h.
 
-def _means(block_means, count=None, name="block_means"):
+def _means(block_means, count=None, name="block_means", dims=None):
+    """The means pointer and its dtype code, from the tensor: float32 rows,
+    bfloat16 rows, or a uint8 buffer of dual means (fp32 rows, their bf16
+    rounding and the row norms: see kin_dual_means_bytes)."""
     if block_means is not None and block_means.dtype == torch.float32:
         return _dev(block_means, name, torch.float32, count=count), KIN_MEANS_F32
+    if block_means is not None and block_means.dtype == torch.uint8:
+        nbytes = kin_dual_means_bytes(dims) if dims is not None else None
+        return _dev(block_means, name, torch.uint8, count=nbytes or None), KIN_MEANS_DUAL
     return _dev(block_means, name, torch.bfloat16, count=count), KIN_MEANS_BF16
+
+
+def kin_dual_means_bytes(dims: kin_dims) -> int:
+    """Bytes of a dual block-means buffer (KIN_MEANS_DUAL) for these dims."""
+    return int(load_library().kin_dual_means_bytes(ctypes.byref(dims)))
+
+
+def alloc_dual_means(dims: kin_dims, device="cuda") -> torch.Tensor:
+    """A dual block-means buffer (uint8, 256-byte aligned as torch allocates),
+    filled by kin_block_means_build_ex / _update_ex and read by
+    kin_block_topk_select_ex."""
+    n = kin_dual_means_bytes(dims)
+    if n == 0:
+        raise KinError(1, "kin_dual_means_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
 def _layout(rows, block_table, c: _Counts):
@@ -330,7 +353,7 @@ def kin_block_means_build_ex(dims, k_rows, seq_lens, block_means, block_table=No
     """per_page: block_means is [num_pages, Hkv, D] (one mean per page; needs block_table)."""
     c = _Counts(dims)
     pages, table, rows = _layout(k_rows, block_table, c)
-    means, dtype = _means(block_means, c.times(pages, c.page_mean) if per_page else c.means)
+    means, dtype = _means(block_means, c.times(pages, c.page_mean) if per_page else c.means, dims=dims)
     dtype |= KIN_MEANS_PER_PAGE if per_page else 0
     rc = load_library().kin_block_means_build_ex(
         ctypes.byref(dims), _dev(k_rows, "k_rows", _BF16, count=rows), pages, table,
@@ -342,7 +365,7 @@ def kin_block_means_update_ex(dims, k_rows, v_rows, block_means, seq_lens, k_new
                               block_table=None, dev_status=None, stream=None, per_page=False):
     c = _Counts(dims)
     pages, table, rows = _layout(k_rows, block_table, c)
-    means, dtype = _means(block_means, c.times(pages, c.page_mean) if per_page else c.means)
+    means, dtype = _means(block_means, c.times(pages, c.page_mean) if per_page else c.means, dims=dims)
     dtype |= KIN_MEANS_PER_PAGE if per_page else 0
     new_rows = c.times(max(int(n_new), 0), c.bkd)
     rc = load_library().kin_block_means_update_ex(
@@ -356,7 +379,7 @@ def kin_block_means_update_ex(dims, k_rows, v_rows, block_means, seq_lens, k_new
 def kin_block_topk_select_ex(dims, q, block_means, seq_lens, k_blocks, sel_idx, sel_cnt, workspace,
                              dev_status=None, stream=None):
     c = _Counts(dims)
-    means, dtype = _means(block_means, c.means)
+    means, dtype = _means(block_means, c.means, dims=dims)
     rc = load_library().kin_block_topk_select_ex(
         ctypes.byref(dims), _dev(q, "q", _BF16, count=c.q), means, dtype,
         _dev(seq_lens, "seq_lens", torch.int32, count=c.lens), int(k_blocks),

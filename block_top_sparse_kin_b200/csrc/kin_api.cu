@@ -130,12 +130,14 @@ cudaError_t ensure_smem_limit(const void* kernel, int slot, size_t bytes) {
   // is read and raised under one lock, so a thread never lowers it under
   // another thread's launch, and the cache (the limit last seen, per slot and
   // device) never exceeds the limit in force.
-  static std::atomic<size_t> done[8][kMaxDevices];
+  // slots in use: 0, 2, 3 and 8, 9, 10 block top-k (256, 512, 1024 threads;
+  // plain and refining), 1 attention, 4 means update, 5 token top-k, 6 token logits
+  static std::atomic<size_t> done[16][kMaxDevices];
   static std::mutex mu;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const bool cached = dev >= 0 && dev < kMaxDevices && slot >= 0 && slot < 8;
+  const bool cached = dev >= 0 && dev < kMaxDevices && slot >= 0 && slot < 16;
   if (cached && done[slot][dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
   std::lock_guard<std::mutex> lock(mu);
   cudaFuncAttributes attr;
@@ -171,11 +173,17 @@ KIN_EXPORT size_t kin_workspace_bytes(const kin_dims* dims, int32_t k_blocks) {
   return ws_layout(*dims, k_blocks).total;
 }
 
+KIN_EXPORT size_t kin_dual_means_bytes(const kin_dims* dims) {
+  if (check_dims(dims) != KIN_OK) return 0;
+  const int64_t rows = (int64_t)dims->batch * dims->num_kv_heads * nbcap_of(*dims);
+  return (size_t)rows * (kHeadDim * 4 + kHeadDim * 2 + 4);
+}
+
 namespace {
 
 kin_status means_build(const kin_dims* dims, const void* k_rows, const PageTable& pt, const int32_t* seq_lens,
                        void* block_means, int means_bf16, int32_t* dev_status, void* stream, int per_page = 0) {
-  MeansBuildParams p;
+  MeansBuildParams p{};  // every field not set below is zero or null
   p.means_per_page = per_page;
   p.k_cache = static_cast<const __nv_bfloat16*>(k_rows);
   p.seq_lens = seq_lens;
@@ -188,13 +196,14 @@ kin_status means_build(const kin_dims* dims, const void* k_rows, const PageTable
   p.Lcap = dims->max_seq_len;
   p.bs = dims->block_size;
   p.nbcap = nbcap_of(*dims);
+  p.mean_rows = (int64_t)p.B * p.Hkv * p.nbcap;
   return from_cuda(launch_means_build(p, static_cast<cudaStream_t>(stream)));
 }
 
 kin_status means_update(const kin_dims* dims, void* k_rows, void* v_rows, const PageTable& pt,
                         void* block_means, int means_bf16, int32_t* seq_lens, const void* k_new,
                         const void* v_new, int32_t n_new, int32_t* dev_status, void* stream, int per_page = 0) {
-  MeansUpdateParams p;
+  MeansUpdateParams p{};
   p.means_per_page = per_page;
   p.k_cache = static_cast<__nv_bfloat16*>(k_rows);
   p.v_cache = static_cast<__nv_bfloat16*>(v_rows);
@@ -210,6 +219,7 @@ kin_status means_update(const kin_dims* dims, void* k_rows, void* v_rows, const 
   p.Lcap = dims->max_seq_len;
   p.bs = dims->block_size;
   p.nbcap = nbcap_of(*dims);
+  p.mean_rows = (int64_t)p.B * p.Hkv * p.nbcap;
   p.n_new = n_new;
   return from_cuda(launch_means_update(p, static_cast<cudaStream_t>(stream)));
 }
@@ -302,10 +312,22 @@ kin_status topk_select(const kin_dims* dims, const void* q, const void* block_me
   kin_status st = check_ws(*dims, k_blocks, workspace, ws_bytes, &w);
   if (st != KIN_OK) return st;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  SelectParams p;
+  SelectParams p{};
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.means = block_means;
   p.means_bf16 = means_bf16;
+  p.refine = 0;
+  p.means_f32 = nullptr;
+  p.norms = nullptr;
+  if (means_bf16 == 2) {  // dual: scan the bf16 rows, rescore from the fp32 rows
+    const int64_t rows = (int64_t)dims->batch * dims->num_kv_heads * nbcap_of(*dims);
+    const float* f = static_cast<const float*>(block_means);
+    p.means = f + rows * kHeadDim;
+    p.means_bf16 = 1;
+    p.refine = 1;
+    p.means_f32 = f;
+    p.norms = f + rows * (kHeadDim + kHeadDim / 2);
+  }
   p.mpages = mpages ? *mpages : contiguous();
   p.seq_lens = seq_lens;
   p.sel_idx = sel_idx;
@@ -324,9 +346,11 @@ kin_status topk_select(const kin_dims* dims, const void* q, const void* block_me
   return from_cuda(launch_select(p, static_cast<cudaStream_t>(stream)));
 }
 
-// means_dtype as a kernel flag (0 fp32, 1 bf16); -1 for an unknown value
+// means_dtype as a kernel flag (0 fp32, 1 bf16, 2 dual); -1 for an unknown
+// value or for dual means stored per page (dual means are logical only)
 int means_flag(int32_t means_dtype) {
   const int32_t t = means_dtype & ~KIN_MEANS_PER_PAGE;
+  if (t == KIN_MEANS_DUAL) return (means_dtype & KIN_MEANS_PER_PAGE) ? -1 : 2;
   return t == KIN_MEANS_F32 ? 0 : t == KIN_MEANS_BF16 ? 1 : -1;
 }
 int per_page_flag(int32_t means_dtype) { return (means_dtype & KIN_MEANS_PER_PAGE) ? 1 : 0; }
@@ -377,7 +401,7 @@ KIN_EXPORT kin_status kin_block_topk_select_paged(const kin_dims* dims, const vo
   kin_status st = check_dims(dims);
   if (st != KIN_OK) return st;
   const int bf = means_flag(means_dtype);
-  if (bf < 0) return KIN_ERR_INVALID_ARG;
+  if (bf < 0 || bf == 2) return KIN_ERR_INVALID_ARG;  // per-page means are fp32 or bf16
   PageTable pt;
   st = check_pages(*dims, page_means, num_pages, block_table, &pt);
   if (st != KIN_OK) return st;
@@ -441,7 +465,7 @@ kin_status sparse_decode_attn(const kin_dims* dims, const void* q, const void* k
   kin_status st = check_ws(*dims, k_blocks, workspace, ws_bytes, &w);
   if (st != KIN_OK) return st;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  AttnParams p;
+  AttnParams p{};
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k_cache = static_cast<const __nv_bfloat16*>(k_rows);
   p.v_cache = static_cast<const __nv_bfloat16*>(v_rows);
@@ -550,7 +574,7 @@ KIN_EXPORT kin_status kin_token_topk_decode_attn(const kin_dims* dims, const voi
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0 || ws_bytes < w.total)
     return KIN_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  TokenParams p;
+  TokenParams p{};
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
   p.v_cache = static_cast<const __nv_bfloat16*>(v_cache);

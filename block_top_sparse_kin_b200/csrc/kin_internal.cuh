@@ -175,6 +175,36 @@ __device__ __forceinline__ void store_mean_row(void* means, int means_bf16, int6
   }
 }
 
+// Dual block means (KIN_MEANS_DUAL; kernel flag 2): one buffer holding the
+// fp32 rows [rows][D], then the same means rounded to bf16 [rows][D], then
+// each row's Euclidean norm [rows] (fp32), rows = the logical mean rows.
+// A select scans the bf16 rows and rescores from the fp32 rows only the
+// blocks its error bound (which uses the norms) cannot place.  Warp-wide:
+// lane l holds dims 4l..4l+3 of the row.
+__device__ __forceinline__ void store_mean_row_dual(void* means, int64_t rows, int64_t row, int lane, float4 m) {
+  float* f = reinterpret_cast<float*>(means);
+  reinterpret_cast<float4*>(f)[row * (kHeadDim / 4) + lane] = m;
+  uint2 v;
+  v.x = pack_bf16x2(m.x, m.y);
+  v.y = pack_bf16x2(m.z, m.w);
+  reinterpret_cast<uint2*>(f + rows * kHeadDim)[row * (kHeadDim / 4) + lane] = v;
+  float ss = m.x * m.x;
+  ss = fmaf(m.y, m.y, ss);
+  ss = fmaf(m.z, m.z, ss);
+  ss = fmaf(m.w, m.w, ss);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  if (lane == 0) f[rows * (kHeadDim + kHeadDim / 2) + row] = sqrtf(ss);
+}
+
+// A mean row in the layout the flag names (0 fp32, 1 bf16, 2 dual).
+__device__ __forceinline__ void store_mean(void* means, int flag, int64_t rows, int64_t row, int lane, float4 m) {
+  if (flag == 2)
+    store_mean_row_dual(means, rows, row, lane, m);
+  else
+    store_mean_row(means, flag, row, lane, m);
+}
+
 // Row of block i of pair (b, h) in the block-means array: logical
 // [B][Hkv][nbcap][D], or per page [num_pages][Hkv][D] (means_per_page: the
 // mean of a page's rows, shared by every sequence whose table maps a block
@@ -191,7 +221,8 @@ struct MeansBuildParams {
   const __nv_bfloat16* k_cache;  // contiguous cache or page pool (see PageTable)
   const int32_t* seq_lens;
   void* means;
-  int means_bf16;
+  int means_bf16;              // 0 fp32, 1 bf16, 2 dual
+  int64_t mean_rows;           // rows of the logical layout (the dual layout's stride)
   int means_per_page;            // means [num_pages][Hkv][D] (needs a page table)
   int32_t* dev_status;
   PageTable pages;
@@ -202,7 +233,8 @@ struct MeansUpdateParams {
   __nv_bfloat16* k_cache;
   __nv_bfloat16* v_cache;
   void* means;
-  int means_bf16;
+  int means_bf16;              // 0 fp32, 1 bf16, 2 dual
+  int64_t mean_rows;
   int means_per_page;
   int32_t* seq_lens;
   const __nv_bfloat16* k_new;
@@ -224,6 +256,11 @@ struct SelectParams {
   int32_t* dev_status;
   int B, Hkv, Hq, g, bs, Lcap, nbcap, k;
   float score_scale;
+  // dual means: the scan reads the bf16 rows (means), the top-k rescores
+  // from the fp32 rows the blocks the norms' error bound cannot place
+  int refine;
+  const float* means_f32;  // [B*Hkv][nbcap][D]
+  const float* norms;      // [B*Hkv][nbcap]
 };
 
 struct AttnParams {

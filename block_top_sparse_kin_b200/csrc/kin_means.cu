@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(256) means_build_kernel(MeansBuildParams p) {
   float4 m = make_float4(__fdiv_rn(acc[0], n), __fdiv_rn(acc[1], n), __fdiv_rn(acc[2], n),
                          __fdiv_rn(acc[3], n));
   const int64_t mrow = means_row_index(p.pages, p.means_per_page, b, h, p.Hkv, p.nbcap, i);
-  if (mrow >= 0) store_mean_row(p.means, p.means_bf16, mrow, lane, m);
+  if (mrow >= 0) store_mean(p.means, p.means_bf16, p.mean_rows, mrow, lane, m);
 }
 
 // grid (B), 256 threads.  One CTA owns a whole sequence so that the length
@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(kUpdThreads) means_update_kernel(MeansUpdatePa
     float4 m = make_float4(__fdiv_rn(acc[0], cnt), __fdiv_rn(acc[1], cnt), __fdiv_rn(acc[2], cnt),
                            __fdiv_rn(acc[3], cnt));
     const int64_t mrow = means_row_index(p.pages, p.means_per_page, b, h, p.Hkv, p.nbcap, i);
-    if (mrow >= 0) store_mean_row(p.means, p.means_bf16, mrow, lane, m);
+    if (mrow >= 0) store_mean(p.means, p.means_bf16, p.mean_rows, mrow, lane, m);
   }
   __syncthreads();
   if (threadIdx.x == 0) p.seq_lens[b] = L1;

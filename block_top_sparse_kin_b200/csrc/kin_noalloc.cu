@@ -73,10 +73,13 @@ KIN_EXPORT kin_status kin_block_topk_select_noalloc(const kin_dims* dims, const 
   float* scratch = scratch_on_current_device(&err);
   if (!scratch) return KIN_ERR_CUDA;
 
-  SelectParams p;
+  SelectParams p{};
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.means = block_means;
   p.means_bf16 = 0;
+  p.refine = 0;  // fp32 means: the plain select (no dual-means refinement)
+  p.means_f32 = nullptr;
+  p.norms = nullptr;
   p.mpages.table = nullptr;  // logical means
   p.mpages.max_blocks = 0;
   p.mpages.num_pages = 0;

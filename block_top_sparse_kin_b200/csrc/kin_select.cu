@@ -1155,10 +1155,191 @@ __global__ void __launch_bounds__(kSelThreads, KIN_SEL_CTAS_PER_SM) select_scan_
 }
 
 
+// ---- dual means: before the exact top-k, make the pair's score row decide
+// exactly.  The scan left s~_i, block i's score from its bf16 mean.  Rounding
+// to bf16 moves each mean element by at most 2^-8 relative, and the fp32
+// arithmetic of either score adds well under 2^-16 relative of the sum of
+// |q||m|, so (Cauchy-Schwarz, 2^-8 of margin, and 2^-119 for subnormal means)
+//   |s~_i - s_i| <= e_i = 2^-8 (1 + 2^-8) scale |q_group|_2 (|m_i|_2 + 2^-119),
+// s_i being the score the fp32 scan computes from the fp32 mean.  With lower
+// and upper bounds l_i = s~_i - e_i, u_i = s~_i + e_i over the candidates:
+//  * T_L <= the kr-th largest l (the lower edge of the bin below the one
+//    that holds it): a candidate with u < T_L has kr candidates strictly
+//    above it and is out;
+//  * T_U >= the kr-th largest u (the upper edge of the bin above the one
+//    that holds it): a candidate with l > T_U has at most kr - 1 candidates
+//    (itself included) that could reach it, so it is in;
+//  * the rest, a narrow band around the boundary, is rescored from the fp32
+//    rows with the fp32 scan's own arithmetic (the same per-lane fma chain;
+//    the same pairing tree, xor 16, 8, 4, 2, 1, which a plain butterfly
+//    reproduces exactly since addition is commutative).
+// The row then holds the band's exact scores, a value above all of them for
+// the candidates that are in and below all of them for those that are out,
+// and the exact top-k that follows returns the fp32 selection bit for bit.
+// Four barriers: bound ranges, histograms, the listing, the rescoring.
+template <int NT>
+__device__ __forceinline__ void refine_scores(const SelectParams& p, int64_t pair, float* row, const Cands& cd,
+                                              TopkSmem<NT>& sm) {
+  constexpr int NW = NT / 32;
+  // candidates per thread: at most 8 below 4096 blocks (256 or 512
+  // threads), 32 at 1024 threads (32768 blocks); beyond, every candidate is
+  // rescored
+  constexpr int kMaxIt = 32;
+  const float kInf = __int_as_float(0x7f800000);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float qs[4];
+  pair_qsum(p, (int)pair, lane, qs);  // the fp32 scan's summed query, lane's 4 dims
+  float qq = qs[0] * qs[0];
+  qq = fmaf(qs[1], qs[1], qq);
+  qq = fmaf(qs[2], qs[2], qq);
+  qq = fmaf(qs[3], qs[3], qq);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) qq += __shfl_xor_sync(0xffffffffu, qq, off);
+  const float escale = __fmul_ru(__fmul_ru(__fsqrt_ru(qq), p.score_scale), 0x1.01p-8f);
+  const float* nrm = p.norms + pair * p.nbcap;
+  auto err = [&](int i) { return __fmul_ru(escale, __fadd_ru(__ldg(nrm + i), 0x1p-119f)); };
+  auto block_min = [&](float v, uint32_t* slots) {  // all threads; slots[NW]
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, off));
+    if (lane == 0) slots[warp] = __float_as_uint(v);
+  };
+  auto block_max = [&](float v, uint32_t* slots) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+    if (lane == 0) slots[warp] = __float_as_uint(v);
+  };
+  auto fold_min = [&](const uint32_t* slots) {
+    float v = __uint_as_float(slots[0]);
+#pragma unroll
+    for (int w = 1; w < NW; ++w) v = fminf(v, __uint_as_float(slots[w]));
+    return v;
+  };
+  auto fold_max = [&](const uint32_t* slots) {
+    float v = __uint_as_float(slots[0]);
+#pragma unroll
+    for (int w = 1; w < NW; ++w) v = fmaxf(v, __uint_as_float(slots[w]));
+    return v;
+  };
+  uint32_t* slot_a = sm.wmin;
+  uint32_t* slot_b = sm.wmax;
+  uint32_t* slot_c = reinterpret_cast<uint32_t*>(sm.warp_cnt[0]);
+  uint32_t* slot_d = reinterpret_cast<uint32_t*>(sm.warp_cnt[1]);
+
+  // 1. ranges of the lower and the upper bounds, and the largest error
+  float l0 = kInf, l1 = -kInf, u0 = kInf, u1 = -kInf, emax = 0.f;
+  for (int i = cd.lo + tid; i <= cd.hi; i += NT) {
+    const float e = err(i), sv = row[i];
+    const float l = __fsub_rd(sv, e), u = __fadd_ru(sv, e);
+    l0 = fminf(l0, l);
+    l1 = fmaxf(l1, l);
+    u0 = fminf(u0, u);
+    u1 = fmaxf(u1, u);
+    emax = fmaxf(emax, e);
+  }
+  block_min(l0, slot_a);
+  block_max(l1, slot_b);
+  block_min(u0, slot_c);
+  block_max(u1, slot_d);
+  block_max(emax, reinterpret_cast<uint32_t*>(sm.slot_cnt));
+  zero_hist(sm, 0);
+  zero_hist(sm, 1);
+  if (tid == 0) sm.list_n = 0;
+  __syncthreads();
+  const float lmin = fold_min(slot_a), lmax = fold_max(slot_b), umin = fold_min(slot_c), umax = fold_max(slot_d);
+  const float emx = fold_max(reinterpret_cast<const uint32_t*>(sm.slot_cnt));
+  const float lr = lmax - lmin, li = 256.f / lr, ur = umax - umin, ui = 256.f / ur;
+  const bool lbin = isfinite(lmin) && isfinite(lmax) && lr > 0.f && isfinite(lr) && isfinite(li);
+  const bool ubin = isfinite(umin) && isfinite(umax) && ur > 0.f && isfinite(ur) && isfinite(ui);
+  auto lbin_of = [&](float l) { return min((int)((l - lmin) * li), 255); };
+  auto ubin_of = [&](float u) { return min((int)((u - umin) * ui), 255); };
+
+  // 2. T_L and T_U from bin edges, one bin wider than the bins found: the
+  //    bin function is monotone and computed to a few ulps, so every bound
+  //    in bin b lies within [lmin + (b - 1) w, lmin + (b + 2) w) (w: the
+  //    bin width); every candidate undecided when the bounds do not spread
+  float TL = -kInf, TU = kInf;
+  if (lbin || ubin) {
+    for (int i = cd.lo + tid; i <= cd.hi; i += NT) {
+      const float e = err(i), sv = row[i];
+      if (lbin) atomicAdd(&sm.hist[0][hidx(lbin_of(__fsub_rd(sv, e)))], 1);
+      if (ubin) atomicAdd(&sm.hist[1][hidx(ubin_of(__fadd_ru(sv, e)))], 1);
+    }
+    __syncthreads();
+    int bl, bu, above, c;
+    if (lbin) {
+      warp_find_bin(sm.hist[0], cd.kr, bl, above, c);  // every warp, same result
+      if (bl >= 1) TL = __fadd_rd(lmin, __fmul_rd((float)(bl - 1), __fdiv_rd(lr, 256.f)));
+    }
+    if (ubin) {
+      warp_find_bin(sm.hist[1], cd.kr, bu, above, c);
+      if (bu <= 253) TU = __fadd_ru(umin, __fmul_ru((float)(bu + 2), __fdiv_ru(ur, 256.f)));
+    }
+  }
+  // a rescored score lies within [T_L - 2 emax, T_U + 2 emax] (to a few ulps,
+  // far below emax): the decided candidates go outside [T_L - 3 emax,
+  // T_U + 3 emax]
+  const float below_all = nextafterf(__fsub_rd(TL, __fmul_ru(3.f, emx)), -kInf);
+  const float above_all = nextafterf(__fadd_ru(TU, __fmul_ru(3.f, emx)), kInf);
+  const bool bracketed = isfinite(below_all) && isfinite(above_all);
+
+  // 3. in (l > T_U), out (u < T_L), or undecided: listed, one reservation per
+  //    warp; the decided ones written now
+  const bool fits = bracketed && cd.hi - cd.lo + 1 <= kMaxIt * NT;
+  for (int j = 0, i = cd.lo + tid; fits && j < kMaxIt; ++j, i += NT) {
+    bool open = false;
+    if (i <= cd.hi) {
+      const float e = err(i), sv = row[i];
+      if (__fsub_rd(sv, e) > TU)
+        row[i] = above_all;
+      else if (__fadd_ru(sv, e) < TL)
+        row[i] = below_all;
+      else
+        open = true;
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, open);
+    if (m) {
+      int slot = 0;
+      if (lane == 0) slot = atomicAdd(&sm.list_n, __popc(m));
+      slot = __shfl_sync(0xffffffffu, slot, 0) + __popc(m & ((1u << lane) - 1u));
+      if (open && slot < kListCap) sm.list[slot] = (uint32_t)i;
+    }
+    if (__all_sync(0xffffffffu, i + NT > cd.hi)) break;
+  }
+  __syncthreads();
+  const int nlist = sm.list_n;
+  // too many to list, or no finite bracket: rescore every candidate (the
+  // decided ones then get their exact scores back, which is as good)
+  const bool all = !fits || nlist > kListCap;
+  const int n = all ? cd.hi - cd.lo + 1 : nlist;
+
+  // 4. rescore them from the fp32 rows, 4 rows in flight per warp
+  const float4* f32 = reinterpret_cast<const float4*>(p.means_f32 + pair * p.nbcap * kHeadDim) + lane;
+  for (int e0 = warp * 4; e0 < n; e0 += NW * 4) {
+    int idx[4];
+    float4 m[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      idx[r] = e0 + r < n ? (all ? cd.lo + e0 + r : (int)sm.list[e0 + r]) : -1;
+      m[r] = idx[r] >= 0 ? __ldg(f32 + (int64_t)idx[r] * (kHeadDim / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      float d = qs[0] * m[r].x;
+      d = fmaf(qs[1], m[r].y, d);
+      d = fmaf(qs[2], m[r].z, d);
+      d = fmaf(qs[3], m[r].w, d);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+      if (idx[r] >= 0 && lane == 0) row[idx[r]] = d * p.score_scale;
+    }
+  }
+  __syncthreads();  // the row is final before the top-k reads it
+}
+
 // ---- kernel 2: one CTA of NT threads per pair: dense shortcut, bad-length
 // flag, or the exact top-k over the scores the scan left in workspace
 // (L2-resident), in registers when nb <= 8 NT.
-template <int NT>
+template <int NT, bool kRefine>
 __global__ void __launch_bounds__(NT, 1024 / NT) select_topk_kernel(SelectParams p) {
   extern __shared__ uint32_t skey[];  // [nbcap] keys (rows beyond 8 NT blocks: then nbcap bytes of bins)
   __shared__ TopkSmem<NT> sm;
@@ -1186,6 +1367,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_topk_kernel(SelectParams
   }
   const uint32_t* row = reinterpret_cast<const uint32_t*>(p.scores + pair * p.nbcap);
   const Cands cd{1, nb - 2, k - 2};  // blocks 0 and nb - 1 forced
+  if constexpr (kRefine) refine_scores<NT>(p, pair, p.scores + pair * p.nbcap, cd, sm);
   if (nb <= 4 * NT) topk_regs<NT, 4>(row, nb, cd, k, sel, skey, sm, p.dev_status);
   else if (nb <= 8 * NT) topk_regs<NT, 8>(row, nb, cd, k, sel, skey, sm, p.dev_status);
   else topk_memory<NT>(row, nb, cd, k, sel, skey, p.nbcap, const_cast<uint32_t*>(row), sm, p.dev_status);
@@ -1252,12 +1434,20 @@ template <int NT>
 cudaError_t launch_topk(const SelectParams& p, cudaStream_t s) {
   // keys (when they do not fit in registers: then also their bins)
   const size_t smem = (size_t)p.nbcap * sizeof(uint32_t) + (p.nbcap > 8 * NT ? ((size_t)p.nbcap + 3) & ~size_t(3) : 0);
+  if (p.refine) {
+    if (smem > 16 * 1024) {
+      cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(select_topk_kernel<NT, true>),
+                                        NT == 256 ? 8 : NT == 512 ? 9 : 10, smem);
+      if (e != cudaSuccess) return e;
+    }
+    return launch_pdl(select_topk_kernel<NT, true>, dim3(p.B * p.Hkv), dim3(NT), smem, s, p);
+  }
   if (smem > 16 * 1024) {
-    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(select_topk_kernel<NT>),
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(select_topk_kernel<NT, false>),
                                       NT == 256 ? 0 : NT == 512 ? 2 : 3, smem);
     if (e != cudaSuccess) return e;
   }
-  return launch_pdl(select_topk_kernel<NT>, dim3(p.B * p.Hkv), dim3(NT), smem, s, p);
+  return launch_pdl(select_topk_kernel<NT, false>, dim3(p.B * p.Hkv), dim3(NT), smem, s, p);
 }
 
 // The selection when the budget covers every block of every sequence the

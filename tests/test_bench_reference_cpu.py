@@ -35,7 +35,7 @@ def test_reference_arm_prints_the_contract_line():
     # its time follows from the rate; the claimed time fits inside the run
     assert "2 sampled" in d["step"]
     import bench
-    assert d["config"] == bench.workload_config(bench.ki.WORKLOADS["qwen3_8b_32k"], 256, 1)
+    assert d["config"] == bench.workload_config(bench.ki.WORKLOADS["qwen3_8b_32k"], 256, 1, means="dual")
     assert abs(d["ms_per_step"] - 2 * 4 / d["value"] * 1e3) < 1e-6 * d["ms_per_step"]
     assert d["steps"] * d["ms_per_step"] / 1e3 <= d["wall_s"]
     p = d["step_us"]
