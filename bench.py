@@ -155,18 +155,32 @@ def kernel_source_digest(name: str) -> str:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def profiled_traffic(kernel_file: str, workload: str, k: int):
+def traffic_key(kernel_file: str, args) -> str:
+    """The key a kernel family's captured traffic is stored under: the source
+    file, plus the block-means kind for the select (fp32, bf16 and dual means
+    move different bytes) and the KV layout when it is not the contiguous one
+    (a paged or shared-prefix run has no capture of its own, so no figure)."""
+    key = kernel_file
+    if kernel_file == "kin_select.cu":
+        key += "@" + means_kind(args)
+    if getattr(args, "paged", False) or getattr(args, "shared_prefix", 1) > 1:
+        key += "@paged"
+    return key
+
+
+def profiled_traffic(kernel_key: str, workload: str, k: int):
     """DRAM bytes per launch from a committed ncu summary, if it matches the
-    current kernel source (profiles/traffic.txt: file workload k sha bytes)."""
+    current kernel source (profiles/traffic.txt: key workload k sha bytes; the
+    key is the source file with the qualifiers traffic_key adds)."""
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(path):
         return None
-    digest = kernel_source_digest(kernel_file)
+    digest = kernel_source_digest(kernel_key.split("@")[0])
     with open(path) as f:
         for line in f:
             parts = line.split()
             if len(parts) == 5 and not line.startswith("#"):
-                if parts[0] == kernel_file and parts[1] == workload and int(parts[2]) == k and parts[3] == digest:
+                if parts[0] == kernel_key and parts[1] == workload and int(parts[2]) == k and parts[3] == digest:
                     return int(float(parts[4]))
     return None
 
@@ -602,18 +616,18 @@ def measure_rank(args, rank, world, local) -> RankRecord:
     def ext_events(n):
         return [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n)]
 
-    # the step's kernel families: (name, call, algorithmic bytes, source file)
+    # the step's kernel families: (name, call, algorithmic bytes, traffic key)
     means_bytes = means_bytes_per_dim(args)
     if args.token_topk:
         parts = [("token_topk_attn", lambda: token_step(st),
-                  token_algorithmic_bytes(w, st["token_kt"], st["lens_final"]), "kin_token.cu")]
+                  token_algorithmic_bytes(w, st["token_kt"], st["lens_final"]), traffic_key("kin_token.cu", args))]
     else:
         if args.shared_prefix > 1:  # shared items counted once (the step's selection, from warm-up)
             sel_b, attn_b = shared_algorithmic_bytes(w, k, st, means_bytes)
         else:
             sel_b, attn_b = algorithmic_bytes(w, k, st["lens_final"], means_bytes)
-        parts = [("select", lambda: select(st), sel_b, "kin_select.cu"),
-                 ("attn", lambda: attend(st), attn_b, "kin_attn.cu")]
+        parts = [("select", lambda: select(st), sel_b, traffic_key("kin_select.cu", args)),
+                 ("attn", lambda: attend(st), attn_b, traffic_key("kin_attn.cu", args))]
 
     # Per-kernel times for the roofline: a graph per kernel family holding
     # KERNEL_REPEATS back-to-back calls between two events.  The means and the

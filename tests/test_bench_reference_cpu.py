@@ -50,3 +50,26 @@ def test_default_sample_keeps_every_host_thread_busy():
     import bench
     assert bench.sample_pairs_default() >= 2 * (os.cpu_count() or 1)
     assert bench.sample_pairs_default() >= 32
+
+
+def test_traffic_lookup_is_keyed_by_means_kind_and_layout():
+    """A captured traffic figure is reported only for the variant it was
+    captured on: the select's bytes depend on the block-means kind, and a
+    paged or shared-prefix run has no capture of its own."""
+    import argparse
+    import bench
+    base = dict(means_fp32=False, means_bf16=False, paged=False, shared_prefix=1)
+    ns = lambda **kw: argparse.Namespace(**{**base, **kw})
+    assert bench.traffic_key("kin_select.cu", ns()) == "kin_select.cu@dual"
+    assert bench.traffic_key("kin_select.cu", ns(means_fp32=True)) == "kin_select.cu@fp32"
+    assert bench.traffic_key("kin_attn.cu", ns()) == "kin_attn.cu"
+    assert bench.traffic_key("kin_attn.cu", ns(paged=True)) == "kin_attn.cu@paged"
+    assert bench.traffic_key("kin_attn.cu", ns(shared_prefix=4)) == "kin_attn.cu@paged"
+    # every line of the table parses, and a line is read only under its own key
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    rows = [l.split() for l in open(path) if l.strip() and not l.startswith("#")]
+    assert rows and all(len(r) == 5 for r in rows)
+    for key, wl, k, digest, nbytes in rows:
+        if digest == bench.kernel_source_digest(key.split("@")[0]):
+            assert bench.profiled_traffic(key, wl, int(k)) == int(float(nbytes))
+            assert bench.profiled_traffic(key + "@paged", wl, int(k)) is None
