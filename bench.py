@@ -414,7 +414,7 @@ def build_device_state(w: ki.Workload, k: int, paged: bool = False, means_bf16: 
     ki.kv_cache_device(w.seed, True, w.B, w.Hkv, w.cap, w.D, w.bs, st["seq"], hh_dev, False, kc)
     ki.kv_cache_device(w.seed, False, w.B, w.Hkv, w.cap, w.D, w.bs, st["seq"], hh_dev, False, vc)
     st["k_cache"], st["v_cache"] = kc, vc
-    if means_dual:  # fp32 means, their bf16 rounding and the row norms in one buffer
+    if means_dual:  # fp32 means, their bf16 rounding and the rows' error radii in one buffer
         st["means"] = kin.alloc_dual_means(dims)
     else:
         st["means"] = torch.zeros((w.B, w.Hkv, w.nbcap, w.D), dtype=torch.bfloat16 if means_bf16 else torch.float32,
@@ -780,7 +780,7 @@ L2_NOTE = ("GPU arm: L2 flushed before every step (256 MiB write + 256 MiB read,
 MEANS_KINDS = {
     "fp32": "fp32",
     "bf16": "bf16",
-    "dual": "dual: the fp32 selection, read from a bf16 copy (fp32 + bf16 means + row norms)",
+    "dual": "dual: the fp32 selection, read from a bf16 copy (fp32 + bf16 means + row error radii)",
 }
 
 
@@ -798,7 +798,7 @@ def means_kind(args) -> str:
 
 def means_bytes_per_dim(args) -> float:
     """Block-mean bytes the select streams per head dim: fp32 4, bf16 2, dual
-    2 + the row norm's 4 bytes spread over the 128 dims (the fp32 rows it
+    2 + the row's 4-byte error radius spread over the 128 dims (the fp32 rows it
     rescores are counted as traffic, not here)."""
     return {"fp32": 4.0, "bf16": 2.0, "dual": 2.0 + 4.0 / 128}[means_kind(args)]
 

@@ -315,7 +315,7 @@ def kin_sparse_decode_attn_paged(dims, q, k_pages, v_pages, block_table, seq_len
 def _means(block_means, count=None, name="block_means", dims=None):
     """The means pointer and its dtype code, from the tensor: float32 rows,
     bfloat16 rows, or a uint8 buffer of dual means (fp32 rows, their bf16
-    rounding and the row norms: see kin_dual_means_bytes)."""
+    rounding and the rows' error radii: see kin_dual_means_bytes)."""
     if block_means is not None and block_means.dtype == torch.float32:
         return _dev(block_means, name, torch.float32, count=count), KIN_MEANS_F32
     if block_means is not None and block_means.dtype == torch.uint8:

@@ -318,7 +318,7 @@ kin_status topk_select(const kin_dims* dims, const void* q, const void* block_me
   p.means_bf16 = means_bf16;
   p.refine = 0;
   p.means_f32 = nullptr;
-  p.norms = nullptr;
+  p.radii = nullptr;
   if (means_bf16 == 2) {  // dual: scan the bf16 rows, rescore from the fp32 rows
     const int64_t rows = (int64_t)dims->batch * dims->num_kv_heads * nbcap_of(*dims);
     const float* f = static_cast<const float*>(block_means);
@@ -326,7 +326,7 @@ kin_status topk_select(const kin_dims* dims, const void* q, const void* block_me
     p.means_bf16 = 1;
     p.refine = 1;
     p.means_f32 = f;
-    p.norms = f + rows * (kHeadDim + kHeadDim / 2);
+    p.radii = f + rows * (kHeadDim + kHeadDim / 2);
   }
   p.mpages = mpages ? *mpages : contiguous();
   p.seq_lens = seq_lens;

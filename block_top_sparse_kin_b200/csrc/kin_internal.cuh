@@ -70,6 +70,10 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 // results; each kernel signals once its own results are written.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// An L2 prefetch hint: moves no data into the program's view of memory, so
+// it may run before pdl_wait (a line that a predecessor later writes is
+// simply fetched again).  The address must lie inside an allocation.
+__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 // Where a kernel lets the next one launch.  griddepcontrol.wait returns
 // only once every prerequisite grid has completed and its memory is visible,
 // so the signal's place never changes results, only overlap: with
@@ -177,10 +181,19 @@ __device__ __forceinline__ void store_mean_row(void* means, int means_bf16, int6
 
 // Dual block means (KIN_MEANS_DUAL; kernel flag 2): one buffer holding the
 // fp32 rows [rows][D], then the same means rounded to bf16 [rows][D], then
-// each row's Euclidean norm [rows] (fp32), rows = the logical mean rows.
-// A select scans the bf16 rows and rescores from the fp32 rows only the
-// blocks its error bound (which uses the norms) cannot place.  Warp-wide:
-// lane l holds dims 4l..4l+3 of the row.
+// each row's error radius [rows] (fp32), rows = the logical mean rows.  A
+// select scans the bf16 rows and rescores from the fp32 rows only the blocks
+// that its error bound cannot place.  The radius of row m with bf16 rounding
+// b (d = m - b, exact in fp32) is an upper bound on
+//   |d|_2 + 2^-19 |m|_2 + 2^-60,
+// rounded up: (1 + 2^-12) |d|_2 + 2^-18 |m|_2 + 2^-59 (the norms' fp32
+// sums of 128 squares are within 2^-20 relative, and underflow of the
+// squares loses less than 2^-60 from a norm).  Warp-wide: lane l holds dims
+// 4l..4l+3 of the row.
+__device__ __forceinline__ float bf16_residual(float x) {
+  return x - __bfloat162float(__float2bfloat16_rn(x));
+}
+
 __device__ __forceinline__ void store_mean_row_dual(void* means, int64_t rows, int64_t row, int lane, float4 m) {
   float* f = reinterpret_cast<float*>(means);
   reinterpret_cast<float4*>(f)[row * (kHeadDim / 4) + lane] = m;
@@ -188,13 +201,24 @@ __device__ __forceinline__ void store_mean_row_dual(void* means, int64_t rows, i
   v.x = pack_bf16x2(m.x, m.y);
   v.y = pack_bf16x2(m.z, m.w);
   reinterpret_cast<uint2*>(f + rows * kHeadDim)[row * (kHeadDim / 4) + lane] = v;
-  float ss = m.x * m.x;
-  ss = fmaf(m.y, m.y, ss);
-  ss = fmaf(m.z, m.z, ss);
-  ss = fmaf(m.w, m.w, ss);
+  const float4 d = make_float4(bf16_residual(m.x), bf16_residual(m.y), bf16_residual(m.z), bf16_residual(m.w));
+  float mm = m.x * m.x, dd = d.x * d.x;
+  mm = fmaf(m.y, m.y, mm);
+  dd = fmaf(d.y, d.y, dd);
+  mm = fmaf(m.z, m.z, mm);
+  dd = fmaf(d.z, d.z, dd);
+  mm = fmaf(m.w, m.w, mm);
+  dd = fmaf(d.w, d.w, dd);
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-  if (lane == 0) f[rows * (kHeadDim + kHeadDim / 2) + row] = sqrtf(ss);
+  for (int off = 16; off > 0; off >>= 1) {
+    mm += __shfl_xor_sync(0xffffffffu, mm, off);
+    dd += __shfl_xor_sync(0xffffffffu, dd, off);
+  }
+  if (lane == 0) {
+    const float rad = __fadd_ru(__fadd_ru(__fmul_ru(__fsqrt_ru(dd), 0x1.001p0f), __fmul_ru(__fsqrt_ru(mm), 0x1p-18f)),
+                                0x1p-59f);
+    f[rows * (kHeadDim + kHeadDim / 2) + row] = rad;
+  }
 }
 
 // A mean row in the layout the flag names (0 fp32, 1 bf16, 2 dual).
@@ -257,10 +281,10 @@ struct SelectParams {
   int B, Hkv, Hq, g, bs, Lcap, nbcap, k;
   float score_scale;
   // dual means: the scan reads the bf16 rows (means), the top-k rescores
-  // from the fp32 rows the blocks the norms' error bound cannot place
+  // from the fp32 rows the blocks that the rows' error radii cannot place
   int refine;
   const float* means_f32;  // [B*Hkv][nbcap][D]
-  const float* norms;      // [B*Hkv][nbcap]
+  const float* radii;      // [B*Hkv][nbcap]
 };
 
 struct AttnParams {

@@ -79,7 +79,7 @@ KIN_EXPORT kin_status kin_block_topk_select_noalloc(const kin_dims* dims, const 
   p.means_bf16 = 0;
   p.refine = 0;  // fp32 means: the plain select (no dual-means refinement)
   p.means_f32 = nullptr;
-  p.norms = nullptr;
+  p.radii = nullptr;
   p.mpages.table = nullptr;  // logical means
   p.mpages.max_blocks = 0;
   p.mpages.num_pages = 0;

@@ -740,33 +740,85 @@ __device__ __forceinline__ void topk_memory(const uint32_t* row, int nb, const C
   select_from_keys(keys, bins, nb, cd, k, kmin, kmax, sel, sm, dev_status);
 }
 
-// The top-k of one pair with nb <= KPT * NT blocks, keys held in registers:
-// thread t owns blocks u * NT + t (u < KPT), so every load and ballot walks
-// the blocks in index order.  Same threshold search as the memory path
-// (equal-width bins; the radix search on a crowded or degenerate range runs
-// from shared memory), and an emit without a second trip through memory:
-// per 32-block slot (u, warp) one ballot pair counts the keys above the
-// threshold (or forced) and the keys equal to it, one barrier publishes the
-// packed counts, every warp scans them, and every thread writes its taken
-// indices at their final positions.
+// The emit of the register path: thread t owns blocks u * NT + t (u < KPT),
+// so every ballot walks the blocks in index order.  Keeps the forced
+// blocks, every candidate whose key is above T, and the first `take`
+// candidates (by index) whose key equals T.  Per 32-block slot (u, warp)
+// one ballot pair counts the keys above the threshold (or forced) and the
+// keys equal to it, one barrier publishes the packed counts, every warp
+// scans them, and every thread writes its taken indices at their final
+// positions.
 template <int NT, int KPT>
-__device__ __forceinline__ void topk_regs(const uint32_t* row, int nb, const Cands& cd, int k, int32_t* sel, uint32_t* skey,
-                                          TopkSmem<NT>& sm, int32_t* dev_status) {
+__device__ __forceinline__ void emit_regs(const uint32_t (&key)[KPT], int nb, const Cands& cd, int k, uint32_t T,
+                                          int take, int32_t* sel, TopkSmem<NT>& sm, int32_t* dev_status) {
   constexpr int NW = NT / 32;
   constexpr int kPerLane = KPT * NW / 32;  // slots per lane in the emit's scan
   static_assert(KPT <= kMaxKPT && kPerLane >= 1 && NW % kPerLane == 0, "slot layout");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  uint32_t key[KPT];
+  // slot s = u * NW + warp covers blocks 32 s .. 32 s + 31, in index order
+  const unsigned lt = (1u << lane) - 1u;
+  auto flags = [&](int u, bool& g, bool& e) {
+    const int i = u * NT + tid;
+    const bool cand = cd.has(i);
+    g = (i < nb && !cand) || (cand && key[u] > T);
+    e = cand && key[u] == T;
+  };
 #pragma unroll
   for (int u = 0; u < KPT; ++u) {
-    const int i = u * NT + tid;
-    key[u] = i < nb ? __ldcg(row + i) : 0u;
+    bool g, e;
+    flags(u, g, e);
+    const unsigned gb = __ballot_sync(0xffffffffu, g), eb = __ballot_sync(0xffffffffu, e);
+    if (lane == 0) sm.slot_cnt[u * NW + warp] = __popc(gb) | (__popc(eb) << 16);
   }
+  __syncthreads();
+  // this warp's slots all sit at offset warp % kPerLane within their owner lane
+  const int jw = warp % kPerLane;
+  int tot = 0, mine = 0;
+#pragma unroll
+  for (int j = 0; j < kPerLane; ++j) {
+    const int v = sm.slot_cnt[lane * kPerLane + j];
+    if (j < jw) mine += v;
+    tot += v;
+  }
+  int inc = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += t;
+  }
+  mine += inc - tot;
+  const int all = __shfl_sync(0xffffffffu, inc, 31);
+#pragma unroll
+  for (int u = 0; u < KPT; ++u) {
+    const int base = __shfl_sync(0xffffffffu, mine, (u * NW + warp) / kPerLane);
+    bool g, e;
+    flags(u, g, e);
+    const unsigned gb = __ballot_sync(0xffffffffu, g), eb = __ballot_sync(0xffffffffu, e);
+    const int gt_before = (base & 0xFFFF) + __popc(gb & lt);
+    const int eq_before = (base >> 16) + __popc(eb & lt);
+    if (g || (e && eq_before < take)) {
+      const int pos = gt_before + min(eq_before, take);
+      if (pos < k) sel[pos] = u * NT + tid;  // never write past the pair's row
+    }
+  }
+  // self-check: exactly k blocks were emitted
+  if (tid == 0 && (all & 0xFFFF) + min(all >> 16, take) != k) set_status(dev_status, KIN_ERR_DEVICE_DATA);
+}
+
+// The threshold search of the register path over keys already in
+// registers (thread t: blocks u * NT + t), then the emit.  Same search as
+// the memory path (equal-width bins; the radix search on a crowded or
+// degenerate range runs from shared memory).  Only the candidates' keys
+// are read.
+template <int NT, int KPT>
+__device__ __forceinline__ void topk_regs_keys(const uint32_t (&key)[KPT], int nb, const Cands& cd, int k, int32_t* sel,
+                                               uint32_t* skey, TopkSmem<NT>& sm, int32_t* dev_status) {
+  constexpr int NW = NT / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t lo = 0xFFFFFFFFu, hi = 0u;
 #pragma unroll
   for (int u = 0; u < KPT; ++u) {
     const int i = u * NT + tid;
-    key[u] = key_of_bits(key[u]);
     if (cd.has(i)) {
       lo = min(lo, key[u]);
       hi = max(hi, key[u]);
@@ -844,54 +896,21 @@ __device__ __forceinline__ void topk_regs(const uint32_t* row, int nb, const Can
     take = sm.thresh_take;
   }
 
-  // ---- emit: slot s = u * NW + warp covers blocks 32 s .. 32 s + 31, in index order
-  const unsigned lt = (1u << lane) - 1u;
-  auto flags = [&](int u, bool& g, bool& e) {
-    const int i = u * NT + tid;
-    const bool cand = cd.has(i);
-    g = (i < nb && !cand) || (cand && key[u] > T);
-    e = cand && key[u] == T;
-  };
+  emit_regs<NT, KPT>(key, nb, cd, k, T, take, sel, sm, dev_status);
+}
+
+// The top-k of one pair with nb <= KPT * NT blocks, keys held in registers:
+// thread t loads blocks u * NT + t (u < KPT) from the score row.
+template <int NT, int KPT>
+__device__ __forceinline__ void topk_regs(const uint32_t* row, int nb, const Cands& cd, int k, int32_t* sel, uint32_t* skey,
+                                          TopkSmem<NT>& sm, int32_t* dev_status) {
+  uint32_t key[KPT];
 #pragma unroll
   for (int u = 0; u < KPT; ++u) {
-    bool g, e;
-    flags(u, g, e);
-    const unsigned gb = __ballot_sync(0xffffffffu, g), eb = __ballot_sync(0xffffffffu, e);
-    if (lane == 0) sm.slot_cnt[u * NW + warp] = __popc(gb) | (__popc(eb) << 16);
+    const int i = u * NT + threadIdx.x;
+    key[u] = i < nb ? key_of_bits(__ldcg(row + i)) : 0u;
   }
-  __syncthreads();
-  // this warp's slots all sit at offset warp % kPerLane within their owner lane
-  const int jw = warp % kPerLane;
-  int tot = 0, mine = 0;
-#pragma unroll
-  for (int j = 0; j < kPerLane; ++j) {
-    const int v = sm.slot_cnt[lane * kPerLane + j];
-    if (j < jw) mine += v;
-    tot += v;
-  }
-  int inc = tot;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int t = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += t;
-  }
-  mine += inc - tot;
-  const int all = __shfl_sync(0xffffffffu, inc, 31);
-#pragma unroll
-  for (int u = 0; u < KPT; ++u) {
-    const int base = __shfl_sync(0xffffffffu, mine, (u * NW + warp) / kPerLane);
-    bool g, e;
-    flags(u, g, e);
-    const unsigned gb = __ballot_sync(0xffffffffu, g), eb = __ballot_sync(0xffffffffu, e);
-    const int gt_before = (base & 0xFFFF) + __popc(gb & lt);
-    const int eq_before = (base >> 16) + __popc(eb & lt);
-    if (g || (e && eq_before < take)) {
-      const int pos = gt_before + min(eq_before, take);
-      if (pos < k) sel[pos] = u * NT + tid;  // never write past the pair's row
-    }
-  }
-  // self-check: exactly k blocks were emitted
-  if (tid == 0 && (all & 0xFFFF) + min(all >> 16, take) != k) set_status(dev_status, KIN_ERR_DEVICE_DATA);
+  topk_regs_keys<NT, KPT>(key, nb, cd, k, sel, skey, sm, dev_status);
 }
 
 // ---- kernel 1: the scan.  Rows are numbered per pair in steps of U
@@ -908,17 +927,26 @@ __device__ __forceinline__ int pair_nb(const SelectParams& p, int pair) {
 }
 
 __device__ __forceinline__ void pair_qsum(const SelectParams& p, int pair, int lane, float (&o)[4]) {
+  // the g query rows read from L2 (ld.global.cg) four at a time, summed in
+  // row order from 0 (the scan's order)
   const int b = pair / p.Hkv, h = pair - b * p.Hkv;
-  const __nv_bfloat16* qg = p.q + ((int64_t)b * p.Hq + (int64_t)h * p.g) * kHeadDim;
+  const uint2* qg = reinterpret_cast<const uint2*>(p.q + ((int64_t)b * p.Hq + (int64_t)h * p.g) * kHeadDim) + lane;
   o[0] = o[1] = o[2] = o[3] = 0.f;
-  for (int j = 0; j < p.g; ++j) {
-    uint2 raw = __ldg(reinterpret_cast<const uint2*>(qg + j * kHeadDim) + lane);
-    float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&raw.x));
-    float2 bb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&raw.y));
-    o[0] += a.x;
-    o[1] += a.y;
-    o[2] += bb.x;
-    o[3] += bb.y;
+  for (int j0 = 0; j0 < p.g; j0 += 4) {
+    uint2 raw[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) raw[j] = j0 + j < p.g ? __ldcg(qg + (j0 + j) * (kHeadDim / 4)) : make_uint2(0u, 0u);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (j0 + j < p.g) {
+        const float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&raw[j].x));
+        const float2 bb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&raw[j].y));
+        o[0] += a.x;
+        o[1] += a.y;
+        o[2] += bb.x;
+        o[3] += bb.y;
+      }
+    }
   }
 }
 
@@ -1156,13 +1184,22 @@ __global__ void __launch_bounds__(kSelThreads, KIN_SEL_CTAS_PER_SM) select_scan_
 
 
 // ---- dual means: before the exact top-k, make the pair's score row decide
-// exactly.  The scan left s~_i, block i's score from its bf16 mean.  Rounding
-// to bf16 moves each mean element by at most 2^-8 relative, and the fp32
-// arithmetic of either score adds well under 2^-16 relative of the sum of
-// |q||m|, so (Cauchy-Schwarz, 2^-8 of margin, and 2^-119 for subnormal means)
-//   |s~_i - s_i| <= e_i = 2^-8 (1 + 2^-8) scale |q_group|_2 (|m_i|_2 + 2^-119),
-// s_i being the score the fp32 scan computes from the fp32 mean.  With lower
-// and upper bounds l_i = s~_i - e_i, u_i = s~_i + e_i over the candidates:
+// exactly.  The scan left s~_i, block i's score from its bf16 mean b_i; s_i
+// is the score the fp32 scan computes from the fp32 mean m_i.  With q the
+// summed query (the same fp32 values on both sides), d_i = m_i - b_i:
+//  * the exact dot products differ by |q . d_i| <= |q|_2 |d_i|_2;
+//  * each fp32 dot product (an fma chain and a pairing tree, depth 9) is
+//    within 9 2^-24 / (1 - 9 2^-24) of sum |q||x|, at most |q|_2 |m_i|_2
+//    (1 + 2^-8) for x = m_i or b_i: 2^-19.8 |q|_2 |m_i|_2 for the two;
+//  * the product with the scale rounds each side once more (2^-23 of it);
+//  * underflow adds at most 2^-141 to a dot product, 2^-149 to a product.
+// The row's stored radius rho_i bounds |d_i|_2 + 2^-19 |m_i|_2 + 2^-60, so
+//   |s~_i - s_i| <= e_i = scale (|q|_2 (1 + 2^-10) + 2^-59) rho_i,
+// computed rounding up (|q|_2's fp32 sum of squares is within 2^-20 of it;
+// the two 2^-59 floors make e_i >= scale 2^-118, above the underflow terms
+// for the select's scale 1/sqrt(128)).
+// With lower and upper bounds l_i = s~_i - e_i, u_i = s~_i + e_i over the
+// candidates:
 //  * T_L <= the kr-th largest l (the lower edge of the bin below the one
 //    that holds it): a candidate with u < T_L has kr candidates strictly
 //    above it and is out;
@@ -1177,6 +1214,100 @@ __global__ void __launch_bounds__(kSelThreads, KIN_SEL_CTAS_PER_SM) select_scan_
 // the candidates that are in and below all of them for those that are out,
 // and the exact top-k that follows returns the fp32 selection bit for bit.
 // Four barriers: bound ranges, histograms, the listing, the rescoring.
+// The error scale of a pair, scale (|q|_2 (1 + 2^-10) + 2^-59) rounding
+// up, from the summed query the scan used (qs: the lane's 4 dims).
+__device__ __forceinline__ float pair_err_scale(const SelectParams& p, const float (&qs)[4]) {
+  float qq = qs[0] * qs[0];
+  qq = fmaf(qs[1], qs[1], qq);
+  qq = fmaf(qs[2], qs[2], qq);
+  qq = fmaf(qs[3], qs[3], qq);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) qq += __shfl_xor_sync(0xffffffffu, qq, off);
+  return __fmul_ru(__fadd_ru(__fmul_ru(__fsqrt_ru(qq), 0x1.004p0f), 0x1p-59f), p.score_scale);
+}
+
+// The warp's minimum / maximum of v into slots[warp] (as float bits), and
+// the fold of NW such slots.
+__device__ __forceinline__ void warp_min_to(float v, uint32_t* slots) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, off));
+  if ((threadIdx.x & 31) == 0) slots[threadIdx.x >> 5] = __float_as_uint(v);
+}
+__device__ __forceinline__ void warp_max_to(float v, uint32_t* slots) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+  if ((threadIdx.x & 31) == 0) slots[threadIdx.x >> 5] = __float_as_uint(v);
+}
+// (every warp folds: lane l reads slot l, then a butterfly)
+template <int NW>
+__device__ __forceinline__ float fold_min(const uint32_t* slots) {
+  const int lane = threadIdx.x & 31;
+  float v = __uint_as_float(slots[lane < NW ? lane : 0]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, off));
+  return v;
+}
+template <int NW>
+__device__ __forceinline__ float fold_max(const uint32_t* slots) {
+  const int lane = threadIdx.x & 31;
+  float v = __uint_as_float(slots[lane < NW ? lane : 0]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+  return v;
+}
+
+// The fp32 scores of n candidates from their fp32 rows, with the fp32
+// scan's own arithmetic: the listed indices list[0..n), or (all) every
+// index lo..lo+n-1.  Four rows in flight per warp; lane 0 hands each
+// result to out(position, index, score).
+template <int NT, typename Out>
+__device__ __forceinline__ void rescore_rows(const SelectParams& p, int64_t pair, const float (&qs)[4], int n, bool all,
+                                             int lo, const uint32_t* list, Out out) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const float4* f32 = reinterpret_cast<const float4*>(p.means_f32 + pair * p.nbcap * kHeadDim) + lane;
+  for (int e0 = warp * 4; e0 < n; e0 += NW * 4) {
+    int idx[4];
+    float4 m[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      idx[r] = e0 + r < n ? (all ? lo + e0 + r : (int)list[e0 + r]) : -1;
+      m[r] = idx[r] >= 0 ? __ldg(f32 + (int64_t)idx[r] * (kHeadDim / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      float d = qs[0] * m[r].x;
+      d = fmaf(qs[1], m[r].y, d);
+      d = fmaf(qs[2], m[r].z, d);
+      d = fmaf(qs[3], m[r].w, d);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+      if (idx[r] >= 0 && lane == 0) out(e0 + r, idx[r], d * p.score_scale);
+    }
+  }
+}
+
+// The bracket of a refinement: T_L and T_U from the histograms of the
+// lower and upper bounds (sm.hist[0], sm.hist[1], when lbin / ubin), one
+// bin wider than the bins found (the bin function is monotone and computed
+// to a few ulps, so every bound in bin b lies within [lo + (b - 1) w,
+// lo + (b + 2) w), w the bin width); -inf / +inf without a histogram.
+__device__ __forceinline__ void bracket_from_hists(const int* hl, const int* hu, int kr, bool lbin, bool ubin,
+                                                   float lmin, float lr, float umin, float ur, float& TL, float& TU) {
+  const float kInf = __int_as_float(0x7f800000);
+  TL = -kInf;
+  TU = kInf;
+  int bl, bu, above, c;
+  if (lbin) {
+    warp_find_bin(hl, kr, bl, above, c);  // every warp, same result
+    if (bl >= 1) TL = __fadd_rd(lmin, __fmul_rd((float)(bl - 1), __fdiv_rd(lr, 256.f)));
+  }
+  if (ubin) {
+    warp_find_bin(hu, kr, bu, above, c);
+    if (bu <= 253) TU = __fadd_ru(umin, __fmul_ru((float)(bu + 2), __fdiv_ru(ur, 256.f)));
+  }
+}
+
 template <int NT>
 __device__ __forceinline__ void refine_scores(const SelectParams& p, int64_t pair, float* row, const Cands& cd,
                                               TopkSmem<NT>& sm) {
@@ -1186,44 +1317,15 @@ __device__ __forceinline__ void refine_scores(const SelectParams& p, int64_t pai
   // rescored
   constexpr int kMaxIt = 32;
   const float kInf = __int_as_float(0x7f800000);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, lane = tid & 31;
   float qs[4];
   pair_qsum(p, (int)pair, lane, qs);  // the fp32 scan's summed query, lane's 4 dims
-  float qq = qs[0] * qs[0];
-  qq = fmaf(qs[1], qs[1], qq);
-  qq = fmaf(qs[2], qs[2], qq);
-  qq = fmaf(qs[3], qs[3], qq);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) qq += __shfl_xor_sync(0xffffffffu, qq, off);
-  const float escale = __fmul_ru(__fmul_ru(__fsqrt_ru(qq), p.score_scale), 0x1.01p-8f);
-  const float* nrm = p.norms + pair * p.nbcap;
-  auto err = [&](int i) { return __fmul_ru(escale, __fadd_ru(__ldg(nrm + i), 0x1p-119f)); };
-  auto block_min = [&](float v, uint32_t* slots) {  // all threads; slots[NW]
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, off));
-    if (lane == 0) slots[warp] = __float_as_uint(v);
-  };
-  auto block_max = [&](float v, uint32_t* slots) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-    if (lane == 0) slots[warp] = __float_as_uint(v);
-  };
-  auto fold_min = [&](const uint32_t* slots) {
-    float v = __uint_as_float(slots[0]);
-#pragma unroll
-    for (int w = 1; w < NW; ++w) v = fminf(v, __uint_as_float(slots[w]));
-    return v;
-  };
-  auto fold_max = [&](const uint32_t* slots) {
-    float v = __uint_as_float(slots[0]);
-#pragma unroll
-    for (int w = 1; w < NW; ++w) v = fmaxf(v, __uint_as_float(slots[w]));
-    return v;
-  };
-  uint32_t* slot_a = sm.wmin;
-  uint32_t* slot_b = sm.wmax;
+  const float escale = pair_err_scale(p, qs);
+  const float* rad = p.radii + pair * p.nbcap;
+  auto err = [&](int i) { return __fmul_ru(escale, __ldg(rad + i)); };
   uint32_t* slot_c = reinterpret_cast<uint32_t*>(sm.warp_cnt[0]);
   uint32_t* slot_d = reinterpret_cast<uint32_t*>(sm.warp_cnt[1]);
+  uint32_t* slot_e = reinterpret_cast<uint32_t*>(sm.slot_cnt);
 
   // 1. ranges of the lower and the upper bounds, and the largest error
   float l0 = kInf, l1 = -kInf, u0 = kInf, u1 = -kInf, emax = 0.f;
@@ -1236,27 +1338,24 @@ __device__ __forceinline__ void refine_scores(const SelectParams& p, int64_t pai
     u1 = fmaxf(u1, u);
     emax = fmaxf(emax, e);
   }
-  block_min(l0, slot_a);
-  block_max(l1, slot_b);
-  block_min(u0, slot_c);
-  block_max(u1, slot_d);
-  block_max(emax, reinterpret_cast<uint32_t*>(sm.slot_cnt));
+  warp_min_to(l0, sm.wmin);
+  warp_max_to(l1, sm.wmax);
+  warp_min_to(u0, slot_c);
+  warp_max_to(u1, slot_d);
+  warp_max_to(emax, slot_e);
   zero_hist(sm, 0);
   zero_hist(sm, 1);
   if (tid == 0) sm.list_n = 0;
   __syncthreads();
-  const float lmin = fold_min(slot_a), lmax = fold_max(slot_b), umin = fold_min(slot_c), umax = fold_max(slot_d);
-  const float emx = fold_max(reinterpret_cast<const uint32_t*>(sm.slot_cnt));
+  const float lmin = fold_min<NW>(sm.wmin), lmax = fold_max<NW>(sm.wmax);
+  const float umin = fold_min<NW>(slot_c), umax = fold_max<NW>(slot_d), emx = fold_max<NW>(slot_e);
   const float lr = lmax - lmin, li = 256.f / lr, ur = umax - umin, ui = 256.f / ur;
   const bool lbin = isfinite(lmin) && isfinite(lmax) && lr > 0.f && isfinite(lr) && isfinite(li);
   const bool ubin = isfinite(umin) && isfinite(umax) && ur > 0.f && isfinite(ur) && isfinite(ui);
   auto lbin_of = [&](float l) { return min((int)((l - lmin) * li), 255); };
   auto ubin_of = [&](float u) { return min((int)((u - umin) * ui), 255); };
 
-  // 2. T_L and T_U from bin edges, one bin wider than the bins found: the
-  //    bin function is monotone and computed to a few ulps, so every bound
-  //    in bin b lies within [lmin + (b - 1) w, lmin + (b + 2) w) (w: the
-  //    bin width); every candidate undecided when the bounds do not spread
+  // 2. T_L and T_U; every candidate undecided when the bounds do not spread
   float TL = -kInf, TU = kInf;
   if (lbin || ubin) {
     for (int i = cd.lo + tid; i <= cd.hi; i += NT) {
@@ -1265,15 +1364,7 @@ __device__ __forceinline__ void refine_scores(const SelectParams& p, int64_t pai
       if (ubin) atomicAdd(&sm.hist[1][hidx(ubin_of(__fadd_ru(sv, e)))], 1);
     }
     __syncthreads();
-    int bl, bu, above, c;
-    if (lbin) {
-      warp_find_bin(sm.hist[0], cd.kr, bl, above, c);  // every warp, same result
-      if (bl >= 1) TL = __fadd_rd(lmin, __fmul_rd((float)(bl - 1), __fdiv_rd(lr, 256.f)));
-    }
-    if (ubin) {
-      warp_find_bin(sm.hist[1], cd.kr, bu, above, c);
-      if (bu <= 253) TU = __fadd_ru(umin, __fmul_ru((float)(bu + 2), __fdiv_ru(ur, 256.f)));
-    }
+    bracket_from_hists(sm.hist[0], sm.hist[1], cd.kr, lbin, ubin, lmin, lr, umin, ur, TL, TU);
   }
   // a rescored score lies within [T_L - 2 emax, T_U + 2 emax] (to a few ulps,
   // far below emax): the decided candidates go outside [T_L - 3 emax,
@@ -1310,30 +1401,172 @@ __device__ __forceinline__ void refine_scores(const SelectParams& p, int64_t pai
   // too many to list, or no finite bracket: rescore every candidate (the
   // decided ones then get their exact scores back, which is as good)
   const bool all = !fits || nlist > kListCap;
-  const int n = all ? cd.hi - cd.lo + 1 : nlist;
 
-  // 4. rescore them from the fp32 rows, 4 rows in flight per warp
-  const float4* f32 = reinterpret_cast<const float4*>(p.means_f32 + pair * p.nbcap * kHeadDim) + lane;
-  for (int e0 = warp * 4; e0 < n; e0 += NW * 4) {
-    int idx[4];
-    float4 m[4];
+  // 4. rescore them from the fp32 rows
+  rescore_rows<NT>(p, pair, qs, all ? cd.hi - cd.lo + 1 : nlist, all, cd.lo, sm.list,
+                   [&](int, int i, float v) { row[i] = v; });
+  __syncthreads();  // the row is final before the top-k reads it
+}
+
+// ---- dual means, register path (nb <= KPT NT): the refinement above and
+// the exact top-k in one pass over registers.  Every candidate's bf16
+// score and radius is loaded once (thread t: blocks u NT + t, the top-k's
+// own layout); the bounds, the histograms and the in / out / band split
+// run from registers; the band is rescored from the fp32 rows and its exact
+// keys come back through shared memory.  The n_in candidates that are in
+// take n_in of the kr places and lie above every band score, so the
+// threshold is the (kr - n_in)-th largest exact key of the band: with at
+// most kRankCap band keys it is found by ranking them pairwise, and the
+// emit follows.  A wider band (or no finite bracket, or a band beyond the
+// list, when every candidate is rescored) goes to the generic search over
+// the refined keys.
+template <int NT, int KPT>
+__device__ __forceinline__ void refine_topk_regs(const SelectParams& p, int64_t pair, int nb, const Cands& cd, int k,
+                                                 int32_t* sel, uint32_t* skey, TopkSmem<NT>& sm) {
+  constexpr int NW = NT / 32;
+  const float kInf = __int_as_float(0x7f800000);
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int kr = cd.kr;
+  if (kr == 0) {  // only the forced blocks are kept
+    pdl_wait();
+    pdl_trigger_early();
+    const uint32_t none[KPT] = {};
+    emit_regs<NT, KPT>(none, nb, cd, k, 0xFFFFFFFFu, 0, sel, sm, p.dev_status);
+    return;
+  }
+  // the radii and the query, before the wait: see select_topk_kernel
+  const float* rad = p.radii + pair * p.nbcap;
+  float ev[KPT];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      idx[r] = e0 + r < n ? (all ? cd.lo + e0 + r : (int)sm.list[e0 + r]) : -1;
-      m[r] = idx[r] >= 0 ? __ldg(f32 + (int64_t)idx[r] * (kHeadDim / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+  for (int u = 0; u < KPT; ++u) {
+    const int i = u * NT + tid;
+    ev[u] = cd.has(i) ? __ldcg(rad + i) : 0.f;
+  }
+  __shared__ float4 qsh[kHeadDim / 4];  // the summed query, for the rescoring
+  float escale;
+  {
+    float qs[4];
+    pair_qsum(p, (int)pair, lane, qs);  // the fp32 scan's summed query, lane's 4 dims
+    escale = pair_err_scale(p, qs);
+    if (tid < 32) qsh[lane] = make_float4(qs[0], qs[1], qs[2], qs[3]);  // read after the next barrier
+  }
+  pdl_wait();  // the scores come from the scan kernel
+  pdl_trigger_early();
+  const float* srow = p.scores + pair * p.nbcap;
+  float sv[KPT];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      float d = qs[0] * m[r].x;
-      d = fmaf(qs[1], m[r].y, d);
-      d = fmaf(qs[2], m[r].z, d);
-      d = fmaf(qs[3], m[r].w, d);
+  for (int u = 0; u < KPT; ++u) {
+    const int i = u * NT + tid;
+    sv[u] = cd.has(i) ? __ldcg(srow + i) : 0.f;
+  }
+  uint32_t* slot_c = reinterpret_cast<uint32_t*>(sm.warp_cnt[0]);
+  uint32_t* slot_d = reinterpret_cast<uint32_t*>(sm.warp_cnt[1]);
+  uint32_t* slot_e = reinterpret_cast<uint32_t*>(sm.slot_cnt);
+
+  // 1. ranges of the lower and the upper bounds, and the largest error
+  float l0 = kInf, l1 = -kInf, u0 = kInf, u1 = -kInf, emax = 0.f;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-      if (idx[r] >= 0 && lane == 0) row[idx[r]] = d * p.score_scale;
+  for (int u = 0; u < KPT; ++u) {
+    ev[u] = __fmul_ru(escale, ev[u]);
+    if (cd.has(u * NT + tid)) {
+      const float l = __fsub_rd(sv[u], ev[u]), h = __fadd_ru(sv[u], ev[u]);
+      l0 = fminf(l0, l);
+      l1 = fmaxf(l1, l);
+      u0 = fminf(u0, h);
+      u1 = fmaxf(u1, h);
+      emax = fmaxf(emax, ev[u]);
     }
   }
-  __syncthreads();  // the row is final before the top-k reads it
+  warp_min_to(l0, sm.wmin);
+  warp_max_to(l1, sm.wmax);
+  warp_min_to(u0, slot_c);
+  warp_max_to(u1, slot_d);
+  warp_max_to(emax, slot_e);
+  zero_hist(sm, 0);
+  zero_hist(sm, 1);
+  if (tid == 0) {
+    sm.list_n = 0;   // band
+    sm.list_n2 = 0;  // in
+  }
+  __syncthreads();
+  const float lmin = fold_min<NW>(sm.wmin), lmax = fold_max<NW>(sm.wmax);
+  const float umin = fold_min<NW>(slot_c), umax = fold_max<NW>(slot_d), emx = fold_max<NW>(slot_e);
+  const float lr = lmax - lmin, li = 256.f / lr, ur = umax - umin, ui = 256.f / ur;
+  const bool lbin = isfinite(lmin) && isfinite(lmax) && lr > 0.f && isfinite(lr) && isfinite(li);
+  const bool ubin = isfinite(umin) && isfinite(umax) && ur > 0.f && isfinite(ur) && isfinite(ui);
+
+  // 2. T_L and T_U (as in refine_scores)
+  float TL = -kInf, TU = kInf;
+  if (lbin || ubin) {
+#pragma unroll
+    for (int u = 0; u < KPT; ++u) {
+      if (cd.has(u * NT + tid)) {
+        if (lbin) atomicAdd(&sm.hist[0][hidx(min((int)((__fsub_rd(sv[u], ev[u]) - lmin) * li), 255))], 1);
+        if (ubin) atomicAdd(&sm.hist[1][hidx(min((int)((__fadd_ru(sv[u], ev[u]) - umin) * ui), 255))], 1);
+      }
+    }
+    __syncthreads();
+    bracket_from_hists(sm.hist[0], sm.hist[1], kr, lbin, ubin, lmin, lr, umin, ur, TL, TU);
+  }
+  const float below_all = nextafterf(__fsub_rd(TL, __fmul_ru(3.f, emx)), -kInf);
+  const float above_all = nextafterf(__fadd_ru(TU, __fmul_ru(3.f, emx)), kInf);
+  const bool bracketed = isfinite(below_all) && isfinite(above_all);
+
+  // 3. in (l > T_U), out (u < T_L), or in the band: band indices listed
+  //    (one reservation per warp), the in ones counted
+  unsigned inm = 0u, bandm = 0u;
+  if (bracketed) {
+#pragma unroll
+    for (int u = 0; u < KPT; ++u) {
+      const int i = u * NT + tid;
+      bool in = false, open = false;
+      if (cd.has(i)) {
+        if (__fsub_rd(sv[u], ev[u]) > TU)
+          in = true;
+        else if (!(__fadd_ru(sv[u], ev[u]) < TL))
+          open = true;
+      }
+      const unsigned mo = __ballot_sync(0xffffffffu, open), mi = __ballot_sync(0xffffffffu, in);
+      if (mo) {
+        int slot = 0;
+        if (lane == 0) slot = atomicAdd(&sm.list_n, __popc(mo));
+        slot = __shfl_sync(0xffffffffu, slot, 0) + __popc(mo & ((1u << lane) - 1u));
+        if (open && slot < kListCap) sm.list[slot] = (uint32_t)i;
+      }
+      if (lane == 0 && mi) atomicAdd(&sm.list_n2, __popc(mi));
+      inm |= (unsigned)in << u;
+      bandm |= (unsigned)open << u;
+    }
+  }
+  __syncthreads();
+  const int nlist = sm.list_n, n_in = sm.list_n2;
+  const bool all = !bracketed || nlist > kListCap;  // then every candidate is rescored
+
+  // 4. the band's (or every candidate's) exact keys, from the fp32 rows
+  const float4 q4 = qsh[lane];
+  const float qs[4] = {q4.x, q4.y, q4.z, q4.w};
+  rescore_rows<NT>(p, pair, qs, all ? cd.hi - cd.lo + 1 : nlist, all, cd.lo, sm.list, [&](int j, int i, float v) {
+    const uint32_t kx = key_of_bits(__float_as_uint(v));
+    skey[i] = kx;
+    if (!all) sm.list[j] = kx;  // the slot this warp just read its index from
+  });
+  __syncthreads();
+  const uint32_t k_in = key_of_bits(__float_as_uint(above_all)), k_out = key_of_bits(__float_as_uint(below_all));
+  uint32_t key[KPT];
+#pragma unroll
+  for (int u = 0; u < KPT; ++u) {
+    const int i = u * NT + tid;
+    key[u] = !cd.has(i) ? 0u : (all || ((bandm >> u) & 1u)) ? skey[i] : ((inm >> u) & 1u) ? k_in : k_out;
+  }
+
+  // 5. the threshold among the band, and the emit
+  const int need = kr - n_in;
+  if (!all && nlist <= kRankCap && need >= 1 && need <= nlist) {
+    rank_keys(0, nlist, need, sm);  // ends with a barrier
+    emit_regs<NT, KPT>(key, nb, cd, k, sm.thresh, sm.thresh_take, sel, sm, p.dev_status);
+  } else {
+    topk_regs_keys<NT, KPT>(key, nb, cd, k, sel, skey, sm, p.dev_status);
+  }
 }
 
 // ---- kernel 2: one CTA of NT threads per pair: dense shortcut, bad-length
@@ -1344,12 +1577,38 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_topk_kernel(SelectParams
   extern __shared__ uint32_t skey[];  // [nbcap] keys (rows beyond 8 NT blocks: then nbcap bytes of bins)
   __shared__ TopkSmem<NT> sm;
   const int tid = threadIdx.x;
-  pdl_wait();  // scores come from the scan kernel
-  pdl_trigger_early();
   const int64_t pair = blockIdx.x;
   const int b = (int)(pair / p.Hkv);
   const int k = p.k;
   int32_t* sel = p.sel_idx + pair * k;
+  if constexpr (kRefine) {
+    // The lengths, the radii and the query are written by work that
+    // completed before the scan's own wait returned (the scan writes only
+    // scores), and this grid starts after every scan CTA passed that wait:
+    // they are read from L2 (ld.global.cg, the point of coherence) before
+    // this grid's wait, while the scan drains.  The register paths wait
+    // inside, before their first score load.
+    const int L = __ldcg(p.seq_lens + b);
+    const int nb = (L >= 1 && L <= p.Lcap) ? (L + p.bs - 1) / p.bs : 0;
+    if (nb > k && nb <= 8 * NT) {
+      const Cands cd{1, nb - 2, k - 2};  // blocks 0 and nb - 1 forced
+      if (nb <= 4 * NT)
+        refine_topk_regs<NT, 4>(p, pair, nb, cd, k, sel, skey, sm);
+      else
+        refine_topk_regs<NT, 8>(p, pair, nb, cd, k, sel, skey, sm);
+      if (tid == 0) p.sel_cnt[pair] = k;
+      return;
+    }
+    if (nb > k) {  // the memory path: warm L2 with this pair's radii and query rows
+      const char* rb = reinterpret_cast<const char*>(p.radii + pair * p.nbcap);
+      for (int t = tid; t < (p.nbcap * 4 + 127) / 128; t += NT) prefetch_l2(rb + t * 128);
+      const int h = (int)(pair - (int64_t)b * p.Hkv);
+      const char* qg = reinterpret_cast<const char*>(p.q + ((int64_t)b * p.Hq + (int64_t)h * p.g) * kHeadDim);
+      if (tid < 2 * p.g) prefetch_l2(qg + tid * 128);  // g rows of 256 bytes
+    }
+  }
+  pdl_wait();  // scores come from the scan kernel
+  pdl_trigger_early();
   const int L = __ldg(p.seq_lens + b);
   if (L < 1 || L > p.Lcap) {
     for (int i = tid; i < k; i += NT) sel[i] = -1;
@@ -1367,10 +1626,16 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_topk_kernel(SelectParams
   }
   const uint32_t* row = reinterpret_cast<const uint32_t*>(p.scores + pair * p.nbcap);
   const Cands cd{1, nb - 2, k - 2};  // blocks 0 and nb - 1 forced
-  if constexpr (kRefine) refine_scores<NT>(p, pair, p.scores + pair * p.nbcap, cd, sm);
-  if (nb <= 4 * NT) topk_regs<NT, 4>(row, nb, cd, k, sel, skey, sm, p.dev_status);
-  else if (nb <= 8 * NT) topk_regs<NT, 8>(row, nb, cd, k, sel, skey, sm, p.dev_status);
-  else topk_memory<NT>(row, nb, cd, k, sel, skey, p.nbcap, const_cast<uint32_t*>(row), sm, p.dev_status);
+  if constexpr (kRefine) {
+    refine_scores<NT>(p, pair, p.scores + pair * p.nbcap, cd, sm);
+    topk_memory<NT>(row, nb, cd, k, sel, skey, p.nbcap, const_cast<uint32_t*>(row), sm, p.dev_status);
+  } else if (nb <= 4 * NT) {
+    topk_regs<NT, 4>(row, nb, cd, k, sel, skey, sm, p.dev_status);
+  } else if (nb <= 8 * NT) {
+    topk_regs<NT, 8>(row, nb, cd, k, sel, skey, sm, p.dev_status);
+  } else {
+    topk_memory<NT>(row, nb, cd, k, sel, skey, p.nbcap, const_cast<uint32_t*>(row), sm, p.dev_status);
+  }
   if (tid == 0) p.sel_cnt[pair] = k;
 }
 

@@ -210,19 +210,22 @@ kin_status kin_sparse_decode_attn_paged(const kin_dims* dims, const void* q, con
 typedef enum { KIN_MEANS_F32 = 0, KIN_MEANS_BF16 = 1, KIN_MEANS_DUAL = 2 } kin_means_dtype;
 /* KIN_MEANS_DUAL: one buffer of kin_dual_means_bytes(dims) bytes (16-byte
  * aligned) holding the fp32 means [B][Hkv][NBcap][D], then the same means
- * rounded to bf16 [B][Hkv][NBcap][D], then each mean row's Euclidean norm
- * [B][Hkv][NBcap] (fp32); the build/update calls write all three.  The
- * select over it returns exactly the selection of the fp32 means (the same
- * indices as kin_block_topk_select on the fp32 part, bit for bit) while it
- * streams the bf16 copy: the scan scores every block from its bf16 mean,
- * each score s~ is within e = 2^-8 (1 + 2^-8) (1/sqrt(D)) |q_group|_2 |m|_2
- * of the fp32 score (bf16 rounding moves a mean element by at most 2^-8
- * relative; the margin covers fp32 rounding), a block whose s~ + e is below
- * the k-th largest s~ - e cannot be kept, one whose s~ - e is above the
- * k-th largest s~ + e is kept, and only the band between is rescored from
- * its fp32 rows with the fp32 scan's own arithmetic before the exact top-k.  Logical layout only: not with KIN_MEANS_PER_PAGE, nor in
- * kin_block_topk_select_paged (KIN_ERR_INVALID_ARG).  Returns 0 for invalid
- * dims. */
+ * rounded to bf16 [B][Hkv][NBcap][D], then each mean row's error radius
+ * [B][Hkv][NBcap] (fp32: an upper bound on |m - bf16(m)|_2 + 2^-19 |m|_2 +
+ * 2^-60 for the row's fp32 mean m); the build/update calls write all three.
+ * The select over it returns exactly the selection of the fp32 means (the
+ * same indices as kin_block_topk_select on the fp32 part, bit for bit)
+ * while it streams the bf16 copy: the scan scores every block from its
+ * bf16 mean, each score s~ is within e = (1/sqrt(D)) |q_group|_2 rho (to a
+ * factor 1 + 2^-10 and an underflow margin) of the fp32 score, rho being
+ * the row's radius (Cauchy-Schwarz on the rounding residual; the 2^-19
+ * |m|_2 term covers the fp32 rounding of both scores), a block whose
+ * s~ + e is below the k-th largest s~ - e cannot be kept, one whose s~ - e
+ * is above the k-th largest s~ + e is kept, and only the band between is
+ * rescored from its fp32 rows with the fp32 scan's own arithmetic before
+ * the exact top-k.  Logical layout only: not with KIN_MEANS_PER_PAGE, nor
+ * in kin_block_topk_select_paged (KIN_ERR_INVALID_ARG).  Returns 0 for
+ * invalid dims. */
 size_t kin_dual_means_bytes(const kin_dims* dims);
 /* OR-ed into means_dtype of the build/update calls (with a block table):
  * block means per page, [num_pages][Hkv][D], read by

@@ -55,7 +55,7 @@ def dims(B=2, Hkv=2, Hq=8, D=128, bs=16, L=256):
 
 
 def test_workspace_bytes(lib):
-    # dual block means: fp32 rows, bf16 rows, one fp32 norm per row
+    # dual block means: fp32 rows, bf16 rows, one fp32 error radius per row
     d = dims()
     rows = d.batch * d.num_kv_heads * -(-d.max_seq_len // d.block_size)
     assert kin.kin_dual_means_bytes(d) == rows * (128 * 4 + 128 * 2 + 4)

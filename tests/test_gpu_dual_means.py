@@ -17,7 +17,7 @@ W = ki.Workload
 
 
 def _parts(dual, dims):
-    """The fp32 rows, bf16 rows and norms of a dual buffer (views)."""
+    """The fp32 rows, bf16 rows and error radii of a dual buffer (views)."""
     rows = dims.batch * dims.num_kv_heads * (-(-dims.max_seq_len // dims.block_size))
     f32 = dual[:rows * D * 4].view(torch.float32).view(rows, D)
     b16 = dual[rows * D * 4:rows * D * 6].view(torch.bfloat16).view(rows, D)
@@ -72,16 +72,23 @@ def _valid_rows(w, dc):
 ], ids=lambda w: w.name)
 def test_dual_layout_build_and_update(w):
     """The fp32 part equals the fp32 means bit for bit, the bf16 part is its
-    round-to-nearest-even bf16 rounding (torch's conversion), the norms are
-    the rows' Euclidean norms; with an append, through the dual update."""
+    round-to-nearest-even bf16 rounding (torch's conversion), and each
+    row's radius bounds |m - bf16(m)|_2 + 2^-19 |m|_2 + 2^-60 from above
+    and exceeds (1 + 2^-12) |m - bf16(m)|_2 + 2^-18 |m|_2 + 2^-59 by no
+    more than fp32 rounding; with an append, through the dual update."""
     a, b, dual = _build_both(w)
-    f32, b16, nrm = _parts(dual, b.dims)
+    f32, b16, rad = _parts(dual, b.dims)
     rows = torch.from_numpy(_valid_rows(w, b)).cuda()
     ref = a.means.view(-1, D)[rows]
     assert torch.equal(f32[rows], ref)
     assert torch.equal(b16[rows], ref.to(torch.bfloat16))
-    want = torch.linalg.vector_norm(ref.double(), dim=-1)
-    assert torch.allclose(nrm[rows].double(), want, rtol=1e-5, atol=0)
+    m = ref.double()
+    dn = torch.linalg.vector_norm(m - ref.to(torch.bfloat16).double(), dim=-1)
+    mn = torch.linalg.vector_norm(m, dim=-1)
+    r = rad[rows].double()
+    assert bool((r >= dn + 2.0 ** -19 * mn + 2.0 ** -60).all())
+    assert bool((r <= ((1 + 2.0 ** -12) * dn + 2.0 ** -18 * mn + 2.0 ** -59) * (1 + 2.0 ** -18)).all())
+    assert bool((dn > 0).any())  # the rounding moved some rows
 
 
 SHAPES = [
@@ -132,6 +139,47 @@ def test_dual_select_with_all_equal_scores(nblocks):
     for r in range(w.B):
         nb = -(-int(b.lens_final[r]) // 16)
         assert list(sb[r, 0]) == list(range(w.k - 1)) + [nb - 1]
+
+
+@pytest.mark.parametrize("nblocks,boosted", [(1024, False), (1024, True), (5000, False)])
+def test_dual_select_with_scores_tied_below_bf16_resolution(nblocks, boosted):
+    """Every block holds the same key rows except one token, moved by a few
+    bf16 ulps in one dim: the fp32 means differ by about 2^-12 relative, far
+    below the bf16 copy's resolution, so the bf16 scores cannot order the
+    blocks and the band is every candidate (listed at 1024 blocks; beyond
+    the list at 5000, so every candidate is rescored).  With `boosted`, a
+    seventh of the blocks are scaled by 1.5: the boundary falls inside that
+    group, whose members are near-tied among themselves, and the rest is out.
+    The dual select must still return the fp32 select's indices."""
+    w = W("dual_subres", 2, 2, 8, D, 16, 0, 0, 40, 94, Lcap=nblocks * 16, lens=(nblocks * 16, nblocks * 16 - 300))
+    a, b = make_device_case(w), make_device_case(w)
+    g = torch.Generator().manual_seed(nblocks + boosted)
+    nb = nblocks
+    kc = torch.randn(w.B, w.Hkv, 1, D, generator=g).to(torch.bfloat16).expand(w.B, w.Hkv, w.cap, D).clone()
+    if boosted:
+        grp = torch.rand(nb, generator=g) < 1 / 7
+        fac = torch.where(grp, 1.5, 1.0).repeat_interleave(16)[:w.cap].view(1, 1, -1, 1)
+        kc = (kc.float() * fac).to(torch.bfloat16)
+    bits = kc.view(torch.int16)
+    dim = torch.randint(0, D, (nb,), generator=g)
+    step = torch.randint(-3, 4, (w.B, w.Hkv, nb), generator=g, dtype=torch.int16)
+    bits[:, :, torch.arange(nb) * 16, dim] += step
+    kc = kc.cuda()
+    for dc in (a, b):
+        dc.k_cache.copy_(kc)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kin.kin_block_means_build(a.dims, a.k_cache, a.seq_lens, a.means, st)
+    dual = kin.alloc_dual_means(b.dims)
+    kin.kin_block_means_build_ex(b.dims, b.k_cache, b.seq_lens, dual, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    sa, ca = _select(a, a.means, w.k)
+    sb, cb = _select(b, dual, w.k)
+    assert np.array_equal(ca, cb) and np.array_equal(sa, sb)
+    # the fp32 means do differ between blocks, below the bf16 copy's resolution
+    f32, b16, _ = _parts(dual, b.dims)
+    assert len(torch.unique(f32.view(w.B, w.Hkv, -1, D)[0, 0, :nb], dim=0)) > 300
+    assert len(torch.unique(b16.view(w.B, w.Hkv, -1, D)[0, 0, :nb], dim=0)) <= 2
 
 
 def test_dual_means_refused_per_page_and_in_the_paged_select():
