@@ -87,6 +87,9 @@ constexpr int kListCap = 4096;   // radix: candidates kept after the first pass
 constexpr int kRankCap = 512;    // equal-width bins: most boundary-bin keys listed
 constexpr int kDirectRank = 64;  // keys in memory: larger boundary bins are ranked through sub-bins
 constexpr int kMaxKPT = 8;       // keys per thread on the register path
+#ifndef KIN_RESCORE_ROWS
+#define KIN_RESCORE_ROWS 4  // fp32 rows in flight per warp when the register path rescores a band
+#endif
 // 256-bin histograms padded by one word per 8 bins, so a lane reading 8
 // consecutive bins (stride 9 words between lanes) hits 32 distinct banks
 constexpr int kHistWords = 256 + 32;
@@ -112,6 +115,7 @@ struct TopkSmem {
   int digit, above, bin;
   uint32_t thresh;
   int thresh_take;
+  int band_n, in_n;            // dual-means refinement: band keys listed, candidates decided in
   int slot_cnt[kMaxKPT * NW];  // register path: packed (> T, == T) counts per 32-block slot
 };
 
@@ -133,12 +137,15 @@ __device__ __forceinline__ void zero_hist(TopkSmem<NT>& sm, int which) {
 // Every lane of the calling warp gets the bin (counted from the top of a
 // 256-bin histogram) holding the kr-th largest key, the count of keys in
 // higher bins, and the bin's own count.  Needs 1 <= kr <= total count.
-__device__ __forceinline__ void warp_find_bin(const int* hist, int kr, int& bin, int& above, int& cnt) {
+// half < 0: whole-word counts; 0 / 1: the low / high 16 bits of each word
+// (two histograms packed in one).
+__device__ __forceinline__ void warp_find_bin(const int* hist, int kr, int& bin, int& above, int& cnt, int half = -1) {
   const int lane = threadIdx.x & 31;
   int c[8], tot = 0;
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
-    c[u] = hist[hidx(255 - (lane * 8 + u))];
+    const int v = hist[hidx(255 - (lane * 8 + u))];
+    c[u] = half < 0 ? v : (v >> (16 * half)) & 0xFFFF;
     tot += c[u];
   }
   int inc = tot;
@@ -1258,24 +1265,24 @@ __device__ __forceinline__ float fold_max(const uint32_t* slots) {
 
 // The fp32 scores of n candidates from their fp32 rows, with the fp32
 // scan's own arithmetic: the listed indices list[0..n), or (all) every
-// index lo..lo+n-1.  Four rows in flight per warp; lane 0 hands each
+// index lo..lo+n-1.  R rows in flight per warp; lane 0 hands each
 // result to out(position, index, score).
-template <int NT, typename Out>
+template <int NT, int R = 4, typename Out>
 __device__ __forceinline__ void rescore_rows(const SelectParams& p, int64_t pair, const float (&qs)[4], int n, bool all,
                                              int lo, const uint32_t* list, Out out) {
   constexpr int NW = NT / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const float4* f32 = reinterpret_cast<const float4*>(p.means_f32 + pair * p.nbcap * kHeadDim) + lane;
-  for (int e0 = warp * 4; e0 < n; e0 += NW * 4) {
-    int idx[4];
-    float4 m[4];
+  for (int e0 = warp * R; e0 < n; e0 += NW * R) {
+    int idx[R];
+    float4 m[R];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
+    for (int r = 0; r < R; ++r) {
       idx[r] = e0 + r < n ? (all ? lo + e0 + r : (int)list[e0 + r]) : -1;
       m[r] = idx[r] >= 0 ? __ldg(f32 + (int64_t)idx[r] * (kHeadDim / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
+    for (int r = 0; r < R; ++r) {
       float d = qs[0] * m[r].x;
       d = fmaf(qs[1], m[r].y, d);
       d = fmaf(qs[2], m[r].z, d);
@@ -1412,14 +1419,14 @@ __device__ __forceinline__ void refine_scores(const SelectParams& p, int64_t pai
 // the exact top-k in one pass over registers.  Every candidate's bf16
 // score and radius is loaded once (thread t: blocks u NT + t, the top-k's
 // own layout); the bounds, the histograms and the in / out / band split
-// run from registers; the band is rescored from the fp32 rows and its exact
-// keys come back through shared memory.  The n_in candidates that are in
-// take n_in of the kr places and lie above every band score, so the
-// threshold is the (kr - n_in)-th largest exact key of the band: with at
-// most kRankCap band keys it is found by ranking them pairwise, and the
-// emit follows.  A wider band (or no finite bracket, or a band beyond the
-// list, when every candidate is rescored) goes to the generic search over
-// the refined keys.
+// run from registers; the band is rescored from the fp32 rows, spread over
+// all warps through a shared list, and its exact keys come back through
+// shared memory.  The n_in candidates that are in take n_in of the kr
+// places and lie above every band score, so the threshold is the
+// (kr - n_in)-th largest exact key of the band: with at most kRankCap band
+// keys it is found by ranking them pairwise, and the emit follows.  A wider
+// band (or no finite bracket, or a band beyond the list, when every
+// candidate is rescored) goes to the generic search over the refined keys.
 template <int NT, int KPT>
 __device__ __forceinline__ void refine_topk_regs(const SelectParams& p, int64_t pair, int nb, const Cands& cd, int k,
                                                  int32_t* sel, uint32_t* skey, TopkSmem<NT>& sm) {
@@ -1459,54 +1466,58 @@ __device__ __forceinline__ void refine_topk_regs(const SelectParams& p, int64_t 
     const int i = u * NT + tid;
     sv[u] = cd.has(i) ? __ldcg(srow + i) : 0.f;
   }
-  uint32_t* slot_c = reinterpret_cast<uint32_t*>(sm.warp_cnt[0]);
-  uint32_t* slot_d = reinterpret_cast<uint32_t*>(sm.warp_cnt[1]);
   uint32_t* slot_e = reinterpret_cast<uint32_t*>(sm.slot_cnt);
 
-  // 1. ranges of the lower and the upper bounds, and the largest error
-  float l0 = kInf, l1 = -kInf, u0 = kInf, u1 = -kInf, emax = 0.f;
+  // 1. the range of the bounds (smallest lower, largest upper), and the
+  //    largest error
+  float l0 = kInf, u1 = -kInf, emax = 0.f;
 #pragma unroll
   for (int u = 0; u < KPT; ++u) {
     ev[u] = __fmul_ru(escale, ev[u]);
     if (cd.has(u * NT + tid)) {
-      const float l = __fsub_rd(sv[u], ev[u]), h = __fadd_ru(sv[u], ev[u]);
-      l0 = fminf(l0, l);
-      l1 = fmaxf(l1, l);
-      u0 = fminf(u0, h);
-      u1 = fmaxf(u1, h);
+      l0 = fminf(l0, __fsub_rd(sv[u], ev[u]));
+      u1 = fmaxf(u1, __fadd_ru(sv[u], ev[u]));
       emax = fmaxf(emax, ev[u]);
     }
   }
   warp_min_to(l0, sm.wmin);
-  warp_max_to(l1, sm.wmax);
-  warp_min_to(u0, slot_c);
-  warp_max_to(u1, slot_d);
+  warp_max_to(u1, sm.wmax);
   warp_max_to(emax, slot_e);
   zero_hist(sm, 0);
-  zero_hist(sm, 1);
   if (tid == 0) {
-    sm.list_n = 0;   // band
-    sm.list_n2 = 0;  // in
+    sm.band_n = 0;
+    sm.in_n = 0;
   }
   __syncthreads();
-  const float lmin = fold_min<NW>(sm.wmin), lmax = fold_max<NW>(sm.wmax);
-  const float umin = fold_min<NW>(slot_c), umax = fold_max<NW>(slot_d), emx = fold_max<NW>(slot_e);
-  const float lr = lmax - lmin, li = 256.f / lr, ur = umax - umin, ui = 256.f / ur;
-  const bool lbin = isfinite(lmin) && isfinite(lmax) && lr > 0.f && isfinite(lr) && isfinite(li);
-  const bool ubin = isfinite(umin) && isfinite(umax) && ur > 0.f && isfinite(ur) && isfinite(ui);
+  const float lo = fold_min<NW>(sm.wmin), hi = fold_max<NW>(sm.wmax), emx = fold_max<NW>(slot_e);
+  const float range = hi - lo, inv = 256.f / range;
+  const bool binned = isfinite(lo) && isfinite(hi) && range > 0.f && isfinite(range) && isfinite(inv);
 
-  // 2. T_L and T_U (as in refine_scores)
+  // 2. T_L and T_U from two histograms over one range, packed in one word
+  //    per bin (lower bounds in the low 16 bits, upper bounds in the high):
+  //    a candidate whose bounds share a bin, the common case, takes one
+  //    atomic.  Bin edges one bin wider, as in refine_scores.
   float TL = -kInf, TU = kInf;
-  if (lbin || ubin) {
+  if (binned) {
 #pragma unroll
     for (int u = 0; u < KPT; ++u) {
       if (cd.has(u * NT + tid)) {
-        if (lbin) atomicAdd(&sm.hist[0][hidx(min((int)((__fsub_rd(sv[u], ev[u]) - lmin) * li), 255))], 1);
-        if (ubin) atomicAdd(&sm.hist[1][hidx(min((int)((__fadd_ru(sv[u], ev[u]) - umin) * ui), 255))], 1);
+        const int bl = min((int)((__fsub_rd(sv[u], ev[u]) - lo) * inv), 255);
+        const int bu = min((int)((__fadd_ru(sv[u], ev[u]) - lo) * inv), 255);
+        if (bl == bu) {
+          atomicAdd(&sm.hist[0][hidx(bl)], 0x10001);
+        } else {
+          atomicAdd(&sm.hist[0][hidx(bl)], 1);
+          atomicAdd(&sm.hist[0][hidx(bu)], 0x10000);
+        }
       }
     }
     __syncthreads();
-    bracket_from_hists(sm.hist[0], sm.hist[1], kr, lbin, ubin, lmin, lr, umin, ur, TL, TU);
+    int bl, bu, above, c;
+    warp_find_bin(sm.hist[0], kr, bl, above, c, 0);  // every warp, same result
+    warp_find_bin(sm.hist[0], kr, bu, above, c, 1);
+    if (bl >= 1) TL = __fadd_rd(lo, __fmul_rd((float)(bl - 1), __fdiv_rd(range, 256.f)));
+    if (bu <= 253) TU = __fadd_ru(lo, __fmul_ru((float)(bu + 2), __fdiv_ru(range, 256.f)));
   }
   const float below_all = nextafterf(__fsub_rd(TL, __fmul_ru(3.f, emx)), -kInf);
   const float above_all = nextafterf(__fadd_ru(TU, __fmul_ru(3.f, emx)), kInf);
@@ -1529,23 +1540,24 @@ __device__ __forceinline__ void refine_topk_regs(const SelectParams& p, int64_t 
       const unsigned mo = __ballot_sync(0xffffffffu, open), mi = __ballot_sync(0xffffffffu, in);
       if (mo) {
         int slot = 0;
-        if (lane == 0) slot = atomicAdd(&sm.list_n, __popc(mo));
+        if (lane == 0) slot = atomicAdd(&sm.band_n, __popc(mo));
         slot = __shfl_sync(0xffffffffu, slot, 0) + __popc(mo & ((1u << lane) - 1u));
         if (open && slot < kListCap) sm.list[slot] = (uint32_t)i;
       }
-      if (lane == 0 && mi) atomicAdd(&sm.list_n2, __popc(mi));
+      if (lane == 0 && mi) atomicAdd(&sm.in_n, __popc(mi));
       inm |= (unsigned)in << u;
       bandm |= (unsigned)open << u;
     }
   }
   __syncthreads();
-  const int nlist = sm.list_n, n_in = sm.list_n2;
+  const int nlist = sm.band_n, n_in = sm.in_n;
   const bool all = !bracketed || nlist > kListCap;  // then every candidate is rescored
 
   // 4. the band's (or every candidate's) exact keys, from the fp32 rows
   const float4 q4 = qsh[lane];
   const float qs[4] = {q4.x, q4.y, q4.z, q4.w};
-  rescore_rows<NT>(p, pair, qs, all ? cd.hi - cd.lo + 1 : nlist, all, cd.lo, sm.list, [&](int j, int i, float v) {
+  rescore_rows<NT, KIN_RESCORE_ROWS>(p, pair, qs, all ? cd.hi - cd.lo + 1 : nlist, all, cd.lo, sm.list,
+                                     [&](int j, int i, float v) {
     const uint32_t kx = key_of_bits(__float_as_uint(v));
     skey[i] = kx;
     if (!all) sm.list[j] = kx;  // the slot this warp just read its index from
