@@ -48,6 +48,12 @@ namespace kin {
 #ifndef KIN_SEL_CTAS_PER_SM
 #define KIN_SEL_CTAS_PER_SM 2
 #endif
+#ifndef KIN_DUAL_SCAN_V
+#define KIN_DUAL_SCAN_V 8  // 16-byte loads per lane per step of the dual-means scan
+#endif
+#ifndef KIN_DUAL_SCAN_CTAS
+#define KIN_DUAL_SCAN_CTAS 2  // its resident CTAs per SM
+#endif
 
 constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
@@ -1045,6 +1051,133 @@ __global__ void __launch_bounds__(kSelThreads, KIN_SEL_CTAS_PER_SM) select_scan_
   pdl_trigger_late();
 }
 
+// ---- kernel 1b: the scan of dual block means' bf16 rows (KIN_MEANS_DUAL).
+// Its scores only have to lie within the refinement's error bound of the
+// fp32 scan's (an fp32 dot product of depth at most 12, from the same fp32
+// summed query), so it is laid out for fewer instructions per byte: a
+// half-warp per row, lane x of a half holding dims 8x..8x+7, so one 16-byte
+// load per lane covers two rows per warp; an 8-term fma chain per row; and
+// a transposing reduction over the 16 lanes of a half: each of the first
+// log2(V) levels (xor 8, 4, ...) hands half of the rows a lane keeps to its
+// partner (V - 1 shuffles for V rows), plain butterfly levels finish (depth
+// 8 + 4 = 12).  V loads per lane per step, U = 2 V rows per warp step,
+// contiguous U-aligned step ranges per warp as in the scan above.
+template <int V>
+__device__ __forceinline__ void dual_qsum(const SelectParams& p, int pair, int x, float (&o)[8]) {
+  // dims 8x..8x+7 of the group-summed query, summed in row order from 0
+  // (the same fp32 values as pair_qsum's)
+  const int b = pair / p.Hkv, h = pair - b * p.Hkv;
+  const uint4* qg = reinterpret_cast<const uint4*>(p.q + ((int64_t)b * p.Hq + (int64_t)h * p.g) * kHeadDim) + x;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) o[c] = 0.f;
+  for (int j0 = 0; j0 < p.g; j0 += 4) {
+    uint4 raw[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) raw[j] = j0 + j < p.g ? __ldcg(qg + (j0 + j) * (kHeadDim / 8)) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (j0 + j < p.g) {
+        const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          o[2 * c] += __uint_as_float(w[c] << 16);
+          o[2 * c + 1] += __uint_as_float(w[c] & 0xFFFF0000u);
+        }
+      }
+    }
+  }
+}
+
+template <int V, int CTAS>
+__global__ void __launch_bounds__(kSelThreads, CTAS) select_scan_dual_kernel(SelectParams p) {
+  static_assert(V == 4 || V == 8, "V loads per lane per step");
+  constexpr int U = 2 * V;     // rows per warp per step
+  constexpr int kGrp = 16 / V;  // lanes of a half that end holding the same row
+  pdl_wait();  // means, lengths and q come from earlier work on the stream
+  pdl_trigger_early();
+  const int lane = threadIdx.x & 31, hh = lane >> 4, x = lane & 15;
+  const int nwarps = gridDim.x * kSelWarps;
+  const int gw = blockIdx.x * kSelWarps + (threadIdx.x >> 5);
+  const int nbp = (p.nbcap + U - 1) / U * U;
+  const int steps = p.B * p.Hkv * (nbp / U);
+  const int per = (steps + nwarps - 1) / nwarps;
+  const int s0 = gw * per, s1 = min(s0 + per, steps);
+  if (s0 >= s1) {
+    pdl_trigger_late();
+    return;
+  }
+  // step-local row r = 2 j + hh comes from the lane's j-th load
+  const uint4* mrow = reinterpret_cast<const uint4*>(p.means) + hh * (kHeadDim / 8) + x;
+  auto load = [&](int pr, int bk, int nbr, bool any, uint4 (&v)[V]) {
+    const uint4* b0 = mrow + ((int64_t)pr * p.nbcap + bk) * (kHeadDim / 8);
+    if (any && bk + U <= nbr) {
+#pragma unroll
+      for (int j = 0; j < V; ++j) v[j] = __ldcs(b0 + j * 2 * (kHeadDim / 8));
+    } else {
+#pragma unroll
+      for (int j = 0; j < V; ++j)
+        v[j] = any && bk + 2 * j + hh < nbr ? __ldcs(b0 + j * 2 * (kHeadDim / 8)) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  int pair = (s0 * U) / nbp;
+  int blk = s0 * U - pair * nbp;
+  int nb = pair_nb(p, pair);
+  float qs[8];
+  dual_qsum<V>(p, pair, x, qs);
+  uint4 cur[V];
+  load(pair, blk, nb, true, cur);
+  for (int s = s0; s < s1; ++s) {
+    int npair = pair, nblk = blk + U, nnb = nb;
+    if (nblk >= nbp) {
+      npair = pair + 1;
+      nblk = 0;
+      nnb = s + 1 < s1 ? pair_nb(p, npair) : 0;
+    }
+    const bool more = s + 1 < s1;
+    uint4 nxt[V];
+    load(npair, nblk, nnb, more, nxt);  // the next step's rows fly during this step's math
+    if (blk < nb) {
+      float d[V];
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        const uint32_t w[4] = {cur[j].x, cur[j].y, cur[j].z, cur[j].w};
+        float t = qs[0] * __uint_as_float(w[0] << 16);
+        t = fmaf(qs[1], __uint_as_float(w[0] & 0xFFFF0000u), t);
+#pragma unroll
+        for (int c = 1; c < 4; ++c) {
+          t = fmaf(qs[2 * c], __uint_as_float(w[c] << 16), t);
+          t = fmaf(qs[2 * c + 1], __uint_as_float(w[c] & 0xFFFF0000u), t);
+        }
+        d[j] = t;
+      }
+      // transposing levels: at offset 8 >> s, the upper lane keeps the upper
+      // half of its rows
+#pragma unroll
+      for (int sl = 0, half = V / 2; half >= 1; ++sl, half >>= 1) {
+        const bool upper = (x >> (3 - sl)) & 1;
+#pragma unroll
+        for (int j = 0; j < half; ++j) {
+          const float keep = upper ? d[j + half] : d[j];
+          const float send = upper ? d[j] : d[j + half];
+          d[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8 >> sl);
+        }
+      }
+      float tot = d[0];
+#pragma unroll
+      for (int off = kGrp / 2; off > 0; off >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, off);
+      const int r = 2 * (x / kGrp) + hh;  // the step-local row this lane holds
+      if ((x & (kGrp - 1)) == 0 && blk + r < nb) p.scores[(int64_t)pair * p.nbcap + blk + r] = tot * p.score_scale;
+    }
+    if (npair != pair && more) dual_qsum<V>(p, npair, x, qs);
+    pair = npair;
+    blk = nblk;
+    nb = nnb;
+#pragma unroll
+    for (int j = 0; j < V; ++j) cur[j] = nxt[j];
+  }
+  pdl_trigger_late();
+}
+
 // The scan over block means stored per page (the shared-prompt layout),
 // found through the page table.  Rows are scattered, so a warp splits into
 // 4 groups of 8 lanes, each group owning one mean row at a time: lane x of a
@@ -1758,6 +1891,19 @@ cudaError_t launch_select(const SelectParams& p, cudaStream_t s) {
     return launch_pdl(select_dense_kernel, dim3(grid), dim3(256), 0, s, p);
   }
   const int64_t rows = (int64_t)p.B * p.Hkv * p.nbcap;
+  if (p.refine) {  // dual means: the bf16 rows' scan, then the refining top-k
+    constexpr int V = KIN_DUAL_SCAN_V, C = KIN_DUAL_SCAN_CTAS;
+    const int64_t res = (int64_t)device_sm_count() * C;
+    const int64_t want = (rows + kSelWarps * 2 * V * 4 - 1) / (kSelWarps * 2 * V * 4);  // >= 4 steps per warp
+    const int grid = (int)(want < res ? (want > 0 ? want : 1) : res);
+    cudaError_t e = launch_pdl(select_scan_dual_kernel<V, C>, dim3(grid), dim3(kSelThreads), 0, s, p);
+    if (e != cudaSuccess) return e;
+    switch (topk_threads(p.nbcap, (int64_t)p.B * p.Hkv)) {
+      case 256: return launch_topk<256>(p, s);
+      case 512: return launch_topk<512>(p, s);
+      default: return launch_topk<1024>(p, s);
+    }
+  }
   const int u = p.means_bf16 ? 2 * kSelU : kSelU;
   const int64_t want = (rows + kSelWarps * u * 4 - 1) / (kSelWarps * u * 4);  // >= 4 steps per warp
   const int grid = (int)(want < resident ? (want > 0 ? want : 1) : resident);
