@@ -178,6 +178,47 @@ __device__ __forceinline__ void warp_find_bin(const int* hist, int kr, int& bin,
   cnt = __shfl_sync(0xffffffffu, cn, src);
 }
 
+// warp_find_bin over the two histograms packed in one word per bin (low
+// and high 16 bits), both searches interleaved over one read of the bins:
+// the bins holding the kr-th largest of each.  Needs 1 <= kr <= each total.
+__device__ __forceinline__ void warp_find_bins_packed(const int* hist, int kr, int& bin_lo, int& bin_hi) {
+  const int lane = threadIdx.x & 31;
+  int c[8], tl = 0, th = 0;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    c[u] = hist[hidx(255 - (lane * 8 + u))];
+    tl += c[u] & 0xFFFF;
+    th += c[u] >> 16;
+  }
+  int il = tl, ih = th;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, il, o), b = __shfl_up_sync(0xffffffffu, ih, o);
+    if (lane >= o) {
+      il += a;
+      ih += b;
+    }
+  }
+  const bool ml = il - tl < kr && kr <= il, mh = ih - th < kr && kr <= ih;
+  int bl = 0, bh = 0, rl = il - tl, rh = ih - th;
+  bool fl = false, fh = false;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    rl += c[u] & 0xFFFF;
+    rh += c[u] >> 16;
+    if (ml && !fl && rl >= kr) {
+      bl = 255 - (lane * 8 + u);
+      fl = true;
+    }
+    if (mh && !fh && rh >= kr) {
+      bh = 255 - (lane * 8 + u);
+      fh = true;
+    }
+  }
+  bin_lo = __shfl_sync(0xffffffffu, bl, __ffs(__ballot_sync(0xffffffffu, ml)) - 1);
+  bin_hi = __shfl_sync(0xffffffffu, bh, __ffs(__ballot_sync(0xffffffffu, mh)) - 1);
+}
+
 // Radix select over the candidate keys keys[1..nb-2]: on entry kr (> 0) is
 // how many of them to keep, sm.hist[0] holds the histogram of their top
 // bytes and sm.hist[1] is zero.  Up to 4 passes of 8 bits from the top: each
@@ -1431,7 +1472,9 @@ __device__ __forceinline__ void rescore_rows(const SelectParams& p, int64_t pair
 // lower and upper bounds (sm.hist[0], sm.hist[1], when lbin / ubin), one
 // bin wider than the bins found (the bin function is monotone and computed
 // to a few ulps, so every bound in bin b lies within [lo + (b - 1) w,
-// lo + (b + 2) w), w the bin width); -inf / +inf without a histogram.
+// lo + (b + 2) w), w the bin width); -inf / +inf without a histogram.  The
+// bin width range / 256 is range * 2^-8 with the same directed rounding (a
+// multiply instead of a slow directed division).
 __device__ __forceinline__ void bracket_from_hists(const int* hl, const int* hu, int kr, bool lbin, bool ubin,
                                                    float lmin, float lr, float umin, float ur, float& TL, float& TU) {
   const float kInf = __int_as_float(0x7f800000);
@@ -1440,11 +1483,11 @@ __device__ __forceinline__ void bracket_from_hists(const int* hl, const int* hu,
   int bl, bu, above, c;
   if (lbin) {
     warp_find_bin(hl, kr, bl, above, c);  // every warp, same result
-    if (bl >= 1) TL = __fadd_rd(lmin, __fmul_rd((float)(bl - 1), __fdiv_rd(lr, 256.f)));
+    if (bl >= 1) TL = __fadd_rd(lmin, __fmul_rd((float)(bl - 1), __fmul_rd(lr, 0x1p-8f)));
   }
   if (ubin) {
     warp_find_bin(hu, kr, bu, above, c);
-    if (bu <= 253) TU = __fadd_ru(umin, __fmul_ru((float)(bu + 2), __fdiv_ru(ur, 256.f)));
+    if (bu <= 253) TU = __fadd_ru(umin, __fmul_ru((float)(bu + 2), __fmul_ru(ur, 0x1p-8f)));
   }
 }
 
@@ -1646,20 +1689,22 @@ __device__ __forceinline__ void refine_topk_regs(const SelectParams& p, int64_t 
       }
     }
     __syncthreads();
-    int bl, bu, above, c;
-    warp_find_bin(sm.hist[0], kr, bl, above, c, 0);  // every warp, same result
-    warp_find_bin(sm.hist[0], kr, bu, above, c, 1);
-    if (bl >= 1) TL = __fadd_rd(lo, __fmul_rd((float)(bl - 1), __fdiv_rd(range, 256.f)));
-    if (bu <= 253) TU = __fadd_ru(lo, __fmul_ru((float)(bu + 2), __fdiv_ru(range, 256.f)));
+    int bl, bu;
+    warp_find_bins_packed(sm.hist[0], kr, bl, bu);  // every warp, same result
+    if (bl >= 1) TL = __fadd_rd(lo, __fmul_rd((float)(bl - 1), __fmul_rd(range, 0x1p-8f)));
+    if (bu <= 253) TU = __fadd_ru(lo, __fmul_ru((float)(bu + 2), __fmul_ru(range, 0x1p-8f)));
   }
   const float below_all = nextafterf(__fsub_rd(TL, __fmul_ru(3.f, emx)), -kInf);
   const float above_all = nextafterf(__fadd_ru(TU, __fmul_ru(3.f, emx)), kInf);
   const bool bracketed = isfinite(below_all) && isfinite(above_all);
 
-  // 3. in (l > T_U), out (u < T_L), or in the band: band indices listed
-  //    (one reservation per warp), the in ones counted
+  // 3. in (l > T_U), out (u < T_L), or in the band: the warp's ballots
+  //    first, then one reservation of list slots and one count of the in
+  //    ones per warp, then the band indices listed
   unsigned inm = 0u, bandm = 0u;
   if (bracketed) {
+    unsigned mo[KPT];
+    int nband = 0, nin = 0;
 #pragma unroll
     for (int u = 0; u < KPT; ++u) {
       const int i = u * NT + tid;
@@ -1670,16 +1715,23 @@ __device__ __forceinline__ void refine_topk_regs(const SelectParams& p, int64_t 
         else if (!(__fadd_ru(sv[u], ev[u]) < TL))
           open = true;
       }
-      const unsigned mo = __ballot_sync(0xffffffffu, open), mi = __ballot_sync(0xffffffffu, in);
-      if (mo) {
-        int slot = 0;
-        if (lane == 0) slot = atomicAdd(&sm.band_n, __popc(mo));
-        slot = __shfl_sync(0xffffffffu, slot, 0) + __popc(mo & ((1u << lane) - 1u));
-        if (open && slot < kListCap) sm.list[slot] = (uint32_t)i;
-      }
-      if (lane == 0 && mi) atomicAdd(&sm.in_n, __popc(mi));
+      mo[u] = __ballot_sync(0xffffffffu, open);
+      nband += __popc(mo[u]);
+      nin += __popc(__ballot_sync(0xffffffffu, in));
       inm |= (unsigned)in << u;
       bandm |= (unsigned)open << u;
+    }
+    int slot = 0;
+    if (lane == 0) {
+      if (nband) slot = atomicAdd(&sm.band_n, nband);
+      if (nin) atomicAdd(&sm.in_n, nin);
+    }
+    slot = __shfl_sync(0xffffffffu, slot, 0);
+#pragma unroll
+    for (int u = 0; u < KPT; ++u) {
+      const int at = slot + __popc(mo[u] & ((1u << lane) - 1u));
+      if (((bandm >> u) & 1u) && at < kListCap) sm.list[at] = (uint32_t)(u * NT + tid);
+      slot += __popc(mo[u]);
     }
   }
   __syncthreads();

@@ -280,3 +280,23 @@ def gpu_step_paged(dc: DeviceCase, pg: Pages, k: int, seq_lens: torch.Tensor, me
     torch.cuda.synchronize()
     return GpuResult(sel.cpu().numpy(), cnt.cpu().numpy(), out.float().cpu().numpy(), lse.cpu().numpy(),
                      int(st.item()))
+
+
+def random_shapes(n, seed, prefix="rand"):
+    """n seeded random workloads: block size 16-128, g 1-8, 1-4 KV heads, batch 1-4, capacity up to
+    20000 tokens, appends of 0, 1 or 5 tokens, k from 2 to a little beyond the block capacity."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        bs = int(rng.choice([16, 32, 64, 128]))
+        g = int(rng.integers(1, 9))
+        Hkv = int(rng.integers(1, 5))
+        B = int(rng.integers(1, 5))
+        n_append = int(rng.choice([0, 0, 1, 5]))
+        Lcap = int(rng.integers(bs, 20000))
+        lens = tuple(int(x) for x in rng.integers(1, Lcap - n_append + 1, size=B))
+        nbcap = -(-Lcap // bs)
+        k = int(rng.integers(2, nbcap + 3))
+        out.append(ki.Workload(f"{prefix}{i}_bs{bs}_g{g}_k{k}", B, Hkv, Hkv * g, D, bs, 0, 0, k, 200 + i, Lcap=Lcap,
+                               lens=tuple(L + n_append for L in lens), n_append=n_append))
+    return out

@@ -10,7 +10,7 @@ import torch
 
 import block_top_sparse_kin_b200 as kin
 import kin_inputs as ki
-from kin_testlib import D, GpuResult, all_pairs, check_pairs, make_device_case
+from kin_testlib import D, GpuResult, all_pairs, check_pairs, make_device_case, random_shapes
 
 pytestmark = pytest.mark.gpu
 W = ki.Workload
@@ -111,6 +111,16 @@ def test_dual_select_equals_fp32_select(w):
     a, b, dual = _build_both(w)
     assert np.array_equal(_select(a, a.means, w.k)[0], _select(b, dual, w.k)[0])
     assert np.array_equal(_select(a, a.means, w.k)[1], _select(b, dual, w.k)[1])
+
+
+@pytest.mark.parametrize("w", random_shapes(16, seed=171, prefix="dual_rand"), ids=lambda w: w.name)
+def test_dual_select_equals_fp32_select_random_shapes(w):
+    """Seeded random shapes (block sizes 16-128, g 1-8, appends, k from 2 to past the block
+    capacity): the dual select's indices and counts equal the fp32 select's."""
+    a, b, dual = _build_both(w)
+    sa, ca = _select(a, a.means, w.k)
+    sb, cb = _select(b, dual, w.k)
+    assert np.array_equal(ca, cb) and np.array_equal(sa, sb)
 
 
 @pytest.mark.parametrize("name,ks", [("qwen3_8b_32k", None), ("qwen3_14b_ragged", None),

@@ -14,7 +14,7 @@ import pytest
 import torch
 
 import kin_inputs as ki
-from kin_testlib import D, all_pairs, check_pairs, gpu_step, make_device_case
+from kin_testlib import D, all_pairs, check_pairs, gpu_step, make_device_case, random_shapes
 
 pytestmark = pytest.mark.gpu
 W = ki.Workload
@@ -42,24 +42,6 @@ HALVING = [
 ]
 
 
-def _random_shapes(n, seed=71):
-    rng = np.random.default_rng(seed)
-    out = []
-    for i in range(n):
-        bs = int(rng.choice([16, 32, 64, 128]))
-        g = int(rng.integers(1, 9))
-        Hkv = int(rng.integers(1, 5))
-        B = int(rng.integers(1, 5))
-        n_append = int(rng.choice([0, 0, 1, 5]))
-        Lcap = int(rng.integers(bs, 20000))
-        lens = tuple(int(x) for x in rng.integers(1, Lcap - n_append + 1, size=B))
-        nbcap = -(-Lcap // bs)
-        k = int(rng.integers(2, nbcap + 3))
-        out.append(W(f"rand{i}_bs{bs}_g{g}_k{k}", B, Hkv, Hkv * g, D, bs, 0, 0, k, 200 + i, Lcap=Lcap,
-                     lens=tuple(L + n_append for L in lens), n_append=n_append))
-    return out
-
-
 def _every_pair(w):
     dc = make_device_case(w)
     gr = gpu_step(dc, w.k)
@@ -81,6 +63,6 @@ def test_topk_thread_halving(w):
     _every_pair(w)
 
 
-@pytest.mark.parametrize("w", _random_shapes(12), ids=lambda w: w.name)
+@pytest.mark.parametrize("w", random_shapes(12, seed=71), ids=lambda w: w.name)
 def test_random_shapes_every_pair(w):
     _every_pair(w)
