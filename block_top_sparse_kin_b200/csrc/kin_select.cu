@@ -1665,7 +1665,19 @@ __device__ __forceinline__ void refine_topk_regs(const SelectParams& p, int64_t 
     sm.in_n = 0;
   }
   __syncthreads();
-  const float lo = fold_min<NW>(sm.wmin), hi = fold_max<NW>(sm.wmax), emx = fold_max<NW>(slot_e);
+  float lo, hi, emx;
+  {  // the three folds interleaved (lane l reads slot l, then one butterfly)
+    const int sl = lane < NW ? lane : 0;
+    lo = __uint_as_float(sm.wmin[sl]);
+    hi = __uint_as_float(sm.wmax[sl]);
+    emx = __uint_as_float(slot_e[sl]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+      emx = fmaxf(emx, __shfl_xor_sync(0xffffffffu, emx, off));
+    }
+  }
   const float range = hi - lo, inv = 256.f / range;
   const bool binned = isfinite(lo) && isfinite(hi) && range > 0.f && isfinite(range) && isfinite(inv);
 
