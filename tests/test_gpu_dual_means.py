@@ -10,7 +10,7 @@ import torch
 
 import block_top_sparse_kin_b200 as kin
 import kin_inputs as ki
-from kin_testlib import D, GpuResult, all_pairs, check_pairs, make_device_case, random_shapes
+from kin_testlib import D, GpuResult, all_pairs, check_pairs, make_device_case, random_shapes, to_pages
 
 pytestmark = pytest.mark.gpu
 W = ki.Workload
@@ -190,6 +190,38 @@ def test_dual_select_with_scores_tied_below_bf16_resolution(nblocks, boosted):
     f32, b16, _ = _parts(dual, b.dims)
     assert len(torch.unique(f32.view(w.B, w.Hkv, -1, D)[0, 0, :nb], dim=0)) > 300
     assert len(torch.unique(b16.view(w.B, w.Hkv, -1, D)[0, 0, :nb], dim=0)) <= 2
+
+
+@pytest.mark.parametrize("w", [
+    W("dual_paged_g4_bs16", 3, 2, 8, D, 16, 300, 1000, 12, 95, Lcap=1024),
+    W("dual_paged_bs128", 2, 2, 4, D, 128, 129, 1000, 3, 96, Lcap=1024),
+    W("dual_paged_append_7", 2, 2, 8, D, 16, 0, 0, 6, 97, Lcap=200, n_append=7, lens=(100, 44)),
+    W("dual_paged_append_1_new_page", 2, 1, 4, D, 32, 0, 0, 3, 98, Lcap=160, n_append=1, lens=(128, 64)),
+], ids=lambda w: w.name)
+def test_dual_means_from_a_paged_cache_equal_the_contiguous_ones(w):
+    """Dual means built (and appended to) through a block table over a shuffled page
+    pool: the fp32 rows, bf16 rows and radii equal those built from the contiguous
+    cache, byte for byte, and the dual select keeps the same blocks."""
+    a, b = make_device_case(w), make_device_case(w)
+    pg = to_pages(b, seed=w.seed)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dual_c, dual_p = kin.alloc_dual_means(a.dims), kin.alloc_dual_means(b.dims)
+    kin.kin_block_means_build_ex(a.dims, a.k_cache, a.seq_lens, dual_c, dev_status=st)
+    kin.kin_block_means_build_ex(b.dims, pg.k, b.seq_lens, dual_p, block_table=pg.table, dev_status=st)
+    if w.n_append:
+        kin.kin_block_means_update_ex(a.dims, a.k_cache, a.v_cache, dual_c, a.seq_lens, a.k_new, a.v_new,
+                                      w.n_append, dev_status=st)
+        kin.kin_block_means_update_ex(b.dims, pg.k, pg.v, dual_p, b.seq_lens, b.k_new, b.v_new, w.n_append,
+                                      block_table=pg.table, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert torch.equal(a.seq_lens, b.seq_lens)
+    rows = torch.from_numpy(_valid_rows(w, a)).cuda()
+    for part_c, part_p in zip(_parts(dual_c, a.dims), _parts(dual_p, b.dims)):
+        assert torch.equal(part_c[rows].view(torch.uint8), part_p[rows].view(torch.uint8))
+    sa, ca = _select(a, dual_c, w.k)
+    sb, cb = _select(b, dual_p, w.k)
+    assert np.array_equal(ca, cb) and np.array_equal(sa, sb)
 
 
 def test_dual_means_refused_per_page_and_in_the_paged_select():
