@@ -70,7 +70,7 @@ def algorithmic_bytes(w: ki.Workload, k: int, lens: np.ndarray, means_bytes: int
     return sel_bytes, attn_bytes
 
 
-def shared_algorithmic_bytes(w: ki.Workload, k: int, st, means_bytes: int = 4):
+def shared_algorithmic_bytes(w: ki.Workload, k: int, st, means_bytes: float = 4.0):
     """Algorithmic bytes when groups of samples share their prompt's pages
     and per-page means, each shared item read once: (select) the distinct
     mean rows (page, head) of the scanned sequences; (attention) the
@@ -442,8 +442,11 @@ def build_device_state(w: ki.Workload, k: int, paged: bool = False, means_bf16: 
     if paged or share_n > 1:
         make_page_pool(st, w.seed, share_n, shuffle_pages)
     if share_n > 1:  # block means per page: the shared prompt's means exist once
-        st["means"] = torch.zeros((st["num_pages"], w.Hkv, w.D),
-                                  dtype=torch.bfloat16 if means_bf16 else torch.float32, device="cuda")
+        if means_dual:
+            st["means"] = kin.alloc_dual_page_means(dims, st["num_pages"])
+        else:
+            st["means"] = torch.zeros((st["num_pages"], w.Hkv, w.D),
+                                      dtype=torch.bfloat16 if means_bf16 else torch.float32, device="cuda")
         st["seq"].copy_(st["seq_pre"])
         kin.kin_block_means_build_ex(dims, st["k_pages"], st["seq"], st["means"], block_table=st["table"],
                                      per_page=True)
@@ -496,7 +499,7 @@ def select(st):
     import block_top_sparse_kin_b200 as kin
     if "page_means" in st:
         kin.kin_block_topk_select_paged(st["dims"], st["q"], st["means"], st["table"], st["seq"], st["k"], st["sel"],
-                                        st["cnt"], st["ws"], st["status"])
+                                        st["cnt"], st["ws"], st["status"], num_pages=st["num_pages"])
     elif str(st["means"].dtype) in ("torch.bfloat16", "torch.uint8"):
         kin.kin_block_topk_select_ex(st["dims"], st["q"], st["means"], st["seq"], st["k"], st["sel"], st["cnt"],
                                      st["ws"], st["status"])
@@ -785,12 +788,17 @@ MEANS_KINDS = {
 
 
 def means_kind(args) -> str:
-    """fp32 (--means-fp32, and always for per-page shared-prompt means), bf16
-    (--means-bf16), else dual: the fp32 selection read from a bf16 copy."""
-    if getattr(args, "means_bf16", False) and getattr(args, "means_fp32", False):
-        raise SystemExit("--means-bf16 and --means-fp32 exclude each other")
+    """bf16 (--means-bf16), dual (--means-dual: the fp32 selection read from a
+    bf16 copy), fp32 (--means-fp32); by default dual, except fp32 for
+    per-page shared-prompt means, whose scan reads mostly from L2 (dual
+    per-page means stay available with --means-dual)."""
+    chosen = [f for f in ("means_bf16", "means_fp32", "means_dual") if getattr(args, f, False)]
+    if len(chosen) > 1:
+        raise SystemExit("--means-bf16, --means-fp32 and --means-dual exclude each other")
     if getattr(args, "means_bf16", False):
         return "bf16"
+    if getattr(args, "means_dual", False):
+        return "dual"
     if getattr(args, "means_fp32", False) or getattr(args, "shared_prefix", 1) > 1:
         return "fp32"
     return "dual"
@@ -1021,6 +1029,8 @@ def main(argv=None):
     ap.add_argument("--means-fp32", action="store_true",
                     help="fp32 block means only: the plain select, which scans them in full (the default keeps dual "
                          "means and returns the same selection from a bf16 copy; see kin.h KIN_MEANS_DUAL)")
+    ap.add_argument("--means-dual", action="store_true",
+                    help="dual block means also with --shared-prefix (per page; the default elsewhere)")
     ap.add_argument("--page-order", default="shuffled", choices=["shuffled", "sequential"],
                     help="page pool order for --paged / --shared-prefix")
     ap.add_argument("--shared-prefix", type=int, default=1,

@@ -29,7 +29,7 @@ EXPORTED = (
     "kin_block_topk_select_noalloc", "kin_block_means_build_paged", "kin_block_means_update_paged",
     "kin_sparse_decode_attn_paged", "kin_block_means_build_ex", "kin_block_means_update_ex",
     "kin_block_topk_select_ex", "kin_token_topk_workspace_bytes", "kin_token_topk_decode_attn",
-    "kin_block_topk_select_paged", "kin_dual_means_bytes",
+    "kin_block_topk_select_paged", "kin_dual_means_bytes", "kin_dual_page_means_bytes",
 )
 KIN_MEANS_F32, KIN_MEANS_BF16, KIN_MEANS_DUAL = 0, 1, 2
 KIN_MEANS_PER_PAGE = 0x100
@@ -111,6 +111,8 @@ def load_library(path: str = LIB_PATH):
     lib.kin_block_topk_select_paged.restype = ctypes.c_int
     lib.kin_dual_means_bytes.argtypes = [dp]
     lib.kin_dual_means_bytes.restype = sz
+    lib.kin_dual_page_means_bytes.argtypes = [dp, i32]
+    lib.kin_dual_page_means_bytes.restype = sz
     _lib = lib
     return lib
 
@@ -312,14 +314,20 @@ def kin_sparse_decode_attn_paged(dims, q, k_pages, v_pages, block_table, seq_len
 # The means dtype follows the block_means tensor (float32 or bfloat16);
 # block_table None selects the contiguous cache.  See include/kin.h.
 
-def _means(block_means, count=None, name="block_means", dims=None):
+def _means(block_means, count=None, name="block_means", dims=None, pages=None):
     """The means pointer and its dtype code, from the tensor: float32 rows,
     bfloat16 rows, or a uint8 buffer of dual means (fp32 rows, their bf16
-    rounding and the rows' error radii: see kin_dual_means_bytes)."""
+    rounding and the rows' error radii: see kin_dual_means_bytes; per page
+    when `pages` is given, see kin_dual_page_means_bytes)."""
     if block_means is not None and block_means.dtype == torch.float32:
         return _dev(block_means, name, torch.float32, count=count), KIN_MEANS_F32
     if block_means is not None and block_means.dtype == torch.uint8:
-        nbytes = kin_dual_means_bytes(dims) if dims is not None else None
+        if dims is None:
+            nbytes = None
+        elif pages is not None:
+            nbytes = kin_dual_page_means_bytes(dims, pages)
+        else:
+            nbytes = kin_dual_means_bytes(dims)
         return _dev(block_means, name, torch.uint8, count=nbytes or None), KIN_MEANS_DUAL
     return _dev(block_means, name, torch.bfloat16, count=count), KIN_MEANS_BF16
 
@@ -327,6 +335,21 @@ def _means(block_means, count=None, name="block_means", dims=None):
 def kin_dual_means_bytes(dims: kin_dims) -> int:
     """Bytes of a dual block-means buffer (KIN_MEANS_DUAL) for these dims."""
     return int(load_library().kin_dual_means_bytes(ctypes.byref(dims)))
+
+
+def kin_dual_page_means_bytes(dims: kin_dims, num_pages: int) -> int:
+    """Bytes of a dual block-means buffer stored per page (KIN_MEANS_DUAL |
+    KIN_MEANS_PER_PAGE) for a pool of num_pages pages."""
+    return int(load_library().kin_dual_page_means_bytes(ctypes.byref(dims), int(num_pages)))
+
+
+def alloc_dual_page_means(dims: kin_dims, num_pages: int, device="cuda") -> torch.Tensor:
+    """A dual block-means buffer per page (uint8), filled by the build/update
+    calls with per_page=True and read by kin_block_topk_select_paged."""
+    n = kin_dual_page_means_bytes(dims, num_pages)
+    if n == 0:
+        raise KinError(1, "kin_dual_page_means_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
 def alloc_dual_means(dims: kin_dims, device="cuda") -> torch.Tensor:
@@ -353,7 +376,8 @@ def kin_block_means_build_ex(dims, k_rows, seq_lens, block_means, block_table=No
     """per_page: block_means is [num_pages, Hkv, D] (one mean per page; needs block_table)."""
     c = _Counts(dims)
     pages, table, rows = _layout(k_rows, block_table, c)
-    means, dtype = _means(block_means, c.times(pages, c.page_mean) if per_page else c.means, dims=dims)
+    means, dtype = _means(block_means, c.times(pages, c.page_mean) if per_page else c.means, dims=dims,
+                          pages=pages if per_page else None)
     dtype |= KIN_MEANS_PER_PAGE if per_page else 0
     rc = load_library().kin_block_means_build_ex(
         ctypes.byref(dims), _dev(k_rows, "k_rows", _BF16, count=rows), pages, table,
@@ -365,7 +389,8 @@ def kin_block_means_update_ex(dims, k_rows, v_rows, block_means, seq_lens, k_new
                               block_table=None, dev_status=None, stream=None, per_page=False):
     c = _Counts(dims)
     pages, table, rows = _layout(k_rows, block_table, c)
-    means, dtype = _means(block_means, c.times(pages, c.page_mean) if per_page else c.means, dims=dims)
+    means, dtype = _means(block_means, c.times(pages, c.page_mean) if per_page else c.means, dims=dims,
+                          pages=pages if per_page else None)
     dtype |= KIN_MEANS_PER_PAGE if per_page else 0
     new_rows = c.times(max(int(n_new), 0), c.bkd)
     rc = load_library().kin_block_means_update_ex(
@@ -417,12 +442,19 @@ def kin_token_topk_decode_attn(dims, q, k_cache, v_cache, seq_lens, k_tokens, so
 
 
 def kin_block_topk_select_paged(dims, q, page_means, block_table, seq_lens, k_blocks, sel_idx, sel_cnt, workspace,
-                                dev_status=None, stream=None):
+                                dev_status=None, stream=None, num_pages=None):
     """The select over per-page block means [num_pages, Hkv, D] (fp32 or bf16),
-    found through block_table: the shared-prompt layout (see include/kin.h)."""
+    or a per-page dual buffer (uint8; num_pages then required), found through
+    block_table: the shared-prompt layout (see include/kin.h)."""
     c = _Counts(dims)
-    pages = int(page_means.shape[0])
-    means, dtype = _means(page_means, c.times(pages, c.page_mean), "page_means")
+    if page_means is not None and page_means.dtype == torch.uint8:
+        if num_pages is None:
+            raise ValueError("page_means: a dual buffer needs num_pages")
+        pages = int(num_pages)
+        means, dtype = _means(page_means, None, "page_means", dims=dims, pages=pages)
+    else:
+        pages = int(page_means.shape[0])
+        means, dtype = _means(page_means, c.times(pages, c.page_mean), "page_means")
     rc = load_library().kin_block_topk_select_paged(
         ctypes.byref(dims), _dev(q, "q", _BF16, count=c.q), means, dtype, pages,
         _dev(block_table, "block_table", torch.int32, count=c.table),

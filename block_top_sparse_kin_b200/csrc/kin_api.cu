@@ -179,6 +179,12 @@ KIN_EXPORT size_t kin_dual_means_bytes(const kin_dims* dims) {
   return (size_t)rows * (kHeadDim * 4 + kHeadDim * 2 + 4);
 }
 
+KIN_EXPORT size_t kin_dual_page_means_bytes(const kin_dims* dims, int32_t num_pages) {
+  if (check_dims(dims) != KIN_OK || num_pages < 1) return 0;
+  const int64_t rows = (int64_t)num_pages * dims->num_kv_heads;
+  return (size_t)rows * (kHeadDim * 4 + kHeadDim * 2 + 4);
+}
+
 namespace {
 
 kin_status means_build(const kin_dims* dims, const void* k_rows, const PageTable& pt, const int32_t* seq_lens,
@@ -196,7 +202,7 @@ kin_status means_build(const kin_dims* dims, const void* k_rows, const PageTable
   p.Lcap = dims->max_seq_len;
   p.bs = dims->block_size;
   p.nbcap = nbcap_of(*dims);
-  p.mean_rows = (int64_t)p.B * p.Hkv * p.nbcap;
+  p.mean_rows = per_page ? (int64_t)pt.num_pages * p.Hkv : (int64_t)p.B * p.Hkv * p.nbcap;
   return from_cuda(launch_means_build(p, static_cast<cudaStream_t>(stream)));
 }
 
@@ -219,7 +225,7 @@ kin_status means_update(const kin_dims* dims, void* k_rows, void* v_rows, const 
   p.Lcap = dims->max_seq_len;
   p.bs = dims->block_size;
   p.nbcap = nbcap_of(*dims);
-  p.mean_rows = (int64_t)p.B * p.Hkv * p.nbcap;
+  p.mean_rows = per_page ? (int64_t)pt.num_pages * p.Hkv : (int64_t)p.B * p.Hkv * p.nbcap;
   p.n_new = n_new;
   return from_cuda(launch_means_update(p, static_cast<cudaStream_t>(stream)));
 }
@@ -320,7 +326,8 @@ kin_status topk_select(const kin_dims* dims, const void* q, const void* block_me
   p.means_f32 = nullptr;
   p.radii = nullptr;
   if (means_bf16 == 2) {  // dual: scan the bf16 rows, rescore from the fp32 rows
-    const int64_t rows = (int64_t)dims->batch * dims->num_kv_heads * nbcap_of(*dims);
+    const int64_t rows = mpages ? (int64_t)mpages->num_pages * dims->num_kv_heads
+                                : (int64_t)dims->batch * dims->num_kv_heads * nbcap_of(*dims);
     const float* f = static_cast<const float*>(block_means);
     p.means = f + rows * kHeadDim;
     p.means_bf16 = 1;
@@ -346,12 +353,10 @@ kin_status topk_select(const kin_dims* dims, const void* q, const void* block_me
   return from_cuda(launch_select(p, static_cast<cudaStream_t>(stream)));
 }
 
-// means_dtype as a kernel flag (0 fp32, 1 bf16, 2 dual); -1 for an unknown
-// value or for dual means stored per page (dual means are logical only)
+// means_dtype as a kernel flag (0 fp32, 1 bf16, 2 dual); -1 for an unknown value
 int means_flag(int32_t means_dtype) {
   const int32_t t = means_dtype & ~KIN_MEANS_PER_PAGE;
-  if (t == KIN_MEANS_DUAL) return (means_dtype & KIN_MEANS_PER_PAGE) ? -1 : 2;
-  return t == KIN_MEANS_F32 ? 0 : t == KIN_MEANS_BF16 ? 1 : -1;
+  return t == KIN_MEANS_F32 ? 0 : t == KIN_MEANS_BF16 ? 1 : t == KIN_MEANS_DUAL ? 2 : -1;
 }
 int per_page_flag(int32_t means_dtype) { return (means_dtype & KIN_MEANS_PER_PAGE) ? 1 : 0; }
 
@@ -401,7 +406,7 @@ KIN_EXPORT kin_status kin_block_topk_select_paged(const kin_dims* dims, const vo
   kin_status st = check_dims(dims);
   if (st != KIN_OK) return st;
   const int bf = means_flag(means_dtype);
-  if (bf < 0 || bf == 2) return KIN_ERR_INVALID_ARG;  // per-page means are fp32 or bf16
+  if (bf < 0) return KIN_ERR_INVALID_ARG;
   PageTable pt;
   st = check_pages(*dims, page_means, num_pages, block_table, &pt);
   if (st != KIN_OK) return st;

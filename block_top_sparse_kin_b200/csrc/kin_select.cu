@@ -1437,6 +1437,32 @@ __device__ __forceinline__ float fold_max(const uint32_t* slots) {
   return v;
 }
 
+// The rows of a pair's blocks in the dual means' arrays: logical, or per
+// page through the table (then -1 for a page index outside the pool: a zero
+// row, as the per-page scan reads it, and no radius).
+struct DualRows {
+  const int32_t* trow;  // the sequence's table row, or null (logical rows)
+  int64_t base;         // logical: pair * nbcap; per page: the head h
+  int Hkv, num_pages;
+  __device__ __forceinline__ DualRows(const SelectParams& p, int64_t pair) {
+    Hkv = p.Hkv;
+    num_pages = p.mpages.num_pages;
+    if (p.mpages.table) {
+      const int64_t b = pair / p.Hkv;
+      trow = p.mpages.table + b * p.mpages.max_blocks;
+      base = pair - b * p.Hkv;
+    } else {
+      trow = nullptr;
+      base = pair * p.nbcap;
+    }
+  }
+  __device__ __forceinline__ int64_t operator()(int i) const {
+    if (!trow) return base + i;
+    const int page = __ldcg(trow + i);
+    return (page < 0 || page >= num_pages) ? -1 : (int64_t)page * Hkv + base;
+  }
+};
+
 // The fp32 scores of n candidates from their fp32 rows, with the fp32
 // scan's own arithmetic: the listed indices list[0..n), or (all) every
 // index lo..lo+n-1.  R rows in flight per warp; lane 0 hands each
@@ -1446,14 +1472,16 @@ __device__ __forceinline__ void rescore_rows(const SelectParams& p, int64_t pair
                                              int lo, const uint32_t* list, Out out) {
   constexpr int NW = NT / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const float4* f32 = reinterpret_cast<const float4*>(p.means_f32 + pair * p.nbcap * kHeadDim) + lane;
+  const float4* f32 = reinterpret_cast<const float4*>(p.means_f32) + lane;
+  const DualRows rows(p, pair);
   for (int e0 = warp * R; e0 < n; e0 += NW * R) {
     int idx[R];
     float4 m[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       idx[r] = e0 + r < n ? (all ? lo + e0 + r : (int)list[e0 + r]) : -1;
-      m[r] = idx[r] >= 0 ? __ldg(f32 + (int64_t)idx[r] * (kHeadDim / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const int64_t row = idx[r] >= 0 ? rows(idx[r]) : -1;
+      m[r] = row >= 0 ? __ldg(f32 + row * (kHeadDim / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -1504,8 +1532,12 @@ __device__ __forceinline__ void refine_scores(const SelectParams& p, int64_t pai
   float qs[4];
   pair_qsum(p, (int)pair, lane, qs);  // the fp32 scan's summed query, lane's 4 dims
   const float escale = pair_err_scale(p, qs);
-  const float* rad = p.radii + pair * p.nbcap;
-  auto err = [&](int i) { return __fmul_ru(escale, __ldg(rad + i)); };
+  const float kInfE = __int_as_float(0x7f800000);
+  const DualRows rows(p, pair);
+  auto err = [&](int i) {  // a block with no page has no radius: undecided
+    const int64_t r = rows(i);
+    return r < 0 ? kInfE : __fmul_ru(escale, __ldg(p.radii + r));
+  };
   uint32_t* slot_c = reinterpret_cast<uint32_t*>(sm.warp_cnt[0]);
   uint32_t* slot_d = reinterpret_cast<uint32_t*>(sm.warp_cnt[1]);
   uint32_t* slot_e = reinterpret_cast<uint32_t*>(sm.slot_cnt);
@@ -1617,13 +1649,15 @@ __device__ __forceinline__ void refine_topk_regs(const SelectParams& p, int64_t 
     emit_regs<NT, KPT>(none, nb, cd, k, 0xFFFFFFFFu, 0, sel, sm, p.dev_status);
     return;
   }
-  // the radii and the query, before the wait: see select_topk_kernel
-  const float* rad = p.radii + pair * p.nbcap;
+  // the radii and the query, before the wait: see select_topk_kernel (a
+  // block with no page has no radius: undecided)
   float ev[KPT];
+  const DualRows rows(p, pair);
 #pragma unroll
   for (int u = 0; u < KPT; ++u) {
     const int i = u * NT + tid;
-    ev[u] = cd.has(i) ? __ldcg(rad + i) : 0.f;
+    const int64_t r = cd.has(i) ? rows(i) : -2;
+    ev[u] = r >= 0 ? __ldcg(p.radii + r) : r == -1 ? kInf : 0.f;
   }
   __shared__ float4 qsh[kHeadDim / 4];  // the summed query, for the rescoring
   float escale;
@@ -1791,11 +1825,11 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_topk_kernel(SelectParams
   const int k = p.k;
   int32_t* sel = p.sel_idx + pair * k;
   if constexpr (kRefine) {
-    // The lengths, the radii and the query are written by work that
-    // completed before the scan's own wait returned (the scan writes only
-    // scores), and this grid starts after every scan CTA passed that wait:
-    // they are read from L2 (ld.global.cg, the point of coherence) before
-    // this grid's wait, while the scan drains.  The register paths wait
+    // The lengths, the radii, the query and the page table are written by
+    // work that completed before the scan's own wait returned (the scan
+    // writes only scores), and this grid starts after every scan CTA passed
+    // that wait: they are read from L2 (ld.global.cg, the point of
+    // coherence) before this grid's wait, while the scan drains.  The register paths wait
     // inside, before their first score load.
     const int L = __ldcg(p.seq_lens + b);
     const int nb = (L >= 1 && L <= p.Lcap) ? (L + p.bs - 1) / p.bs : 0;
@@ -1808,7 +1842,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_topk_kernel(SelectParams
       if (tid == 0) p.sel_cnt[pair] = k;
       return;
     }
-    if (nb > k) {  // the memory path: warm L2 with this pair's radii and query rows
+    if (nb > k && !p.mpages.table) {  // the memory path: warm L2 with this pair's radii and query rows
       const char* rb = reinterpret_cast<const char*>(p.radii + pair * p.nbcap);
       for (int t = tid; t < (p.nbcap * 4 + 127) / 128; t += NT) prefetch_l2(rb + t * 128);
       const int h = (int)(pair - (int64_t)b * p.Hkv);
@@ -1956,11 +1990,18 @@ cudaError_t launch_select(const SelectParams& p, cudaStream_t s) {
   }
   const int64_t rows = (int64_t)p.B * p.Hkv * p.nbcap;
   if (p.refine) {  // dual means: the bf16 rows' scan, then the refining top-k
-    constexpr int V = KIN_DUAL_SCAN_V, C = KIN_DUAL_SCAN_CTAS;
-    const int64_t res = (int64_t)device_sm_count() * C;
-    const int64_t want = (rows + kSelWarps * 2 * V * 4 - 1) / (kSelWarps * 2 * V * 4);  // >= 4 steps per warp
-    const int grid = (int)(want < res ? (want > 0 ? want : 1) : res);
-    cudaError_t e = launch_pdl(select_scan_dual_kernel<V, C>, dim3(grid), dim3(kSelThreads), 0, s, p);
+    cudaError_t e;
+    if (p.mpages.table) {  // per page: the per-page scan of the bf16 rows
+      const int64_t want = (rows + kSelWarps * 2 * kSelU * 4 - 1) / (kSelWarps * 2 * kSelU * 4);
+      const int grid = (int)(want < resident ? (want > 0 ? want : 1) : resident);
+      e = launch_pdl(select_scan_paged_kernel<true>, dim3(grid), dim3(kSelThreads), 0, s, p);
+    } else {
+      constexpr int V = KIN_DUAL_SCAN_V, C = KIN_DUAL_SCAN_CTAS;
+      const int64_t res = (int64_t)device_sm_count() * C;
+      const int64_t want = (rows + kSelWarps * 2 * V * 4 - 1) / (kSelWarps * 2 * V * 4);  // >= 4 steps per warp
+      const int grid = (int)(want < res ? (want > 0 ? want : 1) : res);
+      e = launch_pdl(select_scan_dual_kernel<V, C>, dim3(grid), dim3(kSelThreads), 0, s, p);
+    }
     if (e != cudaSuccess) return e;
     switch (topk_threads(p.nbcap, (int64_t)p.B * p.Hkv)) {
       case 256: return launch_topk<256>(p, s);

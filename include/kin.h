@@ -223,10 +223,15 @@ typedef enum { KIN_MEANS_F32 = 0, KIN_MEANS_BF16 = 1, KIN_MEANS_DUAL = 2 } kin_m
  * s~ + e is below the k-th largest s~ - e cannot be kept, one whose s~ - e
  * is above the k-th largest s~ + e is kept, and only the band between is
  * rescored from its fp32 rows with the fp32 scan's own arithmetic before
- * the exact top-k.  Logical layout only: not with KIN_MEANS_PER_PAGE, nor
- * in kin_block_topk_select_paged (KIN_ERR_INVALID_ARG).  Returns 0 for
- * invalid dims. */
+ * the exact top-k.  Returns 0 for invalid dims.  Stored per page
+ * (KIN_MEANS_DUAL | KIN_MEANS_PER_PAGE, with a block table), the same three
+ * arrays hold one row per (page, KV head): [num_pages][Hkv][D] fp32, then
+ * bf16, then [num_pages][Hkv] radii, in a buffer of
+ * kin_dual_page_means_bytes(dims, num_pages) bytes, read by
+ * kin_block_topk_select_paged (a page index outside the pool is flagged as
+ * for the other means and its block scored from a zero row). */
 size_t kin_dual_means_bytes(const kin_dims* dims);
+size_t kin_dual_page_means_bytes(const kin_dims* dims, int32_t num_pages);
 /* OR-ed into means_dtype of the build/update calls (with a block table):
  * block means per page, [num_pages][Hkv][D], read by
  * kin_block_topk_select_paged below. */
@@ -256,8 +261,9 @@ kin_status kin_block_topk_select_ex(const kin_dims* dims, const void* q, const v
  * calls), the prompt's means are stored once too.  This select reads the
  * per-page means through the table:
  *   page_means  [num_pages][Hkv][D], fp32 or bf16 (means_dtype, without the
- *               per-page flag); block i of (b, h) is page_means[block_table
- *               [b][i]][h].
+ *               per-page flag), or dual means per page (KIN_MEANS_DUAL: the
+ *               fp32 selection read from the bf16 rows, see above); block i
+ *               of (b, h) is page_means[block_table[b][i]][h].
  * A page shared by several sequences must hold full blocks (bs valid rows)
  * in each of them, so its mean is the same for all.  Results equal those
  * of the select over logical means of the same blocks, bit for bit.  A page

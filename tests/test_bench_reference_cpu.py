@@ -3,6 +3,7 @@ on the host cores and prints one JSON line with the contract's keys; its
 step is one pass over the sampled pairs, whose time fits inside the run;
 under a multi-rank launch only rank 0 works and prints."""
 import json
+import pytest
 import os
 import subprocess
 import sys
@@ -73,3 +74,17 @@ def test_traffic_lookup_is_keyed_by_means_kind_and_layout():
         if digest == bench.kernel_source_digest(key.split("@")[0]):
             assert bench.profiled_traffic(key, wl, int(k)) == int(float(nbytes))
             assert bench.profiled_traffic(key + "@paged", wl, int(k)) is None
+
+
+def test_means_kind_follows_the_flags():
+    import argparse
+    import bench
+    base = dict(means_fp32=False, means_bf16=False, means_dual=False, shared_prefix=1)
+    ns = lambda **kw: argparse.Namespace(**{**base, **kw})
+    assert bench.means_kind(ns()) == "dual"
+    assert bench.means_kind(ns(shared_prefix=8)) == "fp32"          # per-page means: fp32 unless asked
+    assert bench.means_kind(ns(shared_prefix=8, means_dual=True)) == "dual"
+    assert bench.means_kind(ns(means_fp32=True)) == "fp32"
+    assert bench.means_kind(ns(means_bf16=True)) == "bf16"
+    with pytest.raises(SystemExit):
+        bench.means_kind(ns(means_fp32=True, means_dual=True))

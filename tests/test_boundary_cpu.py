@@ -60,6 +60,10 @@ def test_workspace_bytes(lib):
     rows = d.batch * d.num_kv_heads * -(-d.max_seq_len // d.block_size)
     assert kin.kin_dual_means_bytes(d) == rows * (128 * 4 + 128 * 2 + 4)
     assert kin.kin_dual_means_bytes(dims(D=64)) == 0
+    # per page: one row per (page, KV head)
+    assert kin.kin_dual_page_means_bytes(d, 5) == 5 * d.num_kv_heads * (128 * 4 + 128 * 2 + 4)
+    assert kin.kin_dual_page_means_bytes(d, 0) == 0
+    assert kin.kin_dual_page_means_bytes(dims(D=64), 5) == 0
     assert kin.kin_workspace_bytes(dims(), 1) == 0
     assert kin.kin_workspace_bytes(dims(D=64), 8) == 0
     assert kin.kin_workspace_bytes(dims(bs=24), 8) == 0
@@ -156,19 +160,19 @@ def test_extended_calls_reject_before_launch(lib):
                                                                   1 << 30, None, None)
     assert sel(dt=3) == 1                          # 0 fp32, 1 bf16, 2 dual
     assert sel(dt=-1) == 1
-    assert sel(dt=2 | 0x100) == 1                  # dual means are never per page
+    assert sel(dt=2 | 0x100) == 1                  # per-page means need the paged select
     assert sel(k=1) == 1
     assert sel(ws=None) == 2
     build = lambda dt=1, pool=FAKE, pages=0, table=None: lib.kin_block_means_build_ex(
         bd, pool, pages, table, FAKE, FAKE, dt, None, None)
     assert build(dt=7) == 1
-    assert build(dt=2 | 0x100, pages=4, table=FAKE) == 1
+    assert build(dt=2 | 0x100, pages=0, table=None) == 1   # per-page (dual) means need a table
     assert build(pool=None) == 1
     assert build(pages=0, table=FAKE) == 1        # a table needs a pool of >= 1 page
     upd = lambda dt=1, n=1, pages=4, table=FAKE: lib.kin_block_means_update_ex(
         bd, FAKE, FAKE, pages, table, FAKE, dt, FAKE, FAKE, FAKE, n, None, None)
     assert upd(dt=3) == 1
-    assert upd(dt=2 | 0x100) == 1
+    assert upd(dt=2 | 0x100, table=None) == 1
     assert upd(n=-1) == 1
     assert upd(n=0) == 0
     assert upd(n=257) == 3
@@ -203,7 +207,7 @@ def test_token_and_page_means_calls_reject_before_launch(lib):
     # the select over means stored per page
     sp = lambda dt=0, pages=4, table=FAKE, pool=FAKE, k=8, ws=FAKE: lib.kin_block_topk_select_paged(
         bd, FAKE, pool, dt, pages, table, FAKE, k, FAKE, FAKE, ws, 1 << 30, None, None)
-    assert sp(dt=2) == 1
+    assert sp(dt=3) == 1                          # an unknown means dtype
     assert sp(pages=0) == 1
     assert sp(table=None) == 1
     assert sp(pool=None) == 1

@@ -224,23 +224,10 @@ def test_dual_means_from_a_paged_cache_equal_the_contiguous_ones(w):
     assert np.array_equal(ca, cb) and np.array_equal(sa, sb)
 
 
-def test_dual_means_refused_per_page_and_in_the_paged_select():
-    import ctypes
+def test_dual_means_size():
     dims = kin.make_dims(2, 2, 8, D, 16, 256)
-    lib = kin.load_library()
-    buf = torch.zeros(kin.kin_dual_means_bytes(dims), dtype=torch.uint8, device="cuda")
-    t = torch.zeros(64, dtype=torch.int32, device="cuda")
-    kc = torch.zeros((2, 2, 256, D), dtype=torch.bfloat16, device="cuda")
-    P = lambda x: ctypes.c_void_p(x.data_ptr())
-    rc = lib.kin_block_means_build_ex(ctypes.byref(dims), P(kc), 4, P(t), P(t), P(buf),
-                                      kin.KIN_MEANS_DUAL | kin.KIN_MEANS_PER_PAGE, None, None)
-    assert rc == 1
-    q = torch.zeros((2, 8, D), dtype=torch.bfloat16, device="cuda")
-    ws = kin.alloc_workspace(dims, 4)
-    rc = lib.kin_block_topk_select_paged(ctypes.byref(dims), P(q), P(buf), kin.KIN_MEANS_DUAL, 4, P(t), P(t), 4,
-                                         P(t), P(t), P(ws), ws.numel(), None, None)
-    assert rc == 1
     assert kin.kin_dual_means_bytes(dims) == 2 * 2 * 16 * (D * 6 + 4)
+    assert kin.kin_dual_page_means_bytes(dims, 7) == 7 * 2 * (D * 6 + 4)
 
 
 @pytest.mark.parametrize("name", ["qwen3_8b_32k", "qwen3_32b_128k_append"])
