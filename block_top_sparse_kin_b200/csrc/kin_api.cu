@@ -130,8 +130,9 @@ cudaError_t ensure_smem_limit(const void* kernel, int slot, size_t bytes) {
   // is read and raised under one lock, so a thread never lowers it under
   // another thread's launch, and the cache (the limit last seen, per slot and
   // device) never exceeds the limit in force.
-  // slots in use: 0, 2, 3 and 8, 9, 10 block top-k (256, 512, 1024 threads;
-  // plain and refining), 1 attention, 4 means update, 5 token top-k, 6 token logits
+  // slots in use: 0, 2, 3, then 8, 9, 10, then 12, 13, 14 block top-k (256,
+  // 512, 1024 threads; plain, refining, refining per page), 1 attention, 4
+  // means update, 5 token top-k, 6 token logits
   static std::atomic<size_t> done[16][kMaxDevices];
   static std::mutex mu;
   int dev = 0;

@@ -1437,17 +1437,18 @@ __device__ __forceinline__ float fold_max(const uint32_t* slots) {
   return v;
 }
 
-// The rows of a pair's blocks in the dual means' arrays: logical, or per
-// page through the table (then -1 for a page index outside the pool: a zero
-// row, as the per-page scan reads it, and no radius).
+// The rows of a pair's blocks in the dual means' arrays: logical, or (kPaged)
+// per page through the table, then -1 for a page index outside the pool: a
+// zero row, as the per-page scan reads it, and no radius.
+template <bool kPaged>
 struct DualRows {
-  const int32_t* trow;  // the sequence's table row, or null (logical rows)
+  const int32_t* trow;  // per page: the sequence's table row
   int64_t base;         // logical: pair * nbcap; per page: the head h
   int Hkv, num_pages;
   __device__ __forceinline__ DualRows(const SelectParams& p, int64_t pair) {
     Hkv = p.Hkv;
     num_pages = p.mpages.num_pages;
-    if (p.mpages.table) {
+    if constexpr (kPaged) {
       const int64_t b = pair / p.Hkv;
       trow = p.mpages.table + b * p.mpages.max_blocks;
       base = pair - b * p.Hkv;
@@ -1457,9 +1458,12 @@ struct DualRows {
     }
   }
   __device__ __forceinline__ int64_t operator()(int i) const {
-    if (!trow) return base + i;
-    const int page = __ldcg(trow + i);
-    return (page < 0 || page >= num_pages) ? -1 : (int64_t)page * Hkv + base;
+    if constexpr (!kPaged) {
+      return base + i;
+    } else {
+      const int page = __ldcg(trow + i);
+      return (page < 0 || page >= num_pages) ? -1 : (int64_t)page * Hkv + base;
+    }
   }
 };
 
@@ -1467,13 +1471,13 @@ struct DualRows {
 // scan's own arithmetic: the listed indices list[0..n), or (all) every
 // index lo..lo+n-1.  R rows in flight per warp; lane 0 hands each
 // result to out(position, index, score).
-template <int NT, int R = 4, typename Out>
+template <int NT, bool kPaged, int R = 4, typename Out>
 __device__ __forceinline__ void rescore_rows(const SelectParams& p, int64_t pair, const float (&qs)[4], int n, bool all,
                                              int lo, const uint32_t* list, Out out) {
   constexpr int NW = NT / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const float4* f32 = reinterpret_cast<const float4*>(p.means_f32) + lane;
-  const DualRows rows(p, pair);
+  const DualRows<kPaged> rows(p, pair);
   for (int e0 = warp * R; e0 < n; e0 += NW * R) {
     int idx[R];
     float4 m[R];
@@ -1519,7 +1523,7 @@ __device__ __forceinline__ void bracket_from_hists(const int* hl, const int* hu,
   }
 }
 
-template <int NT>
+template <int NT, bool kPaged>
 __device__ __forceinline__ void refine_scores(const SelectParams& p, int64_t pair, float* row, const Cands& cd,
                                               TopkSmem<NT>& sm) {
   constexpr int NW = NT / 32;
@@ -1533,7 +1537,7 @@ __device__ __forceinline__ void refine_scores(const SelectParams& p, int64_t pai
   pair_qsum(p, (int)pair, lane, qs);  // the fp32 scan's summed query, lane's 4 dims
   const float escale = pair_err_scale(p, qs);
   const float kInfE = __int_as_float(0x7f800000);
-  const DualRows rows(p, pair);
+  const DualRows<kPaged> rows(p, pair);
   auto err = [&](int i) {  // a block with no page has no radius: undecided
     const int64_t r = rows(i);
     return r < 0 ? kInfE : __fmul_ru(escale, __ldg(p.radii + r));
@@ -1618,7 +1622,7 @@ __device__ __forceinline__ void refine_scores(const SelectParams& p, int64_t pai
   const bool all = !fits || nlist > kListCap;
 
   // 4. rescore them from the fp32 rows
-  rescore_rows<NT>(p, pair, qs, all ? cd.hi - cd.lo + 1 : nlist, all, cd.lo, sm.list,
+  rescore_rows<NT, kPaged>(p, pair, qs, all ? cd.hi - cd.lo + 1 : nlist, all, cd.lo, sm.list,
                    [&](int, int i, float v) { row[i] = v; });
   __syncthreads();  // the row is final before the top-k reads it
 }
@@ -1635,7 +1639,7 @@ __device__ __forceinline__ void refine_scores(const SelectParams& p, int64_t pai
 // keys it is found by ranking them pairwise, and the emit follows.  A wider
 // band (or no finite bracket, or a band beyond the list, when every
 // candidate is rescored) goes to the generic search over the refined keys.
-template <int NT, int KPT>
+template <int NT, int KPT, bool kPaged>
 __device__ __forceinline__ void refine_topk_regs(const SelectParams& p, int64_t pair, int nb, const Cands& cd, int k,
                                                  int32_t* sel, uint32_t* skey, TopkSmem<NT>& sm) {
   constexpr int NW = NT / 32;
@@ -1652,7 +1656,7 @@ __device__ __forceinline__ void refine_topk_regs(const SelectParams& p, int64_t 
   // the radii and the query, before the wait: see select_topk_kernel (a
   // block with no page has no radius: undecided)
   float ev[KPT];
-  const DualRows rows(p, pair);
+  const DualRows<kPaged> rows(p, pair);
 #pragma unroll
   for (int u = 0; u < KPT; ++u) {
     const int i = u * NT + tid;
@@ -1787,7 +1791,7 @@ __device__ __forceinline__ void refine_topk_regs(const SelectParams& p, int64_t 
   // 4. the band's (or every candidate's) exact keys, from the fp32 rows
   const float4 q4 = qsh[lane];
   const float qs[4] = {q4.x, q4.y, q4.z, q4.w};
-  rescore_rows<NT, KIN_RESCORE_ROWS>(p, pair, qs, all ? cd.hi - cd.lo + 1 : nlist, all, cd.lo, sm.list,
+  rescore_rows<NT, kPaged, KIN_RESCORE_ROWS>(p, pair, qs, all ? cd.hi - cd.lo + 1 : nlist, all, cd.lo, sm.list,
                                      [&](int j, int i, float v) {
     const uint32_t kx = key_of_bits(__float_as_uint(v));
     skey[i] = kx;
@@ -1815,7 +1819,7 @@ __device__ __forceinline__ void refine_topk_regs(const SelectParams& p, int64_t 
 // ---- kernel 2: one CTA of NT threads per pair: dense shortcut, bad-length
 // flag, or the exact top-k over the scores the scan left in workspace
 // (L2-resident), in registers when nb <= 8 NT.
-template <int NT, bool kRefine>
+template <int NT, bool kRefine, bool kPaged = false>
 __global__ void __launch_bounds__(NT, 1024 / NT) select_topk_kernel(SelectParams p) {
   extern __shared__ uint32_t skey[];  // [nbcap] keys (rows beyond 8 NT blocks: then nbcap bytes of bins)
   __shared__ TopkSmem<NT> sm;
@@ -1836,13 +1840,13 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_topk_kernel(SelectParams
     if (nb > k && nb <= 8 * NT) {
       const Cands cd{1, nb - 2, k - 2};  // blocks 0 and nb - 1 forced
       if (nb <= 4 * NT)
-        refine_topk_regs<NT, 4>(p, pair, nb, cd, k, sel, skey, sm);
+        refine_topk_regs<NT, 4, kPaged>(p, pair, nb, cd, k, sel, skey, sm);
       else
-        refine_topk_regs<NT, 8>(p, pair, nb, cd, k, sel, skey, sm);
+        refine_topk_regs<NT, 8, kPaged>(p, pair, nb, cd, k, sel, skey, sm);
       if (tid == 0) p.sel_cnt[pair] = k;
       return;
     }
-    if (nb > k && !p.mpages.table) {  // the memory path: warm L2 with this pair's radii and query rows
+    if (nb > k && !kPaged) {  // the memory path: warm L2 with this pair's radii and query rows
       const char* rb = reinterpret_cast<const char*>(p.radii + pair * p.nbcap);
       for (int t = tid; t < (p.nbcap * 4 + 127) / 128; t += NT) prefetch_l2(rb + t * 128);
       const int h = (int)(pair - (int64_t)b * p.Hkv);
@@ -1870,7 +1874,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_topk_kernel(SelectParams
   const uint32_t* row = reinterpret_cast<const uint32_t*>(p.scores + pair * p.nbcap);
   const Cands cd{1, nb - 2, k - 2};  // blocks 0 and nb - 1 forced
   if constexpr (kRefine) {
-    refine_scores<NT>(p, pair, p.scores + pair * p.nbcap, cd, sm);
+    refine_scores<NT, kPaged>(p, pair, p.scores + pair * p.nbcap, cd, sm);
     topk_memory<NT>(row, nb, cd, k, sel, skey, p.nbcap, const_cast<uint32_t*>(row), sm, p.dev_status);
   } else if (nb <= 4 * NT) {
     topk_regs<NT, 4>(row, nb, cd, k, sel, skey, sm, p.dev_status);
@@ -1942,6 +1946,14 @@ template <int NT>
 cudaError_t launch_topk(const SelectParams& p, cudaStream_t s) {
   // keys (when they do not fit in registers: then also their bins)
   const size_t smem = (size_t)p.nbcap * sizeof(uint32_t) + (p.nbcap > 8 * NT ? ((size_t)p.nbcap + 3) & ~size_t(3) : 0);
+  if (p.refine && p.mpages.table) {  // dual means per page
+    if (smem > 16 * 1024) {
+      cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(select_topk_kernel<NT, true, true>),
+                                        NT == 256 ? 12 : NT == 512 ? 13 : 14, smem);
+      if (e != cudaSuccess) return e;
+    }
+    return launch_pdl(select_topk_kernel<NT, true, true>, dim3(p.B * p.Hkv), dim3(NT), smem, s, p);
+  }
   if (p.refine) {
     if (smem > 16 * 1024) {
       cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(select_topk_kernel<NT, true>),
