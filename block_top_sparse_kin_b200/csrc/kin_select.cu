@@ -1484,8 +1484,12 @@ __device__ __forceinline__ void rescore_rows(const SelectParams& p, int64_t pair
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       idx[r] = e0 + r < n ? (all ? lo + e0 + r : (int)list[e0 + r]) : -1;
-      const int64_t row = idx[r] >= 0 ? rows(idx[r]) : -1;
-      m[r] = row >= 0 ? __ldg(f32 + row * (kHeadDim / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      if constexpr (kPaged) {
+        const int64_t row = idx[r] >= 0 ? rows(idx[r]) : -1;
+        m[r] = row >= 0 ? __ldg(f32 + row * (kHeadDim / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      } else {
+        m[r] = idx[r] >= 0 ? __ldg(f32 + rows(idx[r]) * (kHeadDim / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -1660,8 +1664,12 @@ __device__ __forceinline__ void refine_topk_regs(const SelectParams& p, int64_t 
 #pragma unroll
   for (int u = 0; u < KPT; ++u) {
     const int i = u * NT + tid;
-    const int64_t r = cd.has(i) ? rows(i) : -2;
-    ev[u] = r >= 0 ? __ldcg(p.radii + r) : r == -1 ? kInf : 0.f;
+    if constexpr (kPaged) {
+      const int64_t r = cd.has(i) ? rows(i) : -2;
+      ev[u] = r >= 0 ? __ldcg(p.radii + r) : r == -1 ? kInf : 0.f;
+    } else {
+      ev[u] = cd.has(i) ? __ldcg(p.radii + rows(i)) : 0.f;
+    }
   }
   __shared__ float4 qsh[kHeadDim / 4];  // the summed query, for the rescoring
   float escale;
