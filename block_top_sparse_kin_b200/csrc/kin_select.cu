@@ -93,6 +93,9 @@ constexpr int kListCap = 4096;   // radix: candidates kept after the first pass
 constexpr int kRankCap = 512;    // equal-width bins: most boundary-bin keys listed
 constexpr int kDirectRank = 64;  // keys in memory: larger boundary bins are ranked through sub-bins
 constexpr int kMaxKPT = 8;       // keys per thread on the register path
+#ifndef KIN_RANK_SPLIT
+#define KIN_RANK_SPLIT 1  // the refinement ranks a band of <= NT / 4 keys with four threads per key
+#endif
 #ifndef KIN_RESCORE_ROWS
 #define KIN_RESCORE_ROWS 4  // fp32 rows in flight per warp when the register path rescores a band
 #endif
@@ -471,6 +474,34 @@ __device__ __forceinline__ void rank_keys(int off, int c, int need, TopkSmem<NT>
       sm.thresh = kj;
       sm.thresh_take = need - gt;
     }
+  }
+  __syncthreads();
+}
+
+// rank_keys over c <= NT / 4 keys (off 0) with four threads per key: thread
+// 4 j + part counts the keys part, part + 4, ... against key j, and a
+// two-step shuffle sums the four counts (a quarter of the serial loop).
+// Ends with a barrier.
+template <int NT>
+__device__ __forceinline__ void rank_keys_split4(int c, int need, TopkSmem<NT>& sm) {
+  const int j = threadIdx.x >> 2, part = threadIdx.x & 3;
+  const bool mine = j < c;
+  const uint32_t kj = mine ? sm.list[j] : 0u;
+  int gt = 0, ge = 0;
+  if (mine) {
+    for (int i = part; i < c; i += 4) {
+      const uint32_t ki = sm.list[i];
+      gt += ki > kj;
+      ge += ki >= kj;
+    }
+  }
+  gt += __shfl_xor_sync(0xffffffffu, gt, 1);
+  ge += __shfl_xor_sync(0xffffffffu, ge, 1);
+  gt += __shfl_xor_sync(0xffffffffu, gt, 2);
+  ge += __shfl_xor_sync(0xffffffffu, ge, 2);
+  if (mine && part == 0 && gt < need && need <= ge) {
+    sm.thresh = kj;
+    sm.thresh_take = need - gt;
   }
   __syncthreads();
 }
@@ -1817,7 +1848,10 @@ __device__ __forceinline__ void refine_topk_regs(const SelectParams& p, int64_t 
   // 5. the threshold among the band, and the emit
   const int need = kr - n_in;
   if (!all && nlist <= kRankCap && need >= 1 && need <= nlist) {
-    rank_keys(0, nlist, need, sm);  // ends with a barrier
+    if (KIN_RANK_SPLIT && nlist <= NT / 4)
+      rank_keys_split4<NT>(nlist, need, sm);  // ends with a barrier
+    else
+      rank_keys(0, nlist, need, sm);  // ends with a barrier
     emit_regs<NT, KPT>(key, nb, cd, k, sm.thresh, sm.thresh_take, sel, sm, p.dev_status);
   } else {
     topk_regs_keys<NT, KPT>(key, nb, cd, k, sel, skey, sm, p.dev_status);
