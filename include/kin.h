@@ -223,7 +223,8 @@ typedef enum { KIN_MEANS_F32 = 0, KIN_MEANS_BF16 = 1, KIN_MEANS_DUAL = 2 } kin_m
  * s~ + e is below the k-th largest s~ - e cannot be kept, one whose s~ - e
  * is above the k-th largest s~ + e is kept, and only the band between is
  * rescored from its fp32 rows with the fp32 scan's own arithmetic before
- * the exact top-k.  Returns 0 for invalid dims.  Stored per page
+ * the exact top-k.  The sizes are 0 for invalid dims (or num_pages < 1).
+ * Stored per page
  * (KIN_MEANS_DUAL | KIN_MEANS_PER_PAGE, with a block table), the same three
  * arrays hold one row per (page, KV head): [num_pages][Hkv][D] fp32, then
  * bf16, then [num_pages][Hkv] radii, in a buffer of
