@@ -1863,6 +1863,9 @@ __device__ __forceinline__ void refine_topk_regs(const SelectParams& p, int64_t 
 // (L2-resident), in registers when nb <= 8 NT.
 template <int NT, bool kRefine, bool kPaged = false>
 __global__ void __launch_bounds__(NT, 1024 / NT) select_topk_kernel(SelectParams p) {
+  // 4 keys per thread need 8 warps (the emit's slot layout): a 128-thread CTA
+  // (chosen only for rows of at most 8 NT = 1024 blocks) keeps 8 per thread
+  constexpr bool kKpt4 = NT >= 256;
   extern __shared__ uint32_t skey[];  // [nbcap] keys (rows beyond 8 NT blocks: then nbcap bytes of bins)
   __shared__ TopkSmem<NT> sm;
   const int tid = threadIdx.x;
@@ -1881,10 +1884,14 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_topk_kernel(SelectParams
     const int nb = (L >= 1 && L <= p.Lcap) ? (L + p.bs - 1) / p.bs : 0;
     if (nb > k && nb <= 8 * NT) {
       const Cands cd{1, nb - 2, k - 2};  // blocks 0 and nb - 1 forced
-      if (nb <= 4 * NT)
-        refine_topk_regs<NT, 4, kPaged>(p, pair, nb, cd, k, sel, skey, sm);
-      else
-        refine_topk_regs<NT, 8, kPaged>(p, pair, nb, cd, k, sel, skey, sm);
+      bool done = false;
+      if constexpr (kKpt4) {
+        if (nb <= 4 * NT) {
+          refine_topk_regs<NT, 4, kPaged>(p, pair, nb, cd, k, sel, skey, sm);
+          done = true;
+        }
+      }
+      if (!done) refine_topk_regs<NT, 8, kPaged>(p, pair, nb, cd, k, sel, skey, sm);
       if (tid == 0) p.sel_cnt[pair] = k;
       return;
     }
@@ -1918,8 +1925,8 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_topk_kernel(SelectParams
   if constexpr (kRefine) {
     refine_scores<NT, kPaged>(p, pair, p.scores + pair * p.nbcap, cd, sm);
     topk_memory<NT>(row, nb, cd, k, sel, skey, p.nbcap, const_cast<uint32_t*>(row), sm, p.dev_status);
-  } else if (nb <= 4 * NT) {
-    topk_regs<NT, 4>(row, nb, cd, k, sel, skey, sm, p.dev_status);
+  } else if (kKpt4 && nb <= 4 * NT) {
+    if constexpr (kKpt4) topk_regs<NT, 4>(row, nb, cd, k, sel, skey, sm, p.dev_status);
   } else if (nb <= 8 * NT) {
     topk_regs<NT, 8>(row, nb, cd, k, sel, skey, sm, p.dev_status);
   } else {
@@ -1977,10 +1984,10 @@ cudaError_t launch_token_topk(const TokenParams& p, cudaStream_t s) {
 
 // Threads per top-k CTA: enough for 4 keys per thread (up to 4096 blocks),
 // halved (8 keys per thread) while the pairs would need more than one wave
-// of CTAs (the launch bounds allow 1024 / NT CTAs per SM).
+// of CTAs (the launch bounds allow 1024 / NT CTAs per SM), down to 128.
 int topk_threads(int nbcap, int64_t pairs) {
   int nt = nbcap <= 1024 ? 256 : nbcap <= 2048 ? 512 : 1024;
-  while (nt > 256 && nbcap <= 8 * (nt / 2) && pairs > (int64_t)device_sm_count() * (1024 / nt)) nt /= 2;
+  while (nt > 128 && nbcap <= 8 * (nt / 2) && pairs > (int64_t)device_sm_count() * (1024 / nt)) nt /= 2;
   return nt;
 }
 
@@ -1991,7 +1998,7 @@ cudaError_t launch_topk(const SelectParams& p, cudaStream_t s) {
   if (p.refine && p.mpages.table) {  // dual means per page
     if (smem > 16 * 1024) {
       cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(select_topk_kernel<NT, true, true>),
-                                        NT == 256 ? 12 : NT == 512 ? 13 : 14, smem);
+                                        NT <= 256 ? 12 : NT == 512 ? 13 : 14, smem);
       if (e != cudaSuccess) return e;
     }
     return launch_pdl(select_topk_kernel<NT, true, true>, dim3(p.B * p.Hkv), dim3(NT), smem, s, p);
@@ -1999,14 +2006,14 @@ cudaError_t launch_topk(const SelectParams& p, cudaStream_t s) {
   if (p.refine) {
     if (smem > 16 * 1024) {
       cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(select_topk_kernel<NT, true>),
-                                        NT == 256 ? 8 : NT == 512 ? 9 : 10, smem);
+                                        NT <= 256 ? 8 : NT == 512 ? 9 : 10, smem);
       if (e != cudaSuccess) return e;
     }
     return launch_pdl(select_topk_kernel<NT, true>, dim3(p.B * p.Hkv), dim3(NT), smem, s, p);
   }
   if (smem > 16 * 1024) {
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(select_topk_kernel<NT, false>),
-                                      NT == 256 ? 0 : NT == 512 ? 2 : 3, smem);
+                                      NT <= 256 ? 0 : NT == 512 ? 2 : 3, smem);
     if (e != cudaSuccess) return e;
   }
   return launch_pdl(select_topk_kernel<NT, false>, dim3(p.B * p.Hkv), dim3(NT), smem, s, p);
@@ -2058,6 +2065,7 @@ cudaError_t launch_select(const SelectParams& p, cudaStream_t s) {
     }
     if (e != cudaSuccess) return e;
     switch (topk_threads(p.nbcap, (int64_t)p.B * p.Hkv)) {
+      case 128: return launch_topk<128>(p, s);
       case 256: return launch_topk<256>(p, s);
       case 512: return launch_topk<512>(p, s);
       default: return launch_topk<1024>(p, s);
@@ -2076,6 +2084,7 @@ cudaError_t launch_select(const SelectParams& p, cudaStream_t s) {
                      : launch_pdl(select_scan_kernel<false, kSelU>, gd, bd, 0, s, p);
   if (e != cudaSuccess) return e;
   switch (topk_threads(p.nbcap, (int64_t)p.B * p.Hkv)) {
+    case 128: return launch_topk<128>(p, s);
     case 256: return launch_topk<256>(p, s);
     case 512: return launch_topk<512>(p, s);
     default: return launch_topk<1024>(p, s);

@@ -2,8 +2,9 @@
 seeded random shapes; every (batch, kv head) against the oracle.
 
 The top-k CTA has 256, 512 or 1024 threads, picked from the block capacity
-(up to 1024 / 2048 / 4096 blocks), and halved while the capacity still fits
-8 keys per thread and the pairs outnumber the resident CTAs.  Each pair then
+(up to 1024 / 2048 / 4096 blocks), and halved (down to 128) while the
+capacity still fits 8 keys per thread and the pairs outnumber the resident
+CTAs.  Each pair then
 keeps its keys in registers, 4 or 8 per thread, or in shared memory beyond
 8 per thread.  The cases below sit on both sides of every switch, so a
 mistake in a boundary (an off-by-one in a key count, a halving that leaves
@@ -35,10 +36,12 @@ BOUNDARY = [
 ]
 
 # pairs beyond the resident CTAs: 2048 blocks at 512 threads halve to 256
-# (8 keys per thread); 4096 blocks at 1024 halve to 512
+# (8 keys per thread); 4096 blocks at 1024 halve to 512; 1024 blocks at 256
+# halve to 128
 HALVING = [
     W("halve_512_to_256", 38, 8, 8, D, 16, 16400, 32768, 128, 69, Lcap=32768),
     W("halve_1024_to_512", 19, 8, 8, D, 16, 16400, 65536, 128, 70, Lcap=65536),
+    W("halve_256_to_128", 76, 8, 8, D, 16, 500, 16384, 64, 72, Lcap=16384),
 ]
 
 
